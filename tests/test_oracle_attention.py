@@ -1,0 +1,167 @@
+"""Pins for oracle/attention.py: brute-force exact attention, hand-worked examples, and the
+invariants the method fixes (constant V, first causal row, weights sum to one, V * 2^k)."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import attention as A
+from oracle import formats as F
+from oracle import quant as Q
+from golden_io import keyed
+
+
+def _rand(seed, nq, nk, d, scale_k=1.0):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((nq, d))
+    k = rng.standard_normal((nk, d)) * scale_k
+    v = rng.standard_normal((nk, d))
+    return q, k, v
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n", [1, 100, 128, 129, 300])
+def test_tiled_online_softmax_equals_exact_attention(causal, n):
+    q, k, v = _rand(n, n, n, 32, scale_k=2.0)
+    o, _ = A.attention_head(q, k, v, causal, 1 / math.sqrt(32), quantize_p=False)
+    ref = A.exact_attention(q, k, v, causal, 1 / math.sqrt(32))
+    assert np.max(np.abs(o - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def test_hand_worked_examples():
+    g = keyed("attention_examples.txt")
+    d = 64
+    q = np.zeros((1, d)); q[0, 0] = 8.0
+    # example A
+    k = np.zeros((2, d)); k[1, 0] = -1.0
+    v = np.zeros((2, d)); v[0, 0] = 1.0; v[1, 1] = 1.0
+    o, _ = A.attention_head(q, k, v, False, 1 / 8)
+    want = [float(t) for t in g["A"]]
+    assert np.allclose(o[0, :3], want, rtol=0, atol=1e-15)
+    # example B
+    k = np.zeros((129, d)); k[1:128, 0] = -100.0; k[128, 0] = 2.0
+    v = np.zeros((129, d)); v[:, 2] = 1.0; v[0] = 0; v[0, 0] = 1.0; v[128] = 0; v[128, 1] = 1.0
+    o, _ = A.attention_head(q, k, v, False, 1 / 8)
+    want = [float(t) for t in g["B"]]
+    assert np.allclose(o[0, :3], want, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("c", [1.0, 0.375, -2.5])
+def test_constant_v_gives_constant_output(c):
+    q, k, _ = _rand(4, 200, 200, 64, scale_k=3.0)
+    v = np.full((200, 64), c)
+    for causal in (False, True):
+        o, _ = A.attention_head(q, k, v, causal, 0.125)
+        assert np.max(np.abs(o - c)) <= 1e-13 * abs(c)
+
+
+def test_first_causal_row_is_v0():
+    q, k, v = _rand(5, 130, 130, 64)
+    o, _ = A.attention_head(q, k, v, True, 0.125)
+    assert np.array_equal(o[0], v[0])
+
+
+def test_weights_sum_to_one_and_are_e4m3_multiples():
+    """With V = identity, O's row is the weight vector p / l: it sums to one, and l * O is a
+    vector of E4M3 values / 448 (per tile, up to the alpha rescale of earlier tiles)."""
+    n = 100
+    q, k, _ = _rand(6, 3, n, 128, scale_k=2.0)
+    v = np.eye(n, 128)
+    m, l, o = A.attention_rows(q, np.arange(3), k, v, False, 0.1)
+    w = o / l[:, None]
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-14)
+    codes = o * 448.0                              # one tile: no rescale
+    assert np.array_equal(F.e4m3_round(codes), codes)
+
+
+@pytest.mark.parametrize("kexp", [-3, 5])
+def test_v_power_of_two_scaling(kexp):
+    q, k, v = _rand(8, 150, 150, 64, scale_k=2.0)
+    o0, _ = A.attention_head(q, k, v, True, 0.125)
+    o1, _ = A.attention_head(q, k, v * 2.0 ** kexp, True, 0.125)
+    assert np.array_equal(o1, o0 * 2.0 ** kexp)
+
+
+def test_p_quantization_error_is_bounded():
+    """E4M3 rounds each weight by at most 2^-4 relative (or 2^-10/448 absolute), so O moves by
+    at most ~2 * 2^-4 * max|v| from exact attention on the same dequantized operands."""
+    q, k, v = _rand(9, 256, 256, 64, scale_k=2.0)
+    o, _ = A.attention_head(q, k, v, True, 0.125)
+    ref = A.exact_attention(q, k, v, True, 0.125)
+    assert np.max(np.abs(o - ref)) <= 2 * 2.0 ** -4 * np.abs(v).max()
+    assert np.max(np.abs(o - ref)) > 0                  # the quantization is really applied
+
+
+def test_quantized_operands_close_to_unquantized():
+    """Full QK4V8 pipeline on quantized operands stays near exact float attention (a quality
+    figure; the bound here only guards against a grossly wrong dequantization)."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((3, 256, 64)).astype(np.float32)
+    qc, qs, qt = Q.nvfp4_quantize(x[0])
+    kc, ks, kt = Q.nvfp4_quantize(x[1])
+    vc, vs = Q.mxfp8_quantize_v(x[2])
+    qh = Q.nvfp4_dequantize(qc, qs, qt)
+    kh = Q.nvfp4_dequantize(kc, ks, kt)
+    vh = Q.mxfp8_dequantize_v(vc, vs, 256)
+    o, _ = A.attention_head(qh, kh, vh, True, 0.125)
+    ref = A.exact_attention(x[0], x[1], x[2], True, 0.125)
+    rel = np.sqrt(np.mean((o - ref) ** 2)) / np.sqrt(np.mean(ref ** 2))
+    assert rel < 0.15
+
+
+def test_fp16_tiles_everywhere_close_to_exact_on_fp16_operands():
+    q, k, v = _rand(10, 200, 200, 64, scale_k=2.0)
+    q16, k16, v16 = (F.fp16_round(t) for t in (q, k, v))
+    sel_all = lambda qt, t: np.ones(qt.shape, dtype=bool)
+    m, l, o = A.attention_rows(q, np.arange(200), k, v, True, 0.125,
+                               fp16_select=sel_all, q16=q16, k16=k16, v16=v16)
+    out, _ = A.finish(m, l, o)
+    ref = A.exact_attention(q16, k16, v16, True, 0.125)
+    # only the fp16 rounding of 448 p~ remains: 2^-11 relative per weight
+    assert np.max(np.abs(out - ref)) <= 2 * 2.0 ** -11 * np.abs(v16).max()
+    # and without P rounding it is exact attention on the fp16 operands
+    m, l, o = A.attention_rows(q, np.arange(200), k, v, True, 0.125, quantize_p=False,
+                               fp16_select=sel_all, q16=q16, k16=k16, v16=v16)
+    out, _ = A.finish(m, l, o)
+    assert np.max(np.abs(out - ref)) <= 1e-12
+
+
+def test_fp16_selection_only_changes_selected_tiles():
+    q, k, v = _rand(11, 256, 256, 64, scale_k=2.0)
+    q16, k16, v16 = (F.fp16_round(t) for t in (q, k, v))
+    none = lambda qt, t: np.zeros(qt.shape, dtype=bool)
+    base = A.attention_rows(q, np.arange(256), k, v, True, 0.125)
+    same = A.attention_rows(q, np.arange(256), k, v, True, 0.125,
+                            fp16_select=none, q16=q16, k16=k16, v16=v16)
+    assert all(np.array_equal(a, b) for a, b in zip(base, same))
+    only = lambda qt, t: (qt == 1) & (t == 0)
+    mix = A.attention_rows(q, np.arange(256), k, v, True, 0.125,
+                           fp16_select=only, q16=q16, k16=k16, v16=v16)
+    assert np.array_equal(mix[2][:128], base[2][:128])        # q tile 0 untouched
+    assert not np.array_equal(mix[2][128:], base[2][128:])
+
+
+def test_split_merge_is_exact_without_p_rounding():
+    q, k, v = _rand(12, 4, 1000, 64, scale_k=2.0)
+    rows = np.full(4, 999)
+    parts = [A.attention_rows(q, rows, k, v, False, 0.125, quantize_p=False,
+                              key_begin=b, key_end=min(b + 256, 1000)) for b in range(0, 1000, 256)]
+    o, _ = A.finish(*A.merge_splits(parts))
+    ref = A.exact_attention(q, k, v, False, 0.125)
+    assert np.max(np.abs(o - ref)) <= 1e-12
+
+
+def test_decode_one_split_equals_prefill_row():
+    q, k, v = _rand(13, 4, 777, 64, scale_k=2.0)
+    o1, _ = A.decode_rows(q, k, v, 777, 0.125, split_tokens=0)
+    m, l, o = A.attention_rows(q, np.full(4, 776), k, v, False, 0.125)
+    o2, _ = A.finish(m, l, o)
+    assert np.array_equal(o1, o2)
+    o3, _ = A.decode_rows(q, k, v, 777, 0.125, split_tokens=256)   # splits: close, not equal
+    assert np.max(np.abs(o3 - o1)) < 0.1 * np.abs(o1).max()
+
+
+def test_decode_context_length_one_is_v0():
+    q, k, v = _rand(14, 4, 10, 64)
+    o, _ = A.decode_rows(q, k, v, 1, 0.125, split_tokens=128)
+    assert np.array_equal(o, np.repeat(v[:1], 4, axis=0))
