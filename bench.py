@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the QK4V8 hot path on B200; prints ONE JSON line (rank 0).
+
+Default workload: causal prefill, batch 1, 16 heads, 4096 tokens, head_dim 128, bf16 inputs.
+A step = quantize Q and K (NVFP4), quantize V (MXFP8), QK4V8 attention forward. Other
+workloads (--workload): prefill_gqa_n32768, mixed_prefill_n16384 (tile scoring + FP16 tiles
+in the step), paged_decode_s64 (one decode step: quantize the step's Q, paged split-K decode).
+
+Timing: inputs resident in HBM; W warm-up steps; then K steps, each bracketed by CUDA events
+on the launching stream, with a 256 MB L2 flush between steps (outside the events); barrier +
+synchronize on both sides; max over ranks. `e2e` repeats the step through the same public
+API with the inputs copied from pinned host memory and the output read back inside the timed
+region. Multi-GPU (torchrun): independent replicas, one per GPU (no collective in the path).
+`--impl reference` times the CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_block_scaled_nvfp4_b200 import workloads  # noqa: E402
+
+METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of HBM peak"
+FP4_OVER_BF16 = 4.0          # nominal dense ratio 9 PF / 2.25 PF
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def prefill_flops(cfg):
+    """Algorithmic FLOPs: 4 d per visible (query, key) pair (QK^T and PV)."""
+    B, H, N, d = cfg["B"], cfg["Hq"], cfg["N"], cfg["d"]
+    pairs = N * (N + 1) // 2 if cfg["causal"] else N * N
+    return 4.0 * d * pairs * B * H
+
+
+def decode_bytes(lay):
+    """Algorithmic KV bytes of one decode step: per token and KV head 64 + 8 (K codes,
+    scales) + 128 + 4 (V codes, scales) at d = 128, whole pages counted, plus Q, page table,
+    lengths and the output."""
+    cfg = lay.cfg
+    d, hkv, hq, S = cfg["d"], cfg["Hkv"], cfg["Hq"], cfg["S"]
+    per_tok = d // 2 + d // 16 + d + d // 32
+    pages = ((lay.lens.long() + 63) // 64).sum().item()
+    kv = pages * 64 * hkv * per_tok
+    other = S * hq * (d // 2 + d // 16) + lay.page_table.numel() * 4 + S * 4 + S * hq * d * 2
+    return float(kv), float(kv + other)
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in (self.out or "").splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------
+# The steps (our arm)
+# ---------------------------------------------------------------------------------------
+def make_prefill_step(name):
+    from bit_block_scaled_nvfp4_b200 import api
+    w = workloads.make_prefill(name)
+    cfg = w.cfg
+    q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
+    mixed = cfg.get("frac_bp", 0) > 0
+    scale = 1.0 / math.sqrt(cfg["d"])
+    ev = {}
+
+    def step(q=q, k=k, v=v, mark=None):
+        q4 = api.quantize_nvfp4(q, want_fp16=mixed)
+        k4 = api.quantize_nvfp4(k, want_fp16=mixed)
+        v8 = api.quantize_mxfp8_v(v, want_fp16=mixed)
+        bitmap = None
+        if mixed:
+            _, _, bitmap = api.tile_score_select(q4, k4, cfg["causal"], cfg["frac_bp"])
+        if mark is not None:
+            mark[0].record()
+        out = api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=bitmap)
+        if mark is not None:
+            mark[1].record()
+        return out
+
+    launches = 6 + (3 if mixed else 0)
+    host = [w.q.pin_memory(), w.k.pin_memory(), w.v.pin_memory()]
+    return dict(cfg=cfg, step=step, inputs=(q, k, v), host=host, launches=launches,
+                flops=prefill_flops(cfg), kind="prefill", ev=ev)
+
+
+def make_decode_step(name):
+    from bit_block_scaled_nvfp4_b200 import api, paged
+    lay = workloads.make_decode_layout(name)
+    cfg = lay.cfg
+    cache = paged.empty_cache(lay.num_pages, cfg["Hkv"], cfg["d"], workloads.DECODE_K_TENSOR_SCALE, "cuda")
+    lens = lay.lens.tolist()
+    for s in range(cfg["S"]):
+        k, v = workloads.make_decode_sequence(lay, s)
+        paged.write_sequence(cache, k.cuda(), v.cuda(), lay.page_table[s, :(lens[s] + 63) // 64])
+    q = workloads.make_decode_query(lay).cuda()
+    table, ctx = lay.page_table.cuda(), lay.lens.cuda()
+    split = 4096
+    ws = torch.empty(cfg["S"] * cfg["Hq"] * ((max(lens) + split - 1) // split) * (cfg["d"] + 2) * 4,
+                     dtype=torch.uint8, device="cuda")
+
+    def step(q=q, table=table, ctx=ctx, mark=None):
+        q4 = api.quantize_nvfp4(q)
+        if mark is not None:
+            mark[0].record()
+        out = api.attn_qk4v8_decode_paged(q4, cache, table, ctx, max(lens), split, workspace=ws)
+        if mark is not None:
+            mark[1].record()
+        return out
+
+    kv, total = decode_bytes(lay)
+    host = [workloads.make_decode_query(lay).pin_memory(), lay.page_table.pin_memory(), lay.lens.pin_memory()]
+    return dict(cfg=cfg, step=step, inputs=(q, table, ctx), host=host, launches=4, kv_bytes=kv,
+                bytes=total, kind="decode", split=split, lay=lay)
+
+
+def time_steps(st, K, W, world):
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    step = st["step"]
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    k0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    k1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        s_ev[i].record()
+        step(mark=(k0[i], k1[i]))
+        e_ev[i].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    step_ms = sum(s.elapsed_time(e) for s, e in zip(s_ev, e_ev)) / K
+    kern_ms = sum(a.elapsed_time(b) for a, b in zip(k0, k1)) / K
+    return step_ms, kern_ms
+
+
+def time_e2e(st, K, world):
+    """Same step through the public API with H2D of the inputs and D2H of the output."""
+    host = st["host"]
+    dev = [torch.empty_like(h, device="cuda") for h in host]
+    out_host = None
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    h2d = sum(h.numel() * h.element_size() for h in host)
+    d2h = 0
+    tot = 0.0
+    barrier(world)
+    for i in range(K + 1):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for d_, h_ in zip(dev, host):
+            d_.copy_(h_, non_blocking=True)
+        out = st["step"](*dev)
+        if out_host is None:
+            out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        out_host.copy_(out, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        if i > 0:                       # the first pass allocates the pinned output
+            tot += a.elapsed_time(b)
+        d2h = out.numel() * out.element_size()
+    barrier(world)
+    return tot / K, h2d, d2h
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline leg)
+# ---------------------------------------------------------------------------------------
+def oracle_sample(name, rows=256, heads=1):
+    """Time the oracle, as it stands, on a bounded sample of the workload: ``heads`` query
+    heads x ``rows`` query rows spread over the sequence (prefill; the whole-tensor scales
+    are computed once), or ``rows // 64`` sequences' worth of decode steps. Returns
+    (seconds, algorithmic units (FLOPs or bytes) done, description)."""
+    from oracle import attention as OA
+    from oracle import quant as OQ
+    from oracle import paged as OP
+    if name == "paged_decode_s64":
+        lay = workloads.make_decode_layout(name)
+        cfg = lay.cfg
+        q = workloads.make_decode_query(lay).float().numpy()
+        t0 = time.perf_counter()
+        qc, qs, qt = OQ.nvfp4_quantize(q)
+        qh = OQ.nvfp4_dequantize(qc, qs, qt)
+        s = int(np.argmin(lay.lens.numpy()))
+        k, v = workloads.make_decode_sequence(lay, s)
+        n = int(lay.lens[s])
+        kc, ks, vc, vs = OP.quantize_sequence(k.float().numpy(), v.float().numpy(),
+                                              workloads.DECODE_K_TENSOR_SCALE)
+        kh = OQ.nvfp4_dequantize(kc, ks, np.float32(workloads.DECODE_K_TENSOR_SCALE))
+        vh = OQ.mxfp8_dequantize_v(vc, vs, n)
+        g = cfg["Hq"] // cfg["Hkv"]
+        for h in range(cfg["Hkv"]):
+            OA.decode_rows(qh[s, h * g:(h + 1) * g], kh[h], vh[h], n, 1 / math.sqrt(cfg["d"]), 4096)
+        dt = time.perf_counter() - t0
+        per_tok = cfg["d"] // 2 + cfg["d"] // 16 + cfg["d"] + cfg["d"] // 32
+        units = ((n + 63) // 64) * 64 * cfg["Hkv"] * per_tok
+        return dt, float(units), f"1 sequence ({n} tokens) x {cfg['Hkv']} KV heads of one decode step"
+    w = workloads.make_prefill(name)
+    cfg = w.cfg
+    N, d = cfg["N"], cfg["d"]
+    rng = np.random.default_rng(0)
+    row_idx = np.sort(rng.choice(N, size=min(rows, N), replace=False))
+    scale = 1 / math.sqrt(d)
+    q32 = w.q.float().numpy()
+    k32 = w.k.float().numpy()
+    t0 = time.perf_counter()
+    sq = OQ.nvfp4_tensor_scale(q32)
+    sk = OQ.nvfp4_tensor_scale(k32)
+    flops = 0.0
+    for hq in range(heads):
+        hk = hq // (cfg["Hq"] // cfg["Hkv"])
+        qh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(q32[0, hq, row_idx], tensor_scale=sq))
+        kh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(k32[0, hk], tensor_scale=sk))
+        vc, vs = OQ.mxfp8_quantize_v(w.v[0, hk].float().numpy())
+        vh = OQ.mxfp8_dequantize_v(vc, vs, N)
+        OA.attention_rows(qh, row_idx, kh, vh, cfg["causal"], scale)
+        vis = (row_idx + 1).sum() if cfg["causal"] else len(row_idx) * N
+        flops += 4.0 * d * float(vis)
+    dt = time.perf_counter() - t0
+    return dt, flops, f"{heads} query head(s) x {len(row_idx)} seeded query rows (of {N})"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    name = args.workload
+    is_decode = name == "paged_decode_s64"
+    vals = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        dt, units, desc = oracle_sample(name, rows=64, heads=1)
+        if i >= args.warmup:
+            vals.append(units / dt / (1e9 if is_decode else 1e12))
+    v = statistics.mean(vals)
+    unit = "GB/s" if is_decode else "TFLOP/s"
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, **{k: v_ for k, v_ in workloads.WORKLOADS[name].items()}},
+            "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill_h16_n4096",
+                    choices=[n for n in workloads.WORKLOADS if n != "tiny_prefill"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    name = args.workload
+    st = make_decode_step(name) if name == "paged_decode_s64" else make_prefill_step(name)
+    with Clocks(torch.cuda.current_device()) as clk:
+        step_ms, kern_ms = time_steps(st, args.steps, args.warmup, world)
+    e2e_ms, h2d, d2h = time_e2e(st, max(3, args.steps // 3), world)
+    step_ms = max_over_ranks(step_ms, world)
+    kern_ms = max_over_ranks(kern_ms, world)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    pk, src = peaks()
+    cfg = st["cfg"]
+    if st["kind"] == "prefill":
+        units = st["flops"]
+        value = units * world / (step_ms * 1e-3) / 1e12
+        e2e_v = units * world / (e2e_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        ach = units / (kern_ms * 1e-3) / 1e12
+        peak = pk["bf16_tflops"] * FP4_OVER_BF16
+        roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": None,
+                "kernel": "attn_fwd_kernel", "peak_source": f"{src} bf16 x {FP4_OVER_BF16:g} (FP4 dense)",
+                "mixed_fp4_fp8_bound_tflops": peak / 1.5}
+    else:
+        units = st["bytes"]
+        value = units * world / (step_ms * 1e-3) / 1e9
+        e2e_v = units * world / (e2e_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        ach = st["kv_bytes"] / (kern_ms * 1e-3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": None, "kernel": "decode_kernel + decode_merge_kernel",
+                "peak_source": f"{src} hbm_gbs"}
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4/mxfp8 (fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": name, **{k: v_ for k, v_ in workloads.WORKLOADS[name].items()},
+                       "l2": "256 MB flush between timed steps", "parallelism": f"replicas x{world}"},
+            "roofline": roof,
+            "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": st["launches"] * args.steps,
+            "clocks": clk.summary()}
+    if rank == 0 and not args.no_cpu_baseline:
+        dt, u, desc = oracle_sample(name, rows=64 if st["kind"] == "prefill" else 64, heads=1)
+        cv = u / dt / (1e12 if st["kind"] == "prefill" else 1e9)
+        line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
+                                "sample": desc, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+"""Torch-facing binding of libqk4v8.so: the C entry points under the same names.
+
+These functions allocate outputs and workspaces with torch on the input's device, take the
+current CUDA stream, and pass raw pointers to the library. They do no arithmetic of their own:
+every step of the path runs in the library's kernels, and a missing library raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+_DT = {torch.float16: _lib.QK4V8_F16, torch.bfloat16: _lib.QK4V8_BF16}
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise TypeError(f"expected fp16 or bf16, got {t.dtype}")
+    return _DT[t.dtype]
+
+
+@dataclass
+class NVFP4Tensor:
+    """NVFP4 codes [..., D/2], E4M3 scales [..., D/16], FP32 tensor scale (1-element device
+    tensor) and, on request, an fp16 copy of the input [..., D]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    tensor_scale: torch.Tensor
+    fp16: torch.Tensor | None = None
+
+
+@dataclass
+class MXFP8V:
+    """MXFP8 V: codes [..., D, Npad] (token-contiguous), E8M0 scales [..., D, Npad/32], the
+    true token count, and on request an fp16 copy [..., D, Npad]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    n_tokens: int
+    fp16: torch.Tensor | None = None
+
+
+def check_status(stream=None) -> int:
+    """Synchronise the stream and return the device status (0 = ok); see qk4v8_check_status."""
+    s = C.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+    return _lib.load().qk4v8_check_status(s)
+
+
+def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16: bool = False,
+                   workspace: torch.Tensor | None = None) -> NVFP4Tensor:
+    """NVFP4-quantize ``x`` (..., D) along its last axis (contiguous fp16/bf16 CUDA tensor)."""
+    lib = _lib.load()
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    dev = x.device
+    codes = torch.empty(*x.shape[:-1], cols // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(*x.shape[:-1], cols // 16, dtype=torch.uint8, device=dev)
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    x16 = torch.empty(x.shape, dtype=torch.float16, device=dev) if want_fp16 else None
+    if workspace is None:
+        workspace = torch.empty(lib.quantize_nvfp4_workspace_size(), dtype=torch.uint8, device=dev)
+    st = lib.quantize_nvfp4(_ptr(x), _dtype(x), rows, cols, cols,
+                            float(tensor_scale) if tensor_scale else 0.0, _ptr(codes),
+                            _ptr(scales), _ptr(ts), _ptr(x16), _ptr(workspace),
+                            workspace.numel(), _stream())
+    _lib.check(st, "quantize_nvfp4")
+    return NVFP4Tensor(codes, scales, ts, x16)
+
+
+def quantize_mxfp8_v(v: torch.Tensor, want_fp16: bool = False) -> MXFP8V:
+    """MXFP8-quantize V laid out (..., N, D) along the token axis."""
+    lib = _lib.load()
+    if not v.is_cuda or not v.is_contiguous():
+        raise ValueError("v must be a contiguous CUDA tensor")
+    n, d = v.shape[-2], v.shape[-1]
+    bh = v.numel() // (n * d)
+    npad = (n + 127) // 128 * 128
+    lead = v.shape[:-2]
+    codes = torch.empty(*lead, d, npad, dtype=torch.uint8, device=v.device)
+    scales = torch.empty(*lead, d, npad // 32, dtype=torch.uint8, device=v.device)
+    v16 = torch.empty(*lead, d, npad, dtype=torch.float16, device=v.device) if want_fp16 else None
+    st = lib.quantize_mxfp8_v(_ptr(v), _dtype(v), bh, n, d, _ptr(codes), _ptr(scales),
+                              _ptr(v16), _stream())
+    _lib.check(st, "quantize_mxfp8_v")
+    return MXFP8V(codes, scales, n, v16)
+
+
+def tile_score_select(q: NVFP4Tensor, k: NVFP4Tensor, causal: bool, frac_bp: int,
+                      k_max: int | None = None):
+    """Top-fraction tile selection. q.codes [B, Hq, N, D/2], k.codes [B, Hkv, N, D/2].
+    Returns (idx [B*Hq, k_max] rank-ordered, n_sel [B*Hq], bitmap [B*Hq, T, T])."""
+    lib = _lib.load()
+    B, Hq, N, dh = q.codes.shape
+    Hkv = k.codes.shape[1]
+    d = dh * 2
+    T = (N + 127) // 128
+    n_cand = T * (T + 1) // 2 if causal else T * T
+    need = (n_cand * frac_bp + 9999) // 10000
+    k_max = max(need, 1) if k_max is None else k_max
+    dev = q.codes.device
+    idx = torch.full((B * Hq, k_max), -1, dtype=torch.int32, device=dev)
+    n_sel = torch.empty(B * Hq, dtype=torch.int32, device=dev)
+    bitmap = torch.empty(B * Hq, T, T, dtype=torch.uint8, device=dev)
+    wsb = lib.tile_score_select_workspace_size(B, Hq, Hkv, N)
+    ws = torch.empty(max(wsb, 8), dtype=torch.uint8, device=dev)
+    st = lib.tile_score_select(_ptr(q.codes), _ptr(q.scales), _ptr(k.codes), _ptr(k.scales),
+                               B, Hq, Hkv, N, d, int(causal), int(frac_bp), int(k_max),
+                               _ptr(idx), _ptr(n_sel), _ptr(bitmap), _ptr(ws), ws.numel(),
+                               _stream())
+    _lib.check(st, "tile_score_select")
+    return idx, n_sel, bitmap
+
+
+def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
+                   softmax_scale: float | None = None, out_dtype=torch.bfloat16,
+                   fp16_bitmap: torch.Tensor | None = None, want_lse: bool = False):
+    """QK4V8 attention forward. q.codes [B, Hq, Nq, D/2], k.codes [B, Hkv, Nk, D/2],
+    v.codes [B, Hkv, D, Nk_pad]. With ``fp16_bitmap`` the FP16 copies (q.fp16, k.fp16,
+    v.fp16) must be present. Returns out [B, Hq, Nq, D] (and lse [B, Hq, Nq])."""
+    lib = _lib.load()
+    B, Hq, Nq, dh = q.codes.shape
+    Hkv, Nk = k.codes.shape[1], k.codes.shape[2]
+    d = dh * 2
+    out = torch.empty(B, Hq, Nq, d, dtype=out_dtype, device=q.codes.device)
+    lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.codes.device) if want_lse else None
+    p = _lib.FwdParams()
+    p.q_codes, p.q_scales, p.q_tensor_scale = q.codes.data_ptr(), q.scales.data_ptr(), q.tensor_scale.data_ptr()
+    p.k_codes, p.k_scales, p.k_tensor_scale = k.codes.data_ptr(), k.scales.data_ptr(), k.tensor_scale.data_ptr()
+    p.v_codes, p.v_scales = v.codes.data_ptr(), v.scales.data_ptr()
+    p.batch, p.q_heads, p.kv_heads, p.n_q, p.n_k, p.head_dim = B, Hq, Hkv, Nq, Nk, d
+    p.causal = int(causal)
+    p.softmax_scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    if fp16_bitmap is not None:
+        p.fp16_bitmap = fp16_bitmap.data_ptr()
+        p.q16, p.k16, p.v16 = q.fp16.data_ptr(), k.fp16.data_ptr(), v.fp16.data_ptr()
+    p.out_dtype = _DT[out_dtype]
+    p.out = out.data_ptr()
+    p.lse = lse.data_ptr() if lse is not None else None
+    _lib.check(lib.attn_qk4v8_fwd(C.byref(p), _stream()), "attn_qk4v8_fwd")
+    return (out, lse) if want_lse else out
+
+
+@dataclass
+class PagedKV:
+    """Paged NVFP4-K / MXFP8-V cache (64-token pages)."""
+    k_pages: torch.Tensor        # [P, Hkv, 64, D/2]
+    k_scales: torch.Tensor       # [P, Hkv, 64, D/16]
+    k_tensor_scale: torch.Tensor  # [1] float
+    v_pages: torch.Tensor        # [P, Hkv, D, 64]
+    v_scales: torch.Tensor       # [P, Hkv, D, 2]
+
+
+def decode_params(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
+                  context_lens: torch.Tensor, max_context: int, split_tokens: int,
+                  out: torch.Tensor, softmax_scale: float | None = None, lse=None):
+    S, Hq, dh = q.codes.shape
+    P, Hkv = cache.k_pages.shape[0], cache.k_pages.shape[1]
+    d = dh * 2
+    p = _lib.DecodeParams()
+    p.q_codes, p.q_scales, p.q_tensor_scale = q.codes.data_ptr(), q.scales.data_ptr(), q.tensor_scale.data_ptr()
+    p.k_pages, p.k_page_scales, p.k_tensor_scale = (cache.k_pages.data_ptr(), cache.k_scales.data_ptr(),
+                                                    cache.k_tensor_scale.data_ptr())
+    p.v_pages, p.v_page_scales = cache.v_pages.data_ptr(), cache.v_scales.data_ptr()
+    p.page_table, p.context_lens = page_table.data_ptr(), context_lens.data_ptr()
+    p.num_seqs, p.num_pages, p.max_pages = S, P, page_table.shape[1]
+    p.q_heads, p.kv_heads, p.head_dim = Hq, Hkv, d
+    p.max_context, p.split_tokens = int(max_context), int(split_tokens)
+    p.softmax_scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    p.out_dtype = _DT[out.dtype]
+    p.out = out.data_ptr()
+    p.lse = lse.data_ptr() if lse is not None else None
+    return p
+
+
+def attn_qk4v8_decode_paged(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
+                            context_lens: torch.Tensor, max_context: int, split_tokens: int,
+                            softmax_scale: float | None = None, out_dtype=torch.bfloat16,
+                            want_lse: bool = False, workspace: torch.Tensor | None = None):
+    """One decode step. q.codes [S, Hq, D/2]; returns out [S, Hq, D] (and lse [S, Hq])."""
+    lib = _lib.load()
+    S, Hq, dh = q.codes.shape
+    out = torch.empty(S, Hq, dh * 2, dtype=out_dtype, device=q.codes.device)
+    lse = torch.empty(S, Hq, dtype=torch.float32, device=q.codes.device) if want_lse else None
+    p = decode_params(q, cache, page_table, context_lens, max_context, split_tokens, out,
+                      softmax_scale, lse)
+    need = lib.attn_qk4v8_decode_workspace_size(C.byref(p))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.codes.device)
+    st = lib.attn_qk4v8_decode_paged(C.byref(p), _ptr(workspace), workspace.numel(), _stream())
+    _lib.check(st, "attn_qk4v8_decode_paged")
+    return (out, lse) if want_lse else out
+
+
+def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool,
+                    softmax_scale: float | None = None, fp16_frac_bp: int = 0,
+                    out_dtype=None, want_lse: bool = False):
+    """The whole prefill path on bf16/fp16 CUDA tensors q [B, Hq, N, D], k/v [B, Hkv, N, D]:
+    quantize Q, K (NVFP4) and V (MXFP8), optionally score tiles and recompute the top
+    ``fp16_frac_bp`` basis points of them in FP16, then attention."""
+    mixed = fp16_frac_bp > 0
+    q4 = quantize_nvfp4(q, want_fp16=mixed)
+    k4 = quantize_nvfp4(k, want_fp16=mixed)
+    v8 = quantize_mxfp8_v(v, want_fp16=mixed)
+    bitmap = None
+    if mixed:
+        _, _, bitmap = tile_score_select(q4, k4, causal, fp16_frac_bp)
+    return attn_qk4v8_fwd(q4, k4, v8, causal, softmax_scale, out_dtype or q.dtype,
+                          fp16_bitmap=bitmap, want_lse=want_lse)

@@ -1,0 +1,496 @@
+// QK4V8 prefill attention on sm_100a tensor cores.
+//
+// Method (hotelren.com MpFA article §1, §3.3-3.4; problem statement): Q and K in NVFP4, V in
+// MXFP8; S = Q K^T on block-scaled FP4 tensor cores (tcgen05 kind::mxf4nvf4, E4M3 scale per
+// 16 elements) accumulated in FP32; online softmax in FP32 over 128-key tiles; P quantized to
+// E4M3 as P*448 against the running max after the tile; O += P V on block-scaled FP8 tensor
+// cores (kind::mxf8f6f4, E8M0 scale per 32 tokens; P's scale is 1); O / l at the end, where
+// l sums the quantized weights. Optional FP16 tiles (ai-feeds.com ThriftAttention summary,
+// "方法" step 3): a tile marked in the selection bitmap runs QK^T and PV with kind::f16 on
+// FP16 copies of Q, K, V, with P = fp16(448 exp(s - m)), into the same (m, l, O).
+//
+// One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
+//   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
+//              tcgen05 scale layout with plain loads, FP16 tiles when selected
+//   warp 1     TMEM owner and MMA issuer (one thread)
+//   warps 2-5  softmax: each thread owns one query row (its TMEM lane); also rescales O
+//              and writes the output
+// TMEM (512 columns): S double buffer [0,256), O [256, 256+D), scale factors from 384.
+#pragma once
+#include "ptx.cuh"
+
+namespace qk4v8 {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2_448 = 8.807354922057604f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct FwdArgs {
+  const uint8_t* q_scales;
+  const uint8_t* k_scales;
+  const uint8_t* v_scales;
+  const float* q_ts;
+  const float* k_ts;
+  const uint8_t* bitmap;      // [B*Hq, Tq, Tk] or null
+  void* out;
+  float* lse;
+  int32_t B, Hq, Hkv, Nq, Nk, Npad, Tq, Tk;
+  int32_t causal;
+  float softmax_scale;
+  int32_t out_bf16;
+};
+
+template <int D, bool kMixed>
+struct FwdLayout {
+  static constexpr int NS = 3;
+  static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
+  static constexpr int Q_BYTES = 128 * D / 2;
+  static constexpr int K_BYTES = 128 * D / 2;
+  static constexpr int V_BYTES = D * 128;
+  static constexpr int SF_CHUNK = 512;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_QSF = OFF_Q + Q_BYTES;                         // KSTEPS chunks
+  static constexpr int OFF_PSF = OFF_QSF + 1024;
+  static constexpr int OFF_STAGE = OFF_PSF + 1024;
+  static constexpr int ST_K = 0;
+  static constexpr int ST_V = K_BYTES;
+  static constexpr int ST_KSF = ST_V + V_BYTES;
+  static constexpr int ST_VSF = ST_KSF + 1024;
+  static constexpr int STAGE_BYTES = ST_VSF + 1024;
+  static constexpr int OFF_P = OFF_STAGE + NS * STAGE_BYTES;               // 2 x 16 KB
+  static constexpr int OFF_Q16 = OFF_P + 2 * 16384;
+  static constexpr int F16_TILE = 128 * D * 2;
+  static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
+  static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
+  static constexpr int OFF_BAR = OFF_V16 + (kMixed ? F16_TILE : 0);
+  static constexpr int N_BARS = 1 + 2 * NS + 2 * 4 + 3 + 1;
+  static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
+  // TMEM columns
+  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 384, T_PSF = 392, T_KSF = 400,
+                            T_VSF = 424;
+  static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
+  static constexpr uint32_t QK_SBO = 8 * D / 2;
+};
+
+template <int D, bool kMixed>
+__global__ void __launch_bounds__(192, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q16,
+                const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
+                FwdArgs a) {
+  using L = FwdLayout<D, kMixed>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + L::NS;
+  uint64_t* s_full = bars + 1 + 2 * L::NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_full + 4;
+  uint64_t* pv_done = s_full + 6;
+  uint64_t* kv16_full = s_full + 8;
+  uint64_t* kv16_empty = s_full + 9;
+  uint64_t* q16_full = s_full + 10;
+  uint64_t* mma_final = s_full + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::N_BARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BHq = a.B * a.Hq;
+  const int qt = a.Tq - 1 - static_cast<int>(blockIdx.x / BHq);
+  const int bhq = static_cast<int>(blockIdx.x % BHq);
+  const int b = bhq / a.Hq, hq = bhq % a.Hq;
+  const int hk = hq / (a.Hq / a.Hkv);
+  const int bhk = b * a.Hkv + hk;
+  const int nt = a.causal ? min(qt + 1, a.Tk) : a.Tk;
+  const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(bhq) * a.Tq + qt) * a.Tk : nullptr;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1); mbar_init(s_free + i, 4);
+      mbar_init(p_full + i, 4); mbar_init(pv_done + i, 1);
+    }
+    mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1); mbar_init(q16_full, 1);
+    mbar_init(mma_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // P scale factors (E8M0 127 = 1.0) for the PV MMA's A operand.
+  for (int i = threadIdx.x; i < 128; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(sm + L::OFF_PSF)[i] = 0x7F7F7F7Fu;
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  // Producer and softmax warps wait warp-uniformly; the MMA issuer waits alone.
+  auto waitw = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return bounded_wait_warp(bar, parity, abort_flag);
+  };
+  auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return bounded_wait(bar, parity, abort_flag);
+  };
+
+  if (warp == 0) {
+    // ================================ producer ================================
+    if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); }
+    // Q scale factors: row r = r0 + 32 r1 -> chunk byte r0*16 + r1*4 + k (k = 0..3 within a
+    // 64-element MMA step); Q codes by TMA.
+    {
+      const int64_t row0 = static_cast<int64_t>(bhq) * a.Nq + qt * 128;
+      uint32_t w[4][L::KSTEPS];
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) {
+        const int r = r1 * 32 + lane;
+        const bool ok = qt * 128 + r < a.Nq;
+        if constexpr (L::KSTEPS == 2) {
+          uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(a.q_scales + (row0 + r) * (D / 16)))
+                       : make_uint2(0, 0);
+          w[r1][0] = v.x; w[r1][1] = v.y;
+        } else {
+          w[r1][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(a.q_scales + (row0 + r) * (D / 16))) : 0u;
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < L::KSTEPS; ++kk)
+        *reinterpret_cast<uint4*>(sm + L::OFF_QSF + kk * 512 + lane * 16) =
+            make_uint4(w[0][kk], w[1][kk], w[2][kk], w[3][kk]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, L::Q_BYTES);
+        tma_load_3d(sm + L::OFF_Q, &tm_q, q_full, 0, qt * 128, bhq);
+      }
+    }
+    bool q16_loaded = false;
+    int n16 = 0;
+    for (int j = 0; j < nt; ++j) {
+      const int s = j % L::NS;
+      if (j >= L::NS && !waitw(kv_empty + s, ((j / L::NS) - 1) & 1)) break;
+      unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+      // K scale factors of keys j*128 .. j*128+127
+      const int64_t krow0 = static_cast<int64_t>(bhk) * a.Nk + j * 128;
+      uint32_t w[4][L::KSTEPS];
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) {
+        const int r = r1 * 32 + lane;
+        const bool ok = j * 128 + r < a.Nk;
+        if constexpr (L::KSTEPS == 2) {
+          uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(a.k_scales + (krow0 + r) * (D / 16)))
+                       : make_uint2(0, 0);
+          w[r1][0] = v.x; w[r1][1] = v.y;
+        } else {
+          w[r1][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(a.k_scales + (krow0 + r) * (D / 16))) : 0u;
+        }
+      }
+#pragma unroll
+      for (int kk = 0; kk < L::KSTEPS; ++kk)
+        *reinterpret_cast<uint4*>(st + L::ST_KSF + kk * 512 + lane * 16) =
+            make_uint4(w[0][kk], w[1][kk], w[2][kk], w[3][kk]);
+      // V scale factors: channel row c, 4 E8M0 codes (32 tokens each) of this key tile
+      uint32_t vw[4];
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) {
+        const int c = r1 * 32 + lane;
+        vw[r1] = c < D ? __ldg(reinterpret_cast<const uint32_t*>(
+                             a.v_scales + (static_cast<int64_t>(bhk) * D + c) * (a.Npad / 32) + j * 4))
+                       : 0x7F7F7F7Fu;
+      }
+      *reinterpret_cast<uint4*>(st + L::ST_VSF + lane * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_BYTES);
+        tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, bhk);
+        tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, bhk * D);
+      }
+      if constexpr (kMixed) {
+        if (bm_row[j]) {
+          if (!q16_loaded) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(q16_full, L::F16_TILE);
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_3d(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, qt * 128, bhq);
+            }
+            q16_loaded = true;
+          }
+          if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1)) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(kv16_full, 2 * L::F16_TILE);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(sm + L::OFF_K16 + h * 16384, &tm_k16, kv16_full, h * 64, j * 128, bhk);
+            for (int h = 0; h < 2; ++h)
+              tma_load_2d(sm + L::OFF_V16 + h * (D * 128), &tm_v16, kv16_full, j * 128 + h * 64, bhk * D);
+          }
+          ++n16;
+        }
+      }
+    }
+    // Drain: never leave a copy in flight into this CTA's shared memory.
+    for (int s = 0; s < L::NS && s < nt; ++s) {
+      const int last = s + ((nt - 1 - s) / L::NS) * L::NS;
+      mbar_wait(kv_full + s, (last / L::NS) & 1);
+    }
+    mbar_wait(q_full, 0);
+    if (kMixed && n16 > 0) { mbar_wait(kv16_full, (n16 - 1) & 1); mbar_wait(q16_full, 0); }
+  } else if (warp == 1) {
+    // ================================ MMA issuer ================================
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, 128);
+      const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, D);
+      const uint32_t idesc_qk16 = idesc_f16(128, 128);
+      const uint32_t idesc_pv16 = idesc_f16(128, D);
+      const uint32_t sQ = smem_u32(sm + L::OFF_Q);
+      const uint32_t sP = smem_u32(sm + L::OFF_P);
+      bool ok = wait1(q_full, 0);
+      if (ok) {
+        tc_fence_after();
+        for (int kk = 0; kk < L::KSTEPS; ++kk)
+          tmem_cp_sf(tbase + L::T_QSF + 4 * kk, sm + L::OFF_QSF + kk * 512);
+        tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+      }
+      int n16_qk = 0, n16_pv = 0;
+      bool q16_ready = false;
+      auto issue_pv = [&](int jj) -> bool {
+        const int s = jj % L::NS, b2 = jj & 1;
+        const bool f16 = kMixed && bm_row[jj];
+        if (!wait1(p_full + b2, (jj >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t tO = tbase + L::T_O;
+        if (!f16) {
+          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+          const uint32_t tv = tbase + L::T_VSF + 4 * s;
+          tmem_cp_sf(tv, st + L::ST_VSF);
+          const uint32_t sV = smem_u32(st + L::ST_V);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = make_sdesc(sP + b2 * 16384 + kk * 32, 16, 1024, kSw128);
+            const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
+            mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
+                     (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+          const uint32_t sV16 = smem_u32(sm + L::OFF_V16);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
+            const uint64_t db = make_sdesc(sV16 + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024, kSw128);
+            mma_f16(tO, da, db, idesc_pv16, (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(kv16_empty);
+          ++n16_pv;
+        }
+        mma_commit(pv_done + b2);
+        mma_commit(kv_empty + s);
+        return true;
+      };
+      for (int j = 0; ok && j < nt; ++j) {
+        const int s = j % L::NS, b2 = j & 1;
+        const bool f16 = kMixed && bm_row[j];
+        if (!wait1(kv_full + s, (j / L::NS) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (j >= 2 && !wait1(s_free + b2, ((j - 2) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tbase + L::T_S + b2 * 128;
+        if (!f16) {
+          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+          const uint32_t tk = tbase + L::T_KSF + 8 * s;
+          for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, st + L::ST_KSF + kk * 512);
+          const uint32_t sK = smem_u32(st + L::ST_K);
+          for (int kk = 0; kk < L::KSTEPS; ++kk) {
+            const uint64_t da = make_sdesc(sQ + kk * 32, 16, L::QK_SBO, L::QK_SW);
+            const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
+            mma_nvf4(tS, da, db, idesc_qk, tbase + L::T_QSF + 4 * kk, tk + 4 * kk, kk > 0 ? 1u : 0u);
+          }
+        } else {
+          if (!q16_ready) {
+            if (!wait1(q16_full, 0)) { ok = false; break; }
+            q16_ready = true;
+          }
+          if (!wait1(kv16_full, n16_qk & 1)) { ok = false; break; }
+          tc_fence_after();
+          ++n16_qk;
+          const uint32_t sQ16 = smem_u32(sm + L::OFF_Q16), sK16 = smem_u32(sm + L::OFF_K16);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t da = make_sdesc(sQ16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
+            const uint64_t db = make_sdesc(sK16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
+            mma_f16(tS, da, db, idesc_qk16, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(s_full + b2);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && nt > 0) issue_pv(nt - 1);
+      (void)n16_pv;
+      // Everything this thread issued has completed before TMEM is released.
+      mma_commit(mma_final);
+      mbar_wait(mma_final, 0);
+    }
+    __syncwarp();
+  } else {
+    // ================================ softmax ================================
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int qi = qt * 128 + row;
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const float C4 = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
+    const float C16 = a.softmax_scale * kLog2e;
+    float m_run = -INFINITY, l_run = 0.f;
+    unsigned char* sP = sm + L::OFF_P;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int b2 = j & 1;
+      const bool f16 = kMixed && bm_row[j];
+      if (!waitw(s_full + b2, (j >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      float x[128];
+      {
+        uint32_t* xr = reinterpret_cast<uint32_t*>(x);
+        const uint32_t tS = tbase + L::T_S + b2 * 128 + lane_addr;
+        tmem_ld32(tS + 0, xr + 0);
+        tmem_ld32(tS + 32, xr + 32);
+        tmem_ld32(tS + 64, xr + 64);
+        tmem_ld32(tS + 96, xr + 96);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free + b2);
+      const float C = f16 ? C16 : C4;
+      const int kbase = j * 128;
+      const bool need_mask = (a.causal && kbase + 127 > qi) || (kbase + 128 > a.Nk);
+      float mt = -INFINITY;
+      if (need_mask) {
+        const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          x[c] = (c <= lim) ? x[c] * C : -INFINITY;
+          mt = fmaxf(mt, x[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          x[c] = x[c] * C;
+          mt = fmaxf(mt, x[c]);
+        }
+      }
+      const float m_new = fmaxf(m_run, mt);
+      const bool dead = (m_new == -INFINITY);
+      const float moff = dead ? 0.f : m_new - kLog2_448;
+      const float alpha = dead ? 1.f : ex2_approx(m_run - m_new);
+      float lsum = 0.f;
+      uint32_t pw[64];             // e4m3: 32 words used; fp16: 64 words
+      if (!f16) {
+#pragma unroll
+        for (int c = 0; c < 128; c += 4) {
+          const uint32_t lo = cvt_e4m3x2(ex2_approx(x[c] - moff), ex2_approx(x[c + 1] - moff));
+          const uint32_t hi = cvt_e4m3x2(ex2_approx(x[c + 2] - moff), ex2_approx(x[c + 3] - moff));
+          const float2 f0 = __half22float2(e4m3x2_to_half2(lo));
+          const float2 f1 = __half22float2(e4m3x2_to_half2(hi));
+          lsum += (f0.x + f0.y) + (f1.x + f1.y);
+          pw[c >> 2] = lo | (hi << 16);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const __half2 h = __floats2half2_rn(ex2_approx(x[c] - moff), ex2_approx(x[c + 1] - moff));
+          const float2 f = __half22float2(h);
+          lsum += f.x + f.y;
+          pw[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+      }
+      l_run = l_run * alpha + lsum;
+      m_run = m_new;
+      // PV(j-1) must be done: it reads the other P buffer / O, and P(j-2) shares ours.
+      if (j >= 1) {
+        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+      }
+      if (!f16) {
+        unsigned char* prow = sP + b2 * 16384 + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          unsigned char* prow = sP + h * 16384 + row * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+                make_uint4(pw[32 * h + 4 * c], pw[32 * h + 4 * c + 1], pw[32 * h + 4 * c + 2],
+                           pw[32 * h + 4 * c + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      if (j >= 1 && !__all_sync(0xffffffffu, alpha == 1.f)) {
+        const uint32_t tO = tbase + L::T_O + lane_addr;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(tO + c, o);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + b2);
+    }
+    // ---- epilogue ----
+    if (ok && nt > 0 && waitw(pv_done + ((nt - 1) & 1), ((nt - 1) >> 1) & 1)) {
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      const uint32_t tO = tbase + L::T_O + lane_addr;
+      const bool store = qi < a.Nq;
+      const int64_t orow = static_cast<int64_t>(bhq) * a.Nq + qi;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
+        tmem_wait_ld();
+        if (store) {
+          __align__(16) uint32_t packed[16];
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            const float v0 = __uint_as_float(o[k]) * inv, v1 = __uint_as_float(o[k + 1]) * inv;
+            if (a.out_bf16) {
+              __nv_bfloat162 t = __floats2bfloat162_rn(v0, v1);
+              packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
+            } else {
+              __half2 t = __floats2half2_rn(v0, v1);
+              packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
+            }
+          }
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + c);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = reinterpret_cast<uint4*>(packed)[k];
+        }
+      }
+      if (store && a.lse != nullptr) a.lse[orow] = m_run * kLn2 + logf(l_run * (1.f / 448.f));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace qk4v8

@@ -1,0 +1,412 @@
+// Split-K paged decode over an NVFP4-K / MXFP8-V KV cache, and the split merge.
+//
+// Method: sns.style BitDecoding-FP4 summary (the whole KV cache is read once per decoding
+// step; GQA query heads stacked into one tensor-core MMA on a paged cache; probability
+// quantization fused into the kernel), with the QK4V8 arithmetic of the prefill kernel.
+//
+// Grid (split, kv head, sequence). Each CTA walks its split's pages two at a time (128 keys)
+// and keeps (m, l, O) for the g query heads of its KV head. tcgen05 block-scaled MMAs need
+// M = 128, so the g <= 16 query heads form the N dimension (N = 16) and keys / channels form
+// M: S^T = K Q^T (M = 128 keys) and O^T += V^T P^T (M = 128 channels); each softmax thread
+// owns one key, and the row reductions over keys run across the 128 softmax threads.
+// Partials (O unnormalised, m, l) go to the workspace; the merge kernel combines the splits:
+// M = max m_s, O = sum e^(m_s - M) O_s / sum e^(m_s - M) l_s.
+#pragma once
+#include "ptx.cuh"
+#include "attn_fwd.cuh"
+
+namespace qk4v8 {
+
+struct DecArgs {
+  const uint8_t* q_scales;       // [S*Hq, D/16]
+  const float* q_ts;
+  const uint8_t* k_page_scales;  // [P, Hkv, 64, D/16]
+  const float* k_ts;
+  const uint8_t* v_page_scales;  // [P, Hkv, D, 2]
+  const int32_t* page_table;     // [S, max_pages]
+  const int32_t* lens;           // [S]
+  float* ws;                     // [S*Hq, n_splits, D + 2]
+  int32_t S, Hq, Hkv, max_pages, n_splits, split_tokens, num_pages;
+  float softmax_scale;
+};
+
+struct DecLayout {
+  static constexpr int D = 128;
+  static constexpr int NS = 3;
+  static constexpr int OFF_Q = 0;                 // 16 rows x 64 B (SW64)
+  static constexpr int OFF_QSF = 1024;            // 2 chunks
+  static constexpr int OFF_PSF = 2048;            // 1 chunk
+  static constexpr int OFF_P = 3072;              // 2 x [16 rows x 128 B] (SW128), 1024-aligned
+  static constexpr int OFF_STAGE = OFF_P + 2 * 2048;      // 7168, 1024-aligned
+  static constexpr int ST_K = 0;                  // 128 keys x 64 B (SW64)
+  static constexpr int ST_V0 = 8192;              // 128 channels x 64 B (page 0 tokens)
+  static constexpr int ST_V1 = 16384;             // page 1 tokens
+  static constexpr int ST_KSF = 24576;            // 2 chunks
+  static constexpr int ST_VSF = 25600;            // 1 chunk
+  static constexpr int STAGE_BYTES = 26624;
+  static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
+  static constexpr int OFF_RED = OFF_BAR + 256;   // reductions: [4 warps][16] max, [4][16] sum
+  static constexpr int SMEM_BYTES = OFF_RED + 2 * 4 * 16 * 4;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+  static constexpr uint32_t T_S = 0, T_O = 32, T_QSF = 48, T_PSF = 56, T_KSF = 64, T_VSF = 88;
+  static constexpr int NQ = 16;                   // MMA N (query heads, padded)
+};
+
+__global__ void __launch_bounds__(192, 2)
+decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
+              const __grid_constant__ CUtensorMap tm_vp, DecArgs a) {
+  using L = DecLayout;
+  constexpr int D = L::D;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + L::NS;
+  uint64_t* s_full = bars + 1 + 2 * L::NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_full + 4;
+  uint64_t* pv_done = s_full + 6;
+  uint64_t* mma_final = s_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red_max = reinterpret_cast<float*>(sm + L::OFF_RED);
+  float* red_sum = red_max + 64;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const int g = a.Hq / a.Hkv;
+  int len = a.lens[s];
+  if (len < 1 || len > a.n_splits * a.split_tokens || len > a.max_pages * 64) {
+    if (split == 0 && h == 0 && threadIdx.x == 0) flag_error(kStatusBounds);
+    len = 0;                               // every split empty; the merge yields no value
+  }
+  const int k_begin = split * a.split_tokens;
+  const int k_end = min(len, k_begin + a.split_tokens);
+  const int nblk = k_end > k_begin ? (k_end - k_begin + 127) / 128 : 0;
+  const int64_t qrow0 = static_cast<int64_t>(s) * a.Hq + h * g;
+  float* part = a.ws + (qrow0 * a.n_splits + split) * (D + 2);   // + q * n_splits * (D+2)
+  const int64_t q_stride = static_cast<int64_t>(a.n_splits) * (D + 2);
+
+  if (nblk == 0) {                         // empty split: weight zero in the merge
+    for (int q = 0; q < g; ++q)
+      for (int c = threadIdx.x; c < D + 2; c += blockDim.x)
+        part[q * q_stride + c] = (c == D) ? -INFINITY : 0.f;
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < L::NS; ++i) { mbar_init(kv_full + i, 1); mbar_init(kv_empty + i, 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1); mbar_init(s_free + i, 4);
+      mbar_init(p_full + i, 4); mbar_init(pv_done + i, 1);
+    }
+    mbar_init(mma_final, 1);
+    abort_flag[0] = 0;
+    abort_flag[1] = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < 128; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(sm + L::OFF_PSF)[i] = 0x7F7F7F7Fu;
+  for (int i = threadIdx.x; i < 2 * 16 * 128 / 16; i += blockDim.x)   // zero both P^T buffers
+    reinterpret_cast<uint4*>(sm + L::OFF_P)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  // Producer: warp-uniform waits; MMA issuer: single-thread waits (both on abort_flag).
+  // Softmax: warp-uniform waits on its own flag, which it only reads after a barrier of all
+  // four softmax warps, so that the four always leave the loop together.
+  volatile int* soft_flag = abort_flag + 1;
+  auto waitw = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return bounded_wait_warp(bar, parity, abort_flag);
+  };
+  auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
+    return bounded_wait(bar, parity, abort_flag);
+  };
+  auto waits = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int ok = 0;
+    if (lane == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
+  auto page_of = [&](int logical) -> int {
+    int p = a.page_table[static_cast<int64_t>(s) * a.max_pages + logical];
+    if (p < 0 || p >= a.num_pages) { flag_error(kStatusBounds); p = 0; }
+    return p;
+  };
+
+  if (warp == 0) {
+    // ================================ producer ================================
+    {
+      // Q scale factors of the g heads (rows 0..15 of the N = 16 operand; rows >= g are 0).
+      uint32_t w0 = 0, w1 = 0;
+      if (lane < g) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.q_scales + (qrow0 + lane) * (D / 16)));
+        w0 = v.x; w1 = v.y;
+      }
+      *reinterpret_cast<uint4*>(sm + L::OFF_QSF + lane * 16) = make_uint4(w0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(sm + L::OFF_QSF + 512 + lane * 16) = make_uint4(w1, 0, 0, 0);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, 16 * 64);
+        tma_load_2d(sm + L::OFF_Q, &tm_q, q_full, 0, static_cast<int>(qrow0));
+      }
+    }
+    for (int blk = 0; blk < nblk; ++blk) {
+      const int st_i = blk % L::NS;
+      if (blk >= L::NS && !waitw(kv_empty + st_i, ((blk / L::NS) - 1) & 1)) break;
+      unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
+      const int k0 = k_begin + blk * 128;
+      const int lp0 = k0 / 64;
+      const int p0 = page_of(lp0);
+      const int p1 = (k0 + 64 < len) ? page_of(lp0 + 1) : p0;
+      // K scale factors: key rows 0..63 from page p0, 64..127 from p1.
+      uint32_t w[4][2];
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) {
+        const int r = r1 * 32 + lane;
+        const int pp = r < 64 ? p0 : p1;
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(
+            a.k_page_scales + ((static_cast<int64_t>(pp) * a.Hkv + h) * 64 + (r & 63)) * (D / 16)));
+        w[r1][0] = v.x; w[r1][1] = v.y;
+      }
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+        *reinterpret_cast<uint4*>(st + L::ST_KSF + kk * 512 + lane * 16) =
+            make_uint4(w[0][kk], w[1][kk], w[2][kk], w[3][kk]);
+      // V scale factors: channel c, [page0 g0, page0 g1, page1 g0, page1 g1].
+      uint32_t vw[4];
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) {
+        const int c = r1 * 32 + lane;
+        const uint32_t lo = __ldg(reinterpret_cast<const uint16_t*>(
+            a.v_page_scales + ((static_cast<int64_t>(p0) * a.Hkv + h) * D + c) * 2));
+        const uint32_t hi = __ldg(reinterpret_cast<const uint16_t*>(
+            a.v_page_scales + ((static_cast<int64_t>(p1) * a.Hkv + h) * D + c) * 2));
+        vw[r1] = lo | (hi << 16);
+      }
+      *reinterpret_cast<uint4*>(st + L::ST_VSF + lane * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kv_full + st_i, 128 * 64 + 2 * D * 64);
+        tma_load_2d(st + L::ST_K, &tm_kp, kv_full + st_i, 0, (p0 * a.Hkv + h) * 64);
+        tma_load_2d(st + L::ST_K + 4096, &tm_kp, kv_full + st_i, 0, (p1 * a.Hkv + h) * 64);
+        tma_load_2d(st + L::ST_V0, &tm_vp, kv_full + st_i, 0, (p0 * a.Hkv + h) * D);
+        tma_load_2d(st + L::ST_V1, &tm_vp, kv_full + st_i, 0, (p1 * a.Hkv + h) * D);
+      }
+    }
+    for (int i = 0; i < L::NS && i < nblk; ++i) {
+      const int last = i + ((nblk - 1 - i) / L::NS) * L::NS;
+      mbar_wait(kv_full + i, (last / L::NS) & 1);
+    }
+    mbar_wait(q_full, 0);
+  } else if (warp == 1) {
+    // ================================ MMA issuer ================================
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, L::NQ);
+      const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NQ);
+      const uint32_t sQ = smem_u32(sm + L::OFF_Q);
+      const uint32_t sP = smem_u32(sm + L::OFF_P);
+      bool ok = wait1(q_full, 0);
+      if (ok) {
+        tc_fence_after();
+        tmem_cp_sf(tbase + L::T_QSF, sm + L::OFF_QSF);
+        tmem_cp_sf(tbase + L::T_QSF + 4, sm + L::OFF_QSF + 512);
+        tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+      }
+      auto issue_pv = [&](int bb) -> bool {
+        const int st_i = bb % L::NS, b2 = bb & 1;
+        if (!wait1(p_full + b2, (bb >> 1) & 1)) return false;
+        tc_fence_after();
+        unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
+        const uint32_t tv = tbase + L::T_VSF + 4 * st_i;
+        tmem_cp_sf(tv, st + L::ST_VSF);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t sV = smem_u32(st + ((kk >> 1) ? L::ST_V1 : L::ST_V0));
+          const uint64_t da = make_sdesc(sV + (kk & 1) * 32, 16, 512, kSw64);
+          const uint64_t db = make_sdesc(sP + b2 * 2048 + kk * 32, 16, 1024, kSw128);
+          mma_mxf8(tbase + L::T_O, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
+                   tv | (static_cast<uint32_t>(kk) << 30),
+                   (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                   (bb > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(pv_done + b2);
+        mma_commit(kv_empty + st_i);
+        return true;
+      };
+      for (int blk = 0; ok && blk < nblk; ++blk) {
+        const int st_i = blk % L::NS, b2 = blk & 1;
+        if (!wait1(kv_full + st_i, (blk / L::NS) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (blk >= 2 && !wait1(s_free + b2, ((blk - 2) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
+        const uint32_t tk = tbase + L::T_KSF + 8 * st_i;
+        tmem_cp_sf(tk, st + L::ST_KSF);
+        tmem_cp_sf(tk + 4, st + L::ST_KSF + 512);
+        const uint32_t sK = smem_u32(st + L::ST_K);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint64_t da = make_sdesc(sK + kk * 32, 16, 512, kSw64);
+          const uint64_t db = make_sdesc(sQ + kk * 32, 16, 512, kSw64);
+          mma_nvf4(tbase + L::T_S + b2 * 16, da, db, idesc_qk, tk + 4 * kk,
+                   tbase + L::T_QSF + 4 * kk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full + b2);
+        if (blk >= 1 && !issue_pv(blk - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(nblk - 1);
+      mma_commit(mma_final);
+      mbar_wait(mma_final, 0);
+    }
+    __syncwarp();
+  } else {
+    // ============================ softmax (one key per thread) ============================
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
+    float m_run[16], l_run[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) { m_run[q] = -INFINITY; l_run[q] = 0.f; }
+    unsigned char* sP = sm + L::OFF_P;
+    bool failed = false;
+    for (int blk = 0; blk < nblk; ++blk) {
+      const int b2 = blk & 1;
+      // On a timeout the body still runs (on whatever TMEM holds) so that the four warps
+      // meet at both named barriers; the shared flag then ends the loop for all of them.
+      if (!waits(s_full + b2, (blk >> 1) & 1)) failed = true;
+      tc_fence_after();
+      float x[16];
+      tmem_ld16(tbase + L::T_S + b2 * 16 + lane_addr, reinterpret_cast<uint32_t*>(x));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free + b2);
+      const bool valid = k_begin + blk * 128 + r < k_end;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        x[q] = (valid && q < g) ? x[q] * C : -INFINITY;
+        float mm = x[q];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+        if (lane == 0) red_max[wq * 16 + q] = mm;
+      }
+      named_bar_sync(1, 128);
+      float alpha[16], moff[16];
+      bool all_one = true;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float mb = fmaxf(fmaxf(red_max[q], red_max[16 + q]), fmaxf(red_max[32 + q], red_max[48 + q]));
+        const float m_new = fmaxf(m_run[q], mb);
+        const bool dead = (m_new == -INFINITY);
+        moff[q] = dead ? 0.f : m_new - kLog2_448;
+        alpha[q] = dead ? 1.f : ex2_approx(m_run[q] - m_new);
+        all_one = all_one && (alpha[q] == 1.f);
+        m_run[q] = m_new;
+      }
+      uint32_t codes[4];
+#pragma unroll
+      for (int q = 0; q < 16; q += 4) {
+        const uint32_t lo = cvt_e4m3x2(ex2_approx(x[q] - moff[q]), ex2_approx(x[q + 1] - moff[q + 1]));
+        const uint32_t hi = cvt_e4m3x2(ex2_approx(x[q + 2] - moff[q + 2]), ex2_approx(x[q + 3] - moff[q + 3]));
+        codes[q >> 2] = lo | (hi << 16);
+        const float2 f0 = __half22float2(e4m3x2_to_half2(lo));
+        const float2 f1 = __half22float2(e4m3x2_to_half2(hi));
+        float sv[4] = {f0.x, f0.y, f1.x, f1.y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float t = sv[i];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          if (lane == 0) red_sum[wq * 16 + q + i] = t;
+        }
+      }
+      if (blk >= 1) {
+        if (!waits(pv_done + ((blk - 1) & 1), ((blk - 1) >> 1) & 1)) failed = true;
+        tc_fence_after();
+      }
+      // P^T row q (query), column r (key), 128-byte swizzle.
+      unsigned char* pb = sP + b2 * 2048;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        if (q < g)
+          pb[q * 128 + ((((r >> 4) ^ (q & 7))) << 4) + (r & 15)] =
+              static_cast<unsigned char>(codes[q >> 2] >> (8 * (q & 3)));
+      }
+      if (failed && lane == 0) *soft_flag = 1;
+      named_bar_sync(2, 128);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float lb = (red_sum[q] + red_sum[16 + q]) + (red_sum[32 + q] + red_sum[48 + q]);
+        l_run[q] = l_run[q] * alpha[q] + lb;
+      }
+      if (*soft_flag) break;
+      fence_proxy_async_smem();
+      if (blk >= 1 && !all_one) {
+        float o[16];
+        tmem_ld16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) o[q] *= alpha[q];
+        tmem_st16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full + b2);
+    }
+    if (!*soft_flag && waits(pv_done + ((nblk - 1) & 1), ((nblk - 1) >> 1) & 1)) {
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
+      tmem_wait_ld();
+      for (int q = 0; q < g; ++q) {
+        part[q * q_stride + r] = o[q];
+        if (r == 0) { part[q * q_stride + D] = m_run[q]; part[q * q_stride + D + 1] = l_run[q]; }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 128);
+  }
+}
+
+// Merge the splits: one CTA per (sequence, query head), one thread per channel.
+__global__ void __launch_bounds__(128) decode_merge_kernel(const float* __restrict__ ws,
+                                                           int32_t n_splits, int32_t out_bf16,
+                                                           void* __restrict__ out,
+                                                           float* __restrict__ lse) {
+  constexpr int D = 128;
+  const int64_t row = blockIdx.x;
+  const float* p = ws + row * n_splits * (D + 2);
+  float M = -INFINITY;
+  for (int i = 0; i < n_splits; ++i) M = fmaxf(M, p[i * (D + 2) + D]);
+  float Lsum = 0.f, acc = 0.f;
+  for (int i = 0; i < n_splits; ++i) {
+    const float m = p[i * (D + 2) + D];
+    const float w = (m == -INFINITY) ? 0.f : ex2_approx(m - M);
+    Lsum += w * p[i * (D + 2) + D + 1];
+    acc += w * p[i * (D + 2) + threadIdx.x];
+  }
+  const float v = acc / Lsum;
+  if (out_bf16) static_cast<__nv_bfloat16*>(out)[row * D + threadIdx.x] = __float2bfloat16_rn(v);
+  else static_cast<__half*>(out)[row * D + threadIdx.x] = __float2half_rn(v);
+  if (lse != nullptr && threadIdx.x == 0) lse[row] = M * kLn2 + logf(Lsum * (1.f / 448.f));
+}
+
+}  // namespace qk4v8

@@ -1,0 +1,198 @@
+// Quantize kernels: NVFP4 for Q and K (tqpw.cn "块缩放数值格式" article §2.2: E2M1
+// elements, E4M3 scale per 16 elements, FP32 tensor scale) and MXFP8 for V (§2.1: E8M0 scale
+// per 32 elements; here along the token axis, per channel).
+//
+// NVFP4 arithmetic (every step a single IEEE FP32 operation rounded to nearest, subnormals
+// kept):  s_t = amax / 2688 (1 when amax == 0);  s_b = E4M3(amax_b / 6 / s_t);
+// den = s_b * s_t;  code = E2M1(x / den), all codes 0 when s_b == 0.  E2M1 pairs are packed
+// low nibble first. Conversions round to nearest even and saturate; the sign bit of every
+// code is the sign of its input, so a negative value that rounds to zero is negative zero.
+#pragma once
+#include "ptx.cuh"
+
+namespace qk4v8 {
+
+template <typename T> __device__ __forceinline__ float to_float(T v);
+template <> __device__ __forceinline__ float to_float<__half>(__half v) { return __half2float(v); }
+template <> __device__ __forceinline__ float to_float<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+// Eight 16-bit values from one 16-byte load.
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+  const T* h = reinterpret_cast<const T*>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = to_float<T>(h[i]);
+}
+
+__device__ __forceinline__ float e4m3_code_to_float(uint32_t code) {
+  return __low2float(e4m3x2_to_half2(code & 0xFFu));
+}
+
+// ---------------------------------------------------------------------------------------
+// Pass 1: tensor amax (as float bits; non-negative floats order like unsigned integers).
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const T* __restrict__ x, int64_t rows,
+                                                         int32_t cols, int64_t row_stride,
+                                                         unsigned int* __restrict__ amax_bits) {
+  const uint32_t blocks_per_row = static_cast<uint32_t>(cols / 16);
+  const int64_t total = rows * blocks_per_row;
+  float m = 0.f;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / blocks_per_row;
+    const uint32_t cb = static_cast<uint32_t>(i - r * blocks_per_row);
+    const uint4* p = reinterpret_cast<const uint4*>(x + r * row_stride + cb * 16);
+    const uint4 a = __ldg(p), b = __ldg(p + 1);
+    float f[16];
+    unpack8<T>(a, f);
+    unpack8<T>(b, f + 8);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(f[k]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t = fmaxf(t, wm[w]);
+    atomicMax(amax_bits, __float_as_uint(t));
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Pass 2: encode. One thread per 16-element block.
+// ---------------------------------------------------------------------------------------
+template <typename T, bool kWrite16>
+__global__ void __launch_bounds__(256) nvfp4_encode_kernel(
+    const T* __restrict__ x, int64_t rows, int32_t cols, int64_t row_stride,
+    const unsigned int* __restrict__ amax_bits, float tensor_scale_in,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, float* __restrict__ ts_out,
+    __half* __restrict__ x16) {
+  float s_t;
+  if (tensor_scale_in > 0.f) {
+    s_t = tensor_scale_in;
+  } else {
+    const float amax = __uint_as_float(*amax_bits);
+    s_t = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 2688.f);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
+  const uint32_t blocks_per_row = static_cast<uint32_t>(cols / 16);
+  const int64_t total = rows * blocks_per_row;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / blocks_per_row;
+    const uint32_t cb = static_cast<uint32_t>(i - r * blocks_per_row);
+    const uint4* p = reinterpret_cast<const uint4*>(x + r * row_stride + cb * 16);
+    const uint4 a = __ldg(p), b = __ldg(p + 1);
+    float f[16];
+    unpack8<T>(a, f);
+    unpack8<T>(b, f + 8);
+    float amax_b = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(f[k]));
+    const float sbf = __fdiv_rn(__fdiv_rn(amax_b, 6.f), s_t);
+    const uint32_t sc = cvt_e4m3x2(sbf, 0.f) & 0xFFu;
+    const float sbv = e4m3_code_to_float(sc);
+    uint32_t w[2] = {0u, 0u};
+    if (sbv != 0.f) {
+      const float den = __fmul_rn(sbv, s_t);
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        const float q0 = __fdiv_rn(f[k], den), q1 = __fdiv_rn(f[k + 1], den);
+        uint32_t byte = cvt_e2m1x2(q0, q1) & 0x77u;
+        byte |= (__float_as_uint(f[k]) >> 31) << 3;
+        byte |= (__float_as_uint(f[k + 1]) >> 31) << 7;
+        w[k >> 3] |= byte << ((k & 7) * 4);
+      }
+    }
+    const int64_t blk = r * blocks_per_row + cb;
+    *reinterpret_cast<uint2*>(codes + blk * 8) = make_uint2(w[0], w[1]);
+    scales[blk] = static_cast<uint8_t>(sc);
+    if constexpr (kWrite16) {
+      __align__(16) __half h[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) h[k] = __float2half_rn(f[k]);
+      uint4* o = reinterpret_cast<uint4*>(x16 + blk * 16);
+      o[0] = *reinterpret_cast<uint4*>(h);
+      o[1] = *reinterpret_cast<uint4*>(h + 8);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// MXFP8 for V. v: [BH, N, D] token-major. codes: [BH, D, Npad] token-contiguous; scales:
+// [BH, D, Npad/32] E8M0. Npad = N rounded up to 128; padding tokens read as 0.
+// Shared exponent (OCP MX rule): e = floor(log2 amax) - 8 clamped to [-127, 127]; code
+// e + 127; all-zero group -> 127. Elements E4M3(v * 2^-e) (exact power-of-two scaling).
+// Optional fp16 copy written transposed like the codes: [BH, D, Npad].
+// Grid (Npad/128, BH); 256 threads; one 128-token x D tile per CTA.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ int floor_log2_pos(float a) {   // a > 0, finite
+  const uint32_t bits = __float_as_uint(a);
+  const int ef = static_cast<int>(bits >> 23);
+  if (ef > 0) return ef - 127;
+  return (31 - __clz(bits & 0x7FFFFFu)) - 149;              // subnormal
+}
+
+template <typename T, int D, bool kWrite16>
+__global__ void __launch_bounds__(256) mxfp8_v_kernel(const T* __restrict__ v, int32_t N,
+                                                      int32_t Npad, uint8_t* __restrict__ codes,
+                                                      uint8_t* __restrict__ scales,
+                                                      __half* __restrict__ v16t) {
+  constexpr int LD = D + 8;                       // padded row (elements)
+  __shared__ __align__(16) T tile[128 * LD];
+  const int tile_id = blockIdx.x;
+  const int64_t bh = blockIdx.y;
+  const int tok0 = tile_id * 128;
+  // Load 128 tokens x D (16-byte chunks), zero past N.
+  constexpr int CH = D / 8;                       // chunks per token
+  for (int i = threadIdx.x; i < 128 * CH; i += blockDim.x) {
+    const int t = i / CH, c = i % CH;
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (tok0 + t < N) u = __ldg(reinterpret_cast<const uint4*>(v + (bh * N + tok0 + t) * D + c * 8));
+    *reinterpret_cast<uint4*>(&tile[t * LD + c * 8]) = u;
+  }
+  __syncthreads();
+  for (int task = threadIdx.x; task < D * 4; task += blockDim.x) {
+    const int c = task % D, g = task / D;
+    float f[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      f[t] = to_float<T>(tile[(g * 32 + t) * LD + c]);
+      amax = fmaxf(amax, fabsf(f[t]));
+    }
+    int e = 0;
+    if (amax > 0.f) e = max(-127, min(127, floor_log2_pos(amax) - 8));
+    const float mul = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+    __align__(16) uint8_t cb[32];
+#pragma unroll
+    for (int t = 0; t < 32; t += 2) {
+      uint32_t two = cvt_e4m3x2(__fmul_rn(f[t], mul), __fmul_rn(f[t + 1], mul)) & 0x7F7Fu;
+      two |= (__float_as_uint(f[t]) >> 31) << 7;
+      two |= (__float_as_uint(f[t + 1]) >> 31) << 15;
+      cb[t] = static_cast<uint8_t>(two & 0xFF);
+      cb[t + 1] = static_cast<uint8_t>(two >> 8);
+    }
+    const int64_t rowc = bh * D + c;
+    uint4* dst = reinterpret_cast<uint4*>(codes + rowc * Npad + tok0 + g * 32);
+    dst[0] = *reinterpret_cast<uint4*>(cb);
+    dst[1] = *reinterpret_cast<uint4*>(cb + 16);
+    scales[rowc * (Npad / 32) + tile_id * 4 + g] = static_cast<uint8_t>(e + 127);
+    if constexpr (kWrite16) {
+      __align__(16) __half h[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) h[t] = __float2half_rn(f[t]);
+      uint4* o = reinterpret_cast<uint4*>(v16t + rowc * Npad + tok0 + g * 32);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] = reinterpret_cast<uint4*>(h)[k];
+    }
+  }
+}
+
+}  // namespace qk4v8

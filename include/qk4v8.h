@@ -1,0 +1,201 @@
+/*
+ * qk4v8 — block-scaled low-bit FlashAttention (QK4V8) for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libqk4v8.so. Every pointer argument is a DEVICE pointer unless stated otherwise;
+ * the caller allocates and owns every buffer (inputs, outputs and workspaces). The library
+ * never allocates, frees or synchronises, except qk4v8_check_status(), which synchronises the
+ * given stream. All launches are asynchronous on `stream` and deterministic for a fixed shape.
+ *
+ * Errors: arguments are validated on the host before any launch and a bad argument returns
+ * QK4V8_ERR_INVALID_ARG (or QK4V8_ERR_UNSUPPORTED for a valid but unimplemented shape) with
+ * nothing launched. A failed launch returns QK4V8_ERR_CUDA. Problems found on the device (a
+ * pipeline wait that ran past its time limit, a page id out of range) set a device status
+ * word that qk4v8_check_status() reports and clears.
+ *
+ * Formats (tqpw.cn "块缩放数值格式" article §2.1-2.2; zdszero quantization primer, format
+ * table):
+ *   NVFP4  E2M1 elements packed two per byte (element 2i in the low nibble), one E4M3 scale
+ *          per 16 consecutive elements, one FP32 tensor scale.
+ *   MXFP8  E4M3 elements, one E8M0 scale (value 2^(code-127)) per 32 consecutive elements.
+ * Conversions round to nearest even and saturate (E2M1 to +-6, E4M3 to +-448); the sign bit
+ * of a code is the sign of its input.
+ */
+#ifndef QK4V8_H
+#define QK4V8_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QK4V8_OK = 0,
+  QK4V8_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned buffer, ... */
+  QK4V8_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement */
+  QK4V8_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  QK4V8_ERR_TIMEOUT = 4,      /* a device-side pipeline wait passed its time limit */
+  QK4V8_ERR_BOUNDS = 5        /* a device-side index check failed (e.g. page id) */
+} qk4v8_status;
+
+typedef enum { QK4V8_F16 = 0, QK4V8_BF16 = 1 } qk4v8_dtype;
+
+/* Library version (major * 100 + minor). */
+int qk4v8_version(void);
+
+/* sizeof the parameter structs, for bindings that mirror them: which = 0 gives
+ * sizeof(qk4v8_fwd_params), 1 gives sizeof(qk4v8_decode_params), anything else 0. */
+size_t qk4v8_struct_size(int32_t which);
+
+/* Human-readable name of a status code (static string). */
+const char* qk4v8_status_string(qk4v8_status status);
+
+/*
+ * Synchronise `stream`, then report and clear the device status word: QK4V8_ERR_TIMEOUT or
+ * QK4V8_ERR_BOUNDS when a kernel flagged one, QK4V8_ERR_CUDA when the stream reported an
+ * error, else QK4V8_OK.
+ */
+qk4v8_status qk4v8_check_status(cudaStream_t stream);
+
+/*
+ * quantize_nvfp4 — NVFP4 quantization of Q or K (tqpw.cn article §2.2: E2M1 elements, E4M3
+ * scale per 16 elements, FP32 tensor scale). Per call:
+ *   s_t = fl32(amax / 2688) over all of x (2688 = 6 * 448; s_t = 1 when amax is 0), or
+ *         s_t = tensor_scale_in when tensor_scale_in > 0 (e.g. a KV cache's fixed scale);
+ *   per 16-element block: s_b = E4M3(fl32(fl32(amax_b / 6) / s_t));
+ *         code_i = E2M1(fl32(x_i / fl32(s_b * s_t))), every code 0 when s_b is 0.
+ * x       [rows, cols] fp16/bf16, row i at x + i*row_stride elements; 16-byte aligned,
+ *         cols % 16 == 0, row_stride % 8 == 0, row_stride >= cols.
+ * codes   [rows, cols/2] bytes out (8-byte aligned); scales [rows, cols/16] E4M3 codes out.
+ * tensor_scale  one float out (s_t).
+ * x16     optional [rows, cols] fp16 copy of x out (16-byte aligned), for FP16 tiles; or NULL.
+ * workspace     >= quantize_nvfp4_workspace_size() bytes, 4-byte aligned (unused, may be
+ *               NULL, when tensor_scale_in > 0).
+ */
+size_t quantize_nvfp4_workspace_size(void);
+qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,
+                            int64_t row_stride, float tensor_scale_in, uint8_t* codes,
+                            uint8_t* scales, float* tensor_scale, void* x16, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * quantize_mxfp8_v — MXFP8 quantization of V along the token axis (tqpw.cn article §2.1:
+ * E8M0 scale per 32 elements; here the 32 elements are consecutive tokens of one channel,
+ * the contraction axis of P V). Shared exponent e = floor(log2 amax) - 8 clamped to
+ * [-127, 127] (scale code e + 127; 127 for an all-zero group); code_i = E4M3(v_i * 2^-e).
+ * v       [batch_heads, n_tokens, head_dim] fp16/bf16, contiguous, 16-byte aligned.
+ * codes   [batch_heads, head_dim, n_pad] out, n_pad = n_tokens rounded up to 128; token-
+ *         contiguous per channel; padding tokens encode 0. 16-byte aligned.
+ * scales  [batch_heads, head_dim, n_pad/32] E8M0 codes out.
+ * v16     optional [batch_heads, head_dim, n_pad] fp16 copy out (same transposed layout,
+ *         padding 0), for FP16 tiles; or NULL. 16-byte aligned.
+ * head_dim is 64 or 128.
+ */
+qk4v8_status quantize_mxfp8_v(const void* v, qk4v8_dtype dtype, int32_t batch_heads,
+                              int32_t n_tokens, int32_t head_dim, uint8_t* codes,
+                              uint8_t* scales, void* v16, cudaStream_t stream);
+
+/*
+ * tile_score_select — ThriftAttention-style tile importance (ai-feeds.com ThriftAttention
+ * summary, method step 2 and limitations: a cheap L2-norm bound on each 128x128 query-key
+ * tile's largest weight; the top ~5 % of tiles get FP16). Score of tile (qt, kt) =
+ * max_{i in qt} N_i(q) * max_{j in kt} N_j(k), N = |x_hat|^2 * 2^20 / s_t^2 computed exactly
+ * in integers from the NVFP4 codes; exact 128-bit products, so the selection is exact.
+ * Per (batch, query head) it keeps k = ceil(n_candidates * frac_bp / 10000) tiles, where the
+ * candidates are all tiles (causal: kt <= qt), ranked by score descending then by the lower
+ * linear index qt * T + kt (T = ceil(n_tokens / 128)).
+ * q_codes/q_scales  [batch, q_heads, n_tokens, head_dim/2 | head_dim/16] (quantize_nvfp4
+ *                   output); k_codes/k_scales likewise with kv_heads. Query head h uses KV
+ *                   head h / (q_heads / kv_heads).
+ * idx     [batch*q_heads, k_max] out: linear indices in rank order (first n_sel[bh] valid).
+ * n_sel   [batch*q_heads] out.  bitmap  optional [batch*q_heads, T, T] out (1 = selected).
+ * k_max   capacity of idx per head; must be >= k; at most 4096.
+ * workspace >= tile_score_select_workspace_size(...) bytes, 8-byte aligned.
+ */
+size_t tile_score_select_workspace_size(int32_t batch, int32_t q_heads, int32_t kv_heads,
+                                        int32_t n_tokens);
+qk4v8_status tile_score_select(const uint8_t* q_codes, const uint8_t* q_scales,
+                               const uint8_t* k_codes, const uint8_t* k_scales, int32_t batch,
+                               int32_t q_heads, int32_t kv_heads, int32_t n_tokens,
+                               int32_t head_dim, int32_t causal, int32_t frac_bp, int32_t k_max,
+                               int32_t* idx, int32_t* n_sel, uint8_t* bitmap, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * attn_qk4v8_fwd — QK4V8 FlashAttention forward (hotelren.com MpFA article §1, §3.3-3.4;
+ * the pages' mpfa_flash_attn(q, k, v, q_scale, k_scale, v_scale, block_size, num_warps,
+ * causal) call, §4.3). S = Q K^T on block-scaled FP4 tensor cores, FP32 online softmax over
+ * 128-key tiles, P quantized to E4M3 as P*448 against the running max after each tile,
+ * O += P V on block-scaled FP8 tensor cores, O / l with l the sum of the quantized weights.
+ * With fp16_bitmap set, a marked tile (ThriftAttention, method step 3) instead computes
+ * S = fp16(q) fp16(k), P = fp16(448 exp(s - m)), O += P fp16(v) on FP16 tensor cores, merged
+ * into the same (m, l, O).
+ * Causal masking keeps key j <= query i and needs n_q == n_k.
+ */
+typedef struct {
+  const uint8_t* q_codes;      /* [B, Hq, Nq, D/2]   NVFP4 (16-byte aligned) */
+  const uint8_t* q_scales;     /* [B, Hq, Nq, D/16]  E4M3 (8-byte aligned for D = 128) */
+  const float* q_tensor_scale; /* device scalar */
+  const uint8_t* k_codes;      /* [B, Hkv, Nk, D/2] */
+  const uint8_t* k_scales;     /* [B, Hkv, Nk, D/16] */
+  const float* k_tensor_scale; /* device scalar */
+  const uint8_t* v_codes;      /* [B, Hkv, D, Nk_pad] MXFP8 (quantize_mxfp8_v layout) */
+  const uint8_t* v_scales;     /* [B, Hkv, D, Nk_pad/32] E8M0 */
+  int32_t batch, q_heads, kv_heads, n_q, n_k, head_dim; /* head_dim 64 or 128 */
+  int32_t causal;
+  float softmax_scale;         /* e.g. 1/sqrt(head_dim) */
+  const uint8_t* fp16_bitmap;  /* optional [B*Hq, ceil(Nq/128), ceil(Nk/128)]; or NULL */
+  const void* q16;             /* fp16 [B, Hq, Nq, D] when fp16_bitmap is set */
+  const void* k16;             /* fp16 [B, Hkv, Nk, D] */
+  const void* v16;             /* fp16 [B, Hkv, D, Nk_pad] (quantize_mxfp8_v's v16) */
+  qk4v8_dtype out_dtype;
+  void* out;                   /* [B, Hq, Nq, D] out, 16-byte aligned */
+  float* lse;                  /* optional [B, Hq, Nq] natural-log sum-exp out; or NULL */
+} qk4v8_fwd_params;
+
+qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* params, cudaStream_t stream);
+
+/*
+ * attn_qk4v8_decode_paged — one decoding step over a paged NVFP4-K / MXFP8-V KV cache
+ * (sns.style BitDecoding-FP4 summary: the cache is read once per step; GQA queries share one
+ * tensor-core MMA; P quantization fused). Split-K: the keys of a sequence are cut into
+ * splits of split_tokens keys (a multiple of 128); each split runs the QK4V8 online softmax
+ * from its own running max, and the splits merge exactly (M = max m_s,
+ * O = sum e^(m_s - M) O_s / sum e^(m_s - M) l_s).
+ * Page layout (64 tokens per page, per page and KV head):
+ *   K codes [64, D/2], K scales [64, D/16] (NVFP4, one FP32 scale for the whole cache),
+ *   V codes [D, 64] (token-contiguous), V scales [D, 2] (E8M0 per 32 tokens).
+ * Tokens of a sequence's last page at or beyond its context length must hold finite codes
+ * (zero is the usual padding).
+ */
+typedef struct {
+  const uint8_t* q_codes;      /* [S, Hq, D/2] NVFP4 of the step's queries */
+  const uint8_t* q_scales;     /* [S, Hq, D/16] */
+  const float* q_tensor_scale;
+  const uint8_t* k_pages;      /* [num_pages, Hkv, 64, D/2] */
+  const uint8_t* k_page_scales;/* [num_pages, Hkv, 64, D/16] */
+  const float* k_tensor_scale;
+  const uint8_t* v_pages;      /* [num_pages, Hkv, D, 64] */
+  const uint8_t* v_page_scales;/* [num_pages, Hkv, D, 2] */
+  const int32_t* page_table;   /* [S, max_pages] physical page of each logical page */
+  const int32_t* context_lens; /* [S], 1 <= len <= min(max_context, 64 * max_pages) */
+  int32_t num_seqs, num_pages, max_pages, q_heads, kv_heads, head_dim; /* head_dim 128 */
+  int32_t max_context;         /* host-side bound on context_lens (sizes grid and workspace) */
+  int32_t split_tokens;        /* keys per split, a positive multiple of 128 */
+  float softmax_scale;
+  qk4v8_dtype out_dtype;
+  void* out;                   /* [S, Hq, D] out */
+  float* lse;                  /* optional [S, Hq] out; or NULL */
+} qk4v8_decode_params;
+
+size_t attn_qk4v8_decode_workspace_size(const qk4v8_decode_params* params);
+qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* params, void* workspace,
+                                     size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QK4V8_H */

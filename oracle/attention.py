@@ -85,36 +85,34 @@ def attention_rows(q: np.ndarray, row_pos: np.ndarray, k: np.ndarray, v: np.ndar
     for t in range(t_begin, t_end):
         j0, j1 = t * TILE, min((t + 1) * TILE, nk)
         keys = np.arange(j0, j1)
-        valid = np.ones((r, j1 - j0), dtype=bool)
-        if causal:
-            valid &= keys[None, :] <= row_pos[:, None]
-        live = valid.any(axis=1)
-        if not live.any():
+        # rows with at least one visible key in this tile; the others keep their state
+        rows = np.nonzero(row_pos >= j0)[0] if causal else np.arange(r)
+        if rows.size == 0:
             continue
-        s = (q @ k[j0:j1].T) * softmax_scale
-        sel = np.zeros(r, dtype=bool) if fp16_select is None else fp16_select(q_tile, t)
+        valid = np.ones((rows.size, j1 - j0), dtype=bool)
+        if causal:
+            valid &= keys[None, :] <= row_pos[rows, None]
+        s = (q[rows] @ k[j0:j1].T) * softmax_scale
+        sel = np.zeros(rows.size, dtype=bool) if fp16_select is None else fp16_select(q_tile[rows], t)
         if sel.any():
-            s16 = (q16[sel] @ k16[j0:j1].T) * softmax_scale
-            s[sel] = s16
+            s[sel] = (q16[rows[sel]] @ k16[j0:j1].T) * softmax_scale
         s = np.where(valid, s, -np.inf)
-        m_tile = s.max(axis=1)
-        m_new = np.maximum(m, m_tile)
-        m_safe = np.where(live, m_new, 0.0)
-        p_tilde = np.where(valid, np.exp(s - m_safe[:, None]), 0.0)
+        m_old = m[rows]
+        m_new = np.maximum(m_old, s.max(axis=1))
+        p_tilde = np.where(valid, np.exp(s - m_new[:, None]), 0.0)
         if quantize_p:
             p = _p_e4m3(p_tilde)
             if sel.any():
                 p[sel] = _p_fp16(p_tilde[sel])
         else:
             p = p_tilde
-        alpha = np.where(np.isfinite(m), np.exp(np.where(np.isfinite(m), m, 0.0) - m_safe), 0.0)
-        alpha = np.where(live, alpha, 1.0)
+        alpha = np.where(np.isfinite(m_old), np.exp(np.where(np.isfinite(m_old), m_old, 0.0) - m_new), 0.0)
         pv = p @ v[j0:j1]
         if sel.any():
             pv[sel] = p[sel] @ v16[j0:j1]
-        l = np.where(live, alpha * l + p.sum(axis=1), l)
-        o = np.where(live[:, None], alpha[:, None] * o + pv, o)
-        m = np.where(live, m_new, m)
+        l[rows] = alpha * l[rows] + p.sum(axis=1)
+        o[rows] = alpha[:, None] * o[rows] + pv
+        m[rows] = m_new
     return m, l, o
 
 

@@ -1,0 +1,146 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports exactly what
+include/qk4v8.h declares, its structs match the binding, and argument validation rejects bad
+calls before touching the device."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from bit_block_scaled_nvfp4_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qk4v8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)) -
+                  {"if", "defined"})
+
+
+def test_header_declares_the_bound_functions():
+    names = declared_functions()
+    assert set(names) == set(_lib.SIGNATURES), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", out, flags=re.M), name
+
+
+def test_struct_layouts_match(lib):
+    assert lib.qk4v8_struct_size(0) == C.sizeof(_lib.FwdParams)
+    assert lib.qk4v8_struct_size(1) == C.sizeof(_lib.DecodeParams)
+    assert lib.qk4v8_struct_size(7) == 0
+
+
+def test_version_and_status_strings(lib):
+    assert lib.qk4v8_version() == 100
+    assert lib.qk4v8_status_string(0) == b"ok"
+    assert lib.qk4v8_status_string(4) == b"device wait timed out"
+    assert lib.qk4v8_status_string(99) == b"unknown status"
+
+
+FAKE = 1 << 20          # aligned fake device addresses: never dereferenced on these paths
+
+
+def test_quantize_nvfp4_validation(lib):
+    f = lib.quantize_nvfp4
+    ok = dict(x=FAKE, dt=1, rows=4, cols=64, stride=64, ts=0.0, codes=FAKE, scales=FAKE,
+              tsout=FAKE, x16=None, ws=FAKE, wsb=256)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["x"], a["dt"], a["rows"], a["cols"], a["stride"], a["ts"], a["codes"],
+                 a["scales"], a["tsout"], a["x16"], a["ws"], a["wsb"], None)
+    assert call(x=None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert call(cols=40) == _lib.QK4V8_ERR_INVALID_ARG            # not a multiple of 16
+    assert call(stride=32) == _lib.QK4V8_ERR_INVALID_ARG          # stride < cols
+    assert call(stride=68) == _lib.QK4V8_ERR_INVALID_ARG          # stride % 8
+    assert call(x=FAKE + 2) == _lib.QK4V8_ERR_INVALID_ARG         # misaligned input
+    assert call(ws=None) == _lib.QK4V8_ERR_INVALID_ARG            # amax pass needs workspace
+    assert call(wsb=2) == _lib.QK4V8_ERR_INVALID_ARG
+    assert call(dt=7) == _lib.QK4V8_ERR_INVALID_ARG
+
+
+def test_quantize_mxfp8_validation(lib):
+    f = lib.quantize_mxfp8_v
+    assert f(None, 1, 1, 128, 128, FAKE, FAKE, None, None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(FAKE, 1, 1, 0, 128, FAKE, FAKE, None, None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(FAKE, 1, 1, 128, 96, FAKE, FAKE, None, None) == _lib.QK4V8_ERR_UNSUPPORTED
+    assert f(FAKE + 8, 1, 1, 128, 128, FAKE, FAKE, None, None) == _lib.QK4V8_ERR_INVALID_ARG
+
+
+def test_tile_select_validation(lib):
+    f = lib.tile_score_select
+    args = [FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 1000, 128, 1, 500, 64, FAKE, FAKE, None, FAKE, 1 << 20, None]
+    bad_heads = list(args); bad_heads[5] = 3; bad_heads[6] = 2
+    assert f(*bad_heads) == _lib.QK4V8_ERR_INVALID_ARG             # Hq % Hkv
+    small_k = list(args); small_k[11] = 1
+    assert f(*small_k) == _lib.QK4V8_ERR_INVALID_ARG               # k_max < ceil(36 * 5%) = 2
+    big_k = list(args); big_k[11] = 5000
+    assert f(*big_k) == _lib.QK4V8_ERR_UNSUPPORTED
+    frac = list(args); frac[10] = 10001
+    assert f(*frac) == _lib.QK4V8_ERR_INVALID_ARG
+    ws = list(args); ws[16] = 8
+    assert f(*ws) == _lib.QK4V8_ERR_INVALID_ARG
+
+
+def _fwd(**kw):
+    p = _lib.FwdParams()
+    for n in ("q_codes", "q_scales", "q_tensor_scale", "k_codes", "k_scales", "k_tensor_scale",
+              "v_codes", "v_scales", "out"):
+        setattr(p, n, FAKE)
+    p.batch, p.q_heads, p.kv_heads, p.n_q, p.n_k, p.head_dim = 1, 4, 2, 256, 256, 128
+    p.causal, p.softmax_scale, p.out_dtype = 1, 0.125, 1
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_fwd_validation(lib):
+    f = lambda p: lib.attn_qk4v8_fwd(C.byref(p), None)
+    assert f(_fwd(q_codes=None)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_fwd(q_heads=3)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_fwd(n_k=300)) == _lib.QK4V8_ERR_INVALID_ARG        # causal needs Nq == Nk
+    assert f(_fwd(head_dim=96)) == _lib.QK4V8_ERR_UNSUPPORTED
+    assert f(_fwd(out=FAKE + 4)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_fwd(softmax_scale=0.0)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_fwd(fp16_bitmap=FAKE)) == _lib.QK4V8_ERR_INVALID_ARG  # bitmap without fp16 copies
+    assert lib.attn_qk4v8_fwd(None, None) == _lib.QK4V8_ERR_INVALID_ARG
+
+
+def _dec(**kw):
+    p = _lib.DecodeParams()
+    for n in ("q_codes", "q_scales", "q_tensor_scale", "k_pages", "k_page_scales",
+              "k_tensor_scale", "v_pages", "v_page_scales", "page_table", "context_lens", "out"):
+        setattr(p, n, FAKE)
+    p.num_seqs, p.num_pages, p.max_pages = 2, 100, 50
+    p.q_heads, p.kv_heads, p.head_dim = 32, 8, 128
+    p.max_context, p.split_tokens, p.softmax_scale, p.out_dtype = 3000, 1024, 0.088, 1
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_decode_validation_and_workspace(lib):
+    p = _dec()
+    assert lib.attn_qk4v8_decode_workspace_size(C.byref(p)) == 2 * 32 * 3 * 130 * 4
+    f = lambda p, wsb=1 << 30: lib.attn_qk4v8_decode_paged(C.byref(p), FAKE, wsb, None)
+    assert f(_dec(split_tokens=100)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_dec(max_context=50 * 64 + 1)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_dec(head_dim=64)) == _lib.QK4V8_ERR_UNSUPPORTED
+    assert f(_dec(q_heads=64, kv_heads=2)) == _lib.QK4V8_ERR_UNSUPPORTED  # g = 32 > 16
+    assert f(_dec(), wsb=16) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_dec(page_table=None)) == _lib.QK4V8_ERR_INVALID_ARG

@@ -1,0 +1,114 @@
+"""GPU parity of the QK4V8 prefill attention against the oracle (max |dO| <= 2e-2 rms and
+mean <= 2e-3 rms), full outputs on the small workloads and ragged shapes, sampled rows on the
+long-context workload, plus exact invariants on the GPU path itself."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from bit_block_scaled_nvfp4_b200 import api, workloads
+from oracle import attention as OA
+from oracle import quant as OQ
+from helpers import assert_attention_close, f32, oracle_prefill_rows, oracle_tensor_scale
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(q, k, v, causal, scale=None, frac_bp=0, out_dtype=None):
+    return api.qk4v8_attention(q.to(DEV), k.to(DEV), v.to(DEV), causal, scale,
+                               fp16_frac_bp=frac_bp, out_dtype=out_dtype)
+
+
+def _full_oracle(q, k, v, causal, scale):
+    B, Hq, N, D = q.shape
+    out = np.zeros((B, Hq, q.shape[2], D))
+    Hkv = k.shape[1]
+    sq, sk = oracle_tensor_scale(q), oracle_tensor_scale(k)
+    for b in range(B):
+        for hk in range(Hkv):
+            kh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(f32(k[b, hk]), tensor_scale=sk))
+            vc, vs = OQ.mxfp8_quantize_v(f32(v[b, hk]))
+            vh = OQ.mxfp8_dequantize_v(vc, vs, v.shape[2])
+            for hq in range(hk * (Hq // Hkv), (hk + 1) * (Hq // Hkv)):
+                qh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(f32(q[b, hq]), tensor_scale=sq))
+                out[b, hq] = OA.attention_head(qh, kh, vh, causal, scale)[0]
+    return out
+
+
+@pytest.mark.parametrize("name", ["tiny_prefill", "prefill_h16_n4096"])
+def test_workload_full_parity(name):
+    w = workloads.make_prefill(name)
+    D = w.cfg["d"]
+    scale = 1 / math.sqrt(D)
+    out = _run(w.q, w.k, w.v, w.cfg["causal"], scale)
+    ref = _full_oracle(w.q, w.k, w.v, w.cfg["causal"], scale)
+    assert out.dtype == w.q.dtype
+    assert_attention_close(f32(out), ref, name)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,D,causal", [
+    (1, 4, 2, 300, 300, 128, True),      # GQA, ragged tail
+    (2, 2, 1, 1000, 1000, 64, False),    # batch 2, non-causal, D = 64
+    (1, 2, 2, 200, 700, 128, False),     # Nq != Nk
+    (1, 1, 1, 1, 1, 128, True),          # one token
+    (1, 3, 3, 129, 129, 64, True),
+])
+def test_ragged_shapes(B, Hq, Hkv, Nq, Nk, D, causal):
+    g = torch.Generator().manual_seed(Nq * 7 + Nk)
+    q = torch.randn(B, Hq, Nq, D, generator=g).to(torch.bfloat16)
+    k = (torch.randn(B, Hkv, Nk, D, generator=g) * 2).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Nk, D, generator=g).to(torch.bfloat16)
+    out = _run(q, k, v, causal)
+    ref = _full_oracle(q, k, v, causal, 1 / math.sqrt(D))
+    assert_attention_close(f32(out), ref, "ragged")
+
+
+def test_long_context_gqa_sampled():
+    """32 query / 8 KV heads, 32768 tokens, causal; oracle on 2 heads x 256 seeded rows."""
+    w = workloads.make_prefill("prefill_gqa_n32768")
+    scale = 1 / math.sqrt(128)
+    out = _run(w.q, w.k, w.v, True, scale)
+    rng = np.random.default_rng(2)
+    heads = sorted(rng.choice(32, size=2, replace=False).tolist())
+    got, want = [], []
+    for hq in heads:
+        rows = np.sort(rng.choice(32768, size=256, replace=False))
+        o, _ = oracle_prefill_rows(w.q, w.k, w.v, hq, rows, True, scale)
+        want.append(o)
+        got.append(f32(out[0, hq, torch.as_tensor(rows, device=DEV)]))
+    assert_attention_close(np.concatenate(got), np.concatenate(want), "gqa 32k sampled")
+
+
+def test_constant_v_gives_constant_output():
+    g = torch.Generator().manual_seed(0)
+    q = torch.randn(1, 2, 500, 128, generator=g).to(torch.bfloat16)
+    k = (torch.randn(1, 2, 500, 128, generator=g) * 3).to(torch.bfloat16)
+    v = torch.ones(1, 2, 500, 128, dtype=torch.bfloat16)
+    out = _run(q, k, v, True).float()
+    assert torch.all((out - 1.0).abs() <= 2.0 ** -8)
+
+
+def test_first_causal_row_is_dequantized_v0():
+    w = workloads.make_prefill("prefill_h16_n4096")
+    out = _run(w.q, w.k, w.v, True)
+    vc, vs = OQ.mxfp8_quantize_v(f32(w.v[0, 3]))
+    v0 = OQ.mxfp8_dequantize_v(vc, vs, 4096)[0]
+    want = torch.tensor(v0, dtype=torch.float32).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(f32(out[0, 3, 0]), want)
+
+
+def test_lse_matches_oracle():
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(1, 2, 256, 128, generator=g).to(torch.bfloat16)
+    k = torch.randn(1, 2, 256, 128, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 2, 256, 128, generator=g).to(torch.bfloat16)
+    q4, k4, v8 = api.quantize_nvfp4(q.to(DEV)), api.quantize_nvfp4(k.to(DEV)), api.quantize_mxfp8_v(v.to(DEV))
+    _, lse = api.attn_qk4v8_fwd(q4, k4, v8, True, want_lse=True)
+    _, want = oracle_prefill_rows(q, k, v, 1, np.arange(256), True, 1 / math.sqrt(128))
+    assert np.max(np.abs(lse[0, 1].cpu().numpy() - want)) < 1e-3
+
+
+def test_status_clean_after_runs():
+    assert api.check_status() == 0

@@ -1,0 +1,135 @@
+"""GPU parity of the paged split-K decode against the oracle, page-permutation invariance,
+and the device-side page-id bounds check."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from bit_block_scaled_nvfp4_b200 import api, paged, workloads
+from oracle import attention as OA
+from oracle import quant as OQ
+from oracle import paged as OP
+from helpers import assert_attention_close, f32, oracle_tensor_scale
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+KTS = workloads.DECODE_K_TENSOR_SCALE
+
+
+def _build(lens, hkv, d, seed, shuffle=True):
+    g = torch.Generator().manual_seed(seed)
+    pages_per = [(n + 63) // 64 for n in lens]
+    total = sum(pages_per)
+    perm = torch.randperm(total, generator=g)
+    if not shuffle:
+        perm = torch.arange(total)
+    table = torch.full((len(lens), max(pages_per)), -1, dtype=torch.int32)
+    seqs, off = [], 0
+    cache = paged.empty_cache(total, hkv, d, KTS, DEV)
+    for s, n in enumerate(lens):
+        table[s, :pages_per[s]] = perm[off:off + pages_per[s]].int()
+        off += pages_per[s]
+        k = ((torch.randn(n, hkv, d, generator=g) + 0.3) * 3).to(torch.bfloat16)
+        v = torch.randn(n, hkv, d, generator=g).to(torch.bfloat16)
+        seqs.append((k, v))
+        paged.write_sequence(cache, k.to(DEV), v.to(DEV), table[s, :pages_per[s]])
+    return cache, table, seqs
+
+
+def _oracle_decode(q, seqs, lens, hq, hkv, split, scale):
+    """Oracle outputs [S, Hq, D] from the dense per-sequence K/V and the step's q."""
+    S, _, d = q.shape
+    sq = oracle_tensor_scale(q)
+    qc, qs, qt = OQ.nvfp4_quantize(f32(q), tensor_scale=sq)
+    qh = OQ.nvfp4_dequantize(qc, qs, qt)
+    g = hq // hkv
+    out = np.zeros((S, hq, d))
+    lse = np.zeros((S, hq))
+    for s, (k, v) in enumerate(seqs):
+        kc, ks, vc, vs = OP.quantize_sequence(f32(k), f32(v), KTS)
+        kh = OQ.nvfp4_dequantize(kc, ks, np.float32(KTS))
+        vh = OQ.mxfp8_dequantize_v(vc, vs, lens[s])
+        for h in range(hkv):
+            o, l = OA.decode_rows(qh[s, h * g:(h + 1) * g], kh[h], vh[h], lens[s], scale, split)
+            out[s, h * g:(h + 1) * g] = o
+            lse[s, h * g:(h + 1) * g] = l
+    return out, lse
+
+
+@pytest.mark.parametrize("lens,hq,hkv,split", [([1, 200, 1000, 64, 129], 8, 2, 256),
+                                                ([5000, 333], 32, 8, 1024),
+                                                ([777], 16, 1, 128)])
+def test_decode_parity(lens, hq, hkv, split):
+    d = 128
+    cache, table, seqs = _build(lens, hkv, d, seed=sum(lens))
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn(len(lens), hq, d, generator=g).to(torch.bfloat16)
+    q4 = api.quantize_nvfp4(q.to(DEV))
+    ctx = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    out, lse = api.attn_qk4v8_decode_paged(q4, cache, table.to(DEV), ctx, max(lens), split,
+                                           want_lse=True)
+    want, wlse = _oracle_decode(q, seqs, lens, hq, hkv, split, 1 / math.sqrt(d))
+    assert_attention_close(f32(out), want, "decode")
+    assert np.max(np.abs(lse.cpu().numpy() - wlse)) < 1e-3
+    assert api.check_status() == 0
+
+
+def test_page_permutation_is_bit_invariant():
+    lens = [900, 300]
+    c1, t1, seqs = _build(lens, 2, 128, seed=5, shuffle=False)
+    c2, t2, _ = _build(lens, 2, 128, seed=5, shuffle=True)    # same data, other pages
+    q = torch.randn(2, 8, 128, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    q4 = api.quantize_nvfp4(q.to(DEV))
+    ctx = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    o1 = api.attn_qk4v8_decode_paged(q4, c1, t1.to(DEV), ctx, 900, 256)
+    o2 = api.attn_qk4v8_decode_paged(q4, c2, t2.to(DEV), ctx, 900, 256)
+    assert torch.equal(o1, o2)
+
+
+def test_bad_page_id_reports_bounds_error():
+    lens = [300]
+    cache, table, _ = _build(lens, 2, 128, seed=9)
+    table[0, 2] = 10_000                                    # past num_pages
+    q4 = api.quantize_nvfp4(torch.randn(1, 8, 128, dtype=torch.bfloat16, device=DEV))
+    ctx = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    api.attn_qk4v8_decode_paged(q4, cache, table.to(DEV), ctx, 300, 128)
+    assert api.check_status() == 5                          # QK4V8_ERR_BOUNDS
+    assert api.check_status() == 0                          # cleared
+
+
+def test_paged_workload_sampled_sequences():
+    """64 sequences, lengths U[8192, 32768], 32/8 heads, shuffled pages; oracle on the
+    shortest, the longest and two seeded sequences (all heads)."""
+    lay = workloads.make_decode_layout()
+    cfg = lay.cfg
+    cache = paged.empty_cache(lay.num_pages, cfg["Hkv"], cfg["d"], KTS, DEV)
+    seqs = {}
+    lens = lay.lens.tolist()
+    pick = {int(np.argmin(lens)), int(np.argmax(lens)), 7, 40}
+    for s in range(cfg["S"]):
+        k, v = workloads.make_decode_sequence(lay, s)
+        n_pages = (lens[s] + 63) // 64
+        paged.write_sequence(cache, k.to(DEV), v.to(DEV), lay.page_table[s, :n_pages])
+        if s in pick:
+            seqs[s] = (k, v)
+    q = workloads.make_decode_query(lay)
+    q4 = api.quantize_nvfp4(q.to(DEV))
+    split = 4096
+    out = api.attn_qk4v8_decode_paged(q4, cache, lay.page_table.to(DEV), lay.lens.to(DEV),
+                                      max(lens), split)
+    sq = oracle_tensor_scale(q)
+    qc, qs, qt = OQ.nvfp4_quantize(f32(q), tensor_scale=sq)
+    qh = OQ.nvfp4_dequantize(qc, qs, qt)
+    g = cfg["Hq"] // cfg["Hkv"]
+    got, want = [], []
+    for s, (k, v) in sorted(seqs.items()):
+        kc, ks, vc, vs = OP.quantize_sequence(f32(k), f32(v), KTS)
+        kh = OQ.nvfp4_dequantize(kc, ks, np.float32(KTS))
+        vh = OQ.mxfp8_dequantize_v(vc, vs, lens[s])
+        for h in range(cfg["Hkv"]):
+            o, _ = OA.decode_rows(qh[s, h * g:(h + 1) * g], kh[h], vh[h], lens[s],
+                                  1 / math.sqrt(128), split)
+            want.append(o)
+            got.append(f32(out[s, h * g:(h + 1) * g]))
+    assert_attention_close(np.concatenate(got), np.concatenate(want), "paged decode workload")

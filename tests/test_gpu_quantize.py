@@ -1,0 +1,123 @@
+"""GPU parity of the quantize kernels against the oracle: bit-exact codes, scales and tensor
+scales on the workloads' Q/K/V, ragged shapes, and exhaustive sweeps of every fp16 input
+through the E2M1 element, E4M3 block-scale and E4M3 V-element conversions."""
+import numpy as np
+import pytest
+import torch
+
+from bit_block_scaled_nvfp4_b200 import api, workloads
+from oracle import formats as OF
+from oracle import quant as OQ
+from helpers import f32
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _nvfp4_equal(x_cpu, tensor_scale=None, want_fp16=False):
+    g = api.quantize_nvfp4(x_cpu.to(DEV), tensor_scale=tensor_scale, want_fp16=want_fp16)
+    c, s, t = OQ.nvfp4_quantize(f32(x_cpu), tensor_scale=tensor_scale)
+    gc, gs = g.codes.cpu().numpy(), g.scales.cpu().numpy()
+    assert np.array_equal(gs, s), f"scales differ at {np.argwhere(gs != s)[:5]}"
+    assert np.array_equal(gc, c), f"codes differ at {np.argwhere(gc != c)[:5]}"
+    assert np.float32(g.tensor_scale.item()) == t
+    if want_fp16:
+        assert np.array_equal(g.fp16.cpu().numpy(), OF.fp16_round(f32(x_cpu)).astype(np.float16))
+    return g
+
+
+@pytest.mark.parametrize("name", ["tiny_prefill", "prefill_h16_n4096"])
+def test_nvfp4_workload_q_k_bit_exact(name):
+    w = workloads.make_prefill(name)
+    _nvfp4_equal(w.q)
+    _nvfp4_equal(w.k, want_fp16=True)
+
+
+@pytest.mark.parametrize("shape,dtype", [((1000, 64), torch.bfloat16), ((3, 37, 128), torch.float16),
+                                         ((1, 16), torch.bfloat16)])
+def test_nvfp4_ragged_shapes(shape, dtype):
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(shape, generator=g) * torch.rand(shape[:-1] + (1,), generator=g) * 7).to(dtype)
+    _nvfp4_equal(x)
+    _nvfp4_equal(x, tensor_scale=0.0625)
+
+
+def test_nvfp4_zero_tensor():
+    g = api.quantize_nvfp4(torch.zeros(4, 64, dtype=torch.bfloat16, device=DEV))
+    assert g.tensor_scale.item() == 1.0 and not g.codes.any() and not g.scales.any()
+
+
+def _all_fp16_values(lo_bits, hi_bits):
+    return torch.arange(lo_bits, hi_bits, dtype=torch.int32).to(torch.int16).view(torch.float16)
+
+
+def test_e2m1_conversion_exhaustive_fp16():
+    """Tensor scale 2^-8 and a leading 6 in every block give s_b = 256, den = 1: each code is
+    E2M1 of the raw fp16 value. Every fp16 value in [-8, 8] (both signs, zeros) is swept."""
+    pos = _all_fp16_values(0x0000, 0x4801)                  # 0 .. 8
+    vals = torch.cat([pos, -pos])
+    n = vals.numel()
+    nb = (n + 14) // 15
+    x = torch.zeros(nb, 16, dtype=torch.float16)
+    x[:, 0] = 6.0
+    flat = torch.zeros(nb * 15, dtype=torch.float16)
+    flat[:n] = vals
+    x[:, 1:] = flat.view(nb, 15)
+    _nvfp4_equal(x, tensor_scale=2.0 ** -8)
+
+
+def test_e4m3_block_scale_exhaustive_fp16():
+    """Every positive finite fp16 value as a block amax, with tensor scale 2^-4: the block
+    scale is E4M3(amax / 6 / 2^-4) across the whole E4M3 range, subnormals and saturation."""
+    amax = _all_fp16_values(0x0001, 0x7C00)
+    x = torch.zeros(amax.numel(), 16, dtype=torch.float16)
+    x[:, 3] = amax
+    x[:, 7] = -amax / 3
+    _nvfp4_equal(x, tensor_scale=2.0 ** -4)
+
+
+def _mxfp8_equal(v_cpu, want_fp16=False):
+    g = api.quantize_mxfp8_v(v_cpu.to(DEV), want_fp16=want_fp16)
+    c, s = OQ.mxfp8_quantize_v(f32(v_cpu))
+    gc, gs = g.codes.cpu().numpy(), g.scales.cpu().numpy()
+    assert np.array_equal(gs, s), f"scales differ at {np.argwhere(gs != s)[:5]}"
+    assert np.array_equal(gc, c), f"codes differ at {np.argwhere(gc != c)[:5]}"
+    if want_fp16:
+        n = v_cpu.shape[-2]
+        ref = np.zeros(gc.shape, dtype=np.float16)
+        ref[..., :n] = np.swapaxes(OF.fp16_round(f32(v_cpu)), -1, -2)
+        assert np.array_equal(g.fp16.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("name", ["tiny_prefill", "prefill_h16_n4096"])
+def test_mxfp8_workload_v_bit_exact(name):
+    w = workloads.make_prefill(name)
+    _mxfp8_equal(w.v, want_fp16=True)
+
+
+@pytest.mark.parametrize("n,d", [(1, 128), (300, 64), (129, 128)])
+def test_mxfp8_ragged(n, d):
+    g = torch.Generator().manual_seed(n)
+    v = (torch.randn(3, n, d, generator=g) * torch.rand(3, 1, d, generator=g) * 50).to(torch.bfloat16)
+    _mxfp8_equal(v, want_fp16=True)
+
+
+def test_e4m3_element_conversion_exhaustive_fp16():
+    """Groups whose first token is 480 have e = 0 (480 saturates to 448); the other 31 tokens
+    sweep every fp16 value in [-480, 480], so each code is E4M3 of the raw value."""
+    pos = _all_fp16_values(0x0000, 0x5F81)                  # 0 .. 480
+    vals = torch.cat([pos, -pos])
+    n = vals.numel()
+    ng = (n + 30) // 31
+    ng = (ng + 3) // 4 * 4
+    d = 64
+    col = torch.zeros(ng, 32, dtype=torch.float16)
+    col[:, 0] = 480.0
+    flat = torch.zeros(ng * 31, dtype=torch.float16)
+    flat[:n] = vals
+    col[:, 1:] = flat.view(ng, 31)
+    tokens = col.reshape(-1)                                # ng*32 tokens, one channel
+    v = torch.zeros(1, tokens.numel(), d, dtype=torch.float16)
+    v[0, :, 5] = tokens
+    v[0, :, 60] = -tokens
+    _mxfp8_equal(v)
