@@ -20,6 +20,7 @@ QK4V8_ERR_TIMEOUT = 4
 QK4V8_ERR_BOUNDS = 5
 QK4V8_F16 = 0
 QK4V8_BF16 = 1
+QK4V8_F32 = 2
 
 vp = C.c_void_p
 i32 = C.c_int32

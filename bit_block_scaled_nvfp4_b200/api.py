@@ -15,6 +15,7 @@ import torch
 from . import _lib
 
 _DT = {torch.float16: _lib.QK4V8_F16, torch.bfloat16: _lib.QK4V8_BF16}
+_OUT_DT = {**_DT, torch.float32: _lib.QK4V8_F32}
 
 
 def _ptr(t):
@@ -146,7 +147,7 @@ def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
     if fp16_bitmap is not None:
         p.fp16_bitmap = fp16_bitmap.data_ptr()
         p.q16, p.k16, p.v16 = q.fp16.data_ptr(), k.fp16.data_ptr(), v.fp16.data_ptr()
-    p.out_dtype = _DT[out_dtype]
+    p.out_dtype = _OUT_DT[out_dtype]
     p.out = out.data_ptr()
     p.lse = lse.data_ptr() if lse is not None else None
     _lib.check(lib.attn_qk4v8_fwd(C.byref(p), _stream()), "attn_qk4v8_fwd")
@@ -179,7 +180,7 @@ def decode_params(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
     p.q_heads, p.kv_heads, p.head_dim = Hq, Hkv, d
     p.max_context, p.split_tokens = int(max_context), int(split_tokens)
     p.softmax_scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
-    p.out_dtype = _DT[out.dtype]
+    p.out_dtype = _OUT_DT[out.dtype]
     p.out = out.data_ptr()
     p.lse = lse.data_ptr() if lse is not None else None
     return p

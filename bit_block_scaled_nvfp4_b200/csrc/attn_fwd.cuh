@@ -22,7 +22,6 @@
 namespace qk4v8 {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLog2_448 = 8.807354922057604f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct FwdArgs {
@@ -37,7 +36,7 @@ struct FwdArgs {
   int32_t B, Hq, Hkv, Nq, Nk, Npad, Tq, Tk;
   int32_t causal;
   float softmax_scale;
-  int32_t out_bf16;
+  int32_t out_kind;          // 0 fp16, 1 bf16, 2 fp32
 };
 
 template <int D, bool kMixed>
@@ -313,7 +312,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
             mma_nvf4(tS, da, db, idesc_qk, tbase + L::T_QSF + 4 * kk, tk + 4 * kk, kk > 0 ? 1u : 0u);
           }
+          mma_commit(s_full + b2);
+          if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
         } else {
+          // The single FP16 operand buffer is refilled only after the previous FP16 tile's
+          // PV has finished, so PV(j-1) must be issued before waiting for this tile's data.
+          if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
           if (!q16_ready) {
             if (!wait1(q16_full, 0)) { ok = false; break; }
             q16_ready = true;
@@ -327,9 +331,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sK16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
             mma_f16(tS, da, db, idesc_qk16, kk > 0 ? 1u : 0u);
           }
+          mma_commit(s_full + b2);
         }
-        mma_commit(s_full + b2);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && nt > 0) issue_pv(nt - 1);
       (void)n16_pv;
@@ -344,8 +347,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int row = wq * 32 + lane;
     const int qi = qt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    const float C4 = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
-    const float C16 = a.softmax_scale * kLog2e;
+    // Scores stay in the FP4 MMA's raw units (S = sum codes*scales); the running max m is
+    // kept in those units, so (s - m) is exact for the keys near the max, and
+    // p = 2^((s - m) * C) with C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true
+    // dot products and are brought into raw units by 1 / (s_tQ s_tK).
+    const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
+    const float R16 = 1.f / ((*a.q_ts) * (*a.k_ts));
     float m_run = -INFINITY, l_run = 0.f;
     unsigned char* sP = sm + L::OFF_P;
     bool ok = true;
@@ -367,7 +374,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free + b2);
-      const float C = f16 ? C16 : C4;
+      if (f16) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] *= R16;
+      }
       const int kbase = j * 128;
       const bool need_mask = (a.causal && kbase + 127 > qi) || (kbase + 128 > a.Nk);
       float mt = -INFINITY;
@@ -375,27 +385,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
-          x[c] = (c <= lim) ? x[c] * C : -INFINITY;
+          x[c] = (c <= lim) ? x[c] : -INFINITY;
           mt = fmaxf(mt, x[c]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          x[c] = x[c] * C;
-          mt = fmaxf(mt, x[c]);
-        }
+        for (int c = 0; c < 128; ++c) mt = fmaxf(mt, x[c]);
       }
       const float m_new = fmaxf(m_run, mt);
       const bool dead = (m_new == -INFINITY);
-      const float moff = dead ? 0.f : m_new - kLog2_448;
-      const float alpha = dead ? 1.f : ex2_approx(m_run - m_new);
+      const float mref = dead ? 0.f : m_new;
+      const float alpha = dead ? 1.f : ex2_approx((m_run - m_new) * C);
       float lsum = 0.f;
       uint32_t pw[64];             // e4m3: 32 words used; fp16: 64 words
       if (!f16) {
 #pragma unroll
         for (int c = 0; c < 128; c += 4) {
-          const uint32_t lo = cvt_e4m3x2(ex2_approx(x[c] - moff), ex2_approx(x[c + 1] - moff));
-          const uint32_t hi = cvt_e4m3x2(ex2_approx(x[c + 2] - moff), ex2_approx(x[c + 3] - moff));
+          float p[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) p[i] = ex2_approx((x[c + i] - mref) * C) * 448.f;
+          const uint32_t lo = cvt_e4m3x2(p[0], p[1]);
+          const uint32_t hi = cvt_e4m3x2(p[2], p[3]);
           const float2 f0 = __half22float2(e4m3x2_to_half2(lo));
           const float2 f1 = __half22float2(e4m3x2_to_half2(hi));
           lsum += (f0.x + f0.y) + (f1.x + f1.y);
@@ -404,7 +414,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       } else {
 #pragma unroll
         for (int c = 0; c < 128; c += 2) {
-          const __half2 h = __floats2half2_rn(ex2_approx(x[c] - moff), ex2_approx(x[c + 1] - moff));
+          const __half2 h = __floats2half2_rn(ex2_approx((x[c] - mref) * C) * 448.f,
+                                              ex2_approx((x[c + 1] - mref) * C) * 448.f);
           const float2 f = __half22float2(h);
           lsum += f.x + f.y;
           pw[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
@@ -455,7 +466,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ---- epilogue ----
     if (ok && nt > 0 && waitw(pv_done + ((nt - 1) & 1), ((nt - 1) >> 1) & 1)) {
       tc_fence_after();
-      const float inv = 1.f / l_run;
       const uint32_t tO = tbase + L::T_O + lane_addr;
       const bool store = qi < a.Nq;
       const int64_t orow = static_cast<int64_t>(bhq) * a.Nq + qi;
@@ -465,24 +475,35 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_ld32(tO + c, o);
         tmem_wait_ld();
         if (store) {
-          __align__(16) uint32_t packed[16];
+          if (a.out_kind == 2) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c);
 #pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float v0 = __uint_as_float(o[k]) * inv, v1 = __uint_as_float(o[k + 1]) * inv;
-            if (a.out_bf16) {
-              __nv_bfloat162 t = __floats2bfloat162_rn(v0, v1);
-              packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
-            } else {
-              __half2 t = __floats2half2_rn(v0, v1);
-              packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
+            for (int k = 0; k < 8; ++k)
+              dst[k] = make_float4(__fdiv_rn(__uint_as_float(o[4 * k]), l_run),
+                                   __fdiv_rn(__uint_as_float(o[4 * k + 1]), l_run),
+                                   __fdiv_rn(__uint_as_float(o[4 * k + 2]), l_run),
+                                   __fdiv_rn(__uint_as_float(o[4 * k + 3]), l_run));
+          } else {
+            __align__(16) uint32_t packed[16];
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              const float v0 = __fdiv_rn(__uint_as_float(o[k]), l_run);
+              const float v1 = __fdiv_rn(__uint_as_float(o[k + 1]), l_run);
+              if (a.out_kind == 1) {
+                __nv_bfloat162 t = __floats2bfloat162_rn(v0, v1);
+                packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
+              } else {
+                __half2 t = __floats2half2_rn(v0, v1);
+                packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
+              }
             }
-          }
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + c);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + c);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = reinterpret_cast<uint4*>(packed)[k];
+            for (int k = 0; k < 4; ++k) dst[k] = reinterpret_cast<uint4*>(packed)[k];
+          }
         }
       }
-      if (store && a.lse != nullptr) a.lse[orow] = m_run * kLn2 + logf(l_run * (1.f / 448.f));
+      if (store && a.lse != nullptr) a.lse[orow] = m_run * C * kLn2 + logf(l_run * (1.f / 448.f));
     }
   }
   tc_fence_before();

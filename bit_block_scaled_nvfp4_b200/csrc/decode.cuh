@@ -297,7 +297,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const bool valid = k_begin + blk * 128 + r < k_end;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        x[q] = (valid && q < g) ? x[q] * C : -INFINITY;
+        x[q] = (valid && q < g) ? x[q] : -INFINITY;        // raw MMA units
         float mm = x[q];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
@@ -311,16 +311,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float mb = fmaxf(fmaxf(red_max[q], red_max[16 + q]), fmaxf(red_max[32 + q], red_max[48 + q]));
         const float m_new = fmaxf(m_run[q], mb);
         const bool dead = (m_new == -INFINITY);
-        moff[q] = dead ? 0.f : m_new - kLog2_448;
-        alpha[q] = dead ? 1.f : ex2_approx(m_run[q] - m_new);
+        moff[q] = dead ? 0.f : m_new;
+        alpha[q] = dead ? 1.f : ex2_approx((m_run[q] - m_new) * C);
         all_one = all_one && (alpha[q] == 1.f);
         m_run[q] = m_new;
       }
       uint32_t codes[4];
 #pragma unroll
       for (int q = 0; q < 16; q += 4) {
-        const uint32_t lo = cvt_e4m3x2(ex2_approx(x[q] - moff[q]), ex2_approx(x[q + 1] - moff[q + 1]));
-        const uint32_t hi = cvt_e4m3x2(ex2_approx(x[q + 2] - moff[q + 2]), ex2_approx(x[q + 3] - moff[q + 3]));
+        float p[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p[i] = ex2_approx((x[q + i] - moff[q + i]) * C) * 448.f;
+        const uint32_t lo = cvt_e4m3x2(p[0], p[1]);
+        const uint32_t hi = cvt_e4m3x2(p[2], p[3]);
         codes[q >> 2] = lo | (hi << 16);
         const float2 f0 = __half22float2(e4m3x2_to_half2(lo));
         const float2 f1 = __half22float2(e4m3x2_to_half2(hi));
@@ -372,9 +375,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       float o[16];
       tmem_ld16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
       tmem_wait_ld();
-      for (int q = 0; q < g; ++q) {
-        part[q * q_stride + r] = o[q];
-        if (r == 0) { part[q * q_stride + D] = m_run[q]; part[q * q_stride + D + 1] = l_run[q]; }
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        if (q < g) {
+          part[q * q_stride + r] = o[q];
+          // the merge works in log2 units: store m * C
+          if (r == 0) { part[q * q_stride + D] = m_run[q] * C; part[q * q_stride + D + 1] = l_run[q]; }
+        }
       }
     }
   }
@@ -388,7 +395,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
 // Merge the splits: one CTA per (sequence, query head), one thread per channel.
 __global__ void __launch_bounds__(128) decode_merge_kernel(const float* __restrict__ ws,
-                                                           int32_t n_splits, int32_t out_bf16,
+                                                           int32_t n_splits, int32_t out_kind,
                                                            void* __restrict__ out,
                                                            float* __restrict__ lse) {
   constexpr int D = 128;
@@ -404,7 +411,8 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float* __restri
     acc += w * p[i * (D + 2) + threadIdx.x];
   }
   const float v = acc / Lsum;
-  if (out_bf16) static_cast<__nv_bfloat16*>(out)[row * D + threadIdx.x] = __float2bfloat16_rn(v);
+  if (out_kind == 2) static_cast<float*>(out)[row * D + threadIdx.x] = v;
+  else if (out_kind == 1) static_cast<__nv_bfloat16*>(out)[row * D + threadIdx.x] = __float2bfloat16_rn(v);
   else static_cast<__half*>(out)[row * D + threadIdx.x] = __float2half_rn(v);
   if (lse != nullptr && threadIdx.x == 0) lse[row] = M * kLn2 + logf(Lsum * (1.f / 448.f));
 }

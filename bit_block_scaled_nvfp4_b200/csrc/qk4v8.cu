@@ -278,7 +278,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   a.Tq = (Nq + 127) / 128; a.Tk = (Nk + 127) / 128;
   a.causal = p->causal ? 1 : 0;
   a.softmax_scale = p->softmax_scale;
-  a.out_bf16 = p->out_dtype == QK4V8_BF16 ? 1 : 0;
+  a.out_kind = static_cast<int32_t>(p->out_dtype);
   const int64_t grid = static_cast<int64_t>(a.Tq) * B * Hq;
   attn_fwd_kernel<D, kMixed><<<static_cast<unsigned>(grid), 192, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
   return launch_status();
@@ -294,7 +294,8 @@ qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
     return QK4V8_ERR_INVALID_ARG;
   if (p->q_heads % p->kv_heads) return QK4V8_ERR_INVALID_ARG;
   if (p->causal && p->n_q != p->n_k) return QK4V8_ERR_INVALID_ARG;
-  if (p->out_dtype != QK4V8_F16 && p->out_dtype != QK4V8_BF16) return QK4V8_ERR_INVALID_ARG;
+  if (p->out_dtype != QK4V8_F16 && p->out_dtype != QK4V8_BF16 && p->out_dtype != QK4V8_F32)
+    return QK4V8_ERR_INVALID_ARG;
   if (!(p->softmax_scale > 0.f)) return QK4V8_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return QK4V8_ERR_UNSUPPORTED;
   const size_t sa = p->head_dim == 128 ? 8 : 4;
@@ -334,7 +335,8 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
     return QK4V8_ERR_INVALID_ARG;
   if (p->split_tokens <= 0 || p->split_tokens % 128) return QK4V8_ERR_INVALID_ARG;
   if (p->max_context > 64 * p->max_pages) return QK4V8_ERR_INVALID_ARG;
-  if (p->out_dtype != QK4V8_F16 && p->out_dtype != QK4V8_BF16) return QK4V8_ERR_INVALID_ARG;
+  if (p->out_dtype != QK4V8_F16 && p->out_dtype != QK4V8_BF16 && p->out_dtype != QK4V8_F32)
+    return QK4V8_ERR_INVALID_ARG;
   if (!(p->softmax_scale > 0.f)) return QK4V8_ERR_INVALID_ARG;
   if (p->head_dim != 128 || p->q_heads / p->kv_heads > 16) return QK4V8_ERR_UNSUPPORTED;
   if (!aligned(p->q_codes, 16) || !aligned(p->k_pages, 16) || !aligned(p->v_pages, 16) ||
@@ -376,7 +378,7 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   decode_kernel<<<grid, 192, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   decode_merge_kernel<<<p->num_seqs * p->q_heads, 128, 0, stream>>>(
-      a.ws, n_splits, p->out_dtype == QK4V8_BF16 ? 1 : 0, p->out, p->lse);
+      a.ws, n_splits, static_cast<int32_t>(p->out_dtype), p->out, p->lse);
   return launch_status();
 }
 

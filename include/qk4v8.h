@@ -40,7 +40,8 @@ typedef enum {
   QK4V8_ERR_BOUNDS = 5        /* a device-side index check failed (e.g. page id) */
 } qk4v8_status;
 
-typedef enum { QK4V8_F16 = 0, QK4V8_BF16 = 1 } qk4v8_dtype;
+/* Element types. Inputs of the quantizers are F16 or BF16; attention outputs may also be F32. */
+typedef enum { QK4V8_F16 = 0, QK4V8_BF16 = 1, QK4V8_F32 = 2 } qk4v8_dtype;
 
 /* Library version (major * 100 + minor). */
 int qk4v8_version(void);
@@ -151,7 +152,7 @@ typedef struct {
   const void* k16;             /* fp16 [B, Hkv, Nk, D] */
   const void* v16;             /* fp16 [B, Hkv, D, Nk_pad] (quantize_mxfp8_v's v16) */
   qk4v8_dtype out_dtype;
-  void* out;                   /* [B, Hq, Nq, D] out, 16-byte aligned */
+  void* out;                   /* [B, Hq, Nq, D] out (out_dtype), 16-byte aligned */
   float* lse;                  /* optional [B, Hq, Nq] natural-log sum-exp out; or NULL */
 } qk4v8_fwd_params;
 
@@ -186,7 +187,7 @@ typedef struct {
   int32_t split_tokens;        /* keys per split, a positive multiple of 128 */
   float softmax_scale;
   qk4v8_dtype out_dtype;
-  void* out;                   /* [S, Hq, D] out */
+  void* out;                   /* [S, Hq, D] out (out_dtype) */
   float* lse;                  /* optional [S, Hq] out; or NULL */
 } qk4v8_decode_params;
 

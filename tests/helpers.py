@@ -32,6 +32,18 @@ def assert_attention_close(out_gpu, out_oracle, what=""):
     return mx, mean
 
 
+def assert_rounded_output_close(out_gpu, out_oracle, dtype, what=""):
+    """Parity of a 16-bit output: the bar above plus half a unit in the last place of the
+    output format at each element (the output's own rounding)."""
+    rms = float(np.sqrt(np.mean(out_oracle.astype(np.float64) ** 2)))
+    mant = {torch.bfloat16: 8, torch.float16: 11}[dtype]
+    half_ulp = np.ldexp(1.0, np.frexp(np.abs(out_oracle))[1] - mant - 1)
+    d = np.abs(out_gpu.astype(np.float64) - out_oracle)
+    assert np.all(np.isfinite(out_gpu)), what
+    assert np.all(d <= MAX_TOL * rms + half_ulp), f"{what}: worst excess {np.max(d - half_ulp) / rms:.3e}"
+    assert d.mean() <= MEAN_TOL * rms + half_ulp.mean(), what
+
+
 def oracle_tensor_scale(x: torch.Tensor) -> np.float32:
     """The NVFP4 tensor scale of a whole (possibly large) tensor, computed chunk-wise."""
     amax = np.float32(0)

@@ -64,7 +64,8 @@ def test_mixed_workload_selection_and_sampled_attention():
     rng = np.random.default_rng(3)
     heads = sorted(rng.choice(32, size=2, replace=False).tolist())
     _check_selection(w.q, w.k, True, 500, heads=heads)
-    out = api.qk4v8_attention(w.q.to(DEV), w.k.to(DEV), w.v.to(DEV), True, scale, fp16_frac_bp=500)
+    out = api.qk4v8_attention(w.q.to(DEV), w.k.to(DEV), w.v.to(DEV), True, scale, fp16_frac_bp=500,
+                              out_dtype=torch.float32)
     q4, k4 = api.quantize_nvfp4(w.q.to(DEV)), api.quantize_nvfp4(w.k.to(DEV))
     _, _, bitmap = api.tile_score_select(q4, k4, True, 500)
     bitmap = bitmap.cpu().numpy()
@@ -89,7 +90,8 @@ def test_mixed_small_full(frac):
     q = torch.randn(1, 4, 600, 128, generator=g).to(torch.bfloat16)
     k = (torch.randn(1, 2, 600, 128, generator=g) * 2).to(torch.bfloat16)
     v = torch.randn(1, 2, 600, 128, generator=g).to(torch.bfloat16)
-    out = api.qk4v8_attention(q.to(DEV), k.to(DEV), v.to(DEV), True, fp16_frac_bp=frac)
+    out = api.qk4v8_attention(q.to(DEV), k.to(DEV), v.to(DEV), True, fp16_frac_bp=frac,
+                              out_dtype=torch.float32)
     q4, k4 = api.quantize_nvfp4(q.to(DEV)), api.quantize_nvfp4(k.to(DEV))
     _, _, bitmap = api.tile_score_select(q4, k4, True, frac)
     bitmap = bitmap.cpu().numpy()
