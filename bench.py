@@ -366,11 +366,28 @@ def main():
         return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    from bit_block_scaled_nvfp4_b200 import api
     name = args.workload
+    try:
+        apps = subprocess.run(["nvidia-smi", "--query-compute-apps=pid,process_name,used_memory",
+                               "--format=csv,noheader"], capture_output=True, text=True, timeout=20).stdout
+        print(f"bench: compute apps on the GPUs before the run: {apps.strip() or 'none'}", file=sys.stderr)
+    except (OSError, subprocess.TimeoutExpired):
+        pass
     st = make_decode_step(name) if name == "paged_decode_s64" else make_prefill_step(name)
-    with Clocks(torch.cuda.current_device()) as clk:
-        step_ms, kern_ms = time_steps(st, args.steps, args.warmup, world)
-    e2e_ms, h2d, d2h = time_e2e(st, max(3, args.steps // 3), world)
+    # A run in which a device wait timed out (status != 0) produced no valid result: report
+    # where, take the measurement once more, and give up without a number if it repeats.
+    for attempt in range(2):
+        with Clocks(torch.cuda.current_device()) as clk:
+            step_ms, kern_ms = time_steps(st, args.steps, args.warmup, world)
+        e2e_ms, h2d, d2h = time_e2e(st, max(3, args.steps // 3), world)
+        status = api.check_status()
+        if status == 0:
+            break
+        print(f"bench: device status {status}, first timed-out wait {api.timeout_site()}"
+              f" (attempt {attempt + 1})", file=sys.stderr)
+    if status != 0:
+        raise SystemExit(3)
     step_ms = max_over_ranks(step_ms, world)
     kern_ms = max_over_ranks(kern_ms, world)
     e2e_ms = max_over_ranks(e2e_ms, world)
@@ -406,6 +423,7 @@ def main():
             "roofline": roof,
             "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": st["launches"] * args.steps,
+            "device_status": status,
             "clocks": clk.summary()}
     if rank == 0 and not args.no_cpu_baseline:
         dt, u, desc = oracle_sample(name, rows=64 if st["kind"] == "prefill" else 64, heads=1)

@@ -58,6 +58,21 @@ def check_status(stream=None) -> int:
     return _lib.load().qk4v8_check_status(s)
 
 
+def timeout_site() -> dict | None:
+    """Decode qk4v8_timeout_site(): where the first timed-out device wait sat, or None."""
+    v = _lib.load().qk4v8_timeout_site()
+    if v == 0:
+        return None
+    return {"kernel": {1: "attn_fwd", 2: "decode", 3: "selftest"}.get(v >> 56, v >> 56),
+            "role": {0: "producer", 1: "mma", 2: "softmax"}.get((v >> 48) & 0xFF, (v >> 48) & 0xFF),
+            "barrier": (v >> 40) & 0xFF, "tile": (v >> 20) & 0xFFFFF, "block": v & 0xFFFFF}
+
+
+def selftest_wait_timeout() -> None:
+    """Launch the bounded-wait self-test kernel (times out after about a second)."""
+    _lib.check(_lib.load().qk4v8_selftest_wait_timeout(_stream()), "qk4v8_selftest_wait_timeout")
+
+
 def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16: bool = False,
                    workspace: torch.Tensor | None = None) -> NVFP4Tensor:
     """NVFP4-quantize ``x`` (..., D) along its last axis (contiguous fp16/bf16 CUDA tensor)."""

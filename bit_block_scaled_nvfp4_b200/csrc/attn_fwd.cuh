@@ -133,11 +133,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tbase = *tmem_slot;
 
   // Producer and softmax warps wait warp-uniformly; the MMA issuer waits alone.
-  auto waitw = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return bounded_wait_warp(bar, parity, abort_flag);
+  // Barrier ids in timeout reports are their index in the barrier block.
+  const uint32_t role = warp == 0 ? kRoleProducer : warp == 1 ? kRoleMma : kRoleSoftmax;
+  auto site = [&](uint64_t* bar, int tile) {
+    return wait_site(kKernelFwd, role, static_cast<uint32_t>(bar - bars), tile);
   };
-  auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return bounded_wait(bar, parity, abort_flag);
+  auto waitw = [&](uint64_t* bar, uint32_t parity, int tile) -> bool {
+    return bounded_wait_warp(bar, parity, abort_flag, site(bar, tile));
+  };
+  auto wait1 = [&](uint64_t* bar, uint32_t parity, int tile) -> bool {
+    return bounded_wait(bar, parity, abort_flag, site(bar, tile));
   };
 
   if (warp == 0) {
@@ -175,7 +180,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     int n16 = 0;
     for (int j = 0; j < nt; ++j) {
       const int s = j % L::NS;
-      if (j >= L::NS && !waitw(kv_empty + s, ((j / L::NS) - 1) & 1)) break;
+      if (j >= L::NS && !waitw(kv_empty + s, ((j / L::NS) - 1) & 1, j)) break;
       unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
       // K scale factors of keys j*128 .. j*128+127
       const int64_t krow0 = static_cast<int64_t>(bhk) * a.Nk + j * 128;
@@ -223,7 +228,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             q16_loaded = true;
           }
-          if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1)) break;
+          if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1, j)) break;
           if (lane == 0) {
             mbar_arrive_expect_tx(kv16_full, 2 * L::F16_TILE);
             for (int h = 0; h < D / 64; ++h)
@@ -251,7 +256,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t idesc_pv16 = idesc_f16(128, D);
       const uint32_t sQ = smem_u32(sm + L::OFF_Q);
       const uint32_t sP = smem_u32(sm + L::OFF_P);
-      bool ok = wait1(q_full, 0);
+      bool ok = wait1(q_full, 0, -1);
       if (ok) {
         tc_fence_after();
         for (int kk = 0; kk < L::KSTEPS; ++kk)
@@ -263,7 +268,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       auto issue_pv = [&](int jj) -> bool {
         const int s = jj % L::NS, b2 = jj & 1;
         const bool f16 = kMixed && bm_row[jj];
-        if (!wait1(p_full + b2, (jj >> 1) & 1)) return false;
+        if (!wait1(p_full + b2, (jj >> 1) & 1, jj)) return false;
         tc_fence_after();
         const uint32_t tO = tbase + L::T_O;
         if (!f16) {
@@ -297,9 +302,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int j = 0; ok && j < nt; ++j) {
         const int s = j % L::NS, b2 = j & 1;
         const bool f16 = kMixed && bm_row[j];
-        if (!wait1(kv_full + s, (j / L::NS) & 1)) { ok = false; break; }
+        if (!wait1(kv_full + s, (j / L::NS) & 1, j)) { ok = false; break; }
         tc_fence_after();
-        if (j >= 2 && !wait1(s_free + b2, ((j - 2) >> 1) & 1)) { ok = false; break; }
+        if (j >= 2 && !wait1(s_free + b2, ((j - 2) >> 1) & 1, j)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tS = tbase + L::T_S + b2 * 128;
         if (!f16) {
@@ -319,10 +324,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           // PV has finished, so PV(j-1) must be issued before waiting for this tile's data.
           if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
           if (!q16_ready) {
-            if (!wait1(q16_full, 0)) { ok = false; break; }
+            if (!wait1(q16_full, 0, j)) { ok = false; break; }
             q16_ready = true;
           }
-          if (!wait1(kv16_full, n16_qk & 1)) { ok = false; break; }
+          if (!wait1(kv16_full, n16_qk & 1, j)) { ok = false; break; }
           tc_fence_after();
           ++n16_qk;
           const uint32_t sQ16 = smem_u32(sm + L::OFF_Q16), sK16 = smem_u32(sm + L::OFF_K16);
@@ -359,7 +364,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int j = 0; j < nt; ++j) {
       const int b2 = j & 1;
       const bool f16 = kMixed && bm_row[j];
-      if (!waitw(s_full + b2, (j >> 1) & 1)) { ok = false; break; }
+      if (!waitw(s_full + b2, (j >> 1) & 1, j)) { ok = false; break; }
       tc_fence_after();
       float x[128];
       {
@@ -425,7 +430,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       m_run = m_new;
       // PV(j-1) must be done: it reads the other P buffer / O, and P(j-2) shares ours.
       if (j >= 1) {
-        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1)) { ok = false; break; }
+        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
         tc_fence_after();
       }
       if (!f16) {
@@ -464,7 +469,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (lane == 0) mbar_arrive(p_full + b2);
     }
     // ---- epilogue ----
-    if (ok && nt > 0 && waitw(pv_done + ((nt - 1) & 1), ((nt - 1) >> 1) & 1)) {
+    if (ok && nt > 0 && waitw(pv_done + ((nt - 1) & 1), ((nt - 1) >> 1) & 1, nt)) {
       tc_fence_after();
       const uint32_t tO = tbase + L::T_O + lane_addr;
       const bool store = qi < a.Nq;

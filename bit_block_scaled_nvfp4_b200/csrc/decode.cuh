@@ -126,15 +126,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   // Softmax: warp-uniform waits on its own flag, which it only reads after a barrier of all
   // four softmax warps, so that the four always leave the loop together.
   volatile int* soft_flag = abort_flag + 1;
-  auto waitw = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return bounded_wait_warp(bar, parity, abort_flag);
+  const uint32_t role = warp == 0 ? kRoleProducer : warp == 1 ? kRoleMma : kRoleSoftmax;
+  auto site = [&](uint64_t* bar, int blk) {
+    return wait_site(kKernelDecode, role, static_cast<uint32_t>(bar - bars), blk);
   };
-  auto wait1 = [&](uint64_t* bar, uint32_t parity) -> bool {
-    return bounded_wait(bar, parity, abort_flag);
+  auto waitw = [&](uint64_t* bar, uint32_t parity, int blk) -> bool {
+    return bounded_wait_warp(bar, parity, abort_flag, site(bar, blk));
   };
-  auto waits = [&](uint64_t* bar, uint32_t parity) -> bool {
+  auto wait1 = [&](uint64_t* bar, uint32_t parity, int blk) -> bool {
+    return bounded_wait(bar, parity, abort_flag, site(bar, blk));
+  };
+  auto waits = [&](uint64_t* bar, uint32_t parity, int blk) -> bool {
     int ok = 0;
-    if (lane == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
+    if (lane == 0) {
+      ok = mbar_wait(bar, parity) ? 1 : 0;
+      if (!ok) record_timeout(site(bar, blk));
+    }
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
   };
   auto page_of = [&](int logical) -> int {
@@ -163,7 +170,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     for (int blk = 0; blk < nblk; ++blk) {
       const int st_i = blk % L::NS;
-      if (blk >= L::NS && !waitw(kv_empty + st_i, ((blk / L::NS) - 1) & 1)) break;
+      if (blk >= L::NS && !waitw(kv_empty + st_i, ((blk / L::NS) - 1) & 1, blk)) break;
       unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
       const int k0 = k_begin + blk * 128;
       const int lp0 = k0 / 64;
@@ -217,7 +224,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NQ);
       const uint32_t sQ = smem_u32(sm + L::OFF_Q);
       const uint32_t sP = smem_u32(sm + L::OFF_P);
-      bool ok = wait1(q_full, 0);
+      bool ok = wait1(q_full, 0, -1);
       if (ok) {
         tc_fence_after();
         tmem_cp_sf(tbase + L::T_QSF, sm + L::OFF_QSF);
@@ -226,7 +233,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       auto issue_pv = [&](int bb) -> bool {
         const int st_i = bb % L::NS, b2 = bb & 1;
-        if (!wait1(p_full + b2, (bb >> 1) & 1)) return false;
+        if (!wait1(p_full + b2, (bb >> 1) & 1, bb)) return false;
         tc_fence_after();
         unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
         const uint32_t tv = tbase + L::T_VSF + 4 * st_i;
@@ -247,9 +254,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       };
       for (int blk = 0; ok && blk < nblk; ++blk) {
         const int st_i = blk % L::NS, b2 = blk & 1;
-        if (!wait1(kv_full + st_i, (blk / L::NS) & 1)) { ok = false; break; }
+        if (!wait1(kv_full + st_i, (blk / L::NS) & 1, blk)) { ok = false; break; }
         tc_fence_after();
-        if (blk >= 2 && !wait1(s_free + b2, ((blk - 2) >> 1) & 1)) { ok = false; break; }
+        if (blk >= 2 && !wait1(s_free + b2, ((blk - 2) >> 1) & 1, blk)) { ok = false; break; }
         tc_fence_after();
         unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
         const uint32_t tk = tbase + L::T_KSF + 8 * st_i;
@@ -286,7 +293,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const int b2 = blk & 1;
       // On a timeout the body still runs (on whatever TMEM holds) so that the four warps
       // meet at both named barriers; the shared flag then ends the loop for all of them.
-      if (!waits(s_full + b2, (blk >> 1) & 1)) failed = true;
+      if (!waits(s_full + b2, (blk >> 1) & 1, blk)) failed = true;
       tc_fence_after();
       float x[16];
       tmem_ld16(tbase + L::T_S + b2 * 16 + lane_addr, reinterpret_cast<uint32_t*>(x));
@@ -337,7 +344,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
       }
       if (blk >= 1) {
-        if (!waits(pv_done + ((blk - 1) & 1), ((blk - 1) >> 1) & 1)) failed = true;
+        if (!waits(pv_done + ((blk - 1) & 1), ((blk - 1) >> 1) & 1, blk)) failed = true;
         tc_fence_after();
       }
       // P^T row q (query), column r (key), 128-byte swizzle.
@@ -370,7 +377,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + b2);
     }
-    if (!*soft_flag && waits(pv_done + ((nblk - 1) & 1), ((nblk - 1) >> 1) & 1)) {
+    if (!*soft_flag && waits(pv_done + ((nblk - 1) & 1), ((nblk - 1) >> 1) & 1, nblk)) {
       tc_fence_after();
       float o[16];
       tmem_ld16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));

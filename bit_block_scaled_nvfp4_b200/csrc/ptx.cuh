@@ -27,6 +27,22 @@ __device__ __forceinline__ unsigned long long global_ns() {
 
 __device__ __forceinline__ void flag_error(unsigned int bits) { atomicOr(&g_status, bits); }
 
+// First wait that timed out since the last read: kernel id << 56 | role << 48 |
+// barrier id << 40 | (tile & 0xFFFFF) << 20 | (blockIdx.x & 0xFFFFF). Zero when none.
+__device__ unsigned long long g_timeout_site = 0;
+enum : uint32_t { kKernelFwd = 1, kKernelDecode = 2, kKernelSelfTest = 3 };
+enum : uint32_t { kRoleProducer = 0, kRoleMma = 1, kRoleSoftmax = 2 };
+__device__ __forceinline__ uint64_t wait_site(uint32_t kernel, uint32_t role, uint32_t bar_id,
+                                              int tile) {
+  return (static_cast<uint64_t>(kernel) << 56) | (static_cast<uint64_t>(role) << 48) |
+         (static_cast<uint64_t>(bar_id & 0xFF) << 40) |
+         (static_cast<uint64_t>(static_cast<uint32_t>(tile) & 0xFFFFFu) << 20) |
+         static_cast<uint64_t>(blockIdx.x & 0xFFFFFu);
+}
+__device__ __forceinline__ void record_timeout(uint64_t site) {
+  atomicCAS(&g_timeout_site, 0ull, static_cast<unsigned long long>(site));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -71,9 +87,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait that gives up at once when *flag is set, and sets *flag when it times out itself.
-__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* flag) {
+// `site` (wait_site()) is recorded when this wait is the first to time out.
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* flag,
+                                             uint64_t site) {
   if (*flag) return false;
   if (!mbar_wait(bar, parity)) {
+    record_timeout(site);
     *flag = 1;
     return false;
   }
@@ -81,9 +100,9 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
 }
 // The same, taken by lane 0 for the whole (converged) warp, so that every lane agrees.
 __device__ __forceinline__ bool bounded_wait_warp(uint64_t* bar, uint32_t parity,
-                                                  volatile int* flag) {
+                                                  volatile int* flag, uint64_t site) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, flag) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, flag, site) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -291,6 +310,21 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Self-test of the bounded-wait path: one warp waits on a barrier that nothing arrives at.
+// The wait gives up after its time limit, records its site and the timeout status, and the
+// kernel returns normally.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ volatile int flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    flag = 0;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  bounded_wait_warp(&bar, 0, &flag, wait_site(kKernelSelfTest, kRoleProducer, 0, 0));
 }
 
 }  // namespace qk4v8

@@ -96,6 +96,21 @@ qk4v8_status qk4v8_check_status(cudaStream_t stream) {
   return QK4V8_OK;
 }
 
+uint64_t qk4v8_timeout_site(void) {
+  unsigned long long site = 0;
+  if (cudaMemcpyFromSymbol(&site, g_timeout_site, sizeof(site)) != cudaSuccess) return 0;
+  if (site != 0) {
+    const unsigned long long zero = 0;
+    cudaMemcpyToSymbol(g_timeout_site, &zero, sizeof(zero));
+  }
+  return site;
+}
+
+qk4v8_status qk4v8_selftest_wait_timeout(cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>();
+  return launch_status();
+}
+
 // ------------------------------------------------------------------------------------------
 size_t quantize_nvfp4_workspace_size(void) { return 256; }
 

@@ -61,6 +61,22 @@ const char* qk4v8_status_string(qk4v8_status status);
 qk4v8_status qk4v8_check_status(cudaStream_t stream);
 
 /*
+ * Where the first device wait that timed out since the last call sat, then cleared (0 when
+ * none): kernel << 56 (1 prefill, 2 decode) | role << 48 (0 producer warp, 1 MMA issuer,
+ * 2 softmax warps) | barrier index << 40 | (key tile & 0xFFFFF) << 20 | (block & 0xFFFFF).
+ * Synchronous; call it after qk4v8_check_status() reported QK4V8_ERR_TIMEOUT.
+ */
+uint64_t qk4v8_timeout_site(void);
+
+/*
+ * Failure-path self-test: launches one warp that waits on a barrier nothing arrives at. Its
+ * bounded wait gives up after about a second and the kernel returns; the following
+ * qk4v8_check_status() reports QK4V8_ERR_TIMEOUT and qk4v8_timeout_site() names kernel 3.
+ * Nothing faults or hangs; the context stays usable.
+ */
+qk4v8_status qk4v8_selftest_wait_timeout(cudaStream_t stream);
+
+/*
  * quantize_nvfp4 — NVFP4 quantization of Q or K (tqpw.cn article §2.2: E2M1 elements, E4M3
  * scale per 16 elements, FP32 tensor scale). Per call:
  *   s_t = fl32(amax / 2688) over all of x (2688 = 6 * 448; s_t = 1 when amax is 0), or
