@@ -21,6 +21,8 @@ QK4V8_ERR_BOUNDS = 5
 QK4V8_F16 = 0
 QK4V8_BF16 = 1
 QK4V8_F32 = 2
+#: Size of the library's fixed scratch buffer behind attn_qk4v8_decode_paged_noalloc.
+NOALLOC_DECODE_SCRATCH_BYTES = 16 * 1024 * 1024
 
 vp = C.c_void_p
 i32 = C.c_int32
@@ -70,6 +72,7 @@ SIGNATURES = {
     "attn_qk4v8_fwd": (i32, [C.POINTER(FwdParams), vp]),
     "attn_qk4v8_decode_workspace_size": (sz, [C.POINTER(DecodeParams)]),
     "attn_qk4v8_decode_paged": (i32, [C.POINTER(DecodeParams), vp, sz, vp]),
+    "attn_qk4v8_decode_paged_noalloc": (i32, [C.POINTER(DecodeParams), vp]),
 }
 
 _LIB = None

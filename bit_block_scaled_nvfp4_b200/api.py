@@ -220,6 +220,25 @@ def attn_qk4v8_decode_paged(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Te
     return (out, lse) if want_lse else out
 
 
+def attn_qk4v8_decode_paged_noalloc(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
+                                    context_lens: torch.Tensor, max_context: int,
+                                    split_tokens: int, softmax_scale: float | None = None,
+                                    out_dtype=torch.bfloat16, want_lse: bool = False):
+    """The decode step through the library's allocation-free entry point: the library keeps
+    the split partials in its own fixed 16 MiB device buffer instead of a caller workspace,
+    for callers that cannot provide device memory. Only the output (and lse) are allocated
+    here, as for every other entry point of this binding."""
+    lib = _lib.load()
+    S, Hq, dh = q.codes.shape
+    out = torch.empty(S, Hq, dh * 2, dtype=out_dtype, device=q.codes.device)
+    lse = torch.empty(S, Hq, dtype=torch.float32, device=q.codes.device) if want_lse else None
+    p = decode_params(q, cache, page_table, context_lens, max_context, split_tokens, out,
+                      softmax_scale, lse)
+    st = lib.attn_qk4v8_decode_paged_noalloc(C.byref(p), _stream())
+    _lib.check(st, "attn_qk4v8_decode_paged_noalloc")
+    return (out, lse) if want_lse else out
+
+
 def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool,
                     softmax_scale: float | None = None, fp16_frac_bp: int = 0,
                     out_dtype=None, want_lse: bool = False):

@@ -3,6 +3,7 @@
 // decode.cuh); this file only checks, describes memory and launches.
 #include <cudaTypedefs.h>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/qk4v8.h"
 #include "ptx.cuh"
@@ -398,3 +399,38 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free decode: the split partials live in one fixed file-scope device buffer.
+// Host code must not use the array's name as a pointer (on the host it is only a stand-in);
+// its device address is looked up once per device with the device current.
+// ------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_decode_scratch[QK4V8_NOALLOC_DECODE_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
+
+extern "C" qk4v8_status attn_qk4v8_decode_paged_noalloc(const qk4v8_decode_params* p,
+                                                        cudaStream_t stream) {
+  if (p == nullptr) return QK4V8_ERR_INVALID_ARG;
+  const size_t need = attn_qk4v8_decode_workspace_size(p);
+  if (need == 0) return QK4V8_ERR_INVALID_ARG;
+  if (need > QK4V8_NOALLOC_DECODE_SCRATCH_BYTES) return QK4V8_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QK4V8_ERR_CUDA;
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_noalloc_decode_scratch) != cudaSuccess || addr == nullptr)
+        return QK4V8_ERR_CUDA;
+      g_noalloc_ptr[dev] = addr;
+    }
+    ptr = g_noalloc_ptr[dev];
+  }
+  return attn_qk4v8_decode_paged(p, ptr, QK4V8_NOALLOC_DECODE_SCRATCH_BYTES, stream);
+}

@@ -211,6 +211,26 @@ size_t attn_qk4v8_decode_workspace_size(const qk4v8_decode_params* params);
 qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* params, void* workspace,
                                      size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * attn_qk4v8_decode_paged_noalloc — the same decode step for callers that cannot hand the
+ * library device memory for its scratch: an engine that fixed every buffer at start-up and
+ * allows no allocation inside its step loop, a plugin whose host framework owns all device
+ * memory and passes no workspace, or a host program that links only this library and has no
+ * allocator of its own. (The pages have no counterpart; this is an integration variant.)
+ * The split partials go to one file-scope device buffer of
+ * QK4V8_NOALLOC_DECODE_SCRATCH_BYTES (16 MiB), present on every GPU that loads the library
+ * until the process exits; attn_qk4v8_decode_workspace_size(params) must not exceed it,
+ * otherwise QK4V8_ERR_UNSUPPORTED is returned and nothing is launched. Nothing is allocated
+ * or freed. The first call on a device looks up that buffer's device address with the device
+ * current (set-up, once per device); make that first call before any stream capture. All
+ * calls share the one buffer and it keeps the last call's contents (every entry a call reads
+ * it writes first, so nothing needs clearing); calls that overlap on the GPU (other streams,
+ * other host threads) race on it and must be serialised by the caller.
+ */
+#define QK4V8_NOALLOC_DECODE_SCRATCH_BYTES (16u * 1024u * 1024u)
+qk4v8_status attn_qk4v8_decode_paged_noalloc(const qk4v8_decode_params* params,
+                                             cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
