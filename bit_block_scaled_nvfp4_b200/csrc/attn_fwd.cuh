@@ -9,13 +9,19 @@
 // "方法" step 3): a tile marked in the selection bitmap runs QK^T and PV with kind::f16 on
 // FP16 copies of Q, K, V, with P = fp16(448 exp(s - m)), into the same (m, l, O).
 //
+// l comes from the tensor core: every V tile in shared memory carries 16 extra rows of 1.0
+// after its D channel rows, so the PV MMA (N = D + 16) accumulates sum_j P_j into O column D,
+// with the same rescaling as O.
+//
 // One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
 //              tcgen05 scale layout with plain loads, FP16 tiles when selected
 //   warp 1     TMEM owner and MMA issuer (one thread)
-//   warps 2-5  softmax: each thread owns one query row (its TMEM lane); also rescales O
-//              and writes the output
-// TMEM (512 columns): S double buffer [0,256), O [256, 256+D), scale factors from 384.
+//   warps 2-9  softmax: warps w and w+4 share TMEM lane quadrant w % 4 (32 query rows) and
+//              split each row's 128 keys in halves of 64; they exchange the row max through
+//              shared memory, rescale their halves of O and write the output
+// TMEM (512 columns): S double buffer [0,256), O (D + 16 columns) from 256, scale factors
+// from 400.
 #pragma once
 #include "ptx.cuh"
 
@@ -41,15 +47,16 @@ struct FwdArgs {
 
 template <int D, bool kMixed>
 struct FwdLayout {
-  static constexpr int NS = 3;
+  static constexpr int NS = kMixed ? 2 : 3;   // the FP16 operand stage needs the room
   static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
+  static constexpr int NV = D + 16;                     // PV MMA N: D channels + ones rows
   static constexpr int Q_BYTES = 128 * D / 2;
   static constexpr int K_BYTES = 128 * D / 2;
-  static constexpr int V_BYTES = D * 128;
-  static constexpr int SF_CHUNK = 512;
+  static constexpr int V_TMA_BYTES = D * 128;
+  static constexpr int V_BYTES = NV * 128;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_QSF = OFF_Q + Q_BYTES;                         // KSTEPS chunks
-  static constexpr int OFF_PSF = OFF_QSF + 1024;
+  static constexpr int OFF_PSF = OFF_QSF + 1024;                          // all 1.0 (E8M0 127)
   static constexpr int OFF_STAGE = OFF_PSF + 1024;
   static constexpr int ST_K = 0;
   static constexpr int ST_V = K_BYTES;
@@ -57,23 +64,26 @@ struct FwdLayout {
   static constexpr int ST_VSF = ST_KSF + 1024;
   static constexpr int STAGE_BYTES = ST_VSF + 1024;
   static constexpr int OFF_P = OFF_STAGE + NS * STAGE_BYTES;               // 2 x 16 KB
-  static constexpr int OFF_Q16 = OFF_P + 2 * 16384;
+  static constexpr int OFF_RED = OFF_P + 2 * 16384;                        // [2][2][128] floats
+  static constexpr int OFF_Q16 = OFF_RED + 2048;
   static constexpr int F16_TILE = 128 * D * 2;
+  static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
-  static constexpr int OFF_BAR = OFF_V16 + (kMixed ? F16_TILE : 0);
+  static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
   static constexpr int N_BARS = 1 + 2 * NS + 2 * 4 + 3 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   // TMEM columns
-  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 384, T_PSF = 392, T_KSF = 400,
-                            T_VSF = 424;
+  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_PSF = 408, T_KSF = 412,
+                            T_VSF = 436;
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
+  static constexpr int THREADS = 320;
 };
 
 template <int D, bool kMixed>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q16,
                 const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
@@ -111,17 +121,29 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(q_full, 1);
     for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full + i, 1); mbar_init(s_free + i, 4);
-      mbar_init(p_full + i, 4); mbar_init(pv_done + i, 1);
+      mbar_init(s_full + i, 1); mbar_init(s_free + i, 8);
+      mbar_init(p_full + i, 8); mbar_init(pv_done + i, 1);
     }
     mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1); mbar_init(q16_full, 1);
     mbar_init(mma_final, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // P scale factors (E8M0 127 = 1.0) for the PV MMA's A operand.
+  // Constants in shared memory: the P scale factors (E8M0 127 = 1.0, also the second V scale
+  // chunk) and the 16 rows of 1.0 after each V tile (E4M3 0x38; FP16 0x3C00 in the FP16 V).
+  // Every byte of a ones row is equal, so the 128-byte swizzle leaves them unchanged.
   for (int i = threadIdx.x; i < 128; i += blockDim.x)
     reinterpret_cast<uint32_t*>(sm + L::OFF_PSF)[i] = 0x7F7F7F7Fu;
+  for (int s = 0; s < L::NS; ++s)
+    for (int i = threadIdx.x; i < 16 * 128 / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(sm + L::OFF_STAGE + s * L::STAGE_BYTES + L::ST_V + L::V_TMA_BYTES)[i] =
+          make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+  if constexpr (kMixed) {
+    for (int h = 0; h < 2; ++h)
+      for (int i = threadIdx.x; i < 16 * 128 / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(sm + L::OFF_V16 + h * L::V16_ATOM + D * 128)[i] =
+            make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+  }
   fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -132,7 +154,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  // Producer and softmax warps wait warp-uniformly; the MMA issuer waits alone.
   // Barrier ids in timeout reports are their index in the barrier block.
   const uint32_t role = warp == 0 ? kRoleProducer : warp == 1 ? kRoleMma : kRoleSoftmax;
   auto site = [&](uint64_t* bar, int tile) {
@@ -201,7 +222,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int kk = 0; kk < L::KSTEPS; ++kk)
         *reinterpret_cast<uint4*>(st + L::ST_KSF + kk * 512 + lane * 16) =
             make_uint4(w[0][kk], w[1][kk], w[2][kk], w[3][kk]);
-      // V scale factors: channel row c, 4 E8M0 codes (32 tokens each) of this key tile
+      // V scale factors: channel row c, 4 E8M0 codes (32 tokens each) of this key tile; rows
+      // from D on (the ones rows, and padding) get 1.0.
       uint32_t vw[4];
 #pragma unroll
       for (int r1 = 0; r1 < 4; ++r1) {
@@ -214,7 +236,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_BYTES);
+        mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_TMA_BYTES);
         tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, bhk);
         tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, bhk * D);
       }
@@ -230,11 +252,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1, j)) break;
           if (lane == 0) {
-            mbar_arrive_expect_tx(kv16_full, 2 * L::F16_TILE);
+            mbar_arrive_expect_tx(kv16_full, L::F16_TILE + 2 * D * 128);
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(sm + L::OFF_K16 + h * 16384, &tm_k16, kv16_full, h * 64, j * 128, bhk);
             for (int h = 0; h < 2; ++h)
-              tma_load_2d(sm + L::OFF_V16 + h * (D * 128), &tm_v16, kv16_full, j * 128 + h * 64, bhk * D);
+              tma_load_2d(sm + L::OFF_V16 + h * L::V16_ATOM, &tm_v16, kv16_full, j * 128 + h * 64, bhk * D);
           }
           ++n16;
         }
@@ -251,9 +273,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ================================ MMA issuer ================================
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, 128);
-      const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, D);
+      const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NV);
       const uint32_t idesc_qk16 = idesc_f16(128, 128);
-      const uint32_t idesc_pv16 = idesc_f16(128, D);
+      const uint32_t idesc_pv16 = idesc_f16(128, L::NV);
       const uint32_t sQ = smem_u32(sm + L::OFF_Q);
       const uint32_t sP = smem_u32(sm + L::OFF_P);
       bool ok = wait1(q_full, 0, -1);
@@ -262,8 +284,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < L::KSTEPS; ++kk)
           tmem_cp_sf(tbase + L::T_QSF + 4 * kk, sm + L::OFF_QSF + kk * 512);
         tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+        for (int s = 0; s < L::NS; ++s)            // second V scale chunk (rows 128..): 1.0
+          tmem_cp_sf(tbase + L::T_VSF + 8 * s + 4, sm + L::OFF_PSF);
       }
-      int n16_qk = 0, n16_pv = 0;
+      int n16_qk = 0;
       bool q16_ready = false;
       auto issue_pv = [&](int jj) -> bool {
         const int s = jj % L::NS, b2 = jj & 1;
@@ -273,7 +297,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t tO = tbase + L::T_O;
         if (!f16) {
           unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-          const uint32_t tv = tbase + L::T_VSF + 4 * s;
+          const uint32_t tv = tbase + L::T_VSF + 8 * s;
           tmem_cp_sf(tv, st + L::ST_VSF);
           const uint32_t sV = smem_u32(st + L::ST_V);
 #pragma unroll
@@ -289,11 +313,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
-            const uint64_t db = make_sdesc(sV16 + (kk >> 2) * (D * 128) + (kk & 3) * 32, 16, 1024, kSw128);
+            const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
             mma_f16(tO, da, db, idesc_pv16, (jj > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(kv16_empty);
-          ++n16_pv;
         }
         mma_commit(pv_done + b2);
         mma_commit(kv_empty + s);
@@ -340,7 +363,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       if (ok && nt > 0) issue_pv(nt - 1);
-      (void)n16_pv;
       // Everything this thread issued has completed before TMEM is released.
       mma_commit(mma_final);
       mbar_wait(mma_final, 0);
@@ -348,134 +370,161 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncwarp();
   } else {
     // ================================ softmax ================================
-    const int wq = warp & 3;
+    const int wq = warp & 3;                 // TMEM lane quadrant
+    const int half = (warp - 2) >> 2;        // which 64 keys of the tile (and half of O)
     const int row = wq * 32 + lane;
     const int qi = qt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+    float* red = reinterpret_cast<float*>(sm + L::OFF_RED);       // [2 tiles][2 halves][128]
     // Scores stay in the FP4 MMA's raw units (S = sum codes*scales); the running max m is
     // kept in those units, so (s - m) is exact for the keys near the max, and
     // p = 2^((s - m) * C) with C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true
     // dot products and are brought into raw units by 1 / (s_tQ s_tK).
     const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
     const float R16 = 1.f / ((*a.q_ts) * (*a.k_ts));
-    float m_run = -INFINITY, l_run = 0.f;
+    const uint64_t C2 = f2_pack(C, C);
+    const uint64_t P448 = f2_pack(448.f, 448.f);
+    float m_run = -INFINITY;
     unsigned char* sP = sm + L::OFF_P;
+    // A warp whose wait fails keeps iterating without doing work (ok == false), so that the
+    // two partner warps of a quadrant always meet at every named barrier.
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int b2 = j & 1;
       const bool f16 = kMixed && bm_row[j];
-      if (!waitw(s_full + b2, (j >> 1) & 1, j)) { ok = false; break; }
-      tc_fence_after();
-      float x[128];
-      {
+      float x[64];
+      float mt = -INFINITY;
+      if (ok && !waitw(s_full + b2, (j >> 1) & 1, j)) ok = false;
+      if (ok) {
+        tc_fence_after();
         uint32_t* xr = reinterpret_cast<uint32_t*>(x);
-        const uint32_t tS = tbase + L::T_S + b2 * 128 + lane_addr;
+        const uint32_t tS = tbase + L::T_S + b2 * 128 + half * 64 + lane_addr;
         tmem_ld32(tS + 0, xr + 0);
         tmem_ld32(tS + 32, xr + 32);
-        tmem_ld32(tS + 64, xr + 64);
-        tmem_ld32(tS + 96, xr + 96);
         tmem_wait_ld();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + b2);
-      if (f16) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + b2);
+        if (f16) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] *= R16;
-      }
-      const int kbase = j * 128;
-      const bool need_mask = (a.causal && kbase + 127 > qi) || (kbase + 128 > a.Nk);
-      float mt = -INFINITY;
-      if (need_mask) {
-        const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          x[c] = (c <= lim) ? x[c] : -INFINITY;
-          mt = fmaxf(mt, x[c]);
+          for (int c = 0; c < 64; ++c) x[c] *= R16;
         }
-      } else {
+        const int kbase = j * 128 + half * 64;
+        const bool need_mask = (a.causal && kbase + 63 > qi) || (kbase + 64 > a.Nk);
+        if (need_mask) {
+          const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mt = fmaxf(mt, x[c]);
+          for (int c = 0; c < 64; ++c) x[c] = (c <= lim) ? x[c] : -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) mt = fmax3(mt, x[c], x[c + 1]);
       }
+      // Row max over both halves: the partner warp holds the other 64 keys of the row. The
+      // exchange slots alternate between tiles, so a fast warp's next write cannot overwrite
+      // a value its partner has not read yet (both pass the barrier of every tile).
+      red[(b2 * 2 + half) * 128 + row] = mt;
+      named_bar_sync(1 + wq, 64);
+      mt = fmaxf(mt, red[(b2 * 2 + (half ^ 1)) * 128 + row]);
+      if (!ok) continue;
       const float m_new = fmaxf(m_run, mt);
       const bool dead = (m_new == -INFINITY);
       const float mref = dead ? 0.f : m_new;
       const float alpha = dead ? 1.f : ex2_approx((m_run - m_new) * C);
-      float lsum = 0.f;
-      uint32_t pw[64];             // e4m3: 32 words used; fp16: 64 words
+      m_run = m_new;
+      const uint64_t M2 = f2_pack(mref, mref);
+      uint32_t pw[32];             // e4m3: 16 words used; fp16: 32 words
       if (!f16) {
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
+        for (int c = 0; c < 64; c += 4) {
+          float t[4];
+          f2_unpack(f2_mul(f2_sub(f2_pack(x[c], x[c + 1]), M2), C2), t[0], t[1]);
+          f2_unpack(f2_mul(f2_sub(f2_pack(x[c + 2], x[c + 3]), M2), C2), t[2], t[3]);
           float p[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) p[i] = ex2_approx((x[c + i] - mref) * C) * 448.f;
-          const uint32_t lo = cvt_e4m3x2(p[0], p[1]);
-          const uint32_t hi = cvt_e4m3x2(p[2], p[3]);
-          const float2 f0 = __half22float2(e4m3x2_to_half2(lo));
-          const float2 f1 = __half22float2(e4m3x2_to_half2(hi));
-          lsum += (f0.x + f0.y) + (f1.x + f1.y);
-          pw[c >> 2] = lo | (hi << 16);
+          f2_unpack(f2_mul(f2_pack(ex2_approx(t[0]), ex2_approx(t[1])), P448), p[0], p[1]);
+          f2_unpack(f2_mul(f2_pack(ex2_approx(t[2]), ex2_approx(t[3])), P448), p[2], p[3]);
+          pw[c >> 2] = cvt_e4m3x2(p[0], p[1]) | (cvt_e4m3x2(p[2], p[3]) << 16);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const __half2 h = __floats2half2_rn(ex2_approx((x[c] - mref) * C) * 448.f,
-                                              ex2_approx((x[c + 1] - mref) * C) * 448.f);
-          const float2 f = __half22float2(h);
-          lsum += f.x + f.y;
+        for (int c = 0; c < 64; c += 2) {
+          float t0, t1, p0, p1;
+          f2_unpack(f2_mul(f2_sub(f2_pack(x[c], x[c + 1]), M2), C2), t0, t1);
+          f2_unpack(f2_mul(f2_pack(ex2_approx(t0), ex2_approx(t1)), P448), p0, p1);
+          const __half2 h = __floats2half2_rn(p0, p1);
           pw[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
         }
       }
-      l_run = l_run * alpha + lsum;
-      m_run = m_new;
-      // PV(j-1) must be done: it reads the other P buffer / O, and P(j-2) shares ours.
-      if (j >= 1) {
-        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
-        tc_fence_after();
-      }
+      // PV(j-2) read this P buffer and must be done before it is rewritten; an FP16 tile
+      // writes both buffers, so then PV(j-1) too.
+      if (j >= 2 && !waitw(pv_done + b2, ((j - 2) >> 1) & 1, j)) { ok = false; continue; }
+      if (f16 && j >= 1 && !waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; continue; }
       if (!f16) {
         unsigned char* prow = sP + b2 * 16384 + row * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int ch = half * 4 + c;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
+              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        }
+      } else {
+        unsigned char* prow = sP + half * 16384 + row * 128;     // atom = this half's 64 keys
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
               make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-      } else {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          unsigned char* prow = sP + h * 16384 + row * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-                make_uint4(pw[32 * h + 4 * c], pw[32 * h + 4 * c + 1], pw[32 * h + 4 * c + 2],
-                           pw[32 * h + 4 * c + 3]);
-        }
       }
       fence_proxy_async_smem();
-      if (j >= 1 && !__all_sync(0xffffffffu, alpha == 1.f)) {
-        const uint32_t tO = tbase + L::T_O + lane_addr;
+      // PV(j-1) must be done before O is rescaled for this tile.
+      if (j >= 1) {
+        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; continue; }
+        tc_fence_after();
+        if (!__all_sync(0xffffffffu, alpha == 1.f)) {
+          // this warp's columns of O: half 0 -> [0, D/2) and [D, D+16) (l); half 1 -> [D/2, D)
+          const uint32_t tO = tbase + L::T_O + lane_addr;
+          const uint64_t A2 = f2_pack(alpha, alpha);
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + c, o);
-          tmem_wait_ld();
+          for (int cc = 0; cc < D / 2; cc += 32) {
+            const uint32_t col = half * (D / 2) + cc;
+            uint32_t o[32];
+            tmem_ld32(tO + col, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(tO + c, o);
+            for (int k = 0; k < 32; k += 2) {
+              float u0, u1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), A2), u0, u1);
+              o[k] = __float_as_uint(u0);
+              o[k + 1] = __float_as_uint(u1);
+            }
+            tmem_st32(tO + col, o);
+          }
+          if (half == 0) {
+            uint32_t o[16];
+            tmem_ld16(tO + D, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(tO + D, o);
+          }
+          tmem_wait_st();
         }
-        tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + b2);
     }
-    // ---- epilogue ----
+    // ---- epilogue: O / l for this warp's half of the columns ----
     if (ok && nt > 0 && waitw(pv_done + ((nt - 1) & 1), ((nt - 1) >> 1) & 1, nt)) {
       tc_fence_after();
       const uint32_t tO = tbase + L::T_O + lane_addr;
+      uint32_t lr[16];
+      tmem_ld16(tO + D, lr);
+      tmem_wait_ld();
+      const float l_run = __uint_as_float(lr[0]);
       const bool store = qi < a.Nq;
       const int64_t orow = static_cast<int64_t>(bhq) * a.Nq + qi;
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int cc = 0; cc < D / 2; cc += 32) {
+        const int c = half * (D / 2) + cc;
         uint32_t o[32];
         tmem_ld32(tO + c, o);
         tmem_wait_ld();
@@ -508,7 +557,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
         }
       }
-      if (store && a.lse != nullptr) a.lse[orow] = m_run * C * kLn2 + logf(l_run * (1.f / 448.f));
+      if (store && half == 0 && a.lse != nullptr)
+        a.lse[orow] = m_run * C * kLn2 + logf(l_run * (1.f / 448.f));
     }
   }
   tc_fence_before();

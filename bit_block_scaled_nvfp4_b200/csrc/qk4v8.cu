@@ -296,7 +296,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   a.softmax_scale = p->softmax_scale;
   a.out_kind = static_cast<int32_t>(p->out_dtype);
   const int64_t grid = static_cast<int64_t>(a.Tq) * B * Hq;
-  attn_fwd_kernel<D, kMixed><<<static_cast<unsigned>(grid), 192, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
+  attn_fwd_kernel<D, kMixed><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
   return launch_status();
 }
 
