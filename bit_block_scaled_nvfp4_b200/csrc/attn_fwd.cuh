@@ -13,6 +13,11 @@
 // after its D channel rows, so the PV MMA (N = D + 16) accumulates sum_j P_j into O column D,
 // with the same rescaling as O.
 //
+// Two O accumulators: even key tiles accumulate into O_0 and odd ones into O_1, each kept
+// relative to the running max at its last update. Tile j's rescale then touches O_{j&1}, which
+// only needs PV(j-2) finished, so it overlaps PV(j-1) on the tensor core instead of stalling
+// it; the epilogue merges the two exactly (the same result as one accumulator).
+//
 // One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
 //              tcgen05 scale layout with plain loads, FP16 tiles when selected
@@ -20,8 +25,8 @@
 //   warps 2-9  softmax: warps w and w+4 share TMEM lane quadrant w % 4 (32 query rows) and
 //              split each row's 128 keys in halves of 64; they exchange the row max through
 //              shared memory, rescale their halves of O and write the output
-// TMEM (512 columns): S double buffer [0,256), O (D + 16 columns) from 256, scale factors
-// from 400.
+// TMEM (512 columns): S [0,128), O_0 and O_1 (D + 16 columns each) from 128, scale factors
+// from 416.
 #pragma once
 #include "ptx.cuh"
 
@@ -71,12 +76,12 @@ struct FwdLayout {
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int N_BARS = 1 + 2 * NS + 2 * 4 + 3 + 1;
+  static constexpr int N_BARS = 1 + 2 * NS + 2 + 4 + 3 + 1;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   // TMEM columns
-  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_PSF = 408, T_KSF = 412,
-                            T_VSF = 436;
+  static constexpr uint32_t T_S = 0, T_O = 128, T_OSTRIDE = 144, T_QSF = 416, T_PSF = 424,
+                            T_KSF = 428, T_VSF = 452;
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
   static constexpr int THREADS = 320;
@@ -97,13 +102,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = bars + 1 + L::NS;
   uint64_t* s_full = bars + 1 + 2 * L::NS;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_full + 4;
-  uint64_t* pv_done = s_full + 6;
-  uint64_t* kv16_full = s_full + 8;
-  uint64_t* kv16_empty = s_full + 9;
-  uint64_t* q16_full = s_full + 10;
-  uint64_t* mma_final = s_full + 11;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;           // [2], by tile parity
+  uint64_t* pv_done = s_full + 4;          // [2], by tile parity
+  uint64_t* kv16_full = s_full + 6;
+  uint64_t* kv16_empty = s_full + 7;
+  uint64_t* q16_full = s_full + 8;
+  uint64_t* mma_final = s_full + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -118,12 +123,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(bhq) * a.Tq + qt) * a.Tk : nullptr;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full + i, 1); mbar_init(s_free + i, 8);
-      mbar_init(p_full + i, 8); mbar_init(pv_done + i, 1);
-    }
+    // full barriers: the TMA's expect-tx arrival plus one cp.async arrival per producer lane
+    mbar_init(q_full, 33);
+    for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 8);
+    for (int i = 0; i < 2; ++i) { mbar_init(p_full + i, 8); mbar_init(pv_done + i, 1); }
     mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1); mbar_init(q16_full, 1);
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -138,6 +143,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int i = threadIdx.x; i < 16 * 128 / 16; i += blockDim.x)
       reinterpret_cast<uint4*>(sm + L::OFF_STAGE + s * L::STAGE_BYTES + L::ST_V + L::V_TMA_BYTES)[i] =
           make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+  if constexpr (D < 128) {
+    for (int s = 0; s < L::NS; ++s)
+      for (int i = threadIdx.x; i < 128; i += blockDim.x)
+        if (((i >> 2) & 31) + 32 * (i & 3) >= D)       // word i: row (i/4)%32 + 32 (i%4)
+          reinterpret_cast<uint32_t*>(sm + L::OFF_STAGE + s * L::STAGE_BYTES + L::ST_VSF)[i] = 0x7F7F7F7Fu;
+  }
   if constexpr (kMixed) {
     for (int h = 0; h < 2; ++h)
       for (int i = threadIdx.x; i < 16 * 128 / 16; i += blockDim.x)
@@ -169,28 +180,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 0) {
     // ================================ producer ================================
     if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); }
-    // Q scale factors: row r = r0 + 32 r1 -> chunk byte r0*16 + r1*4 + k (k = 0..3 within a
-    // 64-element MMA step); Q codes by TMA.
+    // Scale factors go straight from global memory into the tcgen05 scale layout with 4-byte
+    // asynchronous copies (row r = r0 + 32 r1 of a 128-row chunk -> byte r0*16 + r1*4; one
+    // 4-byte word holds the 4 scales of one 64-element MMA step), completing on the same
+    // barrier as the TMA of the codes, so this warp never waits on their latency.
     {
       const int64_t row0 = static_cast<int64_t>(bhq) * a.Nq + qt * 128;
-      uint32_t w[4][L::KSTEPS];
 #pragma unroll
       for (int r1 = 0; r1 < 4; ++r1) {
         const int r = r1 * 32 + lane;
         const bool ok = qt * 128 + r < a.Nq;
-        if constexpr (L::KSTEPS == 2) {
-          uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(a.q_scales + (row0 + r) * (D / 16)))
-                       : make_uint2(0, 0);
-          w[r1][0] = v.x; w[r1][1] = v.y;
-        } else {
-          w[r1][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(a.q_scales + (row0 + r) * (D / 16))) : 0u;
-        }
-      }
+        const uint8_t* src = a.q_scales + (ok ? (row0 + r) * (D / 16) : 0);
 #pragma unroll
-      for (int kk = 0; kk < L::KSTEPS; ++kk)
-        *reinterpret_cast<uint4*>(sm + L::OFF_QSF + kk * 512 + lane * 16) =
-            make_uint4(w[0][kk], w[1][kk], w[2][kk], w[3][kk]);
-      fence_proxy_async_smem();
+        for (int kk = 0; kk < L::KSTEPS; ++kk)
+          cp_async4(sm + L::OFF_QSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, ok);
+      }
+      cp_async_arrive_noinc(q_full);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(q_full, L::Q_BYTES);
@@ -203,37 +208,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int s = j % L::NS;
       if (j >= L::NS && !waitw(kv_empty + s, ((j / L::NS) - 1) & 1, j)) break;
       unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-      // K scale factors of keys j*128 .. j*128+127
+      // K scale factors of keys j*128 .. j*128+127; V scale factors of this key tile (channel
+      // row c, 4 E8M0 codes of 32 tokens each). Rows past Nk read as zero; V rows from D on
+      // (the ones rows) hold 1.0 set once at start.
       const int64_t krow0 = static_cast<int64_t>(bhk) * a.Nk + j * 128;
-      uint32_t w[4][L::KSTEPS];
 #pragma unroll
       for (int r1 = 0; r1 < 4; ++r1) {
         const int r = r1 * 32 + lane;
         const bool ok = j * 128 + r < a.Nk;
-        if constexpr (L::KSTEPS == 2) {
-          uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(a.k_scales + (krow0 + r) * (D / 16)))
-                       : make_uint2(0, 0);
-          w[r1][0] = v.x; w[r1][1] = v.y;
-        } else {
-          w[r1][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(a.k_scales + (krow0 + r) * (D / 16))) : 0u;
-        }
-      }
+        const uint8_t* src = a.k_scales + (ok ? (krow0 + r) * (D / 16) : 0);
 #pragma unroll
-      for (int kk = 0; kk < L::KSTEPS; ++kk)
-        *reinterpret_cast<uint4*>(st + L::ST_KSF + kk * 512 + lane * 16) =
-            make_uint4(w[0][kk], w[1][kk], w[2][kk], w[3][kk]);
-      // V scale factors: channel row c, 4 E8M0 codes (32 tokens each) of this key tile; rows
-      // from D on (the ones rows, and padding) get 1.0.
-      uint32_t vw[4];
-#pragma unroll
-      for (int r1 = 0; r1 < 4; ++r1) {
-        const int c = r1 * 32 + lane;
-        vw[r1] = c < D ? __ldg(reinterpret_cast<const uint32_t*>(
-                             a.v_scales + (static_cast<int64_t>(bhk) * D + c) * (a.Npad / 32) + j * 4))
-                       : 0x7F7F7F7Fu;
+        for (int kk = 0; kk < L::KSTEPS; ++kk)
+          cp_async4(st + L::ST_KSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, ok);
+        if (r < D)
+          cp_async4(st + L::ST_VSF + lane * 16 + r1 * 4,
+                    a.v_scales + (static_cast<int64_t>(bhk) * D + r) * (a.Npad / 32) + j * 4, true);
       }
-      *reinterpret_cast<uint4*>(st + L::ST_VSF + lane * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
-      fence_proxy_async_smem();
+      cp_async_arrive_noinc(kv_full + s);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_TMA_BYTES);
@@ -294,7 +285,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const bool f16 = kMixed && bm_row[jj];
         if (!wait1(p_full + b2, (jj >> 1) & 1, jj)) return false;
         tc_fence_after();
-        const uint32_t tO = tbase + L::T_O;
+        const uint32_t tO = tbase + L::T_O + b2 * L::T_OSTRIDE;
         if (!f16) {
           unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
           const uint32_t tv = tbase + L::T_VSF + 8 * s;
@@ -306,7 +297,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
             mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
                      (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
-                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 0 || kk > 0) ? 1u : 0u);
+                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 1 || kk > 0) ? 1u : 0u);
           }
         } else {
           const uint32_t sV16 = smem_u32(sm + L::OFF_V16);
@@ -314,7 +305,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
             const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
-            mma_f16(tO, da, db, idesc_pv16, (jj > 0 || kk > 0) ? 1u : 0u);
+            mma_f16(tO, da, db, idesc_pv16, (jj > 1 || kk > 0) ? 1u : 0u);
           }
           mma_commit(kv16_empty);
         }
@@ -327,9 +318,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const bool f16 = kMixed && bm_row[j];
         if (!wait1(kv_full + s, (j / L::NS) & 1, j)) { ok = false; break; }
         tc_fence_after();
-        if (j >= 2 && !wait1(s_free + b2, ((j - 2) >> 1) & 1, j)) { ok = false; break; }
+        if (j >= 1 && !wait1(s_free, (j - 1) & 1, j)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tS = tbase + L::T_S + b2 * 128;
+        const uint32_t tS = tbase + L::T_S;
         if (!f16) {
           unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
           const uint32_t tk = tbase + L::T_KSF + 8 * s;
@@ -340,7 +331,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
             mma_nvf4(tS, da, db, idesc_qk, tbase + L::T_QSF + 4 * kk, tk + 4 * kk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_full + b2);
+          mma_commit(s_full);
           if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
         } else {
           // The single FP16 operand buffer is refilled only after the previous FP16 tile's
@@ -359,7 +350,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sK16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
             mma_f16(tS, da, db, idesc_qk16, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_full + b2);
+          mma_commit(s_full);
         }
       }
       if (ok && nt > 0) issue_pv(nt - 1);
@@ -382,10 +373,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // dot products and are brought into raw units by 1 / (s_tQ s_tK).
     const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
     const float R16 = 1.f / ((*a.q_ts) * (*a.k_ts));
-    const uint64_t C2 = f2_pack(C, C);
-    const uint64_t P448 = f2_pack(448.f, 448.f);
+    const float2 C2 = make_float2(C, C);
+    const float2 P448 = make_float2(448.f, 448.f);
     float m_run = -INFINITY;
+    float m_ref0 = -INFINITY, m_ref1 = -INFINITY;   // max at the last update of O_0 / O_1
     unsigned char* sP = sm + L::OFF_P;
+    bool prev_f16 = false;
     // A warp whose wait fails keeps iterating without doing work (ok == false), so that the
     // two partner warps of a quadrant always meet at every named barrier.
     bool ok = true;
@@ -394,17 +387,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const bool f16 = kMixed && bm_row[j];
       float x[64];
       float mt = -INFINITY;
-      if (ok && !waitw(s_full + b2, (j >> 1) & 1, j)) ok = false;
+      if (ok && !waitw(s_full, j & 1, j)) ok = false;
       if (ok) {
         tc_fence_after();
         uint32_t* xr = reinterpret_cast<uint32_t*>(x);
-        const uint32_t tS = tbase + L::T_S + b2 * 128 + half * 64 + lane_addr;
+        const uint32_t tS = tbase + L::T_S + half * 64 + lane_addr;
         tmem_ld32(tS + 0, xr + 0);
         tmem_ld32(tS + 32, xr + 32);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free + b2);
+        if (lane == 0) mbar_arrive(s_free);
         if (f16) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) x[c] *= R16;
@@ -429,35 +422,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float m_new = fmaxf(m_run, mt);
       const bool dead = (m_new == -INFINITY);
       const float mref = dead ? 0.f : m_new;
-      const float alpha = dead ? 1.f : ex2_approx((m_run - m_new) * C);
       m_run = m_new;
-      const uint64_t M2 = f2_pack(mref, mref);
+      const float2 M2 = make_float2(mref, mref);
       uint32_t pw[32];             // e4m3: 16 words used; fp16: 32 words
       if (!f16) {
 #pragma unroll
         for (int c = 0; c < 64; c += 4) {
-          float t[4];
-          f2_unpack(f2_mul(f2_sub(f2_pack(x[c], x[c + 1]), M2), C2), t[0], t[1]);
-          f2_unpack(f2_mul(f2_sub(f2_pack(x[c + 2], x[c + 3]), M2), C2), t[2], t[3]);
-          float p[4];
-          f2_unpack(f2_mul(f2_pack(ex2_approx(t[0]), ex2_approx(t[1])), P448), p[0], p[1]);
-          f2_unpack(f2_mul(f2_pack(ex2_approx(t[2]), ex2_approx(t[3])), P448), p[2], p[3]);
-          pw[c >> 2] = cvt_e4m3x2(p[0], p[1]) | (cvt_e4m3x2(p[2], p[3]) << 16);
+          const float2 t0 = __fmul2_rn(__fadd2_rn(make_float2(x[c], x[c + 1]), make_float2(-M2.x, -M2.y)), C2);
+          const float2 t1 = __fmul2_rn(__fadd2_rn(make_float2(x[c + 2], x[c + 3]), make_float2(-M2.x, -M2.y)), C2);
+          const float2 p0 = __fmul2_rn(make_float2(ex2_approx(t0.x), ex2_approx(t0.y)), P448);
+          const float2 p1 = __fmul2_rn(make_float2(ex2_approx(t1.x), ex2_approx(t1.y)), P448);
+          pw[c >> 2] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
         }
       } else {
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          float t0, t1, p0, p1;
-          f2_unpack(f2_mul(f2_sub(f2_pack(x[c], x[c + 1]), M2), C2), t0, t1);
-          f2_unpack(f2_mul(f2_pack(ex2_approx(t0), ex2_approx(t1)), P448), p0, p1);
-          const __half2 h = __floats2half2_rn(p0, p1);
+          const float2 t = __fmul2_rn(__fadd2_rn(make_float2(x[c], x[c + 1]), make_float2(-M2.x, -M2.y)), C2);
+          const float2 p = __fmul2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)), P448);
+          const __half2 h = __floats2half2_rn(p.x, p.y);
           pw[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
         }
       }
-      // PV(j-2) read this P buffer and must be done before it is rewritten; an FP16 tile
-      // writes both buffers, so then PV(j-1) too.
+      // P buffer b2 and O_{b2} were last used by PV(j-2). An FP16 tile's P fills both buffers:
+      // writing one needs PV(j-1) done as well, and the tile after an FP16 tile too.
       if (j >= 2 && !waitw(pv_done + b2, ((j - 2) >> 1) & 1, j)) { ok = false; continue; }
-      if (f16 && j >= 1 && !waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; continue; }
+      if ((f16 || prev_f16) && j >= 1 &&
+          !waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; continue; }
+      prev_f16 = f16;
       if (!f16) {
         unsigned char* prow = sP + b2 * 16384 + row * 128;
 #pragma unroll
@@ -474,80 +465,87 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
       }
       fence_proxy_async_smem();
-      // PV(j-1) must be done before O is rescaled for this tile.
-      if (j >= 1) {
-        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; continue; }
+      // Bring O_{b2} from its last reference max to m_new (PV(j-2) is done: waited above).
+      const float m_prev = b2 ? m_ref1 : m_ref0;
+      const float alpha = (m_prev == -INFINITY || dead) ? 1.f : ex2_approx((m_prev - m_new) * C);
+      if (!dead) { if (b2) m_ref1 = m_new; else m_ref0 = m_new; }
+      if (j >= 2 && !__all_sync(0xffffffffu, alpha == 1.f)) {
         tc_fence_after();
-        if (!__all_sync(0xffffffffu, alpha == 1.f)) {
-          // this warp's columns of O: half 0 -> [0, D/2) and [D, D+16) (l); half 1 -> [D/2, D)
-          const uint32_t tO = tbase + L::T_O + lane_addr;
-          const uint64_t A2 = f2_pack(alpha, alpha);
+        // this warp's columns of O_b2: half 0 -> [0, D/2) and [D, D+16) (l); half 1 -> [D/2, D)
+        const uint32_t tO = tbase + L::T_O + b2 * L::T_OSTRIDE + lane_addr;
+        const float2 A2 = make_float2(alpha, alpha);
 #pragma unroll
-          for (int cc = 0; cc < D / 2; cc += 32) {
-            const uint32_t col = half * (D / 2) + cc;
-            uint32_t o[32];
-            tmem_ld32(tO + col, o);
-            tmem_wait_ld();
+        for (int cc = 0; cc < D / 2; cc += 32) {
+          const uint32_t col = half * (D / 2) + cc;
+          uint32_t o[32];
+          tmem_ld32(tO + col, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              float u0, u1;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), A2), u0, u1);
-              o[k] = __float_as_uint(u0);
-              o[k + 1] = __float_as_uint(u1);
-            }
-            tmem_st32(tO + col, o);
+          for (int k = 0; k < 32; k += 2) {
+            const float2 u = __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), A2);
+            o[k] = __float_as_uint(u.x);
+            o[k + 1] = __float_as_uint(u.y);
           }
-          if (half == 0) {
-            uint32_t o[16];
-            tmem_ld16(tO + D, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st16(tO + D, o);
-          }
-          tmem_wait_st();
+          tmem_st32(tO + col, o);
         }
+        if (half == 0) {
+          uint32_t o[16];
+          tmem_ld16(tO + D, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st16(tO + D, o);
+        }
+        tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + b2);
     }
-    // ---- epilogue: O / l for this warp's half of the columns ----
+    // ---- epilogue: merge O_0 and O_1 at the final max, divide by l ----
+    // PV(nt-1)'s completion covers every earlier MMA of the issuing thread.
     if (ok && nt > 0 && waitw(pv_done + ((nt - 1) & 1), ((nt - 1) >> 1) & 1, nt)) {
       tc_fence_after();
-      const uint32_t tO = tbase + L::T_O + lane_addr;
-      uint32_t lr[16];
-      tmem_ld16(tO + D, lr);
+      const uint32_t tO0 = tbase + L::T_O + lane_addr;
+      const uint32_t tO1 = tO0 + L::T_OSTRIDE;
+      uint32_t lr0[16], lr1[16];
+      tmem_ld16(tO0 + D, lr0);
+      tmem_ld16(tO1 + D, lr1);
       tmem_wait_ld();
-      const float l_run = __uint_as_float(lr[0]);
+      const float w0 = (m_ref0 == -INFINITY) ? 0.f : ex2_approx((m_ref0 - m_run) * C);
+      const float w1 = (m_ref1 == -INFINITY) ? 0.f : ex2_approx((m_ref1 - m_run) * C);
+      auto merge = [&](float o0, float o1) {
+        const float v = w0 * o0;
+        return w1 == 0.f ? v : fmaf(w1, o1, v);
+      };
+      const float l_run = merge(__uint_as_float(lr0[0]), __uint_as_float(lr1[0]));
       const bool store = qi < a.Nq;
       const int64_t orow = static_cast<int64_t>(bhq) * a.Nq + qi;
 #pragma unroll
       for (int cc = 0; cc < D / 2; cc += 32) {
         const int c = half * (D / 2) + cc;
-        uint32_t o[32];
-        tmem_ld32(tO + c, o);
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO0 + c, o0);
+        tmem_ld32(tO1 + c, o1);
         tmem_wait_ld();
         if (store) {
+          float v[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            v[k] = __fdiv_rn(merge(__uint_as_float(o0[k]), __uint_as_float(o1[k])), l_run);
           if (a.out_kind == 2) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              dst[k] = make_float4(__fdiv_rn(__uint_as_float(o[4 * k]), l_run),
-                                   __fdiv_rn(__uint_as_float(o[4 * k + 1]), l_run),
-                                   __fdiv_rn(__uint_as_float(o[4 * k + 2]), l_run),
-                                   __fdiv_rn(__uint_as_float(o[4 * k + 3]), l_run));
+            for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
           } else {
             __align__(16) uint32_t packed[16];
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
-              const float v0 = __fdiv_rn(__uint_as_float(o[k]), l_run);
-              const float v1 = __fdiv_rn(__uint_as_float(o[k + 1]), l_run);
               if (a.out_kind == 1) {
-                __nv_bfloat162 t = __floats2bfloat162_rn(v0, v1);
+                __nv_bfloat162 t = __floats2bfloat162_rn(v[k], v[k + 1]);
                 packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
               } else {
-                __half2 t = __floats2half2_rn(v0, v1);
+                __half2 t = __floats2half2_rn(v[k], v[k + 1]);
                 packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
               }
             }

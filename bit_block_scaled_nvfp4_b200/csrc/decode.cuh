@@ -42,11 +42,14 @@ struct DecLayout {
   static constexpr int ST_V0 = 8192;              // 128 channels x 64 B (page 0 tokens)
   static constexpr int ST_V1 = 16384;             // page 1 tokens
   static constexpr int ST_KSF = 24576;            // 2 chunks
-  static constexpr int ST_VSF = 25600;            // 1 chunk
-  static constexpr int STAGE_BYTES = 26624;
+  static constexpr int ST_VSF = 25600;            // 1 chunk (tcgen05 layout)
+  static constexpr int ST_VRAW = 26624;           // the two pages' V scales as stored (2 x 256 B)
+  static constexpr int STAGE_BYTES = 27648;
   static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_BAR + 256;   // reductions: [4 warps][16] max, [4][16] sum
-  static constexpr int SMEM_BYTES = OFF_RED + 2 * 4 * 16 * 4;
+  static constexpr int OFF_PID = OFF_RED + 2 * 4 * 16 * 4;   // page ids of the split
+  static constexpr int MAX_SPLIT_PAGES = 256;                // split_tokens <= 16384
+  static constexpr int SMEM_BYTES = OFF_PID + MAX_SPLIT_PAGES * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   static constexpr uint32_t T_S = 0, T_O = 32, T_QSF = 48, T_PSF = 56, T_KSF = 64, T_VSF = 88;
   static constexpr int NQ = 16;                   // MMA N (query heads, padded)
@@ -98,7 +101,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < L::NS; ++i) { mbar_init(kv_full + i, 1); mbar_init(kv_empty + i, 1); }
+    // kv_full: the producer's expect-tx arrival plus one cp.async arrival per producer lane
+    for (int i = 0; i < L::NS; ++i) { mbar_init(kv_full + i, 33); mbar_init(kv_empty + i, 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1); mbar_init(s_free + i, 4);
       mbar_init(p_full + i, 4); mbar_init(pv_done + i, 1);
@@ -168,48 +172,41 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tma_load_2d(sm + L::OFF_Q, &tm_q, q_full, 0, static_cast<int>(qrow0));
       }
     }
+    // Page ids of this split, checked once, into shared memory.
+    int32_t* pid = reinterpret_cast<int32_t*>(sm + L::OFF_PID);
+    const int n_split_pages = (k_end - k_begin + 63) / 64;
+    for (int i = lane; i < n_split_pages; i += 32) pid[i] = page_of(k_begin / 64 + i);
+    __syncwarp();
     for (int blk = 0; blk < nblk; ++blk) {
       const int st_i = blk % L::NS;
       if (blk >= L::NS && !waitw(kv_empty + st_i, ((blk / L::NS) - 1) & 1, blk)) break;
       unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
       const int k0 = k_begin + blk * 128;
-      const int lp0 = k0 / 64;
-      const int p0 = page_of(lp0);
-      const int p1 = (k0 + 64 < len) ? page_of(lp0 + 1) : p0;
-      // K scale factors: key rows 0..63 from page p0, 64..127 from p1.
-      uint32_t w[4][2];
+      const int p0 = pid[2 * blk];
+      const int p1 = (k0 + 64 < len) ? pid[2 * blk + 1] : p0;
+      // K scale factors straight into the tcgen05 layout with 4-byte asynchronous copies: key
+      // row r = r0 + 32 r1 (rows 0..63 from page p0, 64..127 from p1) -> byte r0*16 + r1*4 of
+      // the chunk of its 64-element MMA step. This warp does not wait for them.
 #pragma unroll
       for (int r1 = 0; r1 < 4; ++r1) {
         const int r = r1 * 32 + lane;
         const int pp = r < 64 ? p0 : p1;
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(
-            a.k_page_scales + ((static_cast<int64_t>(pp) * a.Hkv + h) * 64 + (r & 63)) * (D / 16)));
-        w[r1][0] = v.x; w[r1][1] = v.y;
-      }
+        const uint8_t* src = a.k_page_scales + ((static_cast<int64_t>(pp) * a.Hkv + h) * 64 + (r & 63)) * (D / 16);
 #pragma unroll
-      for (int kk = 0; kk < 2; ++kk)
-        *reinterpret_cast<uint4*>(st + L::ST_KSF + kk * 512 + lane * 16) =
-            make_uint4(w[0][kk], w[1][kk], w[2][kk], w[3][kk]);
-      // V scale factors: channel c, [page0 g0, page0 g1, page1 g0, page1 g1].
-      uint32_t vw[4];
-#pragma unroll
-      for (int r1 = 0; r1 < 4; ++r1) {
-        const int c = r1 * 32 + lane;
-        const uint32_t lo = __ldg(reinterpret_cast<const uint16_t*>(
-            a.v_page_scales + ((static_cast<int64_t>(p0) * a.Hkv + h) * D + c) * 2));
-        const uint32_t hi = __ldg(reinterpret_cast<const uint16_t*>(
-            a.v_page_scales + ((static_cast<int64_t>(p1) * a.Hkv + h) * D + c) * 2));
-        vw[r1] = lo | (hi << 16);
+        for (int kk = 0; kk < 2; ++kk) cp_async4(st + L::ST_KSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, true);
       }
-      *reinterpret_cast<uint4*>(st + L::ST_VSF + lane * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
-      fence_proxy_async_smem();
+      cp_async_arrive_noinc(kv_full + st_i);
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(kv_full + st_i, 128 * 64 + 2 * D * 64);
+        // K and V codes by TMA; the pages' V scales (256 B each, as stored) by bulk copy, to be
+        // rearranged by the MMA warp.
+        mbar_arrive_expect_tx(kv_full + st_i, 128 * 64 + 2 * D * 64 + 2 * D * 2);
         tma_load_2d(st + L::ST_K, &tm_kp, kv_full + st_i, 0, (p0 * a.Hkv + h) * 64);
         tma_load_2d(st + L::ST_K + 4096, &tm_kp, kv_full + st_i, 0, (p1 * a.Hkv + h) * 64);
         tma_load_2d(st + L::ST_V0, &tm_vp, kv_full + st_i, 0, (p0 * a.Hkv + h) * D);
         tma_load_2d(st + L::ST_V1, &tm_vp, kv_full + st_i, 0, (p1 * a.Hkv + h) * D);
+        bulk_load(st + L::ST_VRAW, a.v_page_scales + (static_cast<int64_t>(p0) * a.Hkv + h) * D * 2, D * 2, kv_full + st_i);
+        bulk_load(st + L::ST_VRAW + D * 2, a.v_page_scales + (static_cast<int64_t>(p1) * a.Hkv + h) * D * 2, D * 2, kv_full + st_i);
       }
     }
     for (int i = 0; i < L::NS && i < nblk; ++i) {
@@ -219,21 +216,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_wait(q_full, 0);
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
-    if (lane == 0) {
-      const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, L::NQ);
-      const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NQ);
-      const uint32_t sQ = smem_u32(sm + L::OFF_Q);
-      const uint32_t sP = smem_u32(sm + L::OFF_P);
-      bool ok = wait1(q_full, 0, -1);
-      if (ok) {
-        tc_fence_after();
-        tmem_cp_sf(tbase + L::T_QSF, sm + L::OFF_QSF);
-        tmem_cp_sf(tbase + L::T_QSF + 4, sm + L::OFF_QSF + 512);
-        tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
-      }
-      auto issue_pv = [&](int bb) -> bool {
-        const int st_i = bb % L::NS, b2 = bb & 1;
-        if (!wait1(p_full + b2, (bb >> 1) & 1, bb)) return false;
+    // The whole warp runs the loop: all lanes rearrange the V scales of each block into the
+    // tcgen05 layout; lane 0 alone issues the tcgen05 copies and MMAs and their commits.
+    const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, L::NQ);
+    const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NQ);
+    const uint32_t sQ = smem_u32(sm + L::OFF_Q);
+    const uint32_t sP = smem_u32(sm + L::OFF_P);
+    bool ok = waitw(q_full, 0, -1);
+    if (ok && lane == 0) {
+      tc_fence_after();
+      tmem_cp_sf(tbase + L::T_QSF, sm + L::OFF_QSF);
+      tmem_cp_sf(tbase + L::T_QSF + 4, sm + L::OFF_QSF + 512);
+      tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+    }
+    __syncwarp();
+    auto issue_pv = [&](int bb) -> bool {
+      const int st_i = bb % L::NS, b2 = bb & 1;
+      if (!waitw(p_full + b2, (bb >> 1) & 1, bb)) return false;
+      if (lane == 0) {
         tc_fence_after();
         unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
         const uint32_t tv = tbase + L::T_VSF + 4 * st_i;
@@ -250,15 +250,30 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         mma_commit(pv_done + b2);
         mma_commit(kv_empty + st_i);
-        return true;
-      };
-      for (int blk = 0; ok && blk < nblk; ++blk) {
-        const int st_i = blk % L::NS, b2 = blk & 1;
-        if (!wait1(kv_full + st_i, (blk / L::NS) & 1, blk)) { ok = false; break; }
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int blk = 0; ok && blk < nblk; ++blk) {
+      const int st_i = blk % L::NS, b2 = blk & 1;
+      if (!waitw(kv_full + st_i, (blk / L::NS) & 1, blk)) { ok = false; break; }
+      unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
+      {
+        // channel c = r0 + 32 r1: word [page0 g0, page0 g1, page1 g0, page1 g1] at r0*16 + r1*4
+        const uint16_t* raw = reinterpret_cast<const uint16_t*>(st + L::ST_VRAW);
+        uint32_t vw[4];
+#pragma unroll
+        for (int r1 = 0; r1 < 4; ++r1) {
+          const int c = r1 * 32 + lane;
+          vw[r1] = static_cast<uint32_t>(raw[c]) | (static_cast<uint32_t>(raw[D + c]) << 16);
+        }
+        *reinterpret_cast<uint4*>(st + L::ST_VSF + lane * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (blk >= 2 && !waitw(s_free + b2, ((blk - 2) >> 1) & 1, blk)) { ok = false; break; }
+      if (lane == 0) {
         tc_fence_after();
-        if (blk >= 2 && !wait1(s_free + b2, ((blk - 2) >> 1) & 1, blk)) { ok = false; break; }
-        tc_fence_after();
-        unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
         const uint32_t tk = tbase + L::T_KSF + 8 * st_i;
         tmem_cp_sf(tk, st + L::ST_KSF);
         tmem_cp_sf(tk + 4, st + L::ST_KSF + 512);
@@ -271,9 +286,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                    tbase + L::T_QSF + 4 * kk, kk > 0 ? 1u : 0u);
         }
         mma_commit(s_full + b2);
-        if (blk >= 1 && !issue_pv(blk - 1)) { ok = false; break; }
       }
-      if (ok) issue_pv(nblk - 1);
+      __syncwarp();
+      if (blk >= 1 && !issue_pv(blk - 1)) { ok = false; break; }
+    }
+    if (ok) issue_pv(nblk - 1);
+    if (lane == 0) {
       mma_commit(mma_final);
       mbar_wait(mma_final, 0);
     }

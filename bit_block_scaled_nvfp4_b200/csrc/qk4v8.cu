@@ -5,7 +5,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/qk4v8.h"
+#include "qk4v8.h"
 #include "ptx.cuh"
 #include "quantize.cuh"
 #include "tilescore.cuh"
@@ -350,6 +350,7 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
       p->kv_heads <= 0 || p->q_heads % p->kv_heads || p->max_context <= 0)
     return QK4V8_ERR_INVALID_ARG;
   if (p->split_tokens <= 0 || p->split_tokens % 128) return QK4V8_ERR_INVALID_ARG;
+  if (p->split_tokens > 64 * DecLayout::MAX_SPLIT_PAGES) return QK4V8_ERR_UNSUPPORTED;
   if (p->max_context > 64 * p->max_pages) return QK4V8_ERR_INVALID_ARG;
   if (p->out_dtype != QK4V8_F16 && p->out_dtype != QK4V8_BF16 && p->out_dtype != QK4V8_F32)
     return QK4V8_ERR_INVALID_ARG;

@@ -200,7 +200,7 @@ typedef struct {
   const int32_t* context_lens; /* [S], 1 <= len <= min(max_context, 64 * max_pages) */
   int32_t num_seqs, num_pages, max_pages, q_heads, kv_heads, head_dim; /* head_dim 128 */
   int32_t max_context;         /* host-side bound on context_lens (sizes grid and workspace) */
-  int32_t split_tokens;        /* keys per split, a positive multiple of 128 */
+  int32_t split_tokens;        /* keys per split, a positive multiple of 128, at most 16384 */
   float softmax_scale;
   qk4v8_dtype out_dtype;
   void* out;                   /* [S, Hq, D] out (out_dtype) */
