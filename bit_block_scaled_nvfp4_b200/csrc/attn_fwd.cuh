@@ -13,18 +13,24 @@
 // after its D channel rows, so the PV MMA (N = D + 16) accumulates sum_j P_j into O column D,
 // with the same rescaling as O.
 //
-// Two O accumulators: even key tiles accumulate into O_0 and odd ones into O_1, each kept
-// relative to the running max at its last update. Tile j's rescale then touches O_{j&1}, which
-// only needs PV(j-2) finished, so it overlaps PV(j-1) on the tensor core instead of stalling
-// it; the epilogue merges the two exactly (the same result as one accumulator).
+// Softmax in two groups by key-tile parity. Group 0 (warps 2-5) takes the even key tiles and
+// group 1 (warps 6-9) the odd ones; each thread owns one query row and all 128 keys of the
+// tile. Each group owns one O accumulator (O_0 / O_1), kept relative to the running max at
+// the group's last tile, so a group's rescale never waits on the other group's PV. The only
+// exchange between the groups is the running max, handed on per tile through shared memory
+// right after the tile max (long before the exponentials), so one group's exponentials run
+// while the other loads, reduces and stores: the exp unit, the bound of this kernel, stays
+// busy. The epilogue merges O_0 and O_1 exactly.
+//
+// MMA order: QK(j) then PV(j - LAG) (LAG = 2, 1 with the FP16 operands), so a group has two
+// tile periods to produce P before the tensor core needs it. S is single-buffered but freed
+// as soon as the owning group has copied it to registers.
 //
 // One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
-//              tcgen05 scale layout with plain loads, FP16 tiles when selected
+//              tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles when selected
 //   warp 1     TMEM owner and MMA issuer (one thread)
-//   warps 2-9  softmax: warps w and w+4 share TMEM lane quadrant w % 4 (32 query rows) and
-//              split each row's 128 keys in halves of 64; they exchange the row max through
-//              shared memory, rescale their halves of O and write the output
+//   warps 2-9  softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
 // TMEM (512 columns): S [0,128), O_0 and O_1 (D + 16 columns each) from 128, scale factors
 // from 416.
 #pragma once
@@ -34,6 +40,7 @@ namespace qk4v8 {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
 
 struct FwdArgs {
   const uint8_t* q_scales;
@@ -52,7 +59,11 @@ struct FwdArgs {
 
 template <int D, bool kMixed>
 struct FwdLayout {
-  static constexpr int NS = kMixed ? 2 : 3;   // the FP16 operand stage needs the room
+  static constexpr int NS = kMixed ? 2 : 4;   // the FP16 operand stage needs the room
+  // PV(j - LAG) is issued after QK(j); the producer refills stage s only after PV of its
+  // previous tile, so LAG <= NS - 1 keeps the producer ahead of the MMA issuer.
+  static constexpr int LAG = kMixed ? 1 : 2;
+  static_assert(LAG <= NS - 1, "PV lag must leave the producer a free stage");
   static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
   static constexpr int NV = D + 16;                     // PV MMA N: D channels + ones rows
   static constexpr int Q_BYTES = 128 * D / 2;
@@ -69,19 +80,20 @@ struct FwdLayout {
   static constexpr int ST_VSF = ST_KSF + 1024;
   static constexpr int STAGE_BYTES = ST_VSF + 1024;
   static constexpr int OFF_P = OFF_STAGE + NS * STAGE_BYTES;               // 2 x 16 KB
-  static constexpr int OFF_RED = OFF_P + 2 * 16384;                        // [2][2][128] floats
+  static constexpr int OFF_RED = OFF_P + 2 * 16384;   // running max hand-off [2][128], final [2][128]
   static constexpr int OFF_Q16 = OFF_RED + 2048;
   static constexpr int F16_TILE = 128 * D * 2;
   static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int N_BARS = 1 + 2 * NS + 2 + 4 + 3 + 1;
+  static constexpr int N_BARS = 1 + 2 * NS + 13;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   // TMEM columns
   static constexpr uint32_t T_S = 0, T_O = 128, T_OSTRIDE = 144, T_QSF = 416, T_PSF = 424,
-                            T_KSF = 428, T_VSF = 452;
+                            T_KSF = 428, T_VSF = T_KSF + 8 * NS;
+  static_assert(T_VSF + 8 * NS <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
   static constexpr int THREADS = 320;
@@ -101,14 +113,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = bars + 1 + L::NS;
-  uint64_t* s_full = bars + 1 + 2 * L::NS;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_full + 2;           // [2], by tile parity
-  uint64_t* pv_done = s_full + 4;          // [2], by tile parity
-  uint64_t* kv16_full = s_full + 6;
-  uint64_t* kv16_empty = s_full + 7;
-  uint64_t* q16_full = s_full + 8;
-  uint64_t* mma_final = s_full + 9;
+  // Barriers a group waits on come in pairs by key-tile parity: a waiter must never run more
+  // than one phase ahead of a barrier (a parity wait cannot tell phase k from phase k - 2).
+  uint64_t* s_full = bars + 1 + 2 * L::NS; // [2], by tile parity
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_full + 3;           // [2], by tile parity
+  uint64_t* pv_done = s_full + 5;          // [2], by tile parity
+  uint64_t* m_ready = s_full + 7;          // [2], by tile parity: running max handed on
+  uint64_t* kv16_full = s_full + 9;
+  uint64_t* kv16_empty = s_full + 10;
+  uint64_t* q16_full = s_full + 11;
+  uint64_t* mma_final = s_full + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -126,9 +141,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // full barriers: the TMA's expect-tx arrival plus one cp.async arrival per producer lane
     mbar_init(q_full, 33);
     for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 1); }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 8);
-    for (int i = 0; i < 2; ++i) { mbar_init(p_full + i, 8); mbar_init(pv_done + i, 1); }
+    mbar_init(s_free, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 4);
+      mbar_init(pv_done + i, 1);
+      mbar_init(m_ready + i, 4);
+    }
     mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1); mbar_init(q16_full, 1);
     mbar_init(mma_final, 1);
     *abort_flag = 0;
@@ -203,7 +222,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
     }
     bool q16_loaded = false;
-    int n16 = 0;
+    int n16 = 0, issued = 0;
     for (int j = 0; j < nt; ++j) {
       const int s = j % L::NS;
       if (j >= L::NS && !waitw(kv_empty + s, ((j / L::NS) - 1) & 1, j)) break;
@@ -231,6 +250,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, bhk);
         tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, bhk * D);
       }
+      issued = j + 1;
       if constexpr (kMixed) {
         if (bm_row[j]) {
           if (!q16_loaded) {
@@ -254,8 +274,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
     }
     // Drain: never leave a copy in flight into this CTA's shared memory.
-    for (int s = 0; s < L::NS && s < nt; ++s) {
-      const int last = s + ((nt - 1 - s) / L::NS) * L::NS;
+    for (int s = 0; s < L::NS && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / L::NS) * L::NS;
       mbar_wait(kv_full + s, (last / L::NS) & 1);
     }
     mbar_wait(q_full, 0);
@@ -271,6 +291,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t sP = smem_u32(sm + L::OFF_P);
       bool ok = wait1(q_full, 0, -1);
       if (ok) {
+        // the scale factors arrived by cp.async (generic proxy); the tensor core reads them
+        // through the async proxy
+        fence_proxy_async_smem();
         tc_fence_after();
         for (int kk = 0; kk < L::KSTEPS; ++kk)
           tmem_cp_sf(tbase + L::T_QSF + 4 * kk, sm + L::OFF_QSF + kk * 512);
@@ -313,10 +336,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_commit(kv_empty + s);
         return true;
       };
+      int np = 0;                                  // next tile whose PV is to be issued
       for (int j = 0; ok && j < nt; ++j) {
-        const int s = j % L::NS, b2 = j & 1;
+        const int s = j % L::NS;
         const bool f16 = kMixed && bm_row[j];
+        // The single FP16 operand buffer is refilled only after the previous FP16 tile's PV
+        // has finished, so every pending PV goes out before waiting for this tile's data.
+        if (f16)
+          while (ok && np < j) ok = issue_pv(np++);
+        if (!ok) break;
         if (!wait1(kv_full + s, (j / L::NS) & 1, j)) { ok = false; break; }
+        fence_proxy_async_smem();
         tc_fence_after();
         if (j >= 1 && !wait1(s_free, (j - 1) & 1, j)) { ok = false; break; }
         tc_fence_after();
@@ -331,12 +361,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
             mma_nvf4(tS, da, db, idesc_qk, tbase + L::T_QSF + 4 * kk, tk + 4 * kk, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_full);
-          if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
         } else {
-          // The single FP16 operand buffer is refilled only after the previous FP16 tile's
-          // PV has finished, so PV(j-1) must be issued before waiting for this tile's data.
-          if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
           if (!q16_ready) {
             if (!wait1(q16_full, 0, j)) { ok = false; break; }
             q16_ready = true;
@@ -350,10 +375,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sK16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
             mma_f16(tS, da, db, idesc_qk16, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_full);
         }
+        mma_commit(s_full + (j & 1));
+        while (ok && np <= j - L::LAG) ok = issue_pv(np++);
       }
-      if (ok && nt > 0) issue_pv(nt - 1);
+      while (ok && np < nt) ok = issue_pv(np++);
       // Everything this thread issued has completed before TMEM is released.
       mma_commit(mma_final);
       mbar_wait(mma_final, 0);
@@ -362,123 +388,126 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else {
     // ================================ softmax ================================
     const int wq = warp & 3;                 // TMEM lane quadrant
-    const int half = (warp - 2) >> 2;        // which 64 keys of the tile (and half of O)
+    const int grp = (warp - 2) >> 2;         // key-tile parity this group handles
     const int row = wq * 32 + lane;
     const int qi = qt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-    float* red = reinterpret_cast<float*>(sm + L::OFF_RED);       // [2 tiles][2 halves][128]
+    float* red_m = reinterpret_cast<float*>(sm + L::OFF_RED);         // [2 parities][128]
+    float* red_fin = red_m + 256;                                     // [2 groups][128]
     // Scores stay in the FP4 MMA's raw units (S = sum codes*scales); the running max m is
-    // kept in those units, so (s - m) is exact for the keys near the max, and
-    // p = 2^((s - m) * C) with C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true
-    // dot products and are brought into raw units by 1 / (s_tQ s_tK).
+    // kept in those units and 448 p = 2^(s C + (log2 448 - m C)) with
+    // C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true dot products and are
+    // brought into raw units by 1 / (s_tQ s_tK).
     const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
     const float R16 = 1.f / ((*a.q_ts) * (*a.k_ts));
     const float2 C2 = make_float2(C, C);
-    const float2 P448 = make_float2(448.f, 448.f);
-    float m_run = -INFINITY;
-    float m_ref0 = -INFINITY, m_ref1 = -INFINITY;   // max at the last update of O_0 / O_1
+    float m_own = -INFINITY;        // running max at this group's last tile (O_grp's reference)
     unsigned char* sP = sm + L::OFF_P;
-    bool prev_f16 = false;
-    // A warp whose wait fails keeps iterating without doing work (ok == false), so that the
-    // two partner warps of a quadrant always meet at every named barrier.
+    const uint32_t tO = tbase + L::T_O + grp * L::T_OSTRIDE + lane_addr;
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const int b2 = j & 1;
+    for (int j = grp; j < nt; j += 2) {
+      const int b2 = j & 1;                  // == grp
       const bool f16 = kMixed && bm_row[j];
-      float x[64];
-      float mt = -INFINITY;
-      if (ok && !waitw(s_full, j & 1, j)) ok = false;
-      if (ok) {
-        tc_fence_after();
+      const bool prev_f16 = kMixed && j >= 1 && bm_row[j - 1];
+      float x[128];
+      if (!waitw(s_full + b2, (j >> 1) & 1, j)) { ok = false; break; }
+      tc_fence_after();
+      {
         uint32_t* xr = reinterpret_cast<uint32_t*>(x);
-        const uint32_t tS = tbase + L::T_S + half * 64 + lane_addr;
-        tmem_ld32(tS + 0, xr + 0);
-        tmem_ld32(tS + 32, xr + 32);
+        const uint32_t tS = tbase + L::T_S + lane_addr;
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) tmem_ld32(tS + c, xr + c);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
-        if (f16) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] *= R16;
-        }
-        const int kbase = j * 128 + half * 64;
-        const bool need_mask = (a.causal && kbase + 63 > qi) || (kbase + 64 > a.Nk);
-        if (need_mask) {
-          const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
-#pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = (c <= lim) ? x[c] : -INFINITY;
-        }
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) mt = fmax3(mt, x[c], x[c + 1]);
       }
-      // Row max over both halves: the partner warp holds the other 64 keys of the row. The
-      // exchange slots alternate between tiles, so a fast warp's next write cannot overwrite
-      // a value its partner has not read yet (both pass the barrier of every tile).
-      red[(b2 * 2 + half) * 128 + row] = mt;
-      named_bar_sync(1 + wq, 64);
-      mt = fmaxf(mt, red[(b2 * 2 + (half ^ 1)) * 128 + row]);
-      if (!ok) continue;
-      const float m_new = fmaxf(m_run, mt);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      if (f16) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] *= R16;
+      }
+      const int kbase = j * 128;
+      if ((a.causal && kbase + 127 > qi) || (kbase + 128 > a.Nk)) {
+        const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
+#pragma unroll
+        for (int c = 0; c < 128; ++c) x[c] = (c <= lim) ? x[c] : -INFINITY;
+      }
+      float mt;
+      {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) m4[u] = fmax3(m4[u], x[c + 2 * u], x[c + 2 * u + 1]);
+        }
+        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      }
+      // Running max before this tile: handed on by the group that processed tile j - 1.
+      float m_prev = -INFINITY;
+      if (j >= 1) {
+        if (!waitw(m_ready + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
+        __syncwarp();
+        m_prev = red_m[((j - 1) & 1) * 128 + row];
+      }
+      const float m_new = fmaxf(m_prev, mt);
+      red_m[b2 * 128 + row] = m_new;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(m_ready + b2);
       const bool dead = (m_new == -INFINITY);
-      const float mref = dead ? 0.f : m_new;
-      m_run = m_new;
-      const float2 M2 = make_float2(mref, mref);
-      uint32_t pw[32];             // e4m3: 16 words used; fp16: 32 words
+      const float bias = kLog2_448 - (dead ? 0.f : m_new) * C;
+      const float2 B2 = make_float2(bias, bias);
+      uint32_t pw[kMixed ? 64 : 32];      // e4m3: 32 words; fp16: 64 words
       if (!f16) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-          const float2 t0 = __fmul2_rn(__fadd2_rn(make_float2(x[c], x[c + 1]), make_float2(-M2.x, -M2.y)), C2);
-          const float2 t1 = __fmul2_rn(__fadd2_rn(make_float2(x[c + 2], x[c + 3]), make_float2(-M2.x, -M2.y)), C2);
-          const float2 p0 = __fmul2_rn(make_float2(ex2_approx(t0.x), ex2_approx(t0.y)), P448);
-          const float2 p1 = __fmul2_rn(make_float2(ex2_approx(t1.x), ex2_approx(t1.y)), P448);
-          pw[c >> 2] = cvt_e4m3x2(p0.x, p0.y) | (cvt_e4m3x2(p1.x, p1.y) << 16);
+        for (int c = 0; c < 128; c += 4) {
+          const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
+          const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), C2, B2);
+          pw[c >> 2] = cvt_e4m3x2(ex2_approx(t0.x), ex2_approx(t0.y)) |
+                       (cvt_e4m3x2(ex2_approx(t1.x), ex2_approx(t1.y)) << 16);
         }
-      } else {
+      } else if constexpr (kMixed) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float2 t = __fmul2_rn(__fadd2_rn(make_float2(x[c], x[c + 1]), make_float2(-M2.x, -M2.y)), C2);
-          const float2 p = __fmul2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)), P448);
-          const __half2 h = __floats2half2_rn(p.x, p.y);
+        for (int c = 0; c < 128; c += 2) {
+          const float2 t = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
+          const __half2 h = __floats2half2_rn(ex2_approx(t.x), ex2_approx(t.y));
           pw[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
         }
       }
       // P buffer b2 and O_{b2} were last used by PV(j-2). An FP16 tile's P fills both buffers:
-      // writing one needs PV(j-1) done as well, and the tile after an FP16 tile too.
-      if (j >= 2 && !waitw(pv_done + b2, ((j - 2) >> 1) & 1, j)) { ok = false; continue; }
+      // writing one needs PV(j-1) done as well, and the tile after an FP16 tile too. PV(j-2)'s
+      // completion implies PV(j-3)'s, so the wait on the other parity's barrier is for its
+      // next phase.
+      if (j >= 2 && !waitw(pv_done + b2, ((j - 2) >> 1) & 1, j)) { ok = false; break; }
       if ((f16 || prev_f16) && j >= 1 &&
-          !waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; continue; }
-      prev_f16 = f16;
+          !waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
       if (!f16) {
         unsigned char* prow = sP + b2 * 16384 + row * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int ch = half * 4 + c;
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
-              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-        }
-      } else {
-        unsigned char* prow = sP + half * 16384 + row * 128;     // atom = this half's 64 keys
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
               make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+      } else if constexpr (kMixed) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          unsigned char* prow = sP + h * 16384 + row * 128;     // atom h = keys 64h .. 64h+63
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
+                make_uint4(pw[32 * h + 4 * c], pw[32 * h + 4 * c + 1], pw[32 * h + 4 * c + 2],
+                           pw[32 * h + 4 * c + 3]);
+        }
       }
       fence_proxy_async_smem();
-      // Bring O_{b2} from its last reference max to m_new (PV(j-2) is done: waited above).
-      const float m_prev = b2 ? m_ref1 : m_ref0;
-      const float alpha = (m_prev == -INFINITY || dead) ? 1.f : ex2_approx((m_prev - m_new) * C);
-      if (!dead) { if (b2) m_ref1 = m_new; else m_ref0 = m_new; }
+      // Bring O_{b2} from this group's previous max to m_new (PV(j-2) is done: waited above).
+      const float alpha = (m_own == -INFINITY || dead) ? 1.f : ex2_approx((m_own - m_new) * C);
+      if (!dead) m_own = m_new;
       if (j >= 2 && !__all_sync(0xffffffffu, alpha == 1.f)) {
         tc_fence_after();
-        // this warp's columns of O_b2: half 0 -> [0, D/2) and [D, D+16) (l); half 1 -> [D/2, D)
-        const uint32_t tO = tbase + L::T_O + b2 * L::T_OSTRIDE + lane_addr;
         const float2 A2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int cc = 0; cc < D / 2; cc += 32) {
-          const uint32_t col = half * (D / 2) + cc;
+        for (int cc = 0; cc < D; cc += 32) {
           uint32_t o[32];
-          tmem_ld32(tO + col, o);
+          tmem_ld32(tO + cc, o);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; k += 2) {
@@ -486,9 +515,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             o[k] = __float_as_uint(u.x);
             o[k + 1] = __float_as_uint(u.y);
           }
-          tmem_st32(tO + col, o);
+          tmem_st32(tO + cc, o);
         }
-        if (half == 0) {
+        {
           uint32_t o[16];
           tmem_ld16(tO + D, o);
           tmem_wait_ld();
@@ -503,17 +532,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (lane == 0) mbar_arrive(p_full + b2);
     }
     // ---- epilogue: merge O_0 and O_1 at the final max, divide by l ----
-    // PV(nt-1)'s completion covers every earlier MMA of the issuing thread.
-    if (ok && nt > 0 && waitw(pv_done + ((nt - 1) & 1), ((nt - 1) >> 1) & 1, nt)) {
+    // PV(nt-1)'s completion covers every earlier MMA of the issuing thread; the group that
+    // owns tile nt-1 waits for it (the next phase of its own barrier) and the named barrier
+    // passes that on to the other group.
+    if (ok && grp == ((nt - 1) & 1)) ok = waitw(pv_done + grp, ((nt - 1) >> 1) & 1, nt);
+    red_fin[grp * 128 + row] = m_own;
+    tc_fence_before();
+    named_bar_sync(1, 256);
+    const float m0 = red_fin[row], m1 = red_fin[128 + row];
+    if (ok && !*abort_flag) {
       tc_fence_after();
+      const float m_run = fmaxf(m0, m1);
       const uint32_t tO0 = tbase + L::T_O + lane_addr;
       const uint32_t tO1 = tO0 + L::T_OSTRIDE;
       uint32_t lr0[16], lr1[16];
       tmem_ld16(tO0 + D, lr0);
       tmem_ld16(tO1 + D, lr1);
       tmem_wait_ld();
-      const float w0 = (m_ref0 == -INFINITY) ? 0.f : ex2_approx((m_ref0 - m_run) * C);
-      const float w1 = (m_ref1 == -INFINITY) ? 0.f : ex2_approx((m_ref1 - m_run) * C);
+      // O_1 is never written when there is a single key tile; its weight is then 0.
+      const float w0 = (m0 == -INFINITY) ? 0.f : ex2_approx((m0 - m_run) * C);
+      const float w1 = (m1 == -INFINITY || nt < 2) ? 0.f : ex2_approx((m1 - m_run) * C);
       auto merge = [&](float o0, float o1) {
         const float v = w0 * o0;
         return w1 == 0.f ? v : fmaf(w1, o1, v);
@@ -523,7 +561,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int64_t orow = static_cast<int64_t>(bhq) * a.Nq + qi;
 #pragma unroll
       for (int cc = 0; cc < D / 2; cc += 32) {
-        const int c = half * (D / 2) + cc;
+        const int c = grp * (D / 2) + cc;
         uint32_t o0[32], o1[32];
         tmem_ld32(tO0 + c, o0);
         tmem_ld32(tO1 + c, o1);
@@ -555,7 +593,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
         }
       }
-      if (store && half == 0 && a.lse != nullptr)
+      if (store && grp == 0 && a.lse != nullptr)
         a.lse[orow] = m_run * C * kLn2 + logf(l_run * (1.f / 448.f));
     }
   }
