@@ -22,15 +22,17 @@
 // while the other loads, reduces and stores: the exp unit, the bound of this kernel, stays
 // busy. The epilogue merges O_0 and O_1 exactly.
 //
-// MMA order: QK(j) then PV(j - LAG) (LAG = 2, 1 with the FP16 operands), so a group has two
-// tile periods to produce P before the tensor core needs it. S is single-buffered but freed
-// as soon as the owning group has copied it to registers.
+// Two MMA issuers: one thread issues QK^T, another PV, each waiting only on its own inputs,
+// so neither stream of tensor-core work stalls behind the other's waits (an issuing thread
+// blocks while the tensor core drains what it issued). S is single-buffered but freed as
+// soon as the owning group has copied it to registers.
 //
 // One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
 //              tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles when selected
-//   warp 1     TMEM owner and MMA issuer (one thread)
+//   warp 1     TMEM owner and QK^T issuer (one thread)
 //   warps 2-9  softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
+//   warp 10    PV issuer (one thread)
 // TMEM (512 columns): S [0,128), O_0 and O_1 (D + 16 columns each) from 128, scale factors
 // from 416.
 #pragma once
@@ -60,10 +62,6 @@ struct FwdArgs {
 template <int D, bool kMixed>
 struct FwdLayout {
   static constexpr int NS = kMixed ? 2 : 4;   // the FP16 operand stage needs the room
-  // PV(j - LAG) is issued after QK(j); the producer refills stage s only after PV of its
-  // previous tile, so LAG <= NS - 1 keeps the producer ahead of the MMA issuer.
-  static constexpr int LAG = kMixed ? 1 : 2;
-  static_assert(LAG <= NS - 1, "PV lag must leave the producer a free stage");
   static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
   static constexpr int NV = D + 16;                     // PV MMA N: D channels + ones rows
   static constexpr int Q_BYTES = 128 * D / 2;
@@ -87,7 +85,7 @@ struct FwdLayout {
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int N_BARS = 1 + 2 * NS + 13;
+  static constexpr int N_BARS = 1 + 2 * NS + 14;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   // TMEM columns
@@ -96,11 +94,12 @@ struct FwdLayout {
   static_assert(T_VSF + 8 * NS <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
-  static constexpr int THREADS = 320;
+  static constexpr int PV_WARP = 10;
+  static constexpr int THREADS = 352;
 };
 
 template <int D, bool kMixed>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q16,
                 const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
@@ -123,7 +122,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* kv16_full = s_full + 9;
   uint64_t* kv16_empty = s_full + 10;
   uint64_t* q16_full = s_full + 11;
-  uint64_t* mma_final = s_full + 12;
+  uint64_t* mma_final = s_full + 12;      // [2]: QK issuer, PV issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -140,7 +139,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     // full barriers: the TMA's expect-tx arrival plus one cp.async arrival per producer lane
     mbar_init(q_full, 33);
-    for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 1); }
+    // a stage is free once both the QK^T (K) and the PV (V) issuers are done with it
+    for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 2); }
     mbar_init(s_free, 4);
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
@@ -149,7 +149,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(m_ready + i, 4);
     }
     mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1); mbar_init(q16_full, 1);
-    mbar_init(mma_final, 1);
+    mbar_init(mma_final, 1); mbar_init(mma_final + 1, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -185,7 +185,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tbase = *tmem_slot;
 
   // Barrier ids in timeout reports are their index in the barrier block.
-  const uint32_t role = warp == 0 ? kRoleProducer : warp == 1 ? kRoleMma : kRoleSoftmax;
+  const uint32_t role = warp == 0 ? kRoleProducer : (warp == 1 || warp == L::PV_WARP) ? kRoleMma : kRoleSoftmax;
   auto site = [&](uint64_t* bar, int tile) {
     return wait_site(kKernelFwd, role, static_cast<uint32_t>(bar - bars), tile);
   };
@@ -281,14 +281,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_wait(q_full, 0);
     if (kMixed && n16 > 0) { mbar_wait(kv16_full, (n16 - 1) & 1); mbar_wait(q16_full, 0); }
   } else if (warp == 1) {
-    // ================================ MMA issuer ================================
+    // ============================ QK^T issuer (one thread) ============================
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, 128);
-      const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NV);
       const uint32_t idesc_qk16 = idesc_f16(128, 128);
-      const uint32_t idesc_pv16 = idesc_f16(128, L::NV);
       const uint32_t sQ = smem_u32(sm + L::OFF_Q);
-      const uint32_t sP = smem_u32(sm + L::OFF_P);
       bool ok = wait1(q_full, 0, -1);
       if (ok) {
         // the scale factors arrived by cp.async (generic proxy); the tensor core reads them
@@ -297,54 +294,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         for (int kk = 0; kk < L::KSTEPS; ++kk)
           tmem_cp_sf(tbase + L::T_QSF + 4 * kk, sm + L::OFF_QSF + kk * 512);
-        tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
-        for (int s = 0; s < L::NS; ++s)            // second V scale chunk (rows 128..): 1.0
-          tmem_cp_sf(tbase + L::T_VSF + 8 * s + 4, sm + L::OFF_PSF);
       }
-      int n16_qk = 0;
+      int n16 = 0;
       bool q16_ready = false;
-      auto issue_pv = [&](int jj) -> bool {
-        const int s = jj % L::NS, b2 = jj & 1;
-        const bool f16 = kMixed && bm_row[jj];
-        if (!wait1(p_full + b2, (jj >> 1) & 1, jj)) return false;
-        tc_fence_after();
-        const uint32_t tO = tbase + L::T_O + b2 * L::T_OSTRIDE;
-        if (!f16) {
-          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-          const uint32_t tv = tbase + L::T_VSF + 8 * s;
-          tmem_cp_sf(tv, st + L::ST_VSF);
-          const uint32_t sV = smem_u32(st + L::ST_V);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t da = make_sdesc(sP + b2 * 16384 + kk * 32, 16, 1024, kSw128);
-            const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
-            mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
-                     (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
-                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 1 || kk > 0) ? 1u : 0u);
-          }
-        } else {
-          const uint32_t sV16 = smem_u32(sm + L::OFF_V16);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
-            const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
-            mma_f16(tO, da, db, idesc_pv16, (jj > 1 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(kv16_empty);
-        }
-        mma_commit(pv_done + b2);
-        mma_commit(kv_empty + s);
-        return true;
-      };
-      int np = 0;                                  // next tile whose PV is to be issued
       for (int j = 0; ok && j < nt; ++j) {
         const int s = j % L::NS;
         const bool f16 = kMixed && bm_row[j];
-        // The single FP16 operand buffer is refilled only after the previous FP16 tile's PV
-        // has finished, so every pending PV goes out before waiting for this tile's data.
-        if (f16)
-          while (ok && np < j) ok = issue_pv(np++);
-        if (!ok) break;
         if (!wait1(kv_full + s, (j / L::NS) & 1, j)) { ok = false; break; }
         fence_proxy_async_smem();
         tc_fence_after();
@@ -366,9 +321,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!wait1(q16_full, 0, j)) { ok = false; break; }
             q16_ready = true;
           }
-          if (!wait1(kv16_full, n16_qk & 1, j)) { ok = false; break; }
+          if (!wait1(kv16_full, n16 & 1, j)) { ok = false; break; }
           tc_fence_after();
-          ++n16_qk;
+          ++n16;
           const uint32_t sQ16 = smem_u32(sm + L::OFF_Q16), sK16 = smem_u32(sm + L::OFF_K16);
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t da = make_sdesc(sQ16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
@@ -377,12 +332,63 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
         }
         mma_commit(s_full + (j & 1));
-        while (ok && np <= j - L::LAG) ok = issue_pv(np++);
+        mma_commit(kv_empty + s);                  // K half of the stage is free
       }
-      while (ok && np < nt) ok = issue_pv(np++);
       // Everything this thread issued has completed before TMEM is released.
       mma_commit(mma_final);
       mbar_wait(mma_final, 0);
+    }
+    __syncwarp();
+  } else if (warp == L::PV_WARP) {
+    // ============================== PV issuer (one thread) ==============================
+    if (lane == 0) {
+      const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NV);
+      const uint32_t idesc_pv16 = idesc_f16(128, L::NV);
+      const uint32_t sP = smem_u32(sm + L::OFF_P);
+      tc_fence_after();
+      tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+      for (int s = 0; s < L::NS; ++s)              // second V scale chunk (rows 128..): 1.0
+        tmem_cp_sf(tbase + L::T_VSF + 8 * s + 4, sm + L::OFF_PSF);
+      bool ok = true;
+      int n16 = 0;
+      for (int jj = 0; ok && jj < nt; ++jj) {
+        const int s = jj % L::NS, b2 = jj & 1;
+        const bool f16 = kMixed && bm_row[jj];
+        if (!wait1(p_full + b2, (jj >> 1) & 1, jj)) { ok = false; break; }
+        if (!wait1(kv_full + s, (jj / L::NS) & 1, jj)) { ok = false; break; }
+        if (f16 && !wait1(kv16_full, n16 & 1, jj)) { ok = false; break; }
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t tO = tbase + L::T_O + b2 * L::T_OSTRIDE;
+        if (!f16) {
+          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+          const uint32_t tv = tbase + L::T_VSF + 8 * s;
+          tmem_cp_sf(tv, st + L::ST_VSF);
+          const uint32_t sV = smem_u32(st + L::ST_V);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t da = make_sdesc(sP + b2 * 16384 + kk * 32, 16, 1024, kSw128);
+            const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
+            mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
+                     (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 1 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+          ++n16;
+          const uint32_t sV16 = smem_u32(sm + L::OFF_V16);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
+            const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
+            mma_f16(tO, da, db, idesc_pv16, (jj > 1 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(kv16_empty);
+        }
+        mma_commit(pv_done + b2);
+        mma_commit(kv_empty + s);                  // V half of the stage is free
+      }
+      mma_commit(mma_final + 1);
+      mbar_wait(mma_final + 1, 0);
     }
     __syncwarp();
   } else {
