@@ -65,6 +65,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
                : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
+// The same with a suspend-time hint: a thread whose phase is not complete yet sleeps (up to
+// the hint) until it completes instead of spinning, so waiting warps take no issue slots from
+// the warps that work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\t"
+               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u) : "memory");
+  return ok != 0;
+}
 // Bounded wait for the phase with the given parity to complete. Returns false (and sets the
 // timeout status bit) when the limit passes first. The limit is counted in SM clock cycles
 // (about a second at the B200's clocks) and read only every 32 polls, so the poll loop itself
@@ -76,7 +87,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (mbar_try_wait_sleep(bar, parity)) return true;
     if (clock64() - t0 > kWaitLimitCycles) {
       flag_error(kStatusTimeout);
       return false;
