@@ -15,17 +15,19 @@
 //
 // Softmax in two groups by key-tile parity. Group 0 (warps 2-5) takes the even key tiles and
 // group 1 (warps 6-9) the odd ones; each thread owns one query row and all 128 keys of the
-// tile. Each group owns one O accumulator (O_0 / O_1), kept relative to the running max at
-// the group's last tile, so a group's rescale never waits on the other group's PV. The only
-// exchange between the groups is the running max, handed on per tile through shared memory
-// right after the tile max (long before the exponentials), so one group's exponentials run
-// while the other loads, reduces and stores: the exp unit, the bound of this kernel, stays
-// busy. The epilogue merges O_0 and O_1 exactly.
+// tile. The groups exchange the running max per tile through shared memory right after the
+// tile max (long before the exponentials), so one group's exponentials run while the other
+// loads, reduces and stores: the exp unit, the bound of this kernel, stays busy.
+//
+// S is double-buffered by tile parity, so QK^T of tile j+1 runs while tile j is in the
+// softmax. O is a single accumulator kept relative to the running max of the last tile whose
+// PV went in. Tile j's P is computed against m(j); before PV(j) the rows whose max rose at
+// tile j are rescaled (after PV(j-1) is done). Late in a row the max rarely rises, so most
+// warps skip the rescale and PV(j) follows PV(j-1) without a round trip.
 //
 // Two MMA issuers: one thread issues QK^T, another PV, each waiting only on its own inputs,
 // so neither stream of tensor-core work stalls behind the other's waits (an issuing thread
-// blocks while the tensor core drains what it issued). S is single-buffered but freed as
-// soon as the owning group has copied it to registers.
+// blocks while the tensor core drains what it issued).
 //
 // One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
@@ -33,8 +35,7 @@
 //   warp 1     TMEM owner and QK^T issuer (one thread)
 //   warps 2-9  softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
 //   warp 10    PV issuer (one thread)
-// TMEM (512 columns): S [0,128), O_0 and O_1 (D + 16 columns each) from 128, scale factors
-// from 416.
+// TMEM (512 columns): S_0, S_1 [0,256), O (D + 16 columns) from 256, scale factors from 400.
 #pragma once
 #include "ptx.cuh"
 
@@ -78,20 +79,22 @@ struct FwdLayout {
   static constexpr int ST_VSF = ST_KSF + 1024;
   static constexpr int STAGE_BYTES = ST_VSF + 1024;
   static constexpr int OFF_P = OFF_STAGE + NS * STAGE_BYTES;               // 2 x 16 KB
-  static constexpr int OFF_RED = OFF_P + 2 * 16384;   // running max hand-off [2][128], final [2][128]
+  static constexpr int OFF_RED = OFF_P + 2 * 16384;   // running max hand-off [2][128]
   static constexpr int OFF_Q16 = OFF_RED + 2048;
   static constexpr int F16_TILE = 128 * D * 2;
   static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int N_BARS = 1 + 2 * NS + 14;
+  static constexpr int N_BARS = 1 + 2 * NS + 15;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   // TMEM columns
-  static constexpr uint32_t T_S = 0, T_O = 128, T_OSTRIDE = 144, T_QSF = 416, T_PSF = 424,
-                            T_KSF = 428, T_VSF = T_KSF + 8 * NS;
-  static_assert(T_VSF + 8 * NS <= 512, "TMEM columns");
+  // S_b at T_S + 128 b; K and V scale factors in two slots by tile parity (8 columns each: a
+  // slot is rewritten only after the MMA two tiles back that read it has completed).
+  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_PSF = 408, T_KSF = 412,
+                            T_VSF = 428;
+  static_assert(T_O + NV <= T_QSF && T_VSF + 16 <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
   static constexpr int PV_WARP = 10;
@@ -116,14 +119,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // Barriers a group waits on come in pairs by key-tile parity: a waiter must never run more
   // than one phase ahead of a barrier (a parity wait cannot tell phase k from phase k - 2).
   uint64_t* s_full = bars + 1 + 2 * L::NS; // [2], by tile parity
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_full + 3;           // [2], by tile parity
-  uint64_t* pv_done = s_full + 5;          // [2], by tile parity
-  uint64_t* m_ready = s_full + 7;          // [2], by tile parity: running max handed on
-  uint64_t* kv16_full = s_full + 9;
-  uint64_t* kv16_empty = s_full + 10;
-  uint64_t* q16_full = s_full + 11;
-  uint64_t* mma_final = s_full + 12;      // [2]: QK issuer, PV issuer
+  uint64_t* s_free = s_full + 2;           // [2], by tile parity
+  uint64_t* p_full = s_full + 4;           // [2], by tile parity
+  uint64_t* pv_done = s_full + 6;          // [2], by tile parity
+  uint64_t* m_ready = s_full + 8;          // [2], by tile parity: running max handed on
+  uint64_t* kv16_full = s_full + 10;
+  uint64_t* kv16_empty = s_full + 11;
+  uint64_t* q16_full = s_full + 12;
+  uint64_t* mma_final = s_full + 13;      // [2]: QK issuer, PV issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -142,8 +145,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     mbar_init(q_full, 33);
     // a stage is free once both the QK^T (K) and the PV (V) issuers are done with it
     for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 2); }
-    mbar_init(s_free, 4);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(s_free + i, 4);
       mbar_init(s_full + i, 1);
       mbar_init(p_full + i, 4);
       mbar_init(pv_done + i, 1);
@@ -304,12 +307,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!wait1(kv_full + s, (j / L::NS) & 1, j)) { ok = false; break; }
         fence_proxy_async_smem();
         tc_fence_after();
-        if (j >= 1 && !wait1(s_free, (j - 1) & 1, j)) { ok = false; break; }
+        // S_{j&1} (and K scale slot j&1) were last used by tile j-2
+        if (j >= 2 && !wait1(s_free + (j & 1), ((j - 2) >> 1) & 1, j)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tS = tbase + L::T_S;
+        const uint32_t tS = tbase + L::T_S + (j & 1) * 128;
         if (!f16) {
           unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-          const uint32_t tk = tbase + L::T_KSF + 8 * s;
+          const uint32_t tk = tbase + L::T_KSF + 8 * (j & 1);
           for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, st + L::ST_KSF + kk * 512);
           const uint32_t sK = smem_u32(st + L::ST_K);
           for (int kk = 0; kk < L::KSTEPS; ++kk) {
@@ -348,8 +352,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t sP = smem_u32(sm + L::OFF_P);
       tc_fence_after();
       tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
-      for (int s = 0; s < L::NS; ++s)              // second V scale chunk (rows 128..): 1.0
-        tmem_cp_sf(tbase + L::T_VSF + 8 * s + 4, sm + L::OFF_PSF);
+      for (int b2 = 0; b2 < 2; ++b2)               // second V scale chunk (rows 128..): 1.0
+        tmem_cp_sf(tbase + L::T_VSF + 8 * b2 + 4, sm + L::OFF_PSF);
       bool ok = true;
       int n16 = 0;
       for (int jj = 0; ok && jj < nt; ++jj) {
@@ -360,10 +364,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (f16 && !wait1(kv16_full, n16 & 1, jj)) { ok = false; break; }
         fence_proxy_async_smem();
         tc_fence_after();
-        const uint32_t tO = tbase + L::T_O + b2 * L::T_OSTRIDE;
+        const uint32_t tO = tbase + L::T_O;
         if (!f16) {
           unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-          const uint32_t tv = tbase + L::T_VSF + 8 * s;
+          const uint32_t tv = tbase + L::T_VSF + 8 * b2;   // PV(jj-2), its last reader, is done
           tmem_cp_sf(tv, st + L::ST_VSF);
           const uint32_t sV = smem_u32(st + L::ST_V);
 #pragma unroll
@@ -372,7 +376,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
             mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
                      (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
-                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 1 || kk > 0) ? 1u : 0u);
+                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 0 || kk > 0) ? 1u : 0u);
           }
         } else {
           ++n16;
@@ -381,7 +385,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
             const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
-            mma_f16(tO, da, db, idesc_pv16, (jj > 1 || kk > 0) ? 1u : 0u);
+            mma_f16(tO, da, db, idesc_pv16, (jj > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(kv16_empty);
         }
@@ -400,7 +404,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int qi = qt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     float* red_m = reinterpret_cast<float*>(sm + L::OFF_RED);         // [2 parities][128]
-    float* red_fin = red_m + 256;                                     // [2 groups][128]
     // Scores stay in the FP4 MMA's raw units (S = sum codes*scales); the running max m is
     // kept in those units and 448 p = 2^(s C + (log2 448 - m C)) with
     // C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true dot products and are
@@ -408,9 +411,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
     const float R16 = 1.f / ((*a.q_ts) * (*a.k_ts));
     const float2 C2 = make_float2(C, C);
-    float m_own = -INFINITY;        // running max at this group's last tile (O_grp's reference)
     unsigned char* sP = sm + L::OFF_P;
-    const uint32_t tO = tbase + L::T_O + grp * L::T_OSTRIDE + lane_addr;
+    const uint32_t tO = tbase + L::T_O + lane_addr;
     bool ok = true;
     for (int j = grp; j < nt; j += 2) {
       const int b2 = j & 1;                  // == grp
@@ -421,14 +423,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_after();
       {
         uint32_t* xr = reinterpret_cast<uint32_t*>(x);
-        const uint32_t tS = tbase + L::T_S + lane_addr;
+        const uint32_t tS = tbase + L::T_S + b2 * 128 + lane_addr;
 #pragma unroll
         for (int c = 0; c < 128; c += 32) tmem_ld32(tS + c, xr + c);
         tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
+      if (lane == 0) mbar_arrive(s_free + b2);
       if (f16) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) x[c] *= R16;
@@ -480,7 +482,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           pw[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
         }
       }
-      // P buffer b2 and O_{b2} were last used by PV(j-2). An FP16 tile's P fills both buffers:
+      // P buffer b2 was last used by PV(j-2). An FP16 tile's P fills both buffers:
       // writing one needs PV(j-1) done as well, and the tile after an FP16 tile too. PV(j-2)'s
       // completion implies PV(j-3)'s, so the wait on the other parity's barrier is for its
       // next phase.
@@ -505,10 +507,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       fence_proxy_async_smem();
-      // Bring O_{b2} from this group's previous max to m_new (PV(j-2) is done: waited above).
-      const float alpha = (m_own == -INFINITY || dead) ? 1.f : ex2_approx((m_own - m_new) * C);
-      if (!dead) m_own = m_new;
-      if (j >= 2 && !__all_sync(0xffffffffu, alpha == 1.f)) {
+      // O holds the tiles before j relative to m(j-1) = m_prev. Rows whose max rose at this
+      // tile are brought to m_new once PV(j-1) is done (the next phase of that parity's
+      // barrier: PV(j-2), waited above, implies PV(j-3)); a warp whose rows all kept their
+      // max hands P(j) on at once.
+      const float alpha = (m_prev == -INFINITY || dead) ? 1.f : ex2_approx((m_prev - m_new) * C);
+      if (j >= 1 && !__all_sync(0xffffffffu, alpha == 1.f)) {
+        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
         tc_fence_after();
         const float2 A2 = make_float2(alpha, alpha);
 #pragma unroll
@@ -538,46 +543,32 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + b2);
     }
-    // ---- epilogue: merge O_0 and O_1 at the final max, divide by l ----
+    // ---- epilogue: O / l (O and l already relative to the final max) ----
     // PV(nt-1)'s completion covers every earlier MMA of the issuing thread; the group that
     // owns tile nt-1 waits for it (the next phase of its own barrier) and the named barrier
     // passes that on to the other group.
     if (ok && grp == ((nt - 1) & 1)) ok = waitw(pv_done + grp, ((nt - 1) >> 1) & 1, nt);
-    red_fin[grp * 128 + row] = m_own;
     tc_fence_before();
     named_bar_sync(1, 256);
-    const float m0 = red_fin[row], m1 = red_fin[128 + row];
     if (ok && !*abort_flag) {
       tc_fence_after();
-      const float m_run = fmaxf(m0, m1);
-      const uint32_t tO0 = tbase + L::T_O + lane_addr;
-      const uint32_t tO1 = tO0 + L::T_OSTRIDE;
-      uint32_t lr0[16], lr1[16];
-      tmem_ld16(tO0 + D, lr0);
-      tmem_ld16(tO1 + D, lr1);
+      const float m_run = red_m[((nt - 1) & 1) * 128 + row];   // m(nt-1), published last
+      uint32_t lr[16];
+      tmem_ld16(tO + D, lr);
       tmem_wait_ld();
-      // O_1 is never written when there is a single key tile; its weight is then 0.
-      const float w0 = (m0 == -INFINITY) ? 0.f : ex2_approx((m0 - m_run) * C);
-      const float w1 = (m1 == -INFINITY || nt < 2) ? 0.f : ex2_approx((m1 - m_run) * C);
-      auto merge = [&](float o0, float o1) {
-        const float v = w0 * o0;
-        return w1 == 0.f ? v : fmaf(w1, o1, v);
-      };
-      const float l_run = merge(__uint_as_float(lr0[0]), __uint_as_float(lr1[0]));
+      const float l_run = __uint_as_float(lr[0]);
       const bool store = qi < a.Nq;
       const int64_t orow = static_cast<int64_t>(bhq) * a.Nq + qi;
 #pragma unroll
       for (int cc = 0; cc < D / 2; cc += 32) {
         const int c = grp * (D / 2) + cc;
-        uint32_t o0[32], o1[32];
-        tmem_ld32(tO0 + c, o0);
-        tmem_ld32(tO1 + c, o1);
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
         tmem_wait_ld();
         if (store) {
           float v[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            v[k] = __fdiv_rn(merge(__uint_as_float(o0[k]), __uint_as_float(o1[k])), l_run);
+          for (int k = 0; k < 32; ++k) v[k] = __fdiv_rn(__uint_as_float(o[k]), l_run);
           if (a.out_kind == 2) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c);
 #pragma unroll

@@ -95,23 +95,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Wait that gives up at once when *flag is set, and sets *flag when it times out itself.
-// `site` (wait_site()) is recorded when this wait is the first to time out.
+// Wait that gives up when *flag is set, and sets *flag when it times out itself. `site`
+// (wait_site()) is recorded when this wait is the first to time out. A phase that has
+// already completed is taken on the first poll (the common case in a running pipeline);
+// only then is the flag read, and again between sleeps.
+__device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, volatile int* flag,
+                                               uint64_t site) {
+  const long long t0 = clock64();
+  while (!*flag) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      flag_error(kStatusTimeout);
+      record_timeout(site);
+      *flag = 1;
+      return false;
+    }
+  }
+  return false;
+}
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* flag,
                                              uint64_t site) {
-  if (*flag) return false;
-  if (!mbar_wait(bar, parity)) {
-    record_timeout(site);
-    *flag = 1;
-    return false;
-  }
-  return true;
+  if (mbar_try_wait(bar, parity)) return true;
+  return bounded_wait_slow(bar, parity, flag, site);
 }
-// The same, taken by lane 0 for the whole (converged) warp, so that every lane agrees.
+// The same for a whole (converged) warp: every lane polls once (one instruction, so every
+// lane sees the same phase); a pending phase is then waited for by lane 0 alone and the
+// outcome broadcast, so that every lane agrees.
 __device__ __forceinline__ bool bounded_wait_warp(uint64_t* bar, uint32_t parity,
                                                   volatile int* flag, uint64_t site) {
+  if (__any_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = bounded_wait(bar, parity, flag, site) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = bounded_wait_slow(bar, parity, flag, site) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
