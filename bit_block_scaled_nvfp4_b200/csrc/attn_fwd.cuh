@@ -13,8 +13,8 @@
 // after its D channel rows, so the PV MMA (N = D + 16) accumulates sum_j P_j into O column D,
 // with the same rescaling as O.
 //
-// Softmax in two groups by key-tile parity. Group 0 (warps 2-5) takes the even key tiles and
-// group 1 (warps 6-9) the odd ones; each thread owns one query row and all 128 keys of the
+// Softmax in two groups by key-tile parity. Group 0 (warps 4-7) takes the even key tiles and
+// group 1 (warps 8-11) the odd ones; each thread owns one query row and all 128 keys of the
 // tile. The groups exchange the running max per tile through shared memory right after the
 // tile max (long before the exponentials), so one group's exponentials run while the other
 // loads, reduces and stores: the exp unit, the bound of this kernel, stays busy.
@@ -33,8 +33,9 @@
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
 //              tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles when selected
 //   warp 1     TMEM owner and QK^T issuer (one thread)
-//   warps 2-9  softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
-//   warp 10    PV issuer (one thread)
+//   warp 2     PV issuer (one thread)
+//   warps 4-11 softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4), with
+//              224 registers a thread taken from warpgroup 0 (setmaxnreg)
 // TMEM (512 columns): S_0, S_1 [0,256), O (D + 16 columns) from 256, scale factors from 400.
 #pragma once
 #include "ptx.cuh"
@@ -97,12 +98,20 @@ struct FwdLayout {
   static_assert(T_O + NV <= T_QSF && T_VSF + 16 <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
-  static constexpr int PV_WARP = 10;
-  static constexpr int THREADS = 352;
+  // Warpgroup 0: producer (warp 0), QK^T issuer (1), PV issuer (2), spare (3); warpgroups 1
+  // and 2: the two softmax groups. The softmax warpgroups take the registers warpgroup 0
+  // gives up: 128 x REGS_LOW + 256 x REGS_HIGH = 384 x REGS_LAUNCH.
+  static constexpr int PV_WARP = 2;
+  static constexpr int THREADS = 384;
+  static constexpr int REGS_LAUNCH = 168, REGS_LOW = 56, REGS_HIGH = 224;
+  static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * REGS_LAUNCH, "register split");
+  // The FP16-tile softmax does not fit the higher limit either; that kernel keeps the
+  // launch registers everywhere.
+  static constexpr bool REG_SPLIT = !kMixed;
 };
 
 template <int D, bool kMixed>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q16,
                 const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
@@ -200,6 +209,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     return bounded_wait(bar, parity, abort_flag, site(bar, tile));
   };
 
+  // The register split is taken inside the branch of each warpgroup, so that the compiler
+  // sizes each branch's code to its own limit.
+  if (warp < 4) {
+  if constexpr (L::REG_SPLIT) regs_dealloc<L::REGS_LOW>();
   if (warp == 0) {
     // ================================ producer ================================
     if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); }
@@ -396,10 +409,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_wait(mma_final + 1, 0);
     }
     __syncwarp();
+  }
   } else {
+  if constexpr (L::REG_SPLIT) regs_alloc<L::REGS_HIGH>();
+  {
     // ================================ softmax ================================
     const int wq = warp & 3;                 // TMEM lane quadrant
-    const int grp = (warp - 2) >> 2;         // key-tile parity this group handles
+    const int grp = (warp - 4) >> 2;         // key-tile parity this group handles
     const int row = wq * 32 + lane;
     const int qi = qt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
@@ -594,6 +610,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (store && grp == 0 && a.lse != nullptr)
         a.lse[orow] = m_run * C * kLn2 + logf(l_run * (1.f / 448.f));
     }
+  }
   }
   tc_fence_before();
   __syncthreads();

@@ -99,7 +99,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 // (wait_site()) is recorded when this wait is the first to time out. A phase that has
 // already completed is taken on the first poll (the common case in a running pipeline);
 // only then is the flag read, and again between sleeps.
-__device__ __noinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, volatile int* flag,
+__device__ __forceinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, volatile int* flag,
                                                uint64_t site) {
   const long long t0 = clock64();
   while (!*flag) {
@@ -142,6 +142,17 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Register reallocation between warpgroups (executed by all threads of a warpgroup). An
+// increase waits until decreases elsewhere have freed the registers, so the split must fit
+// the registers the block was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
