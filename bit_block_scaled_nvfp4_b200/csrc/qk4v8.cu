@@ -284,11 +284,6 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   static bool attr = false;
   if (!attr) {
     if (!set_smem(attn_fwd_kernel<D, kMixed>, L::SMEM_ALLOC)) return QK4V8_ERR_CUDA;
-    // The kernel hands registers from its first warpgroup to the softmax warpgroups; that
-    // split is sized for the register count it is launched with, so refuse any other build.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kMixed>) != cudaSuccess) return QK4V8_ERR_CUDA;
-    if (L::REG_SPLIT && fa.numRegs != L::REGS_LAUNCH) return QK4V8_ERR_UNSUPPORTED;
     attr = true;
   }
   FwdArgs a;
