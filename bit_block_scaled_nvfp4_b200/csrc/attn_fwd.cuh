@@ -30,11 +30,10 @@
 // blocks while the tensor core drains what it issued).
 //
 // One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
-//   warp 0     Q/K producer: TMA of Q and K code tiles (swizzled), scale factors gathered into
-//              the tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles if selected
+//   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
+//              tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles when selected
 //   warp 1     TMEM owner and QK^T issuer (one thread)
 //   warp 2     PV issuer (one thread)
-//   warp 3     V producer: TMA of V code tiles, V scale factors
 //   warps 4-11 softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
 // TMEM (512 columns): S_0, S_1 [0,256), O (D + 16 columns) from 256, scale factors from 400.
 #pragma once
@@ -45,6 +44,10 @@ namespace qk4v8 {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
+// Share of the exponentials taken on the FMA pipe, in eighths. 0: all on the special-function
+// unit, the fastest setting measured on B200 for this kernel's instruction mix (2/8 ran 2%
+// slower: the extra FMA-pipe instructions cost more issue slots than the exp unit saved).
+constexpr int kPolyOf8 = 0;
 
 struct FwdArgs {
   const uint8_t* q_scales;
@@ -63,11 +66,7 @@ struct FwdArgs {
 
 template <int D, bool kMixed>
 struct FwdLayout {
-  // Separate K and V rings: a K stage is free once QK^T of its tile is done, a V stage only
-  // after PV, several tile periods later; one shared ring tied the load of tile j to the
-  // softmax of tile j - NS. (The FP16 operands need the room in the mixed kernel.)
-  static constexpr int NK = kMixed ? 2 : 4;
-  static constexpr int NVS = kMixed ? 2 : 3;
+  static constexpr int NS = kMixed ? 2 : 4;   // the FP16 operand stage needs the room
   static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
   static constexpr int NV = D + 16;                     // PV MMA N: D channels + ones rows
   static constexpr int Q_BYTES = 128 * D / 2;
@@ -77,13 +76,13 @@ struct FwdLayout {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_QSF = OFF_Q + Q_BYTES;                         // KSTEPS chunks
   static constexpr int OFF_PSF = OFF_QSF + 1024;                          // all 1.0 (E8M0 127)
-  static constexpr int OFF_KST = OFF_PSF + 1024;          // K stages: codes, then scale factors
-  static constexpr int KST_SF = K_BYTES;
-  static constexpr int KST_BYTES = K_BYTES + 1024;
-  static constexpr int OFF_VST = OFF_KST + NK * KST_BYTES;  // V stages: codes + ones rows, scales
-  static constexpr int VST_SF = V_BYTES;
-  static constexpr int VST_BYTES = V_BYTES + 1024;
-  static constexpr int OFF_P = OFF_VST + NVS * VST_BYTES;                  // 2 x 16 KB
+  static constexpr int OFF_STAGE = OFF_PSF + 1024;
+  static constexpr int ST_K = 0;
+  static constexpr int ST_V = K_BYTES;
+  static constexpr int ST_KSF = ST_V + V_BYTES;
+  static constexpr int ST_VSF = ST_KSF + 1024;
+  static constexpr int STAGE_BYTES = ST_VSF + 1024;
+  static constexpr int OFF_P = OFF_STAGE + NS * STAGE_BYTES;               // 2 x 16 KB
   static constexpr int OFF_RED = OFF_P + 2 * 16384;   // running max hand-off [2][128]
   static constexpr int OFF_Q16 = OFF_RED + 2048;
   static constexpr int F16_TILE = 128 * D * 2;
@@ -91,7 +90,7 @@ struct FwdLayout {
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int N_BARS = 1 + 2 * NK + 2 * NVS + 15;
+  static constexpr int N_BARS = 1 + 2 * NS + 15;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   // TMEM columns
@@ -102,8 +101,8 @@ struct FwdLayout {
   static_assert(T_O + NV <= T_QSF && T_VSF + 16 <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
-  // Warpgroup 0: Q/K producer (warp 0), QK^T issuer (1), PV issuer (2), V producer (3);
-  // warpgroups 1 and 2: the two softmax groups.
+  // Warpgroup 0: producer (warp 0), QK^T issuer (1), PV issuer (2), spare (3); warpgroups 1
+  // and 2: the two softmax groups.
   static constexpr int PV_WARP = 2;
   static constexpr int THREADS = 384;
 };
@@ -121,13 +120,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + L::NK;
-  uint64_t* v_full = k_empty + L::NK;
-  uint64_t* v_empty = v_full + L::NVS;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + L::NS;
   // Barriers a group waits on come in pairs by key-tile parity: a waiter must never run more
   // than one phase ahead of a barrier (a parity wait cannot tell phase k from phase k - 2).
-  uint64_t* s_full = v_empty + L::NVS;     // [2], by tile parity
+  uint64_t* s_full = bars + 1 + 2 * L::NS; // [2], by tile parity
   uint64_t* s_free = s_full + 2;           // [2], by tile parity
   uint64_t* p_full = s_full + 4;           // [2], by tile parity
   uint64_t* pv_done = s_full + 6;          // [2], by tile parity
@@ -153,8 +150,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // full barriers: the TMA's expect-tx arrival plus one cp.async arrival per producer lane
     mbar_init(q_full, 33);
     // a stage is free once both the QK^T (K) and the PV (V) issuers are done with it
-    for (int s = 0; s < L::NK; ++s) { mbar_init(k_full + s, 33); mbar_init(k_empty + s, 1); }
-    for (int s = 0; s < L::NVS; ++s) { mbar_init(v_full + s, 33); mbar_init(v_empty + s, 1); }
+    for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 2); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_free + i, 4);
       mbar_init(s_full + i, 1);
@@ -172,15 +168,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // Every byte of a ones row is equal, so the 128-byte swizzle leaves them unchanged.
   for (int i = threadIdx.x; i < 128; i += blockDim.x)
     reinterpret_cast<uint32_t*>(sm + L::OFF_PSF)[i] = 0x7F7F7F7Fu;
-  for (int s = 0; s < L::NVS; ++s)
+  for (int s = 0; s < L::NS; ++s)
     for (int i = threadIdx.x; i < 16 * 128 / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(sm + L::OFF_VST + s * L::VST_BYTES + L::V_TMA_BYTES)[i] =
+      reinterpret_cast<uint4*>(sm + L::OFF_STAGE + s * L::STAGE_BYTES + L::ST_V + L::V_TMA_BYTES)[i] =
           make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
   if constexpr (D < 128) {
-    for (int s = 0; s < L::NVS; ++s)
+    for (int s = 0; s < L::NS; ++s)
       for (int i = threadIdx.x; i < 128; i += blockDim.x)
         if (((i >> 2) & 31) + 32 * (i & 3) >= D)       // word i: row (i/4)%32 + 32 (i%4)
-          reinterpret_cast<uint32_t*>(sm + L::OFF_VST + s * L::VST_BYTES + L::VST_SF)[i] = 0x7F7F7F7Fu;
+          reinterpret_cast<uint32_t*>(sm + L::OFF_STAGE + s * L::STAGE_BYTES + L::ST_VSF)[i] = 0x7F7F7F7Fu;
   }
   if constexpr (kMixed) {
     for (int h = 0; h < 2; ++h)
@@ -199,8 +195,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tbase = *tmem_slot;
 
   // Barrier ids in timeout reports are their index in the barrier block.
-  const uint32_t role = (warp == 0 || warp == 3) ? kRoleProducer
-                        : (warp == 1 || warp == L::PV_WARP) ? kRoleMma : kRoleSoftmax;
+  const uint32_t role = warp == 0 ? kRoleProducer : (warp == 1 || warp == L::PV_WARP) ? kRoleMma : kRoleSoftmax;
   auto site = [&](uint64_t* bar, int tile) {
     return wait_site(kKernelFwd, role, static_cast<uint32_t>(bar - bars), tile);
   };
@@ -213,7 +208,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (warp == 0) {
     // ================================ producer ================================
-    if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); }
+    if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); }
     // Scale factors go straight from global memory into the tcgen05 scale layout with 4-byte
     // asynchronous copies (row r = r0 + 32 r1 of a 128-row chunk -> byte r0*16 + r1*4; one
     // 4-byte word holds the 4 scales of one 64-element MMA step), completing on the same
@@ -239,10 +234,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool q16_loaded = false;
     int n16 = 0, issued = 0;
     for (int j = 0; j < nt; ++j) {
-      const int s = j % L::NK;
-      if (j >= L::NK && !waitw(k_empty + s, ((j / L::NK) - 1) & 1, j)) break;
-      unsigned char* st = sm + L::OFF_KST + s * L::KST_BYTES;
-      // K scale factors of keys j*128 .. j*128+127; rows past Nk read as zero.
+      const int s = j % L::NS;
+      if (j >= L::NS && !waitw(kv_empty + s, ((j / L::NS) - 1) & 1, j)) break;
+      unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+      // K scale factors of keys j*128 .. j*128+127; V scale factors of this key tile (channel
+      // row c, 4 E8M0 codes of 32 tokens each). Rows past Nk read as zero; V rows from D on
+      // (the ones rows) hold 1.0 set once at start.
       const int64_t krow0 = static_cast<int64_t>(bhk) * a.Nk + j * 128;
 #pragma unroll
       for (int r1 = 0; r1 < 4; ++r1) {
@@ -251,13 +248,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint8_t* src = a.k_scales + (ok ? (krow0 + r) * (D / 16) : 0);
 #pragma unroll
         for (int kk = 0; kk < L::KSTEPS; ++kk)
-          cp_async4(st + L::KST_SF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, ok);
+          cp_async4(st + L::ST_KSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, ok);
+        if (r < D)
+          cp_async4(st + L::ST_VSF + lane * 16 + r1 * 4,
+                    a.v_scales + (static_cast<int64_t>(bhk) * D + r) * (a.Npad / 32) + j * 4, true);
       }
-      cp_async_arrive_noinc(k_full + s);
+      cp_async_arrive_noinc(kv_full + s);
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(k_full + s, L::K_BYTES);
-        tma_load_3d(st, &tm_k, k_full + s, 0, j * 128, bhk);
+        mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_TMA_BYTES);
+        tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, bhk);
+        tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, bhk * D);
       }
       issued = j + 1;
       if constexpr (kMixed) {
@@ -283,9 +284,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
     }
     // Drain: never leave a copy in flight into this CTA's shared memory.
-    for (int s = 0; s < L::NK && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / L::NK) * L::NK;
-      mbar_wait(k_full + s, (last / L::NK) & 1);
+    for (int s = 0; s < L::NS && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / L::NS) * L::NS;
+      mbar_wait(kv_full + s, (last / L::NS) & 1);
     }
     mbar_wait(q_full, 0);
     if (kMixed && n16 > 0) { mbar_wait(kv16_full, (n16 - 1) & 1); mbar_wait(q16_full, 0); }
@@ -307,9 +308,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int n16 = 0;
       bool q16_ready = false;
       for (int j = 0; ok && j < nt; ++j) {
-        const int s = j % L::NK;
+        const int s = j % L::NS;
         const bool f16 = kMixed && bm_row[j];
-        if (!wait1(k_full + s, (j / L::NK) & 1, j)) { ok = false; break; }
+        if (!wait1(kv_full + s, (j / L::NS) & 1, j)) { ok = false; break; }
         fence_proxy_async_smem();
         tc_fence_after();
         // S_{j&1} (and K scale slot j&1) were last used by tile j-2
@@ -317,10 +318,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         const uint32_t tS = tbase + L::T_S + (j & 1) * 128;
         if (!f16) {
-          unsigned char* st = sm + L::OFF_KST + s * L::KST_BYTES;
+          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
           const uint32_t tk = tbase + L::T_KSF + 8 * (j & 1);
-          for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, st + L::KST_SF + kk * 512);
-          const uint32_t sK = smem_u32(st);
+          for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, st + L::ST_KSF + kk * 512);
+          const uint32_t sK = smem_u32(st + L::ST_K);
           for (int kk = 0; kk < L::KSTEPS; ++kk) {
             const uint64_t da = make_sdesc(sQ + kk * 32, 16, L::QK_SBO, L::QK_SW);
             const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
@@ -342,7 +343,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
         }
         mma_commit(s_full + (j & 1));
-        mma_commit(k_empty + s);
+        mma_commit(kv_empty + s);                  // K half of the stage is free
       }
       // Everything this thread issued has completed before TMEM is released.
       mma_commit(mma_final);
@@ -362,19 +363,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bool ok = true;
       int n16 = 0;
       for (int jj = 0; ok && jj < nt; ++jj) {
-        const int s = jj % L::NVS, b2 = jj & 1;
+        const int s = jj % L::NS, b2 = jj & 1;
         const bool f16 = kMixed && bm_row[jj];
         if (!wait1(p_full + b2, (jj >> 1) & 1, jj)) { ok = false; break; }
-        if (!wait1(v_full + s, (jj / L::NVS) & 1, jj)) { ok = false; break; }
+        if (!wait1(kv_full + s, (jj / L::NS) & 1, jj)) { ok = false; break; }
         if (f16 && !wait1(kv16_full, n16 & 1, jj)) { ok = false; break; }
         fence_proxy_async_smem();
         tc_fence_after();
         const uint32_t tO = tbase + L::T_O;
         if (!f16) {
-          unsigned char* st = sm + L::OFF_VST + s * L::VST_BYTES;
+          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
           const uint32_t tv = tbase + L::T_VSF + 8 * b2;   // PV(jj-2), its last reader, is done
-          tmem_cp_sf(tv, st + L::VST_SF);
-          const uint32_t sV = smem_u32(st);
+          tmem_cp_sf(tv, st + L::ST_VSF);
+          const uint32_t sV = smem_u32(st + L::ST_V);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t da = make_sdesc(sP + b2 * 16384 + kk * 32, 16, 1024, kSw128);
@@ -395,41 +396,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mma_commit(kv16_empty);
         }
         mma_commit(pv_done + b2);
-        mma_commit(v_empty + s);
+        mma_commit(kv_empty + s);                  // V half of the stage is free
       }
       mma_commit(mma_final + 1);
       mbar_wait(mma_final + 1, 0);
     }
     __syncwarp();
-  } else if (warp == 3) {
-    // ============================ V producer ============================
-    if (lane == 0) prefetch_tmap(&tm_v);
-    int issued = 0;
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % L::NVS;
-      if (j >= L::NVS && !waitw(v_empty + s, ((j / L::NVS) - 1) & 1, j)) break;
-      unsigned char* st = sm + L::OFF_VST + s * L::VST_BYTES;
-      // V scale factors of this key tile (channel row c, 4 E8M0 codes of 32 tokens each);
-      // rows from D on (the ones rows) hold 1.0 set once at start.
-#pragma unroll
-      for (int r1 = 0; r1 < 4; ++r1) {
-        const int r = r1 * 32 + lane;
-        if (r < D)
-          cp_async4(st + L::VST_SF + lane * 16 + r1 * 4,
-                    a.v_scales + (static_cast<int64_t>(bhk) * D + r) * (a.Npad / 32) + j * 4, true);
-      }
-      cp_async_arrive_noinc(v_full + s);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(v_full + s, L::V_TMA_BYTES);
-        tma_load_2d(st, &tm_v, v_full + s, j * 128, bhk * D);
-      }
-      issued = j + 1;
-    }
-    for (int s = 0; s < L::NVS && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / L::NVS) * L::NVS;
-      mbar_wait(v_full + s, (last / L::NVS) & 1);
-    }
   } else if (warp >= 4) {
     // ================================ softmax ================================
     const int wq = warp & 3;                 // TMEM lane quadrant
@@ -501,12 +473,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float2 B2 = make_float2(bias, bias);
       uint32_t pw[kMixed ? 64 : 32];      // e4m3: 32 words; fp16: 64 words
       if (!f16) {
+        // kPolyOf8 of every 8 groups of 4 scores take the FMA-pipe exponential, the rest the
+        // special-function unit, so both pipes work on the tile.
 #pragma unroll
         for (int c = 0; c < 128; c += 4) {
           const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
           const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), C2, B2);
-          pw[c >> 2] = cvt_e4m3x2(ex2_approx(t0.x), ex2_approx(t0.y)) |
-                       (cvt_e4m3x2(ex2_approx(t1.x), ex2_approx(t1.y)) << 16);
+          float2 e0, e1;
+          if (((c >> 2) & 7) < kPolyOf8) {
+            e0 = exp2_poly2(t0);
+            e1 = exp2_poly2(t1);
+          } else {
+            e0 = make_float2(ex2_approx(t0.x), ex2_approx(t0.y));
+            e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
+          }
+          pw[c >> 2] = cvt_e4m3x2(e0.x, e0.y) | (cvt_e4m3x2(e1.x, e1.y) << 16);
         }
       } else if constexpr (kMixed) {
 #pragma unroll

@@ -107,6 +107,13 @@ uint64_t qk4v8_timeout_site(void) {
   return site;
 }
 
+qk4v8_status qk4v8_selftest_exp2(const float* t, float* out, int32_t n, cudaStream_t stream) {
+  if (t == nullptr || out == nullptr || n < 0 || (n & 1)) return QK4V8_ERR_INVALID_ARG;
+  if (n == 0) return QK4V8_OK;
+  exp2_selftest_kernel<<<(n / 2 + 255) / 256, 256, 0, stream>>>(t, out, n);
+  return launch_status();
+}
+
 qk4v8_status qk4v8_selftest_wait_timeout(cudaStream_t stream) {
   wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>();
   return launch_status();
