@@ -32,12 +32,13 @@ struct DecArgs {
 
 struct DecLayout {
   static constexpr int D = 128;
-  static constexpr int NS = 3;
+  static constexpr int NS = 2;                    // two stages, three CTAs per SM
   static constexpr int OFF_Q = 0;                 // 16 rows x 64 B (SW64)
   static constexpr int OFF_QSF = 1024;            // 2 chunks
   static constexpr int OFF_PSF = 2048;            // 1 chunk
   static constexpr int OFF_P = 3072;              // 2 x [16 rows x 128 B] (SW128), 1024-aligned
-  static constexpr int OFF_STAGE = OFF_P + 2 * 2048;      // 7168, 1024-aligned
+  static constexpr int OFF_ONES = OFF_P + 2 * 2048;       // 128 x 32 B of E4M3 1.0 (SW32)
+  static constexpr int OFF_STAGE = OFF_ONES + 4096;       // 11264, 1024-aligned
   static constexpr int ST_K = 0;                  // 128 keys x 64 B (SW64)
   static constexpr int ST_V0 = 8192;              // 128 channels x 64 B (page 0 tokens)
   static constexpr int ST_V1 = 16384;             // page 1 tokens
@@ -46,16 +47,20 @@ struct DecLayout {
   static constexpr int ST_VRAW = 26624;           // the two pages' V scales as stored (2 x 256 B)
   static constexpr int STAGE_BYTES = 27648;
   static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
-  static constexpr int OFF_RED = OFF_BAR + 256;   // reductions: [4 warps][16] max, [4][16] sum
+  static constexpr int OFF_RED = OFF_BAR + 256;   // block max exchange [2 parities][4 warps][16]
   static constexpr int OFF_PID = OFF_RED + 2 * 4 * 16 * 4;   // page ids of the split
   static constexpr int MAX_SPLIT_PAGES = 256;                // split_tokens <= 16384
   static constexpr int SMEM_BYTES = OFF_PID + MAX_SPLIT_PAGES * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-  static constexpr uint32_t T_S = 0, T_O = 32, T_QSF = 48, T_PSF = 56, T_KSF = 64, T_VSF = 88;
+  // S^T x2 [0,32), O^T [32,48), L^T [48,64) (every row: l), Q / P scales, K and V scales by
+  // stage
+  static constexpr uint32_t T_S = 0, T_O = 32, T_L = 48, T_QSF = 64, T_PSF = 72, T_KSF = 76,
+                            T_VSF = T_KSF + 8 * NS;
+  static_assert(T_VSF + 4 * NS <= 128, "TMEM columns");
   static constexpr int NQ = 16;                   // MMA N (query heads, padded)
 };
 
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(192, 3)
 decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
               const __grid_constant__ CUtensorMap tm_vp, DecArgs a) {
   using L = DecLayout;
@@ -75,7 +80,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red_max = reinterpret_cast<float*>(sm + L::OFF_RED);
-  float* red_sum = red_max + 64;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
@@ -116,6 +120,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     reinterpret_cast<uint32_t*>(sm + L::OFF_PSF)[i] = 0x7F7F7F7Fu;
   for (int i = threadIdx.x; i < 2 * 16 * 128 / 16; i += blockDim.x)   // zero both P^T buffers
     reinterpret_cast<uint4*>(sm + L::OFF_P)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < 4096 / 16; i += blockDim.x)            // the ones operand
+    reinterpret_cast<uint4*>(sm + L::OFF_ONES)[i] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
   fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_slot, 128);
@@ -248,6 +254,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                    (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
                    (bb > 0 || kk > 0) ? 1u : 0u);
         }
+        // l on the tensor core: L^T += 1 P^T (A = 128 rows of E4M3 1.0, the same 32-key slice
+        // for every step), so every row of L^T holds the row sums of the quantized P, rescaled
+        // with O^T.
+        const uint64_t d1 = make_sdesc(smem_u32(sm + L::OFF_ONES), 16, 256, kSw32);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t db = make_sdesc(sP + b2 * 2048 + kk * 32, 16, 1024, kSw128);
+          mma_mxf8(tbase + L::T_L, d1, db, idesc_with_sf_ids(idesc_pv, kk, kk),
+                   (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                   (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                   (bb > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(pv_done + b2);
         mma_commit(kv_empty + st_i);
       }
@@ -302,15 +320,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int r = wq * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
-    float m_run[16], l_run[16];
+    float m_run[16];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) { m_run[q] = -INFINITY; l_run[q] = 0.f; }
+    for (int q = 0; q < 16; ++q) m_run[q] = -INFINITY;
     unsigned char* sP = sm + L::OFF_P;
     bool failed = false;
     for (int blk = 0; blk < nblk; ++blk) {
       const int b2 = blk & 1;
       // On a timeout the body still runs (on whatever TMEM holds) so that the four warps
-      // meet at both named barriers; the shared flag then ends the loop for all of them.
+      // meet at the named barrier; the shared flag, set before it, then ends the loop for all.
       if (!waits(s_full + b2, (blk >> 1) & 1, blk)) failed = true;
       tc_fence_after();
       float x[16];
@@ -320,20 +338,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free + b2);
       const bool valid = k_begin + blk * 128 + r < k_end;
+      // Block max per query: over this warp's 32 keys in one warp reduction, then over the
+      // four warps through shared memory (slots alternate by block parity, so a fast warp's
+      // next write cannot land before the others have read).
+      float* rm = red_max + b2 * 64;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
         x[q] = (valid && q < g) ? x[q] : -INFINITY;        // raw MMA units
-        float mm = x[q];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
-        if (lane == 0) red_max[wq * 16 + q] = mm;
+        float mm;
+        asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(mm) : "f"(x[q]));
+        if (lane == 0) rm[wq * 16 + q] = mm;
       }
+      if (failed && lane == 0) *soft_flag = 1;
       named_bar_sync(1, 128);
+      if (*soft_flag) break;
       float alpha[16], moff[16];
       bool all_one = true;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const float mb = fmaxf(fmaxf(red_max[q], red_max[16 + q]), fmaxf(red_max[32 + q], red_max[48 + q]));
+        const float mb = fmaxf(fmaxf(rm[q], rm[16 + q]), fmaxf(rm[32 + q], rm[48 + q]));
         const float m_new = fmaxf(m_run[q], mb);
         const bool dead = (m_new == -INFINITY);
         moff[q] = dead ? 0.f : m_new;
@@ -347,20 +370,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         float p[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) p[i] = ex2_approx((x[q + i] - moff[q + i]) * C) * 448.f;
-        const uint32_t lo = cvt_e4m3x2(p[0], p[1]);
-        const uint32_t hi = cvt_e4m3x2(p[2], p[3]);
-        codes[q >> 2] = lo | (hi << 16);
-        const float2 f0 = __half22float2(e4m3x2_to_half2(lo));
-        const float2 f1 = __half22float2(e4m3x2_to_half2(hi));
-        float sv[4] = {f0.x, f0.y, f1.x, f1.y};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float t = sv[i];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          if (lane == 0) red_sum[wq * 16 + q + i] = t;
-        }
+        codes[q >> 2] = cvt_e4m3x2(p[0], p[1]) | (cvt_e4m3x2(p[2], p[3]) << 16);
       }
+      // P^T buffer b2 was read by PV(blk-2); O^T and L^T are rescaled below after PV(blk-1).
       if (blk >= 1) {
         if (!waits(pv_done + ((blk - 1) & 1), ((blk - 1) >> 1) & 1, blk)) failed = true;
         tc_fence_after();
@@ -373,39 +385,34 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           pb[q * 128 + ((((r >> 4) ^ (q & 7))) << 4) + (r & 15)] =
               static_cast<unsigned char>(codes[q >> 2] >> (8 * (q & 3)));
       }
-      if (failed && lane == 0) *soft_flag = 1;
-      named_bar_sync(2, 128);
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float lb = (red_sum[q] + red_sum[16 + q]) + (red_sum[32 + q] + red_sum[48 + q]);
-        l_run[q] = l_run[q] * alpha[q] + lb;
-      }
-      if (*soft_flag) break;
       fence_proxy_async_smem();
-      if (blk >= 1 && !all_one) {
-        float o[16];
+      if (blk >= 1 && !__all_sync(0xffffffffu, all_one)) {
+        float o[16], l[16];
         tmem_ld16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
+        tmem_ld16(tbase + L::T_L + lane_addr, reinterpret_cast<uint32_t*>(l));
         tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) o[q] *= alpha[q];
+        for (int q = 0; q < 16; ++q) { o[q] *= alpha[q]; l[q] *= alpha[q]; }
         tmem_st16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
+        tmem_st16(tbase + L::T_L + lane_addr, reinterpret_cast<uint32_t*>(l));
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + b2);
     }
-    if (!*soft_flag && waits(pv_done + ((nblk - 1) & 1), ((nblk - 1) >> 1) & 1, nblk)) {
+    if (!*soft_flag && !failed && waits(pv_done + ((nblk - 1) & 1), ((nblk - 1) >> 1) & 1, nblk)) {
       tc_fence_after();
-      float o[16];
+      float o[16], l[16];
       tmem_ld16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
+      tmem_ld16(tbase + L::T_L + lane_addr, reinterpret_cast<uint32_t*>(l));
       tmem_wait_ld();
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
         if (q < g) {
           part[q * q_stride + r] = o[q];
           // the merge works in log2 units: store m * C
-          if (r == 0) { part[q * q_stride + D] = m_run[q] * C; part[q * q_stride + D + 1] = l_run[q]; }
+          if (r == 0) { part[q * q_stride + D] = m_run[q] * C; part[q * q_stride + D + 1] = l[q]; }
         }
       }
     }
