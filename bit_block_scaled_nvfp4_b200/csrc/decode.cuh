@@ -8,9 +8,16 @@
 // and keeps (m, l, O) for the g query heads of its KV head. tcgen05 block-scaled MMAs need
 // M = 128, so the g <= 16 query heads form the N dimension (N = 16) and keys / channels form
 // M: S^T = K Q^T (M = 128 keys) and O^T += V^T P^T (M = 128 channels); each softmax thread
-// owns one key, and the row reductions over keys run across the 128 softmax threads.
+// owns one key; the block max per query is one warp reduction (redux.sync) and an exchange
+// of the four warps' maxima through shared memory. l comes from the tensor core: a second MMA
+// with an all-ones A operand (L^T += 1 P^T) sums the quantized P per query, rescaled with O.
 // Partials (O unnormalised, m, l) go to the workspace; the merge kernel combines the splits:
 // M = max m_s, O = sum e^(m_s - M) O_s / sum e^(m_s - M) l_s.
+//
+// Warp roles (two CTAs per SM): warp 0 K producer (TMA of the two pages' K codes, K scale
+// factors by 4-byte asynchronous copies into the tcgen05 layout), warp 7 V producer (TMA of V
+// codes, bulk copy of the pages' V scales), warp 1 QK^T issuer, warp 6 PV issuer (and the V
+// scale rearrangement), warps 2-5 softmax. K and V stages form separate rings.
 #pragma once
 #include "ptx.cuh"
 #include "attn_fwd.cuh"
@@ -32,21 +39,25 @@ struct DecArgs {
 
 struct DecLayout {
   static constexpr int D = 128;
-  static constexpr int NS = 2;                    // two stages, three CTAs per SM
+  // Separate K and V rings (two CTAs per SM): a K stage is free after QK^T of its block, a
+  // V stage only after PV, so the next blocks' K loads do not wait for the softmax.
+  static constexpr int NK = 3, NVS = 3;
   static constexpr int OFF_Q = 0;                 // 16 rows x 64 B (SW64)
   static constexpr int OFF_QSF = 1024;            // 2 chunks
   static constexpr int OFF_PSF = 2048;            // 1 chunk
   static constexpr int OFF_P = 3072;              // 2 x [16 rows x 128 B] (SW128), 1024-aligned
   static constexpr int OFF_ONES = OFF_P + 2 * 2048;       // 128 x 32 B of E4M3 1.0 (SW32)
-  static constexpr int OFF_STAGE = OFF_ONES + 4096;       // 11264, 1024-aligned
+  static constexpr int OFF_KST = OFF_ONES + 4096;         // 11264, 1024-aligned
   static constexpr int ST_K = 0;                  // 128 keys x 64 B (SW64)
-  static constexpr int ST_V0 = 8192;              // 128 channels x 64 B (page 0 tokens)
-  static constexpr int ST_V1 = 16384;             // page 1 tokens
-  static constexpr int ST_KSF = 24576;            // 2 chunks
-  static constexpr int ST_VSF = 25600;            // 1 chunk (tcgen05 layout)
-  static constexpr int ST_VRAW = 26624;           // the two pages' V scales as stored (2 x 256 B)
-  static constexpr int STAGE_BYTES = 27648;
-  static constexpr int OFF_BAR = OFF_STAGE + NS * STAGE_BYTES;
+  static constexpr int ST_KSF = 8192;             // 2 chunks
+  static constexpr int KST_BYTES = 9216;
+  static constexpr int OFF_VST = OFF_KST + NK * KST_BYTES;
+  static constexpr int ST_V0 = 0;                 // 128 channels x 64 B (page 0 tokens)
+  static constexpr int ST_V1 = 8192;              // page 1 tokens
+  static constexpr int ST_VSF = 16384;            // 1 chunk (tcgen05 layout)
+  static constexpr int ST_VRAW = 16896;           // the two pages' V scales as stored (2 x 256 B)
+  static constexpr int VST_BYTES = 17408;
+  static constexpr int OFF_BAR = OFF_VST + NVS * VST_BYTES;
   static constexpr int OFF_RED = OFF_BAR + 256;   // block max exchange [2 parities][4 warps][16]
   static constexpr int OFF_PID = OFF_RED + 2 * 4 * 16 * 4;   // page ids of the split
   static constexpr int MAX_SPLIT_PAGES = 256;                // split_tokens <= 16384
@@ -55,12 +66,15 @@ struct DecLayout {
   // S^T x2 [0,32), O^T [32,48), L^T [48,64) (every row: l), Q / P scales, K and V scales by
   // stage
   static constexpr uint32_t T_S = 0, T_O = 32, T_L = 48, T_QSF = 64, T_PSF = 72, T_KSF = 76,
-                            T_VSF = T_KSF + 8 * NS;
-  static_assert(T_VSF + 4 * NS <= 128, "TMEM columns");
+                            T_VSF = T_KSF + 8 * NK;
+  static_assert(T_VSF + 4 * NVS <= 128, "TMEM columns");
   static constexpr int NQ = 16;                   // MMA N (query heads, padded)
+  static constexpr int PV_WARP = 6;
+  static constexpr int VLOAD_WARP = 7;
+  static constexpr int THREADS = 256;
 };
 
-__global__ void __launch_bounds__(192, 3)
+__global__ void __launch_bounds__(256, 2)
 decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
               const __grid_constant__ CUtensorMap tm_vp, DecArgs a) {
   using L = DecLayout;
@@ -70,14 +84,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + L::NS;
-  uint64_t* s_full = bars + 1 + 2 * L::NS;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + L::NK;
+  uint64_t* v_full = k_empty + L::NK;
+  uint64_t* v_empty = v_full + L::NVS;
+  uint64_t* s_full = v_empty + L::NVS;
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_full + 4;
   uint64_t* pv_done = s_full + 6;
-  uint64_t* mma_final = s_full + 8;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 9);
+  uint64_t* mma_final = s_full + 8;        // [2]: QK^T issuer, PV issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red_max = reinterpret_cast<float*>(sm + L::OFF_RED);
 
@@ -105,13 +121,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    // kv_full: the producer's expect-tx arrival plus one cp.async arrival per producer lane
-    for (int i = 0; i < L::NS; ++i) { mbar_init(kv_full + i, 33); mbar_init(kv_empty + i, 1); }
+    // k_full: the producer's expect-tx arrival plus one cp.async arrival per producer lane
+    for (int i = 0; i < L::NK; ++i) { mbar_init(k_full + i, 33); mbar_init(k_empty + i, 1); }
+    for (int i = 0; i < L::NVS; ++i) { mbar_init(v_full + i, 1); mbar_init(v_empty + i, 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1); mbar_init(s_free + i, 4);
       mbar_init(p_full + i, 4); mbar_init(pv_done + i, 1);
     }
     mbar_init(mma_final, 1);
+    mbar_init(mma_final + 1, 1);
     abort_flag[0] = 0;
     abort_flag[1] = 0;
     fence_mbar_init();
@@ -122,6 +140,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     reinterpret_cast<uint4*>(sm + L::OFF_P)[i] = make_uint4(0, 0, 0, 0);
   for (int i = threadIdx.x; i < 4096 / 16; i += blockDim.x)            // the ones operand
     reinterpret_cast<uint4*>(sm + L::OFF_ONES)[i] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+  // Page ids of this split, checked once, into shared memory (read by both producers).
+  int32_t* pid = reinterpret_cast<int32_t*>(sm + L::OFF_PID);
+  {
+    const int n_split_pages = (k_end - k_begin + 63) / 64;
+    for (int i = threadIdx.x; i < n_split_pages; i += blockDim.x) {
+      int p = a.page_table[static_cast<int64_t>(s) * a.max_pages + k_begin / 64 + i];
+      if (p < 0 || p >= a.num_pages) { flag_error(kStatusBounds); p = 0; }
+      pid[i] = p;
+    }
+  }
   fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_slot, 128);
@@ -136,7 +164,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   // Softmax: warp-uniform waits on its own flag, which it only reads after a barrier of all
   // four softmax warps, so that the four always leave the loop together.
   volatile int* soft_flag = abort_flag + 1;
-  const uint32_t role = warp == 0 ? kRoleProducer : warp == 1 ? kRoleMma : kRoleSoftmax;
+  const uint32_t role = (warp == 0 || warp == L::VLOAD_WARP) ? kRoleProducer
+                        : (warp == 1 || warp == L::PV_WARP) ? kRoleMma : kRoleSoftmax;
   auto site = [&](uint64_t* bar, int blk) {
     return wait_site(kKernelDecode, role, static_cast<uint32_t>(bar - bars), blk);
   };
@@ -153,11 +182,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (!ok) record_timeout(site(bar, blk));
     }
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
-  };
-  auto page_of = [&](int logical) -> int {
-    int p = a.page_table[static_cast<int64_t>(s) * a.max_pages + logical];
-    if (p < 0 || p >= a.num_pages) { flag_error(kStatusBounds); p = 0; }
-    return p;
   };
 
   if (warp == 0) {
@@ -178,15 +202,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tma_load_2d(sm + L::OFF_Q, &tm_q, q_full, 0, static_cast<int>(qrow0));
       }
     }
-    // Page ids of this split, checked once, into shared memory.
-    int32_t* pid = reinterpret_cast<int32_t*>(sm + L::OFF_PID);
-    const int n_split_pages = (k_end - k_begin + 63) / 64;
-    for (int i = lane; i < n_split_pages; i += 32) pid[i] = page_of(k_begin / 64 + i);
-    __syncwarp();
+    int issued = 0;
     for (int blk = 0; blk < nblk; ++blk) {
-      const int st_i = blk % L::NS;
-      if (blk >= L::NS && !waitw(kv_empty + st_i, ((blk / L::NS) - 1) & 1, blk)) break;
-      unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
+      const int st_i = blk % L::NK;
+      if (blk >= L::NK && !waitw(k_empty + st_i, ((blk / L::NK) - 1) & 1, blk)) break;
+      unsigned char* st = sm + L::OFF_KST + st_i * L::KST_BYTES;
       const int k0 = k_begin + blk * 128;
       const int p0 = pid[2 * blk];
       const int p1 = (k0 + 64 < len) ? pid[2 * blk + 1] : p0;
@@ -201,47 +221,117 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) cp_async4(st + L::ST_KSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, true);
       }
-      cp_async_arrive_noinc(kv_full + st_i);
+      cp_async_arrive_noinc(k_full + st_i);
       __syncwarp();
       if (lane == 0) {
-        // K and V codes by TMA; the pages' V scales (256 B each, as stored) by bulk copy, to be
-        // rearranged by the MMA warp.
-        mbar_arrive_expect_tx(kv_full + st_i, 128 * 64 + 2 * D * 64 + 2 * D * 2);
-        tma_load_2d(st + L::ST_K, &tm_kp, kv_full + st_i, 0, (p0 * a.Hkv + h) * 64);
-        tma_load_2d(st + L::ST_K + 4096, &tm_kp, kv_full + st_i, 0, (p1 * a.Hkv + h) * 64);
-        tma_load_2d(st + L::ST_V0, &tm_vp, kv_full + st_i, 0, (p0 * a.Hkv + h) * D);
-        tma_load_2d(st + L::ST_V1, &tm_vp, kv_full + st_i, 0, (p1 * a.Hkv + h) * D);
-        bulk_load(st + L::ST_VRAW, a.v_page_scales + (static_cast<int64_t>(p0) * a.Hkv + h) * D * 2, D * 2, kv_full + st_i);
-        bulk_load(st + L::ST_VRAW + D * 2, a.v_page_scales + (static_cast<int64_t>(p1) * a.Hkv + h) * D * 2, D * 2, kv_full + st_i);
+        mbar_arrive_expect_tx(k_full + st_i, 128 * 64);
+        tma_load_2d(st + L::ST_K, &tm_kp, k_full + st_i, 0, (p0 * a.Hkv + h) * 64);
+        tma_load_2d(st + L::ST_K + 4096, &tm_kp, k_full + st_i, 0, (p1 * a.Hkv + h) * 64);
       }
+      issued = blk + 1;
     }
-    for (int i = 0; i < L::NS && i < nblk; ++i) {
-      const int last = i + ((nblk - 1 - i) / L::NS) * L::NS;
-      mbar_wait(kv_full + i, (last / L::NS) & 1);
+    // Drain: never leave a copy in flight into this CTA's shared memory.
+    for (int i = 0; i < L::NK && i < issued; ++i) {
+      const int last = i + ((issued - 1 - i) / L::NK) * L::NK;
+      mbar_wait(k_full + i, (last / L::NK) & 1);
     }
     mbar_wait(q_full, 0);
-  } else if (warp == 1) {
-    // ================================ MMA issuer ================================
-    // The whole warp runs the loop: all lanes rearrange the V scales of each block into the
-    // tcgen05 layout; lane 0 alone issues the tcgen05 copies and MMAs and their commits.
-    const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, L::NQ);
-    const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NQ);
-    const uint32_t sQ = smem_u32(sm + L::OFF_Q);
-    const uint32_t sP = smem_u32(sm + L::OFF_P);
-    bool ok = waitw(q_full, 0, -1);
-    if (ok && lane == 0) {
-      tc_fence_after();
-      tmem_cp_sf(tbase + L::T_QSF, sm + L::OFF_QSF);
-      tmem_cp_sf(tbase + L::T_QSF + 4, sm + L::OFF_QSF + 512);
-      tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+  } else if (warp == L::VLOAD_WARP) {
+    // ============================== V producer ==============================
+    // V codes of the block's two pages by TMA; their V scales (256 B each, as stored) by bulk
+    // copy, to be rearranged into the tcgen05 layout by the PV warp.
+    if (lane == 0) {
+      int issued = 0;
+      for (int blk = 0; blk < nblk; ++blk) {
+        const int st_i = blk % L::NVS;
+        if (blk >= L::NVS && !wait1(v_empty + st_i, ((blk / L::NVS) - 1) & 1, blk)) break;
+        unsigned char* st = sm + L::OFF_VST + st_i * L::VST_BYTES;
+        const int k0 = k_begin + blk * 128;
+        const int p0 = pid[2 * blk];
+        const int p1 = (k0 + 64 < len) ? pid[2 * blk + 1] : p0;
+        mbar_arrive_expect_tx(v_full + st_i, 2 * D * 64 + 2 * D * 2);
+        tma_load_2d(st + L::ST_V0, &tm_vp, v_full + st_i, 0, (p0 * a.Hkv + h) * D);
+        tma_load_2d(st + L::ST_V1, &tm_vp, v_full + st_i, 0, (p1 * a.Hkv + h) * D);
+        bulk_load(st + L::ST_VRAW, a.v_page_scales + (static_cast<int64_t>(p0) * a.Hkv + h) * D * 2, D * 2, v_full + st_i);
+        bulk_load(st + L::ST_VRAW + D * 2, a.v_page_scales + (static_cast<int64_t>(p1) * a.Hkv + h) * D * 2, D * 2, v_full + st_i);
+        issued = blk + 1;
+      }
+      for (int i = 0; i < L::NVS && i < issued; ++i) {
+        const int last = i + ((issued - 1 - i) / L::NVS) * L::NVS;
+        mbar_wait(v_full + i, (last / L::NVS) & 1);
+      }
     }
     __syncwarp();
-    auto issue_pv = [&](int bb) -> bool {
-      const int st_i = bb % L::NS, b2 = bb & 1;
-      if (!waitw(p_full + b2, (bb >> 1) & 1, bb)) return false;
+  } else if (warp == 1) {
+    // ============================ QK^T issuer (one thread) ============================
+    const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, L::NQ);
+    const uint32_t sQ = smem_u32(sm + L::OFF_Q);
+    if (lane == 0) {
+      bool ok = wait1(q_full, 0, -1);
+      if (ok) {
+        tc_fence_after();
+        tmem_cp_sf(tbase + L::T_QSF, sm + L::OFF_QSF);
+        tmem_cp_sf(tbase + L::T_QSF + 4, sm + L::OFF_QSF + 512);
+      }
+      for (int blk = 0; ok && blk < nblk; ++blk) {
+        const int st_i = blk % L::NK, b2 = blk & 1;
+        if (!wait1(k_full + st_i, (blk / L::NK) & 1, blk)) { ok = false; break; }
+        // the K scale factors arrived by cp.async (generic proxy); the tensor core reads them
+        // through the async proxy
+        fence_proxy_async_smem();
+        if (blk >= 2 && !wait1(s_free + b2, ((blk - 2) >> 1) & 1, blk)) { ok = false; break; }
+        tc_fence_after();
+        unsigned char* st = sm + L::OFF_KST + st_i * L::KST_BYTES;
+        const uint32_t tk = tbase + L::T_KSF + 8 * st_i;
+        tmem_cp_sf(tk, st + L::ST_KSF);
+        tmem_cp_sf(tk + 4, st + L::ST_KSF + 512);
+        const uint32_t sK = smem_u32(st + L::ST_K);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint64_t da = make_sdesc(sK + kk * 32, 16, 512, kSw64);
+          const uint64_t db = make_sdesc(sQ + kk * 32, 16, 512, kSw64);
+          mma_nvf4(tbase + L::T_S + b2 * 16, da, db, idesc_qk, tk + 4 * kk,
+                   tbase + L::T_QSF + 4 * kk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full + b2);
+        mma_commit(k_empty + st_i);
+      }
+      mma_commit(mma_final);
+      mbar_wait(mma_final, 0);
+    }
+    __syncwarp();
+  } else if (warp == L::PV_WARP) {
+    // ============================== PV issuer ==============================
+    // The whole warp rearranges the V scales of each block into the tcgen05 layout; lane 0
+    // issues the tcgen05 copies and MMAs and their commits. PV(blk) goes out as soon as P(blk)
+    // is ready, independently of the QK^T stream (which waits for the next block's loads).
+    const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NQ);
+    const uint32_t sP = smem_u32(sm + L::OFF_P);
+    if (lane == 0) {
+      tc_fence_after();
+      tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+    }
+    bool ok = true;
+    for (int bb = 0; ok && bb < nblk; ++bb) {
+      const int st_i = bb % L::NVS, b2 = bb & 1;
+      if (!waitw(p_full + b2, (bb >> 1) & 1, bb)) { ok = false; break; }
+      if (!waitw(v_full + st_i, (bb / L::NVS) & 1, bb)) { ok = false; break; }
+      unsigned char* st = sm + L::OFF_VST + st_i * L::VST_BYTES;
+      {
+        // channel c = r0 + 32 r1: word [page0 g0, page0 g1, page1 g0, page1 g1] at r0*16 + r1*4
+        const uint16_t* raw = reinterpret_cast<const uint16_t*>(st + L::ST_VRAW);
+        uint32_t vw[4];
+#pragma unroll
+        for (int r1 = 0; r1 < 4; ++r1) {
+          const int c = r1 * 32 + lane;
+          vw[r1] = static_cast<uint32_t>(raw[c]) | (static_cast<uint32_t>(raw[D + c]) << 16);
+        }
+        *reinterpret_cast<uint4*>(st + L::ST_VSF + lane * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
       if (lane == 0) {
         tc_fence_after();
-        unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
         const uint32_t tv = tbase + L::T_VSF + 4 * st_i;
         tmem_cp_sf(tv, st + L::ST_VSF);
 #pragma unroll
@@ -267,51 +357,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                    (bb > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(pv_done + b2);
-        mma_commit(kv_empty + st_i);
+        mma_commit(v_empty + st_i);
       }
       __syncwarp();
-      return true;
-    };
-    for (int blk = 0; ok && blk < nblk; ++blk) {
-      const int st_i = blk % L::NS, b2 = blk & 1;
-      if (!waitw(kv_full + st_i, (blk / L::NS) & 1, blk)) { ok = false; break; }
-      unsigned char* st = sm + L::OFF_STAGE + st_i * L::STAGE_BYTES;
-      {
-        // channel c = r0 + 32 r1: word [page0 g0, page0 g1, page1 g0, page1 g1] at r0*16 + r1*4
-        const uint16_t* raw = reinterpret_cast<const uint16_t*>(st + L::ST_VRAW);
-        uint32_t vw[4];
-#pragma unroll
-        for (int r1 = 0; r1 < 4; ++r1) {
-          const int c = r1 * 32 + lane;
-          vw[r1] = static_cast<uint32_t>(raw[c]) | (static_cast<uint32_t>(raw[D + c]) << 16);
-        }
-        *reinterpret_cast<uint4*>(st + L::ST_VSF + lane * 16) = make_uint4(vw[0], vw[1], vw[2], vw[3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-      if (blk >= 2 && !waitw(s_free + b2, ((blk - 2) >> 1) & 1, blk)) { ok = false; break; }
-      if (lane == 0) {
-        tc_fence_after();
-        const uint32_t tk = tbase + L::T_KSF + 8 * st_i;
-        tmem_cp_sf(tk, st + L::ST_KSF);
-        tmem_cp_sf(tk + 4, st + L::ST_KSF + 512);
-        const uint32_t sK = smem_u32(st + L::ST_K);
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint64_t da = make_sdesc(sK + kk * 32, 16, 512, kSw64);
-          const uint64_t db = make_sdesc(sQ + kk * 32, 16, 512, kSw64);
-          mma_nvf4(tbase + L::T_S + b2 * 16, da, db, idesc_qk, tk + 4 * kk,
-                   tbase + L::T_QSF + 4 * kk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(s_full + b2);
-      }
-      __syncwarp();
-      if (blk >= 1 && !issue_pv(blk - 1)) { ok = false; break; }
     }
-    if (ok) issue_pv(nblk - 1);
     if (lane == 0) {
-      mma_commit(mma_final);
-      mbar_wait(mma_final, 0);
+      mma_commit(mma_final + 1);
+      mbar_wait(mma_final + 1, 0);
     }
     __syncwarp();
   } else {

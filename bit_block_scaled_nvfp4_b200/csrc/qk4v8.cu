@@ -399,7 +399,7 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   a.n_splits = n_splits; a.split_tokens = p->split_tokens; a.num_pages = p->num_pages;
   a.softmax_scale = p->softmax_scale;
   dim3 grid(n_splits, p->kv_heads, p->num_seqs);
-  decode_kernel<<<grid, 192, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  decode_kernel<<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   decode_merge_kernel<<<p->num_seqs * p->q_heads, 128, 0, stream>>>(
       a.ws, n_splits, static_cast<int32_t>(p->out_dtype), p->out, p->lse);
