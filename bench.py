@@ -33,6 +33,14 @@ sys.path.insert(0, ROOT)
 from bit_block_scaled_nvfp4_b200 import workloads  # noqa: E402
 
 METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of HBM peak"
+
+# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu capture summarised
+# in profiles/ (attn_fwd_prefill_h16_n4096.md, decode_paged_decode_s64.md). Only workloads with
+# a capture of the current kernel have an entry; the others report null.
+NCU_TRAFFIC_BYTES = {
+    "prefill_h16_n4096": 18_160_384 + 512,
+    "paged_decode_s64": 2_170_615_000 + 13_027_072,
+}
 FP4_OVER_BF16 = 4.0          # nominal dense ratio 9 PF / 2.25 PF
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -401,7 +409,7 @@ def main():
         ach = units / (kern_ms * 1e-3) / 1e12
         peak = pk["bf16_tflops"] * FP4_OVER_BF16
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": None,
+                "frac": ach / peak, "traffic": NCU_TRAFFIC_BYTES.get(name),
                 "kernel": "attn_fwd_kernel", "peak_source": f"{src} bf16 x {FP4_OVER_BF16:g} (FP4 dense)",
                 "mixed_fp4_fp8_bound_tflops": peak / 1.5}
     else:
@@ -412,7 +420,8 @@ def main():
         ach = st["kv_bytes"] / (kern_ms * 1e-3) / 1e9
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": None, "kernel": "decode_kernel + decode_merge_kernel",
+                "traffic": NCU_TRAFFIC_BYTES.get(name), "traffic_kernel": "decode_kernel",
+                "kernel": "decode_kernel + decode_merge_kernel",
                 "peak_source": f"{src} hbm_gbs"}
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
