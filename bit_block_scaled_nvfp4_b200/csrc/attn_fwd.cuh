@@ -13,23 +13,25 @@
 // after its D channel rows, so the PV MMA (N = D + 16) accumulates sum_j P_j into O column D,
 // with the same rescaling as O.
 //
-// Softmax in two groups by key-tile parity. Group 0 (warps 4-7) takes the even key tiles and
-// group 1 (warps 8-11) the odd ones; each thread owns one query row and all 128 keys of the
-// tile. The groups exchange the running max per tile through shared memory right after the
-// tile max (long before the exponentials), so one group's exponentials run while the other
-// loads, reduces and stores: the exp unit, the bound of this kernel, stays busy.
+// Persistent: one CTA per SM walks a list of work items (128-query tile, batch, query head),
+// heaviest causal items first, dealt to the CTAs in a zigzag so their loads even out. All
+// pipelines run on across items (a CTA-wide key-tile counter g numbers the stages and
+// buffers), so the next item's Q, K and V loads and its first QK^T overlap the current
+// item's last tiles and epilogue; Q has two buffers.
 //
-// S is double-buffered by tile parity, so QK^T of tile j+1 runs while tile j is in the
+// Softmax in two groups by the parity of g. Group 0 (warps 4-7) and group 1 (warps 8-11);
+// each thread owns one query row and all 128 keys of its tile. The groups hand the running max
+// on per tile through shared memory right after the tile max (long before the exponentials),
+// so one group's exponentials run while the other loads, reduces and stores.
+//
+// S is double-buffered by tile parity, so QK^T of the next tile runs while a tile is in the
 // softmax. O is a single accumulator kept relative to the running max of the last tile whose
-// PV went in. Tile j's P is computed against m(j); before PV(j) the rows whose max rose at
-// tile j are rescaled (after PV(j-1) is done). Late in a row the max rarely rises, so most
-// warps skip the rescale and PV(j) follows PV(j-1) without a round trip.
+// PV went in; before PV(j) the rows whose max rose at tile j are rescaled (after PV(j-1) is
+// done); late in a row the max rarely rises, so most warps skip the rescale. Two MMA issuer
+// threads (QK^T and PV) each wait only on their own inputs (an issuing thread blocks while the
+// tensor core drains what it issued).
 //
-// Two MMA issuers: one thread issues QK^T, another PV, each waiting only on its own inputs,
-// so neither stream of tensor-core work stalls behind the other's waits (an issuing thread
-// blocks while the tensor core drains what it issued).
-//
-// One CTA per (128-query tile, batch, query head), heaviest causal tiles first. Warp roles:
+// Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
 //              tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles when selected
 //   warp 1     TMEM owner and QK^T issuer (one thread)
@@ -64,6 +66,27 @@ struct FwdArgs {
   int32_t out_kind;          // 0 fp16, 1 bf16, 2 fp32
 };
 
+// A work item of the persistent prefill kernel: the 128-query tile, batch and query head it
+// covers, heaviest causal items first (item = (Tq - 1 - qt) * B*Hq + b*Hq + hq).
+struct FwdItem {
+  int qt, bhq, bhk, nt;
+};
+__device__ __forceinline__ FwdItem fwd_item(const FwdArgs& a, int idx) {
+  const int BHq = a.B * a.Hq;
+  FwdItem w;
+  w.qt = a.Tq - 1 - idx / BHq;
+  w.bhq = idx % BHq;
+  const int b = w.bhq / a.Hq, hq = w.bhq % a.Hq;
+  w.bhk = b * a.Hkv + hq / (a.Hq / a.Hkv);
+  w.nt = a.causal ? min(w.qt + 1, a.Tk) : a.Tk;
+  return w;
+}
+// Item of round `it` for CTA c of G: c, 2G-1-c, 2G+c, 4G-1-c, ... (zigzag over the heaviest-
+// first order, so the CTAs' total work evens out).
+__device__ __forceinline__ int fwd_item_index(int it, int G, int c) {
+  return it * G + ((it & 1) ? (G - 1 - c) : c);
+}
+
 template <int D, bool kMixed>
 struct FwdLayout {
   static constexpr int NS = kMixed ? 2 : 4;   // the FP16 operand stage needs the room
@@ -73,9 +96,9 @@ struct FwdLayout {
   static constexpr int K_BYTES = 128 * D / 2;
   static constexpr int V_TMA_BYTES = D * 128;
   static constexpr int V_BYTES = NV * 128;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_QSF = OFF_Q + Q_BYTES;                         // KSTEPS chunks
-  static constexpr int OFF_PSF = OFF_QSF + 1024;                          // all 1.0 (E8M0 127)
+  static constexpr int OFF_Q = 0;                                         // 2 buffers
+  static constexpr int OFF_QSF = OFF_Q + 2 * Q_BYTES;                     // 2 x KSTEPS chunks
+  static constexpr int OFF_PSF = OFF_QSF + 2048;                          // all 1.0 (E8M0 127)
   static constexpr int OFF_STAGE = OFF_PSF + 1024;
   static constexpr int ST_K = 0;
   static constexpr int ST_V = K_BYTES;
@@ -83,26 +106,25 @@ struct FwdLayout {
   static constexpr int ST_VSF = ST_KSF + 1024;
   static constexpr int STAGE_BYTES = ST_VSF + 1024;
   static constexpr int OFF_P = OFF_STAGE + NS * STAGE_BYTES;               // 2 x 16 KB
-  static constexpr int OFF_RED = OFF_P + 2 * 16384;   // running max hand-off [2][128]
+  static constexpr int OFF_RED = OFF_P + 2 * 16384;   // running max hand-off [2][128], final [128]
   static constexpr int OFF_Q16 = OFF_RED + 2048;
   static constexpr int F16_TILE = 128 * D * 2;
   static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int N_BARS = 1 + 2 * NS + 15;
+  static constexpr int N_BARS = 2 * NS + 21;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
-  // TMEM columns
-  // S_b at T_S + 128 b; K and V scale factors in two slots by tile parity (8 columns each: a
-  // slot is rewritten only after the MMA two tiles back that read it has completed).
-  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_PSF = 408, T_KSF = 412,
-                            T_VSF = 428;
+  static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
+  // TMEM columns. S_b at T_S + 128 b; Q scale factors in two slots by item parity, K and V
+  // scale factors in two slots by tile parity (8 columns each: a slot is rewritten only after
+  // the MMA two items / tiles back that read it has completed).
+  static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_PSF = 416, T_KSF = 420,
+                            T_VSF = 436;
   static_assert(T_O + NV <= T_QSF && T_VSF + 16 <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
-  // Warpgroup 0: producer (warp 0), QK^T issuer (1), PV issuer (2), spare (3); warpgroups 1
-  // and 2: the two softmax groups.
   static constexpr int PV_WARP = 2;
   static constexpr int THREADS = 384;
 };
@@ -119,36 +141,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // still sees shared-memory accesses (not generic ones)
   unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + L::NS;
-  // Barriers a group waits on come in pairs by key-tile parity: a waiter must never run more
+  // Barriers a waiter uses come in pairs by parity where needed: a waiter must never run more
   // than one phase ahead of a barrier (a parity wait cannot tell phase k from phase k - 2).
-  uint64_t* s_full = bars + 1 + 2 * L::NS; // [2], by tile parity
+  uint64_t* q_full = bars + 0;             // [2], by item parity
+  uint64_t* q_empty = bars + 2;            // [2], by item parity
+  uint64_t* kv_full = bars + 4;
+  uint64_t* kv_empty = kv_full + L::NS;
+  uint64_t* s_full = kv_empty + L::NS;     // [2], by tile parity
   uint64_t* s_free = s_full + 2;           // [2], by tile parity
   uint64_t* p_full = s_full + 4;           // [2], by tile parity
   uint64_t* pv_done = s_full + 6;          // [2], by tile parity
   uint64_t* m_ready = s_full + 8;          // [2], by tile parity: running max handed on
-  uint64_t* kv16_full = s_full + 10;
-  uint64_t* kv16_empty = s_full + 11;
-  uint64_t* q16_full = s_full + 12;
-  uint64_t* mma_final = s_full + 13;      // [2]: QK issuer, PV issuer
+  uint64_t* o_free = s_full + 10;          // the epilogue has read O
+  uint64_t* kv16_full = s_full + 11;
+  uint64_t* kv16_empty = s_full + 12;
+  uint64_t* q16_full = s_full + 13;
+  uint64_t* q16_empty = s_full + 14;
+  uint64_t* mma_final = s_full + 15;       // [2]: QK issuer, PV issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BHq = a.B * a.Hq;
-  const int qt = a.Tq - 1 - static_cast<int>(blockIdx.x / BHq);
-  const int bhq = static_cast<int>(blockIdx.x % BHq);
-  const int b = bhq / a.Hq, hq = bhq % a.Hq;
-  const int hk = hq / (a.Hq / a.Hkv);
-  const int bhk = b * a.Hkv + hk;
-  const int nt = a.causal ? min(qt + 1, a.Tk) : a.Tk;
-  const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(bhq) * a.Tq + qt) * a.Tk : nullptr;
+  const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+  const int n_items = a.Tq * a.B * a.Hq;
 
   if (threadIdx.x == 0) {
     // full barriers: the TMA's expect-tx arrival plus one cp.async arrival per producer lane
-    mbar_init(q_full, 33);
+    for (int i = 0; i < 2; ++i) { mbar_init(q_full + i, 33); mbar_init(q_empty + i, 1); }
     // a stage is free once both the QK^T (K) and the PV (V) issuers are done with it
     for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 2); }
     for (int i = 0; i < 2; ++i) {
@@ -158,7 +177,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(pv_done + i, 1);
       mbar_init(m_ready + i, 4);
     }
-    mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1); mbar_init(q16_full, 1);
+    mbar_init(o_free, 8);
+    mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1);
+    mbar_init(q16_full, 1); mbar_init(q16_empty, 1);
     mbar_init(mma_final, 1); mbar_init(mma_final + 1, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -194,7 +215,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  // Barrier ids in timeout reports are their index in the barrier block.
+  // Barrier ids in timeout reports are their index in the barrier block; the tile number is
+  // the CTA's running key-tile counter.
   const uint32_t role = warp == 0 ? kRoleProducer : (warp == 1 || warp == L::PV_WARP) ? kRoleMma : kRoleSoftmax;
   auto site = [&](uint64_t* bar, int tile) {
     return wait_site(kKernelFwd, role, static_cast<uint32_t>(bar - bars), tile);
@@ -213,137 +235,168 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // asynchronous copies (row r = r0 + 32 r1 of a 128-row chunk -> byte r0*16 + r1*4; one
     // 4-byte word holds the 4 scales of one 64-element MMA step), completing on the same
     // barrier as the TMA of the codes, so this warp never waits on their latency.
-    {
-      const int64_t row0 = static_cast<int64_t>(bhq) * a.Nq + qt * 128;
+    int g = 0, n16 = 0, nq16 = 0, q_issued = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int idx = fwd_item_index(it, G, cta);
+      if (idx >= n_items) break;
+      const FwdItem w = fwd_item(a, idx);
+      const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk : nullptr;
+      const int qb = it & 1;
+      // Q buffer qb was last read by the QK^T MMAs of item it - 2.
+      if (it >= 2 && !waitw(q_empty + qb, ((it - 2) >> 1) & 1, g)) { ok = false; break; }
+      {
+        const int64_t row0 = static_cast<int64_t>(w.bhq) * a.Nq + w.qt * 128;
 #pragma unroll
-      for (int r1 = 0; r1 < 4; ++r1) {
-        const int r = r1 * 32 + lane;
-        const bool ok = qt * 128 + r < a.Nq;
-        const uint8_t* src = a.q_scales + (ok ? (row0 + r) * (D / 16) : 0);
+        for (int r1 = 0; r1 < 4; ++r1) {
+          const int r = r1 * 32 + lane;
+          const bool valid = w.qt * 128 + r < a.Nq;
+          const uint8_t* src = a.q_scales + (valid ? (row0 + r) * (D / 16) : 0);
 #pragma unroll
-        for (int kk = 0; kk < L::KSTEPS; ++kk)
-          cp_async4(sm + L::OFF_QSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, ok);
+          for (int kk = 0; kk < L::KSTEPS; ++kk)
+            cp_async4(sm + L::OFF_QSF + qb * 1024 + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
+        }
+        cp_async_arrive_noinc(q_full + qb);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(q_full + qb, L::Q_BYTES);
+          tma_load_3d(sm + L::OFF_Q + qb * L::Q_BYTES, &tm_q, q_full + qb, 0, w.qt * 128, w.bhq);
+        }
+        q_issued = it + 1;
       }
-      cp_async_arrive_noinc(q_full);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, L::Q_BYTES);
-        tma_load_3d(sm + L::OFF_Q, &tm_q, q_full, 0, qt * 128, bhq);
-      }
-    }
-    bool q16_loaded = false;
-    int n16 = 0, issued = 0;
-    for (int j = 0; j < nt; ++j) {
-      const int s = j % L::NS;
-      if (j >= L::NS && !waitw(kv_empty + s, ((j / L::NS) - 1) & 1, j)) break;
-      unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-      // K scale factors of keys j*128 .. j*128+127; V scale factors of this key tile (channel
-      // row c, 4 E8M0 codes of 32 tokens each). Rows past Nk read as zero; V rows from D on
-      // (the ones rows) hold 1.0 set once at start.
-      const int64_t krow0 = static_cast<int64_t>(bhk) * a.Nk + j * 128;
+      bool q16_loaded = false;
+      for (int j = 0; j < w.nt; ++j, ++g) {
+        const int s = g % L::NS;
+        if (g >= L::NS && !waitw(kv_empty + s, ((g / L::NS) - 1) & 1, g)) { ok = false; break; }
+        unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+        // K scale factors of keys j*128 .. j*128+127; V scale factors of this key tile
+        // (channel row c, 4 E8M0 codes of 32 tokens each). Rows past Nk read as zero; V rows
+        // from D on (the ones rows) hold 1.0 set once at start.
+        const int64_t krow0 = static_cast<int64_t>(w.bhk) * a.Nk + j * 128;
 #pragma unroll
-      for (int r1 = 0; r1 < 4; ++r1) {
-        const int r = r1 * 32 + lane;
-        const bool ok = j * 128 + r < a.Nk;
-        const uint8_t* src = a.k_scales + (ok ? (krow0 + r) * (D / 16) : 0);
+        for (int r1 = 0; r1 < 4; ++r1) {
+          const int r = r1 * 32 + lane;
+          const bool valid = j * 128 + r < a.Nk;
+          const uint8_t* src = a.k_scales + (valid ? (krow0 + r) * (D / 16) : 0);
 #pragma unroll
-        for (int kk = 0; kk < L::KSTEPS; ++kk)
-          cp_async4(st + L::ST_KSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, ok);
-        if (r < D)
-          cp_async4(st + L::ST_VSF + lane * 16 + r1 * 4,
-                    a.v_scales + (static_cast<int64_t>(bhk) * D + r) * (a.Npad / 32) + j * 4, true);
-      }
-      cp_async_arrive_noinc(kv_full + s);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_TMA_BYTES);
-        tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, bhk);
-        tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, bhk * D);
-      }
-      issued = j + 1;
-      if constexpr (kMixed) {
-        if (bm_row[j]) {
-          if (!q16_loaded) {
-            if (lane == 0) {
-              mbar_arrive_expect_tx(q16_full, L::F16_TILE);
-              for (int h = 0; h < D / 64; ++h)
-                tma_load_3d(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, qt * 128, bhq);
+          for (int kk = 0; kk < L::KSTEPS; ++kk)
+            cp_async4(st + L::ST_KSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
+          if (r < D)
+            cp_async4(st + L::ST_VSF + lane * 16 + r1 * 4,
+                      a.v_scales + (static_cast<int64_t>(w.bhk) * D + r) * (a.Npad / 32) + j * 4, true);
+        }
+        cp_async_arrive_noinc(kv_full + s);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_TMA_BYTES);
+          tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, w.bhk);
+          tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, w.bhk * D);
+        }
+        if constexpr (kMixed) {
+          if (bm_row[j]) {
+            if (!q16_loaded) {
+              // the single FP16 Q buffer was last read by the FP16 QK^Ts of an earlier item
+              if (nq16 >= 1 && !waitw(q16_empty, (nq16 - 1) & 1, g)) { ok = false; ++g; break; }
+              if (lane == 0) {
+                mbar_arrive_expect_tx(q16_full, L::F16_TILE);
+                for (int h = 0; h < D / 64; ++h)
+                  tma_load_3d(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, w.qt * 128, w.bhq);
+              }
+              q16_loaded = true;
+              ++nq16;
             }
-            q16_loaded = true;
+            if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1, g)) { ok = false; ++g; break; }
+            if (lane == 0) {
+              mbar_arrive_expect_tx(kv16_full, L::F16_TILE + 2 * D * 128);
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_3d(sm + L::OFF_K16 + h * 16384, &tm_k16, kv16_full, h * 64, j * 128, w.bhk);
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(sm + L::OFF_V16 + h * L::V16_ATOM, &tm_v16, kv16_full, j * 128 + h * 64, w.bhk * D);
+            }
+            ++n16;
           }
-          if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1, j)) break;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(kv16_full, L::F16_TILE + 2 * D * 128);
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_3d(sm + L::OFF_K16 + h * 16384, &tm_k16, kv16_full, h * 64, j * 128, bhk);
-            for (int h = 0; h < 2; ++h)
-              tma_load_2d(sm + L::OFF_V16 + h * L::V16_ATOM, &tm_v16, kv16_full, j * 128 + h * 64, bhk * D);
-          }
-          ++n16;
         }
       }
     }
-    // Drain: never leave a copy in flight into this CTA's shared memory.
-    for (int s = 0; s < L::NS && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / L::NS) * L::NS;
+    // Drain: never leave a copy in flight into this CTA's shared memory (g = tiles issued).
+    for (int s = 0; s < L::NS && s < g; ++s) {
+      const int last = s + ((g - 1 - s) / L::NS) * L::NS;
       mbar_wait(kv_full + s, (last / L::NS) & 1);
     }
-    mbar_wait(q_full, 0);
-    if (kMixed && n16 > 0) { mbar_wait(kv16_full, (n16 - 1) & 1); mbar_wait(q16_full, 0); }
+    for (int qb = 0; qb < 2 && qb < q_issued; ++qb) {
+      const int last = qb + ((q_issued - 1 - qb) / 2) * 2;
+      mbar_wait(q_full + qb, (last >> 1) & 1);
+    }
+    if (kMixed && n16 > 0) mbar_wait(kv16_full, (n16 - 1) & 1);
+    if (kMixed && nq16 > 0) mbar_wait(q16_full, (nq16 - 1) & 1);
   } else if (warp == 1) {
     // ============================ QK^T issuer (one thread) ============================
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, 128);
       const uint32_t idesc_qk16 = idesc_f16(128, 128);
-      const uint32_t sQ = smem_u32(sm + L::OFF_Q);
-      bool ok = wait1(q_full, 0, -1);
-      if (ok) {
+      bool ok = true;
+      int g = 0, n16 = 0, nq16 = 0;
+      for (int it = 0; ok; ++it) {
+        const int idx = fwd_item_index(it, G, cta);
+        if (idx >= n_items) break;
+        const FwdItem w = fwd_item(a, idx);
+        const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk : nullptr;
+        const int qb = it & 1;
+        if (!wait1(q_full + qb, (it >> 1) & 1, g)) { ok = false; break; }
+        // Q scale slot qb was last read by item it - 2, whose QK^Ts are done once tile g - 2
+        // (the latest tile it can own) has been read out of S.
+        if (g >= 2 && !wait1(s_free + (g & 1), ((g - 2) >> 1) & 1, g)) { ok = false; break; }
         // the scale factors arrived by cp.async (generic proxy); the tensor core reads them
         // through the async proxy
         fence_proxy_async_smem();
         tc_fence_after();
+        const uint32_t tq = tbase + L::T_QSF + 8 * qb;
         for (int kk = 0; kk < L::KSTEPS; ++kk)
-          tmem_cp_sf(tbase + L::T_QSF + 4 * kk, sm + L::OFF_QSF + kk * 512);
-      }
-      int n16 = 0;
-      bool q16_ready = false;
-      for (int j = 0; ok && j < nt; ++j) {
-        const int s = j % L::NS;
-        const bool f16 = kMixed && bm_row[j];
-        if (!wait1(kv_full + s, (j / L::NS) & 1, j)) { ok = false; break; }
-        fence_proxy_async_smem();
-        tc_fence_after();
-        // S_{j&1} (and K scale slot j&1) were last used by tile j-2
-        if (j >= 2 && !wait1(s_free + (j & 1), ((j - 2) >> 1) & 1, j)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tS = tbase + L::T_S + (j & 1) * 128;
-        if (!f16) {
-          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-          const uint32_t tk = tbase + L::T_KSF + 8 * (j & 1);
-          for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, st + L::ST_KSF + kk * 512);
-          const uint32_t sK = smem_u32(st + L::ST_K);
-          for (int kk = 0; kk < L::KSTEPS; ++kk) {
-            const uint64_t da = make_sdesc(sQ + kk * 32, 16, L::QK_SBO, L::QK_SW);
-            const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
-            mma_nvf4(tS, da, db, idesc_qk, tbase + L::T_QSF + 4 * kk, tk + 4 * kk, kk > 0 ? 1u : 0u);
-          }
-        } else {
-          if (!q16_ready) {
-            if (!wait1(q16_full, 0, j)) { ok = false; break; }
-            q16_ready = true;
-          }
-          if (!wait1(kv16_full, n16 & 1, j)) { ok = false; break; }
+          tmem_cp_sf(tq + 4 * kk, sm + L::OFF_QSF + qb * 1024 + kk * 512);
+        const uint32_t sQ = smem_u32(sm + L::OFF_Q + qb * L::Q_BYTES);
+        bool q16_ready = false, had16 = false;
+        for (int j = 0; j < w.nt; ++j, ++g) {
+          const int s = g % L::NS;
+          const bool f16 = kMixed && bm_row[j];
+          if (!wait1(kv_full + s, (g / L::NS) & 1, g)) { ok = false; break; }
+          fence_proxy_async_smem();
+          // S_{g&1} (and K scale slot g&1) were last used by tile g - 2
+          if (g >= 2 && !wait1(s_free + (g & 1), ((g - 2) >> 1) & 1, g)) { ok = false; break; }
           tc_fence_after();
-          ++n16;
-          const uint32_t sQ16 = smem_u32(sm + L::OFF_Q16), sK16 = smem_u32(sm + L::OFF_K16);
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t da = make_sdesc(sQ16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
-            const uint64_t db = make_sdesc(sK16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
-            mma_f16(tS, da, db, idesc_qk16, kk > 0 ? 1u : 0u);
+          const uint32_t tS = tbase + L::T_S + (g & 1) * 128;
+          if (!f16) {
+            unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+            const uint32_t tk = tbase + L::T_KSF + 8 * (g & 1);
+            for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, st + L::ST_KSF + kk * 512);
+            const uint32_t sK = smem_u32(st + L::ST_K);
+            for (int kk = 0; kk < L::KSTEPS; ++kk) {
+              const uint64_t da = make_sdesc(sQ + kk * 32, 16, L::QK_SBO, L::QK_SW);
+              const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
+              mma_nvf4(tS, da, db, idesc_qk, tq + 4 * kk, tk + 4 * kk, kk > 0 ? 1u : 0u);
+            }
+          } else {
+            if (!q16_ready) {
+              if (!wait1(q16_full, nq16 & 1, g)) { ok = false; break; }
+              ++nq16;
+              q16_ready = true;
+            }
+            if (!wait1(kv16_full, n16 & 1, g)) { ok = false; break; }
+            tc_fence_after();
+            ++n16;
+            had16 = true;
+            const uint32_t sQ16 = smem_u32(sm + L::OFF_Q16), sK16 = smem_u32(sm + L::OFF_K16);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t da = make_sdesc(sQ16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
+              const uint64_t db = make_sdesc(sK16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
+              mma_f16(tS, da, db, idesc_qk16, kk > 0 ? 1u : 0u);
+            }
           }
+          mma_commit(s_full + (g & 1));
+          mma_commit(kv_empty + s);                  // K half of the stage is free
         }
-        mma_commit(s_full + (j & 1));
-        mma_commit(kv_empty + s);                  // K half of the stage is free
+        if (!ok) break;
+        mma_commit(q_empty + qb);                    // Q buffer qb is free
+        if (kMixed && had16) mma_commit(q16_empty);
       }
       // Everything this thread issued has completed before TMEM is released.
       mma_commit(mma_final);
@@ -356,47 +409,55 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NV);
       const uint32_t idesc_pv16 = idesc_f16(128, L::NV);
       const uint32_t sP = smem_u32(sm + L::OFF_P);
+      const uint32_t tO = tbase + L::T_O;
       tc_fence_after();
       tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
       for (int b2 = 0; b2 < 2; ++b2)               // second V scale chunk (rows 128..): 1.0
         tmem_cp_sf(tbase + L::T_VSF + 8 * b2 + 4, sm + L::OFF_PSF);
       bool ok = true;
-      int n16 = 0;
-      for (int jj = 0; ok && jj < nt; ++jj) {
-        const int s = jj % L::NS, b2 = jj & 1;
-        const bool f16 = kMixed && bm_row[jj];
-        if (!wait1(p_full + b2, (jj >> 1) & 1, jj)) { ok = false; break; }
-        if (!wait1(kv_full + s, (jj / L::NS) & 1, jj)) { ok = false; break; }
-        if (f16 && !wait1(kv16_full, n16 & 1, jj)) { ok = false; break; }
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint32_t tO = tbase + L::T_O;
-        if (!f16) {
-          unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-          const uint32_t tv = tbase + L::T_VSF + 8 * b2;   // PV(jj-2), its last reader, is done
-          tmem_cp_sf(tv, st + L::ST_VSF);
-          const uint32_t sV = smem_u32(st + L::ST_V);
+      int g = 0, n16 = 0;
+      for (int it = 0; ok; ++it) {
+        const int idx = fwd_item_index(it, G, cta);
+        if (idx >= n_items) break;
+        const FwdItem w = fwd_item(a, idx);
+        const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk : nullptr;
+        // the first PV of an item overwrites O: the previous item's epilogue must have read it
+        if (it >= 1 && !wait1(o_free, (it - 1) & 1, g)) { ok = false; break; }
+        for (int j = 0; j < w.nt; ++j, ++g) {
+          const int s = g % L::NS, b2 = g & 1;
+          const bool f16 = kMixed && bm_row[j];
+          if (!wait1(p_full + b2, (g >> 1) & 1, g)) { ok = false; break; }
+          if (!wait1(kv_full + s, (g / L::NS) & 1, g)) { ok = false; break; }
+          if (f16 && !wait1(kv16_full, n16 & 1, g)) { ok = false; break; }
+          fence_proxy_async_smem();
+          tc_fence_after();
+          if (!f16) {
+            unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
+            const uint32_t tv = tbase + L::T_VSF + 8 * b2;   // PV(g-2), its last reader, is done
+            tmem_cp_sf(tv, st + L::ST_VSF);
+            const uint32_t sV = smem_u32(st + L::ST_V);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t da = make_sdesc(sP + b2 * 16384 + kk * 32, 16, 1024, kSw128);
-            const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
-            mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
-                     (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
-                     tv | (static_cast<uint32_t>(kk) << 30), (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-        } else {
-          ++n16;
-          const uint32_t sV16 = smem_u32(sm + L::OFF_V16);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t da = make_sdesc(sP + b2 * 16384 + kk * 32, 16, 1024, kSw128);
+              const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
+              mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
+                       (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                       tv | (static_cast<uint32_t>(kk) << 30), (j > 0 || kk > 0) ? 1u : 0u);
+            }
+          } else {
+            ++n16;
+            const uint32_t sV16 = smem_u32(sm + L::OFF_V16);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
-            const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
-            mma_f16(tO, da, db, idesc_pv16, (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
+              const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
+              mma_f16(tO, da, db, idesc_pv16, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(kv16_empty);
           }
-          mma_commit(kv16_empty);
+          mma_commit(pv_done + b2);
+          mma_commit(kv_empty + s);                  // V half of the stage is free
         }
-        mma_commit(pv_done + b2);
-        mma_commit(kv_empty + s);                  // V half of the stage is free
       }
       mma_commit(mma_final + 1);
       mbar_wait(mma_final + 1, 0);
@@ -407,9 +468,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int wq = warp & 3;                 // TMEM lane quadrant
     const int grp = (warp - 4) >> 2;         // key-tile parity this group handles
     const int row = wq * 32 + lane;
-    const int qi = qt * 128 + row;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     float* red_m = reinterpret_cast<float*>(sm + L::OFF_RED);         // [2 parities][128]
+    float* red_fin = red_m + 256;                                     // [2 items][128]
     // Scores stay in the FP4 MMA's raw units (S = sum codes*scales); the running max m is
     // kept in those units and 448 p = 2^(s C + (log2 448 - m C)) with
     // C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true dot products and are
@@ -419,195 +480,224 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float2 C2 = make_float2(C, C);
     unsigned char* sP = sm + L::OFF_P;
     const uint32_t tO = tbase + L::T_O + lane_addr;
+    // A warp whose wait fails keeps walking the items without doing work (ok == false), so
+    // that the two groups always meet at every item's named barrier.
     bool ok = true;
-    for (int j = grp; j < nt; j += 2) {
-      const int b2 = j & 1;                  // == grp
-      const bool f16 = kMixed && bm_row[j];
-      const bool prev_f16 = kMixed && j >= 1 && bm_row[j - 1];
-      float x[128];
-      if (!waitw(s_full + b2, (j >> 1) & 1, j)) { ok = false; break; }
-      tc_fence_after();
-      {
-        uint32_t* xr = reinterpret_cast<uint32_t*>(x);
-        const uint32_t tS = tbase + L::T_S + b2 * 128 + lane_addr;
-#pragma unroll
-        for (int c = 0; c < 128; c += 32) tmem_ld32(tS + c, xr + c);
-        tmem_wait_ld();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + b2);
-      if (f16) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] *= R16;
-      }
-      const int kbase = j * 128;
-      if ((a.causal && kbase + 127 > qi) || (kbase + 128 > a.Nk)) {
-        const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (c <= lim) ? x[c] : -INFINITY;
-      }
-      float mt;
-      {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < 128; c += 8) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) m4[u] = fmax3(m4[u], x[c + 2 * u], x[c + 2 * u + 1]);
-        }
-        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      }
-      // Running max before this tile: handed on by the group that processed tile j - 1.
-      float m_prev = -INFINITY;
-      if (j >= 1) {
-        if (!waitw(m_ready + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
-        __syncwarp();
-        m_prev = red_m[((j - 1) & 1) * 128 + row];
-      }
-      const float m_new = fmaxf(m_prev, mt);
-      red_m[b2 * 128 + row] = m_new;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(m_ready + b2);
-      const bool dead = (m_new == -INFINITY);
-      const float bias = kLog2_448 - (dead ? 0.f : m_new) * C;
-      const float2 B2 = make_float2(bias, bias);
-      uint32_t pw[kMixed ? 64 : 32];      // e4m3: 32 words; fp16: 64 words
-      if (!f16) {
-        // kPolyOf8 of every 8 groups of 4 scores take the FMA-pipe exponential, the rest the
-        // special-function unit, so both pipes work on the tile.
-#pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
-          const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), C2, B2);
-          float2 e0, e1;
-          if (((c >> 2) & 7) < kPolyOf8) {
-            e0 = exp2_poly2(t0);
-            e1 = exp2_poly2(t1);
-          } else {
-            e0 = make_float2(ex2_approx(t0.x), ex2_approx(t0.y));
-            e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
-          }
-          pw[c >> 2] = cvt_e4m3x2(e0.x, e0.y) | (cvt_e4m3x2(e1.x, e1.y) << 16);
-        }
-      } else if constexpr (kMixed) {
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float2 t = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
-          const __half2 h = __floats2half2_rn(ex2_approx(t.x), ex2_approx(t.y));
-          pw[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-      }
-      // P buffer b2 was last used by PV(j-2). An FP16 tile's P fills both buffers:
-      // writing one needs PV(j-1) done as well, and the tile after an FP16 tile too. PV(j-2)'s
-      // completion implies PV(j-3)'s, so the wait on the other parity's barrier is for its
-      // next phase.
-      if (j >= 2 && !waitw(pv_done + b2, ((j - 2) >> 1) & 1, j)) { ok = false; break; }
-      if ((f16 || prev_f16) && j >= 1 &&
-          !waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
-      if (!f16) {
-        unsigned char* prow = sP + b2 * 16384 + row * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-      } else if constexpr (kMixed) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          unsigned char* prow = sP + h * 16384 + row * 128;     // atom h = keys 64h .. 64h+63
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) =
-                make_uint4(pw[32 * h + 4 * c], pw[32 * h + 4 * c + 1], pw[32 * h + 4 * c + 2],
-                           pw[32 * h + 4 * c + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      // O holds the tiles before j relative to m(j-1) = m_prev. Rows whose max rose at this
-      // tile are brought to m_new once PV(j-1) is done (the next phase of that parity's
-      // barrier: PV(j-2), waited above, implies PV(j-3)); a warp whose rows all kept their
-      // max hands P(j) on at once.
-      const float alpha = (m_prev == -INFINITY || dead) ? 1.f : ex2_approx((m_prev - m_new) * C);
-      if (j >= 1 && !__all_sync(0xffffffffu, alpha == 1.f)) {
-        if (!waitw(pv_done + ((j - 1) & 1), ((j - 1) >> 1) & 1, j)) { ok = false; break; }
+    bool prev_last_f16 = false;              // the previous item's last tile ran in FP16
+    int g = 0;
+    for (int it = 0;; ++it) {
+      const int idx = fwd_item_index(it, G, cta);
+      if (idx >= n_items) break;
+      const FwdItem w = fwd_item(a, idx);
+      const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk : nullptr;
+      const int qi = w.qt * 128 + row;
+      const int g0 = g;
+      float m_last = -INFINITY;              // running max after this group's latest tile
+      for (int j = (grp - g0) & 1; j < w.nt; j += 2) {
+        if (!ok) continue;
+        const int gg = g0 + j;
+        const int b2 = gg & 1;               // == grp
+        const bool f16 = kMixed && bm_row[j];
+        const bool prev_f16 = kMixed && (j >= 1 ? bm_row[j - 1] != 0 : prev_last_f16);
+        float x[128];
+        if (!waitw(s_full + b2, (gg >> 1) & 1, gg)) { ok = false; continue; }
         tc_fence_after();
-        const float2 A2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            const float2 u = __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), A2);
-            o[k] = __float_as_uint(u.x);
-            o[k + 1] = __float_as_uint(u.y);
-          }
-          tmem_st32(tO + cc, o);
-        }
         {
-          uint32_t o[16];
-          tmem_ld16(tO + D, o);
+          uint32_t* xr = reinterpret_cast<uint32_t*>(x);
+          const uint32_t tS = tbase + L::T_S + b2 * 128 + lane_addr;
+#pragma unroll
+          for (int c = 0; c < 128; c += 32) tmem_ld32(tS + c, xr + c);
           tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st16(tO + D, o);
         }
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full + b2);
-    }
-    // ---- epilogue: O / l (O and l already relative to the final max) ----
-    // PV(nt-1)'s completion covers every earlier MMA of the issuing thread; the group that
-    // owns tile nt-1 waits for it (the next phase of its own barrier) and the named barrier
-    // passes that on to the other group.
-    if (ok && grp == ((nt - 1) & 1)) ok = waitw(pv_done + grp, ((nt - 1) >> 1) & 1, nt);
-    tc_fence_before();
-    named_bar_sync(1, 256);
-    if (ok && !*abort_flag) {
-      tc_fence_after();
-      const float m_run = red_m[((nt - 1) & 1) * 128 + row];   // m(nt-1), published last
-      uint32_t lr[16];
-      tmem_ld16(tO + D, lr);
-      tmem_wait_ld();
-      const float l_run = __uint_as_float(lr[0]);
-      const bool store = qi < a.Nq;
-      const int64_t orow = static_cast<int64_t>(bhq) * a.Nq + qi;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free + b2);
+        if (f16) {
 #pragma unroll
-      for (int cc = 0; cc < D / 2; cc += 32) {
-        const int c = grp * (D / 2) + cc;
-        uint32_t o[32];
-        tmem_ld32(tO + c, o);
-        tmem_wait_ld();
-        if (store) {
-          float v[32];
+          for (int c = 0; c < 128; ++c) x[c] *= R16;
+        }
+        const int kbase = j * 128;
+        if ((a.causal && kbase + 127 > qi) || (kbase + 128 > a.Nk)) {
+          const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
 #pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = __fdiv_rn(__uint_as_float(o[k]), l_run);
-          if (a.out_kind == 2) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c);
+          for (int c = 0; c < 128; ++c) x[c] = (c <= lim) ? x[c] : -INFINITY;
+        }
+        float mt;
+        {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-          } else {
-            __align__(16) uint32_t packed[16];
+          for (int c = 0; c < 128; c += 8) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m4[u] = fmax3(m4[u], x[c + 2 * u], x[c + 2 * u + 1]);
+          }
+          mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        }
+        // Running max before this tile: handed on by the group that processed tile gg - 1 of
+        // the same item (the first tile of an item starts from -inf).
+        float m_prev = -INFINITY;
+        if (j >= 1) {
+          if (!waitw(m_ready + ((gg - 1) & 1), ((gg - 1) >> 1) & 1, gg)) { ok = false; continue; }
+          __syncwarp();
+          m_prev = red_m[((gg - 1) & 1) * 128 + row];
+        }
+        const float m_new = fmaxf(m_prev, mt);
+        m_last = m_new;
+        red_m[b2 * 128 + row] = m_new;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(m_ready + b2);
+        const bool dead = (m_new == -INFINITY);
+        const float bias = kLog2_448 - (dead ? 0.f : m_new) * C;
+        const float2 B2 = make_float2(bias, bias);
+        // P buffer b2 was last used by PV(gg-2). An FP16 tile's P fills both buffers: writing
+        // one needs PV(gg-1) done as well, and the tile after an FP16 tile too. PV(gg-2)'s
+        // completion implies PV(gg-3)'s, so the wait on the other parity's barrier is for its
+        // next phase. The waits come before the exponentials so that P can be stored 16 bytes
+        // at a time as it is produced (no register copy of the whole row).
+        if (gg >= 2 && !waitw(pv_done + b2, ((gg - 2) >> 1) & 1, gg)) { ok = false; continue; }
+        if ((f16 || prev_f16) && gg >= 1 &&
+            !waitw(pv_done + ((gg - 1) & 1), ((gg - 1) >> 1) & 1, gg)) { ok = false; continue; }
+        if (!f16) {
+          // kPolyOf8 of every 8 groups of 4 scores take the FMA-pipe exponential, the rest the
+          // special-function unit.
+          unsigned char* prow = sP + b2 * 16384 + row * 128;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {               // 16 keys per 16-byte chunk
+            uint32_t w4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int c = ch * 16 + q * 4;
+              const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
+              const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), C2, B2);
+              float2 e0, e1;
+              if (((c >> 2) & 7) < kPolyOf8) {
+                e0 = exp2_poly2(t0);
+                e1 = exp2_poly2(t1);
+              } else {
+                e0 = make_float2(ex2_approx(t0.x), ex2_approx(t0.y));
+                e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
+              }
+              w4[q] = cvt_e4m3x2(e0.x, e0.y) | (cvt_e4m3x2(e1.x, e1.y) << 16);
+            }
+            *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        } else if constexpr (kMixed) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            unsigned char* prow = sP + h * 16384 + row * 128;     // atom h = keys 64h .. 64h+63
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {             // 8 keys per 16-byte chunk
+              uint32_t w4[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int c = h * 64 + ch * 8 + q * 2;
+                const float2 t = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
+                const __half2 hv = __floats2half2_rn(ex2_approx(t.x), ex2_approx(t.y));
+                w4[q] = *reinterpret_cast<const uint32_t*>(&hv);
+              }
+              *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        // O holds the item's tiles before j relative to m(j-1) = m_prev. Rows whose max rose
+        // at this tile are brought to m_new once PV(gg-1) is done (the next phase of that
+        // parity's barrier: PV(gg-2), waited above, implies PV(gg-3)); a warp whose rows all
+        // kept their max hands P on at once.
+        const float alpha = (m_prev == -INFINITY || dead) ? 1.f : ex2_approx((m_prev - m_new) * C);
+        if (j >= 1 && !__all_sync(0xffffffffu, alpha == 1.f)) {
+          if (!waitw(pv_done + ((gg - 1) & 1), ((gg - 1) >> 1) & 1, gg)) { ok = false; continue; }
+          tc_fence_after();
+          const float2 A2 = make_float2(alpha, alpha);
+#pragma unroll
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc, o);
+            tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
-              if (a.out_kind == 1) {
-                __nv_bfloat162 t = __floats2bfloat162_rn(v[k], v[k + 1]);
-                packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
-              } else {
-                __half2 t = __floats2half2_rn(v[k], v[k + 1]);
-                packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
-              }
+              const float2 u = __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), A2);
+              o[k] = __float_as_uint(u.x);
+              o[k + 1] = __float_as_uint(u.y);
             }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + c);
+            tmem_st32(tO + cc, o);
+          }
+          {
+            uint32_t o[16];
+            tmem_ld16(tO + D, o);
+            tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 4; ++k) dst[k] = reinterpret_cast<uint4*>(packed)[k];
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st16(tO + D, o);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full + b2);
+      }
+      g = g0 + w.nt;
+      if constexpr (kMixed) prev_last_f16 = bm_row[w.nt - 1] != 0;
+      // ---- epilogue of this item: O / l (O and l already relative to the final max) ----
+      // PV of the item's last tile covers every earlier MMA of its issuing thread; the group
+      // that owns that tile waits for it (the next phase of its own barrier) and publishes the
+      // final max, and the named barrier passes both on to the other group.
+      const int owner = (g - 1) & 1;
+      if (ok && grp == owner) {
+        ok = waitw(pv_done + owner, ((g - 1) >> 1) & 1, g - 1);
+        red_fin[(it & 1) * 128 + row] = m_last;
+      }
+      tc_fence_before();
+      named_bar_sync(1, 256);
+      const bool live = ok && !*abort_flag;
+      if (live) {
+        tc_fence_after();
+        uint32_t lr[16];
+        tmem_ld16(tO + D, lr);
+        tmem_wait_ld();
+        const float m_run = red_fin[(it & 1) * 128 + row];
+        const float l_run = __uint_as_float(lr[0]);
+        const bool store = qi < a.Nq;
+        const int64_t orow = static_cast<int64_t>(w.bhq) * a.Nq + qi;
+#pragma unroll
+        for (int cc = 0; cc < D / 2; cc += 32) {
+          const int c = grp * (D / 2) + cc;
+          uint32_t o[32];
+          tmem_ld32(tO + c, o);
+          tmem_wait_ld();
+          if (store) {
+            float v[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = __fdiv_rn(__uint_as_float(o[k]), l_run);
+            if (a.out_kind == 2) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+            } else {
+              __align__(16) uint32_t packed[16];
+#pragma unroll
+              for (int k = 0; k < 32; k += 2) {
+                if (a.out_kind == 1) {
+                  __nv_bfloat162 t = __floats2bfloat162_rn(v[k], v[k + 1]);
+                  packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
+                } else {
+                  __half2 t = __floats2half2_rn(v[k], v[k + 1]);
+                  packed[k >> 1] = *reinterpret_cast<uint32_t*>(&t);
+                }
+              }
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + c);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) dst[k] = reinterpret_cast<uint4*>(packed)[k];
+            }
           }
         }
+        if (store && grp == 0 && a.lse != nullptr)
+          a.lse[orow] = m_run * C * kLn2 + logf(l_run * (1.f / 448.f));
       }
-      if (store && grp == 0 && a.lse != nullptr)
-        a.lse[orow] = m_run * C * kLn2 + logf(l_run * (1.f / 448.f));
+      // O has been read (every tcgen05.ld above waited): the next item's first PV may
+      // overwrite it.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
     }
   }
   tc_fence_before();

@@ -65,17 +65,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
                : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
-// The same with a suspend-time hint: a thread whose phase is not complete yet sleeps (up to
-// the hint) until it completes instead of spinning, so waiting warps take no issue slots from
-// the warps that work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile("{\n\t.reg .pred p;\n\t"
-               "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-               "selp.u32 %0, 1, 0, p;\n\t}"
-               : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u) : "memory");
-  return ok != 0;
-}
 // Bounded wait for the phase with the given parity to complete. Returns false (and sets the
 // timeout status bit) when the limit passes first. The limit is counted in SM clock cycles
 // (about a second at the B200's clocks) and read only every 32 polls, so the poll loop itself
@@ -87,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_sleep(bar, parity)) return true;
+      if (mbar_try_wait(bar, parity)) return true;
     if (clock64() - t0 > kWaitLimitCycles) {
       flag_error(kStatusTimeout);
       return false;
@@ -98,14 +87,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 // Wait that gives up when *flag is set, and sets *flag when it times out itself. `site`
 // (wait_site()) is recorded when this wait is the first to time out. A phase that has
 // already completed is taken on the first poll (the common case in a running pipeline);
-// only then is the flag read, and again between sleeps.
+// only then is the flag read, and again every 32 polls (try_wait itself suspends the thread
+// for a short, hardware-chosen time while the phase is pending).
 __device__ __forceinline__ bool bounded_wait_slow(uint64_t* bar, uint32_t parity, volatile int* flag,
                                                uint64_t site) {
   const long long t0 = clock64();
   while (!*flag) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_sleep(bar, parity)) return true;
+      if (mbar_try_wait(bar, parity)) return true;
     if (clock64() - t0 > kWaitLimitCycles) {
       flag_error(kStatusTimeout);
       record_timeout(site);

@@ -51,6 +51,19 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Number of SMs of the current device (queried once per device).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 int grid_for(int64_t work, int threads) {
   int64_t g = (work + threads - 1) / threads;
   if (g > kNumSMs * 16) g = kNumSMs * 16;
@@ -302,7 +315,10 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   a.causal = p->causal ? 1 : 0;
   a.softmax_scale = p->softmax_scale;
   a.out_kind = static_cast<int32_t>(p->out_dtype);
-  const int64_t grid = static_cast<int64_t>(a.Tq) * B * Hq;
+  // Persistent: one CTA per SM (or per work item when there are fewer items).
+  const int64_t items = static_cast<int64_t>(a.Tq) * B * Hq;
+  if (items > INT32_MAX / 2) return QK4V8_ERR_UNSUPPORTED;
+  const int64_t grid = items < sm_count() ? items : sm_count();
   attn_fwd_kernel<D, kMixed><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
   return launch_status();
 }
