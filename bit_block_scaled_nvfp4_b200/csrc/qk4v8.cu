@@ -245,11 +245,11 @@ qk4v8_status tile_score_select(const uint8_t* q_codes, const uint8_t* q_scales,
   const int64_t qrows = static_cast<int64_t>(batch) * q_heads * n_tokens;
   const int64_t krows = static_cast<int64_t>(batch) * kv_heads * n_tokens;
   if (head_dim == 128) {
-    row_norm_tile_max_kernel<128><<<(qrows + 255) / 256, 256, 0, stream>>>(q_codes, q_scales, static_cast<int64_t>(batch) * q_heads, n_tokens, T, qmax);
-    row_norm_tile_max_kernel<128><<<(krows + 255) / 256, 256, 0, stream>>>(k_codes, k_scales, static_cast<int64_t>(batch) * kv_heads, n_tokens, T, kmax);
+    row_norm_tile_max_kernel<128><<<(qrows * 4 + 255) / 256, 256, 0, stream>>>(q_codes, q_scales, static_cast<int64_t>(batch) * q_heads, n_tokens, T, qmax);
+    row_norm_tile_max_kernel<128><<<(krows * 4 + 255) / 256, 256, 0, stream>>>(k_codes, k_scales, static_cast<int64_t>(batch) * kv_heads, n_tokens, T, kmax);
   } else {
-    row_norm_tile_max_kernel<64><<<(qrows + 255) / 256, 256, 0, stream>>>(q_codes, q_scales, static_cast<int64_t>(batch) * q_heads, n_tokens, T, qmax);
-    row_norm_tile_max_kernel<64><<<(krows + 255) / 256, 256, 0, stream>>>(k_codes, k_scales, static_cast<int64_t>(batch) * kv_heads, n_tokens, T, kmax);
+    row_norm_tile_max_kernel<64><<<(qrows * 2 + 255) / 256, 256, 0, stream>>>(q_codes, q_scales, static_cast<int64_t>(batch) * q_heads, n_tokens, T, qmax);
+    row_norm_tile_max_kernel<64><<<(krows * 2 + 255) / 256, 256, 0, stream>>>(k_codes, k_scales, static_cast<int64_t>(batch) * kv_heads, n_tokens, T, kmax);
   }
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   const int smem = (2 * T + 2) * 8 + kSelectMax * (16 + 4);

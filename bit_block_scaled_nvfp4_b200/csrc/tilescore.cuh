@@ -19,21 +19,27 @@ __device__ __forceinline__ uint64_t e4m3_times512(uint32_t c) {
   return e == 0 ? m : static_cast<uint64_t>(8 + m) << (e - 1);
 }
 
-// Squares of (2 * E2M1 magnitude) for the 8 magnitude codes: 0,1,4,9,16,36,64,144.
-__device__ __forceinline__ uint32_t e2m1_sq2(uint32_t c) {
-  switch (c & 7u) {
-    case 0: return 0; case 1: return 1; case 2: return 4; case 3: return 9;
-    case 4: return 16; case 5: return 36; case 6: return 64; default: return 144;
-  }
+// Sum over the 8 E2M1 codes of a 32-bit word of (2 * magnitude)^2: the squares
+// 0,1,4,9,16,36,64,144 of the 8 magnitude codes as a byte table, looked up four codes at a time
+// with a byte permute (the sign bit of each code masked off) and summed with dp4a.
+__device__ __forceinline__ uint32_t e2m1_sq2_sum(uint32_t w) {
+  constexpr uint32_t kLo = 0x09040100u, kHi = 0x90402410u;
+  const uint32_t a = __byte_perm(kLo, kHi, w & 0x7777u);
+  const uint32_t b = __byte_perm(kLo, kHi, (w >> 16) & 0x7777u);
+  return __dp4a(b, 0x01010101u, __dp4a(a, 0x01010101u, 0u));
 }
 
 // Per-row exact norm and per-tile maximum. rows of one tensor [BH, N, D] in NVFP4.
-// tile_max: [BH, T] u64, zeroed by the caller. One thread per row.
+// tile_max: [BH, T] u64, zeroed by the caller. D/32 consecutive threads share a row, each
+// taking 16 bytes of codes (two 16-element blocks), so the loads are coalesced.
 template <int D>
 __global__ void __launch_bounds__(256) row_norm_tile_max_kernel(
     const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, int64_t BH, int32_t N,
     int32_t T, unsigned long long* __restrict__ tile_max) {
-  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  constexpr int TPR = D / 32;                    // threads per row
+  const int64_t gtid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t row = gtid / TPR;
+  const int part = static_cast<int>(gtid % TPR);
   const bool live = row < BH * N;
   uint64_t nr = 0;
   int64_t bh = 0;
@@ -42,26 +48,16 @@ __global__ void __launch_bounds__(256) row_norm_tile_max_kernel(
     bh = row / N;
     const int n = static_cast<int>(row - bh * N);
     tile = n / 128;
-    const uint4* c4 = reinterpret_cast<const uint4*>(codes + row * (D / 2));
-    const uint8_t* sc = scales + row * (D / 16);
-#pragma unroll
-    for (int b = 0; b < D / 16; b += 2) {       // two 16-element blocks per 16-byte load
-      const uint4 u = __ldg(c4 + b / 2);
-      const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t s = 0;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const uint32_t w = wds[h * 2 + k];
-#pragma unroll
-          for (int nib = 0; nib < 8; ++nib) s += e2m1_sq2(w >> (4 * nib));
-        }
-        const uint64_t f = e4m3_times512(sc[b + h]);
-        nr += f * f * s;
-      }
-    }
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(codes + row * (D / 2)) + part);
+    const uint8_t* sc = scales + row * (D / 16) + part * 2;
+    const uint32_t s0 = e2m1_sq2_sum(u.x) + e2m1_sq2_sum(u.y);
+    const uint32_t s1 = e2m1_sq2_sum(u.z) + e2m1_sq2_sum(u.w);
+    const uint64_t f0 = e4m3_times512(sc[0]), f1 = e4m3_times512(sc[1]);
+    nr = f0 * f0 * s0 + f1 * f1 * s1;
   }
+  // whole-row sums in every lane of the row's group
+#pragma unroll
+  for (int o = 1; o < TPR; o <<= 1) nr += __shfl_xor_sync(0xffffffffu, nr, o);
   // One atomic per warp when all its rows fall in the same (bh, tile); else one per row.
   const int64_t key = live ? bh * T + tile : -1;
   const int64_t key0 = __shfl_sync(0xffffffffu, key, 0);
@@ -73,7 +69,7 @@ __global__ void __launch_bounds__(256) row_norm_tile_max_kernel(
       m = other > m ? other : m;
     }
     if ((threadIdx.x & 31) == 0 && key0 >= 0) atomicMax(tile_max + key0, m);
-  } else if (live) {
+  } else if (live && part == 0) {
     atomicMax(tile_max + key, static_cast<unsigned long long>(nr));
   }
 }
@@ -142,15 +138,28 @@ __global__ void __launch_bounds__(kSelectThreads) tile_select_kernel(
   // --- radix select the k-th largest score (tau) -------------------------------------
   U128 pre{0, 0};
   uint32_t k_rem = static_cast<uint32_t>(k);
+  // Row norms are below 2^51, so scores are below 2^102: bytes 13-15 are always zero.
   if (k > 0) {
-    for (int p = 15; p >= 0; --p) {
+    for (int p = 12; p >= 0; --p) {
       for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
       __syncthreads();
-      for (int64_t c = tid; c < total; c += blockDim.x) {
-        const int qt = static_cast<int>(c / Tk), kt = static_cast<int>(c % Tk);
-        if (causal && kt > qt) continue;
-        const U128 v = mul_u64(mq[qt], mk[kt]);
-        if (prefix_match(v, pre, p)) atomicAdd(&hist[byte_of(v, p)], 1u);
+      // Warp per query-tile row, lanes over key tiles (no index division). Lanes with the
+      // same digit add once per warp (most scores share their high bytes, and one shared-
+      // memory atomic per candidate would serialise on a few bins).
+      const int lane = tid & 31;
+      for (int qt = tid >> 5; qt < Tq; qt += kSelectThreads / 32) {
+        const uint64_t a = mq[qt];
+        const int kt_end = causal ? min(qt + 1, Tk) : Tk;
+        for (int kb = 0; kb < kt_end; kb += 32) {
+          const int kt = kb + lane;
+          int bin = -1;
+          if (kt < kt_end) {
+            const U128 v = mul_u64(a, mk[kt]);
+            if (prefix_match(v, pre, p)) bin = static_cast<int>(byte_of(v, p));
+          }
+          const unsigned same = __match_any_sync(0xffffffffu, bin);
+          if (bin >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(same)));
+        }
       }
       __syncthreads();
       if (tid == 0) {
@@ -181,7 +190,8 @@ __global__ void __launch_bounds__(kSelectThreads) tile_select_kernel(
       bool gt = false, eq = false;
       U128 v{0, 0};
       if (c < total) {
-        const int qt = static_cast<int>(c / Tk), kt = static_cast<int>(c % Tk);
+        const int qt = static_cast<int>(static_cast<uint32_t>(c) / static_cast<uint32_t>(Tk));
+        const int kt = static_cast<int>(c) - qt * Tk;
         if (!(causal && kt > qt)) {
           v = mul_u64(mq[qt], mk[kt]);
           gt = u128_gt(v, pre);
