@@ -36,6 +36,7 @@
 //              tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles when selected
 //   warp 1     TMEM owner and QK^T issuer (one thread)
 //   warp 2     PV issuer (one thread)
+//   warp 3     FP16 operand producer (FP16-tile kernel only)
 //   warps 4-11 softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
 // TMEM (512 columns): S_0, S_1 [0,256), O (D + 16 columns) from 256, scale factors from 400.
 #pragma once
@@ -217,7 +218,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   // Barrier ids in timeout reports are their index in the barrier block; the tile number is
   // the CTA's running key-tile counter.
-  const uint32_t role = warp == 0 ? kRoleProducer : (warp == 1 || warp == L::PV_WARP) ? kRoleMma : kRoleSoftmax;
+  const uint32_t role = (warp == 0 || warp == 3) ? kRoleProducer
+                        : (warp == 1 || warp == L::PV_WARP) ? kRoleMma : kRoleSoftmax;
   auto site = [&](uint64_t* bar, int tile) {
     return wait_site(kKernelFwd, role, static_cast<uint32_t>(bar - bars), tile);
   };
@@ -235,13 +237,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // asynchronous copies (row r = r0 + 32 r1 of a 128-row chunk -> byte r0*16 + r1*4; one
     // 4-byte word holds the 4 scales of one 64-element MMA step), completing on the same
     // barrier as the TMA of the codes, so this warp never waits on their latency.
-    int g = 0, n16 = 0, nq16 = 0, q_issued = 0;
+    int g = 0, q_issued = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const int idx = fwd_item_index(it, G, cta);
       if (idx >= n_items) break;
       const FwdItem w = fwd_item(a, idx);
-      const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk : nullptr;
       const int qb = it & 1;
       // Q buffer qb was last read by the QK^T MMAs of item it - 2.
       if (it >= 2 && !waitw(q_empty + qb, ((it - 2) >> 1) & 1, g)) { ok = false; break; }
@@ -264,7 +265,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         q_issued = it + 1;
       }
-      bool q16_loaded = false;
       for (int j = 0; j < w.nt; ++j, ++g) {
         const int s = g % L::NS;
         if (g >= L::NS && !waitw(kv_empty + s, ((g / L::NS) - 1) & 1, g)) { ok = false; break; }
@@ -292,30 +292,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, w.bhk);
           tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, w.bhk * D);
         }
-        if constexpr (kMixed) {
-          if (bm_row[j]) {
-            if (!q16_loaded) {
-              // the single FP16 Q buffer was last read by the FP16 QK^Ts of an earlier item
-              if (nq16 >= 1 && !waitw(q16_empty, (nq16 - 1) & 1, g)) { ok = false; ++g; break; }
-              if (lane == 0) {
-                mbar_arrive_expect_tx(q16_full, L::F16_TILE);
-                for (int h = 0; h < D / 64; ++h)
-                  tma_load_3d(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, w.qt * 128, w.bhq);
-              }
-              q16_loaded = true;
-              ++nq16;
-            }
-            if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1, g)) { ok = false; ++g; break; }
-            if (lane == 0) {
-              mbar_arrive_expect_tx(kv16_full, L::F16_TILE + 2 * D * 128);
-              for (int h = 0; h < D / 64; ++h)
-                tma_load_3d(sm + L::OFF_K16 + h * 16384, &tm_k16, kv16_full, h * 64, j * 128, w.bhk);
-              for (int h = 0; h < 2; ++h)
-                tma_load_2d(sm + L::OFF_V16 + h * L::V16_ATOM, &tm_v16, kv16_full, j * 128 + h * 64, w.bhk * D);
-            }
-            ++n16;
-          }
-        }
       }
     }
     // Drain: never leave a copy in flight into this CTA's shared memory (g = tiles issued).
@@ -327,8 +303,46 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int last = qb + ((q_issued - 1 - qb) / 2) * 2;
       mbar_wait(q_full + qb, (last >> 1) & 1);
     }
-    if (kMixed && n16 > 0) mbar_wait(kv16_full, (n16 - 1) & 1);
-    if (kMixed && nq16 > 0) mbar_wait(q16_full, (nq16 - 1) & 1);
+  } else if (kMixed && warp == 3) {
+    // ========================== FP16 operand producer ==========================
+    // The FP16 Q of an item and the FP16 K / V of each selected tile, on a warp of their own
+    // so that the FP4 producer never waits for the single FP16 operand buffer to drain.
+    if (lane == 0) { prefetch_tmap(&tm_q16); prefetch_tmap(&tm_k16); prefetch_tmap(&tm_v16); }
+    int g = 0, n16 = 0, nq16 = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int idx = fwd_item_index(it, G, cta);
+      if (idx >= n_items) break;
+      const FwdItem w = fwd_item(a, idx);
+      const uint8_t* bm_row = a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk;
+      bool q16_loaded = false;
+      for (int j = 0; j < w.nt; ++j, ++g) {
+        if (!bm_row[j]) continue;
+        if (!q16_loaded) {
+          // the single FP16 Q buffer was last read by the FP16 QK^Ts of an earlier item
+          if (nq16 >= 1 && !waitw(q16_empty, (nq16 - 1) & 1, g)) { ok = false; break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(q16_full, L::F16_TILE);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_3d(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, w.qt * 128, w.bhq);
+          }
+          q16_loaded = true;
+          ++nq16;
+        }
+        if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1, g)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(kv16_full, L::F16_TILE + 2 * D * 128);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(sm + L::OFF_K16 + h * 16384, &tm_k16, kv16_full, h * 64, j * 128, w.bhk);
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(sm + L::OFF_V16 + h * L::V16_ATOM, &tm_v16, kv16_full, j * 128 + h * 64, w.bhk * D);
+        }
+        ++n16;
+      }
+    }
+    // Drain: never leave a copy in flight into this CTA's shared memory.
+    if (n16 > 0) mbar_wait(kv16_full, (n16 - 1) & 1);
+    if (nq16 > 0) mbar_wait(q16_full, (nq16 - 1) & 1);
   } else if (warp == 1) {
     // ============================ QK^T issuer (one thread) ============================
     if (lane == 0) {
