@@ -90,7 +90,17 @@ __device__ __forceinline__ int fwd_item_index(int it, int G, int c) {
 
 template <int D, bool kMixed>
 struct FwdLayout {
-  static constexpr int NS = kMixed ? 2 : 4;   // the FP16 operand stage needs the room
+  // K and V stages. In the FP16-tile kernel, whose FP16 operands take 100 KB, K and V form
+  // rings of their own (three K, two V stages): a K stage is free once QK^T of its tile is
+  // done, a V stage only once PV is, so K runs ahead. Otherwise stage s of both arrays is one
+  // stage of a single ring of four (one full and one empty barrier), which measured faster:
+  // with K running ahead the two softmax groups fall into step and contend for the
+  // exponential unit at the same time.
+  static constexpr bool kSplit = kMixed;
+  static constexpr int NK = kMixed ? 3 : 4;
+  static constexpr int NVS = kMixed ? 2 : 4;
+  // P buffers, one per tile parity: the exponentials of tile g wait for PV(g - 2).
+  static constexpr int NP = 2;
   static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
   static constexpr int NV = D + 16;                     // PV MMA N: D channels + ones rows
   static constexpr int Q_BYTES = 128 * D / 2;
@@ -100,24 +110,39 @@ struct FwdLayout {
   static constexpr int OFF_Q = 0;                                         // 2 buffers
   static constexpr int OFF_QSF = OFF_Q + 2 * Q_BYTES;                     // 2 x KSTEPS chunks
   static constexpr int OFF_PSF = OFF_QSF + 2048;                          // all 1.0 (E8M0 127)
-  static constexpr int OFF_STAGE = OFF_PSF + 1024;
-  static constexpr int ST_K = 0;
-  static constexpr int ST_V = K_BYTES;
-  static constexpr int ST_KSF = ST_V + V_BYTES;
-  static constexpr int ST_VSF = ST_KSF + 1024;
-  static constexpr int STAGE_BYTES = ST_VSF + 1024;
-  static constexpr int OFF_P = OFF_STAGE + NS * STAGE_BYTES;               // 2 x 16 KB
-  static constexpr int OFF_RED = OFF_P + 2 * 16384;   // running max hand-off [2][128], final [128]
+  // Stage s of K and of V: with rings of equal depth, one block [K | V (+ ones rows) | K scales
+  // | V scales] per s (measured faster than two separate arrays); otherwise K blocks
+  // [K | K scales] followed by V blocks [V | V scales].
+  static constexpr bool kInterleaved = (NK == NVS);
+  static constexpr int OFF_STG = OFF_PSF + 1024;
+  static constexpr int STG_BYTES = K_BYTES + V_BYTES + 2048;
+  static constexpr int OFF_VSTG = OFF_STG + NK * (K_BYTES + 1024);
+  __device__ static constexpr int k_off(int s) {
+    return kInterleaved ? OFF_STG + s * STG_BYTES : OFF_STG + s * (K_BYTES + 1024);
+  }
+  __device__ static constexpr int k_sf_off(int s) {
+    return kInterleaved ? k_off(s) + K_BYTES + V_BYTES : k_off(s) + K_BYTES;
+  }
+  __device__ static constexpr int v_off(int s) {
+    return kInterleaved ? k_off(s) + K_BYTES : OFF_VSTG + s * (V_BYTES + 1024);
+  }
+  __device__ static constexpr int v_sf_off(int s) {
+    return kInterleaved ? k_off(s) + K_BYTES + V_BYTES + 1024 : v_off(s) + V_BYTES;
+  }
+  static constexpr int OFF_P = kInterleaved ? OFF_STG + NK * STG_BYTES
+                                            : OFF_VSTG + NVS * (V_BYTES + 1024);  // NP x 16 KB
+  static constexpr int OFF_RED = OFF_P + NP * 16384;   // running max hand-off [2][128], final [128]
   static constexpr int OFF_Q16 = OFF_RED + 2048;
   static constexpr int F16_TILE = 128 * D * 2;
   static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int N_BARS = 2 * NS + 21;
+  static constexpr int N_BARS = 2 * NK + 2 * NVS + 2 * NP + 17;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
+  static_assert(kSplit || NK == NVS, "a single ring has one stage count");
   // TMEM columns. S_b at T_S + 128 b; Q scale factors in two slots by item parity, K and V
   // scale factors in two slots by tile parity (8 columns each: a slot is rewritten only after
   // the MMA two items / tiles back that read it has completed).
@@ -146,19 +171,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // than one phase ahead of a barrier (a parity wait cannot tell phase k from phase k - 2).
   uint64_t* q_full = bars + 0;             // [2], by item parity
   uint64_t* q_empty = bars + 2;            // [2], by item parity
-  uint64_t* kv_full = bars + 4;
-  uint64_t* kv_empty = kv_full + L::NS;
-  uint64_t* s_full = kv_empty + L::NS;     // [2], by tile parity
+  uint64_t* k_full = bars + 4;             // [NK]
+  uint64_t* k_empty = k_full + L::NK;
+  uint64_t* v_full = L::kSplit ? k_empty + L::NK : k_full;       // [NVS]
+  uint64_t* v_empty = L::kSplit ? v_full + L::NVS : k_empty;
+  uint64_t* s_full = bars + 4 + 2 * L::NK + 2 * L::NVS;          // [2], by tile parity
   uint64_t* s_free = s_full + 2;           // [2], by tile parity
-  uint64_t* p_full = s_full + 4;           // [2], by tile parity
-  uint64_t* pv_done = s_full + 6;          // [2], by tile parity
-  uint64_t* m_ready = s_full + 8;          // [2], by tile parity: running max handed on
-  uint64_t* o_free = s_full + 10;          // the epilogue has read O
-  uint64_t* kv16_full = s_full + 11;
-  uint64_t* kv16_empty = s_full + 12;
-  uint64_t* q16_full = s_full + 13;
-  uint64_t* q16_empty = s_full + 14;
-  uint64_t* mma_final = s_full + 15;       // [2]: QK issuer, PV issuer
+  uint64_t* m_ready = s_full + 4;          // [2], by tile parity: running max handed on
+  uint64_t* o_free = s_full + 6;           // the epilogue has read O
+  uint64_t* kv16_full = s_full + 7;
+  uint64_t* kv16_empty = s_full + 8;
+  uint64_t* q16_full = s_full + 9;
+  uint64_t* q16_empty = s_full + 10;
+  uint64_t* mma_final = s_full + 11;       // [2]: QK issuer, PV issuer
+  uint64_t* p_full = s_full + 13;          // [NP], by tile number mod NP
+  uint64_t* pv_done = p_full + L::NP;      // [NP], by tile number mod NP
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L::N_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -169,15 +196,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     // full barriers: the TMA's expect-tx arrival plus one cp.async arrival per producer lane
     for (int i = 0; i < 2; ++i) { mbar_init(q_full + i, 33); mbar_init(q_empty + i, 1); }
-    // a stage is free once both the QK^T (K) and the PV (V) issuers are done with it
-    for (int s = 0; s < L::NS; ++s) { mbar_init(kv_full + s, 33); mbar_init(kv_empty + s, 2); }
+    // full: the TMA's expect-tx arrival plus one cp.async arrival per producer lane (a single
+    // ring: K and V on one barrier; its empty barrier takes both issuers' commits)
+    if constexpr (L::kSplit) {
+      for (int s = 0; s < L::NK; ++s) { mbar_init(k_full + s, 33); mbar_init(k_empty + s, 1); }
+      for (int s = 0; s < L::NVS; ++s) { mbar_init(v_full + s, 33); mbar_init(v_empty + s, 1); }
+    } else {
+      for (int s = 0; s < L::NK; ++s) { mbar_init(k_full + s, 33); mbar_init(k_empty + s, 2); }
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_free + i, 4);
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 4);
-      mbar_init(pv_done + i, 1);
       mbar_init(m_ready + i, 4);
     }
+    for (int i = 0; i < L::NP; ++i) { mbar_init(p_full + i, 4); mbar_init(pv_done + i, 1); }
     mbar_init(o_free, 8);
     mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1);
     mbar_init(q16_full, 1); mbar_init(q16_empty, 1);
@@ -190,15 +222,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // Every byte of a ones row is equal, so the 128-byte swizzle leaves them unchanged.
   for (int i = threadIdx.x; i < 128; i += blockDim.x)
     reinterpret_cast<uint32_t*>(sm + L::OFF_PSF)[i] = 0x7F7F7F7Fu;
-  for (int s = 0; s < L::NS; ++s)
+  for (int s = 0; s < L::NVS; ++s)
     for (int i = threadIdx.x; i < 16 * 128 / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(sm + L::OFF_STAGE + s * L::STAGE_BYTES + L::ST_V + L::V_TMA_BYTES)[i] =
+      reinterpret_cast<uint4*>(sm + L::v_off(s) + L::V_TMA_BYTES)[i] =
           make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
   if constexpr (D < 128) {
-    for (int s = 0; s < L::NS; ++s)
+    for (int s = 0; s < L::NVS; ++s)
       for (int i = threadIdx.x; i < 128; i += blockDim.x)
         if (((i >> 2) & 31) + 32 * (i & 3) >= D)       // word i: row (i/4)%32 + 32 (i%4)
-          reinterpret_cast<uint32_t*>(sm + L::OFF_STAGE + s * L::STAGE_BYTES + L::ST_VSF)[i] = 0x7F7F7F7Fu;
+          reinterpret_cast<uint32_t*>(sm + L::v_sf_off(s))[i] = 0x7F7F7F7Fu;
   }
   if constexpr (kMixed) {
     for (int h = 0; h < 2; ++h)
@@ -229,15 +261,97 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   auto wait1 = [&](uint64_t* bar, uint32_t parity, int tile) -> bool {
     return bounded_wait(bar, parity, abort_flag, site(bar, tile));
   };
+  // Producer steps (one warp): key tile j (the CTA's g-th) of an item into K stage g % NK /
+  // V stage g % NVS. Scale factors go straight from global memory into the tcgen05 scale
+  // layout with 4-byte asynchronous copies (row r = r0 + 32 r1 of a 128-row chunk -> byte
+  // r0*16 + r1*4; one 4-byte word holds the 4 scales of one 64-element MMA step, or the 4
+  // E8M0 scales of a V channel row), completing on the same barrier as the TMA of the codes,
+  // so the producer never waits on their latency.
+  auto load_k = [&](int g, int j, const FwdItem& w) -> bool {
+    const int s = g % L::NK;
+    if (g >= L::NK && !waitw(k_empty + s, ((g / L::NK) - 1) & 1, g)) return false;
+    unsigned char* st = sm + L::k_off(s);
+    unsigned char* sf = sm + L::k_sf_off(s);
+    const int64_t krow0 = static_cast<int64_t>(w.bhk) * a.Nk + j * 128;
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) {
+      const int r = r1 * 32 + lane;
+      const bool valid = j * 128 + r < a.Nk;             // rows past Nk read as zero
+      const uint8_t* src = a.k_scales + (valid ? (krow0 + r) * (D / 16) : 0);
+#pragma unroll
+      for (int kk = 0; kk < L::KSTEPS; ++kk)
+        cp_async4(sf + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
+    }
+    cp_async_arrive_noinc(k_full + s);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(k_full + s, L::K_BYTES);
+      tma_load_3d(st, &tm_k, k_full + s, 0, j * 128, w.bhk);
+    }
+    return true;
+  };
+  auto load_v = [&](int g, int j, const FwdItem& w) -> bool {
+    const int s = g % L::NVS;
+    if (g >= L::NVS && !waitw(v_empty + s, ((g / L::NVS) - 1) & 1, g)) return false;
+    unsigned char* st = sm + L::v_off(s);
+    unsigned char* sf = sm + L::v_sf_off(s);
+    // rows from D on (the ones rows) hold 1.0 set once at start
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) {
+      const int r = r1 * 32 + lane;
+      if (r < D)
+        cp_async4(sf + lane * 16 + r1 * 4,
+                  a.v_scales + (static_cast<int64_t>(w.bhk) * D + r) * (a.Npad / 32) + j * 4, true);
+    }
+    cp_async_arrive_noinc(v_full + s);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(v_full + s, L::V_TMA_BYTES);
+      tma_load_2d(st, &tm_v, v_full + s, j * 128, w.bhk * D);
+    }
+    return true;
+  };
+  // Both halves of a single-ring stage with one arrival per lane and one TMA transaction count
+  // (measured faster than two arrivals on the same barrier).
+  auto load_kv = [&](int g, int j, const FwdItem& w) -> bool {
+    const int s = g % L::NK;
+    if (g >= L::NK && !waitw(k_empty + s, ((g / L::NK) - 1) & 1, g)) return false;
+    unsigned char* ksf = sm + L::k_sf_off(s);
+    unsigned char* vsf = sm + L::v_sf_off(s);
+    const int64_t krow0 = static_cast<int64_t>(w.bhk) * a.Nk + j * 128;
+#pragma unroll
+    for (int r1 = 0; r1 < 4; ++r1) {
+      const int r = r1 * 32 + lane;
+      const bool valid = j * 128 + r < a.Nk;
+      const uint8_t* src = a.k_scales + (valid ? (krow0 + r) * (D / 16) : 0);
+#pragma unroll
+      for (int kk = 0; kk < L::KSTEPS; ++kk)
+        cp_async4(ksf + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
+      if (r < D)
+        cp_async4(vsf + lane * 16 + r1 * 4,
+                  a.v_scales + (static_cast<int64_t>(w.bhk) * D + r) * (a.Npad / 32) + j * 4, true);
+    }
+    cp_async_arrive_noinc(k_full + s);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(k_full + s, L::K_BYTES + L::V_TMA_BYTES);
+      tma_load_3d(sm + L::k_off(s), &tm_k, k_full + s, 0, j * 128, w.bhk);
+      tma_load_2d(sm + L::v_off(s), &tm_v, k_full + s, j * 128, w.bhk * D);
+    }
+    return true;
+  };
+  // Drain of a ring: wait for the last copy issued into each stage (n = tiles issued).
+  auto drain = [&](uint64_t* full, int n_stages, int n) {
+    for (int s = 0; s < n_stages && s < n; ++s) {
+      const int last = s + ((n - 1 - s) / n_stages) * n_stages;
+      mbar_wait(full + s, (last / n_stages) & 1);
+    }
+  };
 
   if (warp == 0) {
     // ================================ producer ================================
     if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); }
-    // Scale factors go straight from global memory into the tcgen05 scale layout with 4-byte
-    // asynchronous copies (row r = r0 + 32 r1 of a 128-row chunk -> byte r0*16 + r1*4; one
-    // 4-byte word holds the 4 scales of one 64-element MMA step), completing on the same
-    // barrier as the TMA of the codes, so this warp never waits on their latency.
-    int g = 0, q_issued = 0;
+    int g = 0, q_issued = 0, k_issued = 0, v_issued = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const int idx = fwd_item_index(it, G, cta);
@@ -266,39 +380,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         q_issued = it + 1;
       }
       for (int j = 0; j < w.nt; ++j, ++g) {
-        const int s = g % L::NS;
-        if (g >= L::NS && !waitw(kv_empty + s, ((g / L::NS) - 1) & 1, g)) { ok = false; break; }
-        unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
-        // K scale factors of keys j*128 .. j*128+127; V scale factors of this key tile
-        // (channel row c, 4 E8M0 codes of 32 tokens each). Rows past Nk read as zero; V rows
-        // from D on (the ones rows) hold 1.0 set once at start.
-        const int64_t krow0 = static_cast<int64_t>(w.bhk) * a.Nk + j * 128;
-#pragma unroll
-        for (int r1 = 0; r1 < 4; ++r1) {
-          const int r = r1 * 32 + lane;
-          const bool valid = j * 128 + r < a.Nk;
-          const uint8_t* src = a.k_scales + (valid ? (krow0 + r) * (D / 16) : 0);
-#pragma unroll
-          for (int kk = 0; kk < L::KSTEPS; ++kk)
-            cp_async4(st + L::ST_KSF + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
-          if (r < D)
-            cp_async4(st + L::ST_VSF + lane * 16 + r1 * 4,
-                      a.v_scales + (static_cast<int64_t>(w.bhk) * D + r) * (a.Npad / 32) + j * 4, true);
-        }
-        cp_async_arrive_noinc(kv_full + s);
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(kv_full + s, L::K_BYTES + L::V_TMA_BYTES);
-          tma_load_3d(st + L::ST_K, &tm_k, kv_full + s, 0, j * 128, w.bhk);
-          tma_load_2d(st + L::ST_V, &tm_v, kv_full + s, j * 128, w.bhk * D);
+        if constexpr (L::kSplit) {
+          if (!load_k(g, j, w)) { ok = false; break; }
+          k_issued = g + 1;
+          if (!load_v(g, j, w)) { ok = false; break; }
+          v_issued = g + 1;
+        } else {
+          if (!load_kv(g, j, w)) { ok = false; break; }
+          k_issued = g + 1;
         }
       }
     }
-    // Drain: never leave a copy in flight into this CTA's shared memory (g = tiles issued).
-    for (int s = 0; s < L::NS && s < g; ++s) {
-      const int last = s + ((g - 1 - s) / L::NS) * L::NS;
-      mbar_wait(kv_full + s, (last / L::NS) & 1);
-    }
+    // Drain: never leave a copy in flight into this CTA's shared memory.
+    drain(k_full, L::NK, k_issued);
+    drain(v_full, L::NVS, v_issued);
     for (int qb = 0; qb < 2 && qb < q_issued; ++qb) {
       const int last = qb + ((q_issued - 1 - qb) / 2) * 2;
       mbar_wait(q_full + qb, (last >> 1) & 1);
@@ -370,19 +465,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t sQ = smem_u32(sm + L::OFF_Q + qb * L::Q_BYTES);
         bool q16_ready = false, had16 = false;
         for (int j = 0; j < w.nt; ++j, ++g) {
-          const int s = g % L::NS;
+          const int s = g % L::NK;
           const bool f16 = kMixed && bm_row[j];
-          if (!wait1(kv_full + s, (g / L::NS) & 1, g)) { ok = false; break; }
+          if (!wait1(k_full + s, (g / L::NK) & 1, g)) { ok = false; break; }
           fence_proxy_async_smem();
           // S_{g&1} (and K scale slot g&1) were last used by tile g - 2
           if (g >= 2 && !wait1(s_free + (g & 1), ((g - 2) >> 1) & 1, g)) { ok = false; break; }
           tc_fence_after();
           const uint32_t tS = tbase + L::T_S + (g & 1) * 128;
           if (!f16) {
-            unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
             const uint32_t tk = tbase + L::T_KSF + 8 * (g & 1);
-            for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, st + L::ST_KSF + kk * 512);
-            const uint32_t sK = smem_u32(st + L::ST_K);
+            for (int kk = 0; kk < L::KSTEPS; ++kk) tmem_cp_sf(tk + 4 * kk, sm + L::k_sf_off(s) + kk * 512);
+            const uint32_t sK = smem_u32(sm + L::k_off(s));
             for (int kk = 0; kk < L::KSTEPS; ++kk) {
               const uint64_t da = make_sdesc(sQ + kk * 32, 16, L::QK_SBO, L::QK_SW);
               const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
@@ -406,7 +500,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
           }
           mma_commit(s_full + (g & 1));
-          mma_commit(kv_empty + s);                  // K half of the stage is free
+          mma_commit(k_empty + s);
         }
         if (!ok) break;
         mma_commit(q_empty + qb);                    // Q buffer qb is free
@@ -438,21 +532,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // the first PV of an item overwrites O: the previous item's epilogue must have read it
         if (it >= 1 && !wait1(o_free, (it - 1) & 1, g)) { ok = false; break; }
         for (int j = 0; j < w.nt; ++j, ++g) {
-          const int s = g % L::NS, b2 = g & 1;
+          const int s = g % L::NVS, b2 = g & 1, pb = g % L::NP;
           const bool f16 = kMixed && bm_row[j];
-          if (!wait1(p_full + b2, (g >> 1) & 1, g)) { ok = false; break; }
-          if (!wait1(kv_full + s, (g / L::NS) & 1, g)) { ok = false; break; }
+          if (!wait1(p_full + pb, (g / L::NP) & 1, g)) { ok = false; break; }
+          if (!wait1(v_full + s, (g / L::NVS) & 1, g)) { ok = false; break; }
           if (f16 && !wait1(kv16_full, n16 & 1, g)) { ok = false; break; }
           fence_proxy_async_smem();
           tc_fence_after();
           if (!f16) {
-            unsigned char* st = sm + L::OFF_STAGE + s * L::STAGE_BYTES;
             const uint32_t tv = tbase + L::T_VSF + 8 * b2;   // PV(g-2), its last reader, is done
-            tmem_cp_sf(tv, st + L::ST_VSF);
-            const uint32_t sV = smem_u32(st + L::ST_V);
+            tmem_cp_sf(tv, sm + L::v_sf_off(s));
+            const uint32_t sV = smem_u32(sm + L::v_off(s));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t da = make_sdesc(sP + b2 * 16384 + kk * 32, 16, 1024, kSw128);
+              const uint64_t da = make_sdesc(sP + pb * 16384 + kk * 32, 16, 1024, kSw128);
               const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
               mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
                        (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
@@ -469,8 +562,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             mma_commit(kv16_empty);
           }
-          mma_commit(pv_done + b2);
-          mma_commit(kv_empty + s);                  // V half of the stage is free
+          mma_commit(pv_done + pb);
+          mma_commit(v_empty + s);
         }
       }
       mma_commit(mma_final + 1);
@@ -511,6 +604,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!ok) continue;
         const int gg = g0 + j;
         const int b2 = gg & 1;               // == grp
+        const int pb = gg % L::NP;           // P buffer
         const bool f16 = kMixed && bm_row[j];
         const bool prev_f16 = kMixed && (j >= 1 ? bm_row[j - 1] != 0 : prev_last_f16);
         float x[128];
@@ -562,18 +656,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const bool dead = (m_new == -INFINITY);
         const float bias = kLog2_448 - (dead ? 0.f : m_new) * C;
         const float2 B2 = make_float2(bias, bias);
-        // P buffer b2 was last used by PV(gg-2). An FP16 tile's P fills both buffers: writing
-        // one needs PV(gg-1) done as well, and the tile after an FP16 tile too. PV(gg-2)'s
-        // completion implies PV(gg-3)'s, so the wait on the other parity's barrier is for its
-        // next phase. The waits come before the exponentials so that P can be stored 16 bytes
-        // at a time as it is produced (no register copy of the whole row).
-        if (gg >= 2 && !waitw(pv_done + b2, ((gg - 2) >> 1) & 1, gg)) { ok = false; continue; }
+        // P buffer pb was last used by PV(gg-NP), the last phase of its barrier that can have
+        // completed. An FP16 tile's P fills both buffers (NP = 2 in that kernel): writing one
+        // needs PV(gg-1) done as well, and the tile after an FP16 tile too. The waits come
+        // before the exponentials so that P can be stored 16 bytes at a time as it is produced
+        // (no register copy of the whole row).
+        if (gg >= L::NP && !waitw(pv_done + pb, ((gg - L::NP) / L::NP) & 1, gg)) { ok = false; continue; }
         if ((f16 || prev_f16) && gg >= 1 &&
-            !waitw(pv_done + ((gg - 1) & 1), ((gg - 1) >> 1) & 1, gg)) { ok = false; continue; }
+            !waitw(pv_done + (gg - 1) % L::NP, ((gg - 1) / L::NP) & 1, gg)) { ok = false; continue; }
         if (!f16) {
           // kPolyOf8 of every 8 groups of 4 scores take the FMA-pipe exponential, the rest the
           // special-function unit.
-          unsigned char* prow = sP + b2 * 16384 + row * 128;
+          unsigned char* prow = sP + pb * 16384 + row * 128;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {               // 16 keys per 16-byte chunk
             uint32_t w4[4];
@@ -614,40 +708,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         fence_proxy_async_smem();
         // O holds the item's tiles before j relative to m(j-1) = m_prev. Rows whose max rose
-        // at this tile are brought to m_new once PV(gg-1) is done (the next phase of that
-        // parity's barrier: PV(gg-2), waited above, implies PV(gg-3)); a warp whose rows all
-        // kept their max hands P on at once.
+        // at this tile are brought to m_new once PV(gg-1) is done; a warp whose rows all kept
+        // their max hands P on at once. Of the 16 ones columns only column D (l) is read, so
+        // only it is rescaled. All loads are issued before one wait.
         const float alpha = (m_prev == -INFINITY || dead) ? 1.f : ex2_approx((m_prev - m_new) * C);
         if (j >= 1 && !__all_sync(0xffffffffu, alpha == 1.f)) {
-          if (!waitw(pv_done + ((gg - 1) & 1), ((gg - 1) >> 1) & 1, gg)) { ok = false; continue; }
+          if (!waitw(pv_done + (gg - 1) % L::NP, ((gg - 1) / L::NP) & 1, gg)) { ok = false; continue; }
           tc_fence_after();
           const float2 A2 = make_float2(alpha, alpha);
+          uint32_t o[D], ol;
 #pragma unroll
-          for (int cc = 0; cc < D; cc += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + cc, o);
-            tmem_wait_ld();
+          for (int cc = 0; cc < D; cc += 32) tmem_ld32(tO + cc, o + cc);
+          tmem_ld1(tO + D, &ol);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              const float2 u = __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), A2);
-              o[k] = __float_as_uint(u.x);
-              o[k + 1] = __float_as_uint(u.y);
-            }
-            tmem_st32(tO + cc, o);
+          for (int k = 0; k < D; k += 2) {
+            const float2 u = __fmul2_rn(make_float2(__uint_as_float(o[k]), __uint_as_float(o[k + 1])), A2);
+            o[k] = __float_as_uint(u.x);
+            o[k + 1] = __float_as_uint(u.y);
           }
-          {
-            uint32_t o[16];
-            tmem_ld16(tO + D, o);
-            tmem_wait_ld();
+          ol = __float_as_uint(__uint_as_float(ol) * alpha);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st16(tO + D, o);
-          }
+          for (int cc = 0; cc < D; cc += 32) tmem_st32(tO + cc, o + cc);
+          tmem_st1(tO + D, &ol);
           tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full + b2);
+        if (lane == 0) mbar_arrive(p_full + pb);
       }
       g = g0 + w.nt;
       if constexpr (kMixed) prev_last_f16 = bm_row[w.nt - 1] != 0;
@@ -657,7 +745,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // final max, and the named barrier passes both on to the other group.
       const int owner = (g - 1) & 1;
       if (ok && grp == owner) {
-        ok = waitw(pv_done + owner, ((g - 1) >> 1) & 1, g - 1);
+        ok = waitw(pv_done + (g - 1) % L::NP, ((g - 1) / L::NP) & 1, g - 1);
         red_fin[(it & 1) * 128 + row] = m_last;
       }
       tc_fence_before();

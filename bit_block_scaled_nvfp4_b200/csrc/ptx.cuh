@@ -280,6 +280,12 @@ __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, const void* smem_chun
 // ---------------------------------------------------------------------------------------
 // tcgen05: TMEM <-> registers (32 lanes x 32-bit pattern; each thread owns one lane)
 // ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r[0]) : "memory");
+}
 #define QK4V8_R8(b) "=r"(r[b+0]), "=r"(r[b+1]), "=r"(r[b+2]), "=r"(r[b+3]), \
                     "=r"(r[b+4]), "=r"(r[b+5]), "=r"(r[b+6]), "=r"(r[b+7])
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
