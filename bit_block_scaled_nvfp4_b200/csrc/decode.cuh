@@ -74,6 +74,9 @@ struct DecLayout {
   static constexpr int THREADS = 256;
 };
 
+// GM: a compile-time bound on g (4, 8 or 16); the softmax reduces and exponentiates only
+// the first GM query columns of the N = 16 MMA operand (rows >= g of Q^T and P^T are zero).
+template <int GM>
 __global__ void __launch_bounds__(256, 2)
 decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
               const __grid_constant__ CUtensorMap tm_vp, DecArgs a) {
@@ -372,9 +375,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int r = wq * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
     const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
-    float m_run[16];
+    float m_run[GM];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) m_run[q] = -INFINITY;
+    for (int q = 0; q < GM; ++q) m_run[q] = -INFINITY;
     unsigned char* sP = sm + L::OFF_P;
     bool failed = false;
     for (int blk = 0; blk < nblk; ++blk) {
@@ -395,7 +398,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // next write cannot land before the others have read).
       float* rm = red_max + b2 * 64;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
+      for (int q = 0; q < GM; ++q) {
         x[q] = (valid && q < g) ? x[q] : -INFINITY;        // raw MMA units
         float mm;
         asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(mm) : "f"(x[q]));
@@ -404,10 +407,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (failed && lane == 0) *soft_flag = 1;
       named_bar_sync(1, 128);
       if (*soft_flag) break;
-      float alpha[16], moff[16];
+      float alpha[GM], moff[GM];
       bool all_one = true;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
+      for (int q = 0; q < GM; ++q) {
         const float mb = fmaxf(fmaxf(rm[q], rm[16 + q]), fmaxf(rm[32 + q], rm[48 + q]));
         const float m_new = fmaxf(m_run[q], mb);
         const bool dead = (m_new == -INFINITY);
@@ -416,9 +419,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         all_one = all_one && (alpha[q] == 1.f);
         m_run[q] = m_new;
       }
-      uint32_t codes[4];
+      uint32_t codes[GM / 4];
 #pragma unroll
-      for (int q = 0; q < 16; q += 4) {
+      for (int q = 0; q < GM; q += 4) {
         float p[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) p[i] = ex2_approx((x[q + i] - moff[q + i]) * C) * 448.f;
@@ -432,7 +435,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // P^T row q (query), column r (key), 128-byte swizzle.
       unsigned char* pb = sP + b2 * 2048;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
+      for (int q = 0; q < GM; ++q) {
         if (q < g)
           pb[q * 128 + ((((r >> 4) ^ (q & 7))) << 4) + (r & 15)] =
               static_cast<unsigned char>(codes[q >> 2] >> (8 * (q & 3)));
@@ -444,7 +447,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_ld16(tbase + L::T_L + lane_addr, reinterpret_cast<uint32_t*>(l));
         tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) { o[q] *= alpha[q]; l[q] *= alpha[q]; }
+        for (int q = 0; q < GM; ++q) { o[q] *= alpha[q]; l[q] *= alpha[q]; }
         tmem_st16(tbase + L::T_O + lane_addr, reinterpret_cast<uint32_t*>(o));
         tmem_st16(tbase + L::T_L + lane_addr, reinterpret_cast<uint32_t*>(l));
         tmem_wait_st();
@@ -460,7 +463,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_ld16(tbase + L::T_L + lane_addr, reinterpret_cast<uint32_t*>(l));
       tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
+      for (int q = 0; q < GM; ++q) {
         if (q < g) {
           part[q * q_stride + r] = o[q];
           // the merge works in log2 units: store m * C

@@ -403,7 +403,9 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   }
   static bool attr = false;
   if (!attr) {
-    if (!set_smem(decode_kernel, DecLayout::SMEM_ALLOC)) return QK4V8_ERR_CUDA;
+    if (!set_smem(decode_kernel<4>, DecLayout::SMEM_ALLOC) || !set_smem(decode_kernel<8>, DecLayout::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<16>, DecLayout::SMEM_ALLOC))
+      return QK4V8_ERR_CUDA;
     attr = true;
   }
   DecArgs a;
@@ -415,7 +417,11 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   a.n_splits = n_splits; a.split_tokens = p->split_tokens; a.num_pages = p->num_pages;
   a.softmax_scale = p->softmax_scale;
   dim3 grid(n_splits, p->kv_heads, p->num_seqs);
-  decode_kernel<<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  // the softmax handles the g = Hq / Hkv real query columns: an instance per bound on g
+  const int g = p->q_heads / p->kv_heads;
+  if (g <= 4) decode_kernel<4><<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  else if (g <= 8) decode_kernel<8><<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  else decode_kernel<16><<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   decode_merge_kernel<<<p->num_seqs * p->q_heads, 128, 0, stream>>>(
       a.ws, n_splits, static_cast<int32_t>(p->out_dtype), p->out, p->lse);

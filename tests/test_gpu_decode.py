@@ -59,7 +59,13 @@ def _oracle_decode(q, seqs, lens, hq, hkv, split, scale):
 
 @pytest.mark.parametrize("lens,hq,hkv,split", [([1, 200, 1000, 64, 129], 8, 2, 256),
                                                 ([5000, 333], 32, 8, 1024),
-                                                ([777], 16, 1, 128)])
+                                                ([777], 16, 1, 128),
+                                                # g = 8, 1, 3, 6: every softmax instance and
+                                                # partial groups of four query columns
+                                                ([300, 4100], 16, 2, 512),
+                                                ([64, 513], 4, 4, 128),
+                                                ([900], 6, 2, 256),
+                                                ([130, 700], 12, 2, 256)])
 def test_decode_parity(lens, hq, hkv, split):
     d = 128
     cache, table, seqs = _build(lens, hkv, d, seed=sum(lens))
