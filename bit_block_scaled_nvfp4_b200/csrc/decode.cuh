@@ -14,7 +14,7 @@
 // Partials (O unnormalised, m, l) go to the workspace; the merge kernel combines the splits:
 // M = max m_s, O = sum e^(m_s - M) O_s / sum e^(m_s - M) l_s.
 //
-// Warp roles (two CTAs per SM): warp 0 K producer (TMA of the two pages' K codes, K scale
+// Warp roles (two or three CTAs per SM): warp 0 K producer (TMA of the two pages' K codes, K scale
 // factors by 4-byte asynchronous copies into the tcgen05 layout), warp 7 V producer (TMA of V
 // codes, bulk copy of the pages' V scales), warp 1 QK^T issuer, warp 6 PV issuer (and the V
 // scale rearrangement), warps 2-5 softmax. K and V stages form separate rings.
@@ -37,11 +37,17 @@ struct DecArgs {
   float softmax_scale;
 };
 
+// GM: a compile-time bound on g (4, 8 or 16); the softmax reduces and exponentiates only
+// the first GM query columns of the N = 16 MMA operand (rows >= g of Q^T and P^T are zero).
+// With GM = 4 the kernel fits three CTAs per SM (80 registers, two stages per ring); the
+// wider instances keep two CTAs per SM and three stages.
+template <int GM>
 struct DecLayout {
+  static constexpr int CTAS_PER_SM = GM <= 4 ? 3 : 2;
   static constexpr int D = 128;
-  // Separate K and V rings (two CTAs per SM): a K stage is free after QK^T of its block, a
-  // V stage only after PV, so the next blocks' K loads do not wait for the softmax.
-  static constexpr int NK = 3, NVS = 3;
+  // Separate K and V rings: a K stage is free after QK^T of its block, a V stage only after
+  // PV, so the next blocks' K loads do not wait for the softmax.
+  static constexpr int NK = GM <= 4 ? 2 : 3, NVS = NK;
   static constexpr int OFF_Q = 0;                 // 16 rows x 64 B (SW64)
   static constexpr int OFF_QSF = 1024;            // 2 chunks
   static constexpr int OFF_PSF = 2048;            // 1 chunk
@@ -74,13 +80,11 @@ struct DecLayout {
   static constexpr int THREADS = 256;
 };
 
-// GM: a compile-time bound on g (4, 8 or 16); the softmax reduces and exponentiates only
-// the first GM query columns of the N = 16 MMA operand (rows >= g of Q^T and P^T are zero).
 template <int GM>
-__global__ void __launch_bounds__(256, 2)
+__global__ void __launch_bounds__(256, DecLayout<GM>::CTAS_PER_SM)
 decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
               const __grid_constant__ CUtensorMap tm_vp, DecArgs a) {
-  using L = DecLayout;
+  using L = DecLayout<GM>;
   constexpr int D = L::D;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(

@@ -373,7 +373,7 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
       p->kv_heads <= 0 || p->q_heads % p->kv_heads || p->max_context <= 0)
     return QK4V8_ERR_INVALID_ARG;
   if (p->split_tokens <= 0 || p->split_tokens % 128) return QK4V8_ERR_INVALID_ARG;
-  if (p->split_tokens > 64 * DecLayout::MAX_SPLIT_PAGES) return QK4V8_ERR_UNSUPPORTED;
+  if (p->split_tokens > 64 * DecLayout<4>::MAX_SPLIT_PAGES) return QK4V8_ERR_UNSUPPORTED;
   if (p->max_context > 64 * p->max_pages) return QK4V8_ERR_INVALID_ARG;
   if (p->out_dtype != QK4V8_F16 && p->out_dtype != QK4V8_BF16 && p->out_dtype != QK4V8_F32)
     return QK4V8_ERR_INVALID_ARG;
@@ -403,8 +403,8 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   }
   static bool attr = false;
   if (!attr) {
-    if (!set_smem(decode_kernel<4>, DecLayout::SMEM_ALLOC) || !set_smem(decode_kernel<8>, DecLayout::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<16>, DecLayout::SMEM_ALLOC))
+    if (!set_smem(decode_kernel<4>, DecLayout<4>::SMEM_ALLOC) || !set_smem(decode_kernel<8>, DecLayout<8>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<16>, DecLayout<16>::SMEM_ALLOC))
       return QK4V8_ERR_CUDA;
     attr = true;
   }
@@ -419,9 +419,9 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   dim3 grid(n_splits, p->kv_heads, p->num_seqs);
   // the softmax handles the g = Hq / Hkv real query columns: an instance per bound on g
   const int g = p->q_heads / p->kv_heads;
-  if (g <= 4) decode_kernel<4><<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
-  else if (g <= 8) decode_kernel<8><<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
-  else decode_kernel<16><<<grid, DecLayout::THREADS, DecLayout::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  if (g <= 4) decode_kernel<4><<<grid, DecLayout<4>::THREADS, DecLayout<4>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  else if (g <= 8) decode_kernel<8><<<grid, DecLayout<8>::THREADS, DecLayout<8>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  else decode_kernel<16><<<grid, DecLayout<16>::THREADS, DecLayout<16>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   decode_merge_kernel<<<p->num_seqs * p->q_heads, 128, 0, stream>>>(
       a.ws, n_splits, static_cast<int32_t>(p->out_dtype), p->out, p->lse);
