@@ -133,7 +133,9 @@ qk4v8_status qk4v8_selftest_wait_timeout(cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------------------------------------
-size_t quantize_nvfp4_workspace_size(void) { return 256; }
+// the amax pass's per-CTA maxima (at most kAmaxPartials)
+constexpr int kAmaxPartials = 1024;
+size_t quantize_nvfp4_workspace_size(void) { return 4 * kAmaxPartials; }
 
 qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,
                             int64_t row_stride, float tensor_scale_in, uint8_t* codes,
@@ -147,30 +149,34 @@ qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int3
   if (!aligned(x, 16) || !aligned(codes, 8) || (x16 != nullptr && !aligned(x16, 16)))
     return QK4V8_ERR_INVALID_ARG;
   if (!(tensor_scale_in > 0.f) &&
-      (workspace == nullptr || workspace_bytes < 4 || !aligned(workspace, 4)))
+      (workspace == nullptr || workspace_bytes < quantize_nvfp4_workspace_size() || !aligned(workspace, 4)))
     return QK4V8_ERR_INVALID_ARG;
   const int64_t blocks = rows * (cols / 16);
   const int grid = grid_for(blocks, 256);
-  unsigned int* amax = static_cast<unsigned int*>(workspace);
+  // amax pass: two CTAs per SM (at most kAmaxPartials), each writing one partial maximum
+  int64_t ag = (blocks + 255) / 256;
+  if (ag > 2 * kNumSMs) ag = 2 * kNumSMs;
+  const int agrid = static_cast<int>(ag < 1 ? 1 : ag);
+  static_assert(2 * kNumSMs <= kAmaxPartials, "amax partials");
+  float* amax = static_cast<float*>(workspace);
   if (!(tensor_scale_in > 0.f)) {
-    if (cudaMemsetAsync(amax, 0, 4, stream) != cudaSuccess) return QK4V8_ERR_CUDA;
     if (dtype == QK4V8_BF16)
-      nvfp4_amax_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+      nvfp4_amax_kernel<__nv_bfloat16><<<agrid, 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(x), rows, cols, row_stride, amax);
     else
-      nvfp4_amax_kernel<__half><<<grid, 256, 0, stream>>>(static_cast<const __half*>(x), rows,
-                                                          cols, row_stride, amax);
+      nvfp4_amax_kernel<__half><<<agrid, 256, 0, stream>>>(static_cast<const __half*>(x), rows,
+                                                           cols, row_stride, amax);
     if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   }
   __half* h = static_cast<__half*>(x16);
   if (dtype == QK4V8_BF16) {
     auto xb = static_cast<const __nv_bfloat16*>(x);
-    if (h) nvfp4_encode_kernel<__nv_bfloat16, true><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, tensor_scale_in, codes, scales, tensor_scale, h);
-    else nvfp4_encode_kernel<__nv_bfloat16, false><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, tensor_scale_in, codes, scales, tensor_scale, h);
+    if (h) nvfp4_encode_kernel<__nv_bfloat16, true><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
+    else nvfp4_encode_kernel<__nv_bfloat16, false><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
   } else {
     auto xh = static_cast<const __half*>(x);
-    if (h) nvfp4_encode_kernel<__half, true><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, tensor_scale_in, codes, scales, tensor_scale, h);
-    else nvfp4_encode_kernel<__half, false><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, tensor_scale_in, codes, scales, tensor_scale, h);
+    if (h) nvfp4_encode_kernel<__half, true><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
+    else nvfp4_encode_kernel<__half, false><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
   }
   return launch_status();
 }

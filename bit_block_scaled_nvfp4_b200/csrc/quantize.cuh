@@ -30,27 +30,49 @@ __device__ __forceinline__ float e4m3_code_to_float(uint32_t code) {
   return __low2float(e4m3x2_to_half2(code & 0xFFu));
 }
 
+// Element offset of 16-element block i (row i / bpr, block i % bpr of that row); a dense
+// tensor needs no division.
+__device__ __forceinline__ int64_t block_offset(int64_t i, uint32_t bpr, int64_t row_stride,
+                                                bool contiguous) {
+  if (contiguous) return i * 16;
+  const int64_t r = i / bpr;
+  return r * row_stride + static_cast<int64_t>(i - r * bpr) * 16;
+}
+
 // ---------------------------------------------------------------------------------------
-// Pass 1: tensor amax (as float bits; non-negative floats order like unsigned integers).
+// Pass 1: tensor amax. A grid of a few CTAs per SM; CTA c writes the maximum of |x| over its
+// share to partial[c] (no atomics, nothing to clear), and the encode pass reduces the
+// partials. Four blocks of 16 per thread are loaded before any is reduced.
 // ---------------------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const T* __restrict__ x, int64_t rows,
                                                          int32_t cols, int64_t row_stride,
-                                                         unsigned int* __restrict__ amax_bits) {
+                                                         float* __restrict__ partial) {
   const uint32_t blocks_per_row = static_cast<uint32_t>(cols / 16);
   const int64_t total = rows * blocks_per_row;
+  const bool contiguous = (row_stride == cols);
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
   float m = 0.f;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / blocks_per_row;
-    const uint32_t cb = static_cast<uint32_t>(i - r * blocks_per_row);
-    const uint4* p = reinterpret_cast<const uint4*>(x + r * row_stride + cb * 16);
-    const uint4 a = __ldg(p), b = __ldg(p + 1);
-    float f[16];
-    unpack8<T>(a, f);
-    unpack8<T>(b, f + 8);
+  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < total;
+       i0 += 4 * step) {
+    uint4 u[8];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) m = fmaxf(m, fabsf(f[k]));
+    for (int k = 0; k < 4; ++k) {
+      const int64_t i = i0 + k * step;
+      u[2 * k] = u[2 * k + 1] = make_uint4(0, 0, 0, 0);
+      if (i < total) {
+        const uint4* p = reinterpret_cast<const uint4*>(x + block_offset(i, blocks_per_row, row_stride, contiguous));
+        u[2 * k] = __ldg(p);
+        u[2 * k + 1] = __ldg(p + 1);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float f[8];
+      unpack8<T>(u[k], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -60,8 +82,23 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const T* __restrict__ x
   if (threadIdx.x == 0) {
     float t = 0.f;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t = fmaxf(t, wm[w]);
-    atomicMax(amax_bits, __float_as_uint(t));
+    partial[blockIdx.x] = t;
   }
+}
+
+// Maximum of n (<= 1024) partial maxima, by every thread of a 256-thread CTA.
+__device__ __forceinline__ float reduce_partials(const float* __restrict__ partial, int n) {
+  float m = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, partial[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) t = fmaxf(t, wm[w]);
+  return t;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -70,24 +107,23 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const T* __restrict__ x
 template <typename T, bool kWrite16>
 __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
     const T* __restrict__ x, int64_t rows, int32_t cols, int64_t row_stride,
-    const unsigned int* __restrict__ amax_bits, float tensor_scale_in,
+    const float* __restrict__ amax_partial, int32_t n_partial, float tensor_scale_in,
     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, float* __restrict__ ts_out,
     __half* __restrict__ x16) {
   float s_t;
   if (tensor_scale_in > 0.f) {
     s_t = tensor_scale_in;
   } else {
-    const float amax = __uint_as_float(*amax_bits);
+    const float amax = reduce_partials(amax_partial, n_partial);
     s_t = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 2688.f);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
   const uint32_t blocks_per_row = static_cast<uint32_t>(cols / 16);
   const int64_t total = rows * blocks_per_row;
+  const bool contiguous = (row_stride == cols);
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / blocks_per_row;
-    const uint32_t cb = static_cast<uint32_t>(i - r * blocks_per_row);
-    const uint4* p = reinterpret_cast<const uint4*>(x + r * row_stride + cb * 16);
+    const uint4* p = reinterpret_cast<const uint4*>(x + block_offset(i, blocks_per_row, row_stride, contiguous));
     const uint4 a = __ldg(p), b = __ldg(p + 1);
     float f[16];
     unpack8<T>(a, f);
@@ -110,7 +146,7 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
         w[k >> 3] |= byte << ((k & 7) * 4);
       }
     }
-    const int64_t blk = r * blocks_per_row + cb;
+    const int64_t blk = i;                        // outputs are dense: block i of row i / bpr
     *reinterpret_cast<uint2*>(codes + blk * 8) = make_uint2(w[0], w[1]);
     scales[blk] = static_cast<uint8_t>(sc);
     if constexpr (kWrite16) {
@@ -150,12 +186,20 @@ __global__ void __launch_bounds__(256) mxfp8_v_kernel(const T* __restrict__ v, i
   const int64_t bh = blockIdx.y;
   const int tok0 = tile_id * 128;
   // Load 128 tokens x D (16-byte chunks), zero past N.
+  // (256 threads: every load of the tile is in flight before the first shared store)
   constexpr int CH = D / 8;                       // chunks per token
-  for (int i = threadIdx.x; i < 128 * CH; i += blockDim.x) {
-    const int t = i / CH, c = i % CH;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (tok0 + t < N) u = __ldg(reinterpret_cast<const uint4*>(v + (bh * N + tok0 + t) * D + c * 8));
-    *reinterpret_cast<uint4*>(&tile[t * LD + c * 8]) = u;
+  constexpr int ITER = 128 * CH / 256;
+  uint4 u[ITER];
+#pragma unroll
+  for (int k = 0; k < ITER; ++k) {
+    const int i = threadIdx.x + k * 256, t = i / CH, c = i % CH;
+    u[k] = make_uint4(0, 0, 0, 0);
+    if (tok0 + t < N) u[k] = __ldg(reinterpret_cast<const uint4*>(v + (bh * N + tok0 + t) * D + c * 8));
+  }
+#pragma unroll
+  for (int k = 0; k < ITER; ++k) {
+    const int i = threadIdx.x + k * 256, t = i / CH, c = i % CH;
+    *reinterpret_cast<uint4*>(&tile[t * LD + c * 8]) = u[k];
   }
   __syncthreads();
   for (int task = threadIdx.x; task < D * 4; task += blockDim.x) {

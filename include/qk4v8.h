@@ -97,8 +97,8 @@ qk4v8_status qk4v8_selftest_exp2(const float* t, float* out, int32_t n, cudaStre
  * codes   [rows, cols/2] bytes out (8-byte aligned); scales [rows, cols/16] E4M3 codes out.
  * tensor_scale  one float out (s_t).
  * x16     optional [rows, cols] fp16 copy of x out (16-byte aligned), for FP16 tiles; or NULL.
- * workspace     >= quantize_nvfp4_workspace_size() bytes, 4-byte aligned (unused, may be
- *               NULL, when tensor_scale_in > 0).
+ * workspace     >= quantize_nvfp4_workspace_size() bytes, 4-byte aligned: the per-CTA
+ *               maxima of the amax pass (unused, may be NULL, when tensor_scale_in > 0).
  */
 size_t quantize_nvfp4_workspace_size(void);
 qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,

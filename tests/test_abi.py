@@ -58,7 +58,7 @@ FAKE = 1 << 20          # aligned fake device addresses: never dereferenced on t
 def test_quantize_nvfp4_validation(lib):
     f = lib.quantize_nvfp4
     ok = dict(x=FAKE, dt=1, rows=4, cols=64, stride=64, ts=0.0, codes=FAKE, scales=FAKE,
-              tsout=FAKE, x16=None, ws=FAKE, wsb=256)
+              tsout=FAKE, x16=None, ws=FAKE, wsb=4096)
 
     def call(**kw):
         a = dict(ok, **kw)
