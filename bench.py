@@ -35,12 +35,15 @@ from bit_block_scaled_nvfp4_b200 import workloads  # noqa: E402
 METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of HBM peak"
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu capture summarised
-# in profiles/ (attn_fwd_prefill_h16_n4096.md, decode_paged_decode_s64.md). Only workloads with
+# in profiles/ (attn_fwd_prefill_h16_n4096.md, attn_fwd_prefill_gqa_n32768.md,
+# decode_paged_decode_s64.md). Only workloads with
 # a capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
-    "prefill_h16_n4096": 18_160_384 + 512,
-    "paged_decode_s64": 2_170_615_000 + 13_027_072,
+    "prefill_h16_n4096": 18_165_760 + 1_024,
+    "prefill_gqa_n32768": 167_058_944 + 216_239_616,
+    "paged_decode_s64": 2_170_641_000 + 11_350_272,
 }
+KERNEL_TIMING = "CUDA graph of the kernel(s) alone, replayed after a 256 MB L2 flush, CUDA events"
 FP4_OVER_BF16 = 4.0          # nominal dense ratio 9 PF / 2.25 PF
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -165,26 +168,38 @@ def make_prefill_step(name):
     q, k, v = w.q.cuda(), w.k.cuda(), w.v.cuda()
     mixed = cfg.get("frac_bp", 0) > 0
     scale = 1.0 / math.sqrt(cfg["d"])
-    ev = {}
 
-    def step(q=q, k=k, v=v, mark=None):
-        q4 = api.quantize_nvfp4(q, want_fp16=mixed)
-        k4 = api.quantize_nvfp4(k, want_fp16=mixed)
-        v8 = api.quantize_mxfp8_v(v, want_fp16=mixed)
+    def quant(q=q, k=k, v=v):
+        return (api.quantize_nvfp4(q, want_fp16=mixed), api.quantize_nvfp4(k, want_fp16=mixed),
+                api.quantize_mxfp8_v(v, want_fp16=mixed))
+
+    def step(q=q, k=k, v=v):
+        q4, k4, v8 = quant(q, k, v)
         bitmap = None
         if mixed:
             _, _, bitmap = api.tile_score_select(q4, k4, cfg["causal"], cfg["frac_bp"])
-        if mark is not None:
-            mark[0].record()
-        out = api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=bitmap)
-        if mark is not None:
-            mark[1].record()
-        return out
+        return api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=bitmap)
+
+    prep = {}
+
+    def attn_only():
+        # the attention kernel alone, on inputs quantized (and scored) once beforehand
+        if not prep:
+            prep["in"] = quant()
+            prep["bm"] = (api.tile_score_select(prep["in"][0], prep["in"][1], cfg["causal"],
+                                                cfg["frac_bp"])[2] if mixed else None)
+        q4, k4, v8 = prep["in"]
+        return api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=prep["bm"])
 
     launches = 6 + (3 if mixed else 0)
     host = [w.q.pin_memory(), w.k.pin_memory(), w.v.pin_memory()]
+    # algorithmic quantize bytes: bf16 read once, NVFP4 codes + E4M3 scales (Q, K) and MXFP8
+    # codes + E8M0 scales (V) written, plus the fp16 copies the FP16 tiles read
+    nq, nk, nv = q.numel(), k.numel(), v.numel()
+    qbytes = (nq + nk) * (2 + 0.5 + 1 / 16) + nv * (2 + 1 + 1 / 32) + (2 * (nq + nk + nv) if mixed else 0)
     return dict(cfg=cfg, step=step, inputs=(q, k, v), host=host, launches=launches,
-                flops=prefill_flops(cfg), kind="prefill", ev=ev)
+                flops=prefill_flops(cfg), kind="prefill", quant=quant, quant_bytes=qbytes,
+                attn_only=attn_only)
 
 
 def make_decode_step(name):
@@ -202,19 +217,25 @@ def make_decode_step(name):
     ws = torch.empty(cfg["S"] * cfg["Hq"] * ((max(lens) + split - 1) // split) * (cfg["d"] + 2) * 4,
                      dtype=torch.uint8, device="cuda")
 
-    def step(q=q, table=table, ctx=ctx, mark=None):
-        q4 = api.quantize_nvfp4(q)
-        if mark is not None:
-            mark[0].record()
-        out = api.attn_qk4v8_decode_paged(q4, cache, table, ctx, max(lens), split, workspace=ws)
-        if mark is not None:
-            mark[1].record()
-        return out
+    def quant(q=q):
+        return api.quantize_nvfp4(q)
+
+    def step(q=q, table=table, ctx=ctx):
+        return api.attn_qk4v8_decode_paged(quant(q), cache, table, ctx, max(lens), split, workspace=ws)
+
+    prep = {}
+
+    def attn_only():
+        # decode + merge alone, on a query quantized once beforehand
+        if not prep:
+            prep["q4"] = quant()
+        return api.attn_qk4v8_decode_paged(prep["q4"], cache, table, ctx, max(lens), split, workspace=ws)
 
     kv, total = decode_bytes(lay)
     host = [workloads.make_decode_query(lay).pin_memory(), lay.page_table.pin_memory(), lay.lens.pin_memory()]
     return dict(cfg=cfg, step=step, inputs=(q, table, ctx), host=host, launches=4, kv_bytes=kv,
-                bytes=total, kind="decode", split=split, lay=lay)
+                bytes=total, kind="decode", split=split, lay=lay, quant=quant, attn_only=attn_only,
+                quant_bytes=q.numel() * (2 + 0.5 + 1 / 16))
 
 
 def capture_step(step):
@@ -246,6 +267,10 @@ def time_steps(st, K, W, world):
     e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     k0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     k1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    q0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    q1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    qgraph, _ = capture_step(st["quant"])      # the quantize kernels alone, as one graph
+    kgraph, _ = capture_step(st["attn_only"])  # the attention (or decode) kernels alone
     barrier(world)
     torch.cuda.synchronize()
     for i in range(K):                  # the step: one graph replay per step
@@ -254,13 +279,22 @@ def time_steps(st, K, W, world):
         graph.replay()
         e_ev[i].record()
     torch.cuda.synchronize()
-    for i in range(K):                  # the dominant kernel alone (eager launches, marked)
+    for i in range(K):                  # the dominant kernel alone, as a graph of its own
         flush.zero_()
-        step(mark=(k0[i], k1[i]))
+        k0[i].record()
+        kgraph.replay()
+        k1[i].record()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        q0[i].record()
+        qgraph.replay()
+        q1[i].record()
     torch.cuda.synchronize()
     barrier(world)
     step_ms = sum(s.elapsed_time(e) for s, e in zip(s_ev, e_ev)) / K
     kern_ms = sum(a.elapsed_time(b) for a, b in zip(k0, k1)) / K
+    st["quant_ms"] = sum(a.elapsed_time(b) for a, b in zip(q0, q1)) / K
     return step_ms, kern_ms
 
 
@@ -433,7 +467,7 @@ def main():
         peak = pk["bf16_tflops"] * FP4_OVER_BF16
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": NCU_TRAFFIC_BYTES.get(name),
-                "kernel": "attn_fwd_kernel", "peak_source": f"{src} bf16 x {FP4_OVER_BF16:g} (FP4 dense)",
+                "kernel": "attn_fwd_kernel", "timing": KERNEL_TIMING, "peak_source": f"{src} bf16 x {FP4_OVER_BF16:g} (FP4 dense)",
                 "mixed_fp4_fp8_bound_tflops": peak / 1.5}
     else:
         units = st["bytes"]
@@ -444,7 +478,7 @@ def main():
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "traffic": NCU_TRAFFIC_BYTES.get(name), "traffic_kernel": "decode_kernel",
-                "kernel": "decode_kernel + decode_merge_kernel",
+                "kernel": "decode_kernel + decode_merge_kernel", "timing": KERNEL_TIMING,
                 "peak_source": f"{src} hbm_gbs"}
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -456,6 +490,12 @@ def main():
             "roofline": roof,
             "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": st["launches"] * args.steps,
+            # the quantize kernels of the step, timed as a graph of their own after an L2 flush
+            # (algorithmic bytes: the amax pass's second read of each input is not counted)
+            "quantize": {"achieved_gbs": st["quant_bytes"] / (st["quant_ms"] * 1e-3) / 1e9,
+                         "peak_gbs": pk["hbm_gbs"],
+                         "frac": st["quant_bytes"] / (st["quant_ms"] * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "ms": st["quant_ms"], "bytes": st["quant_bytes"]},
             "device_status": status,
             "clocks": clk.summary()}
     if rank == 0 and not args.no_cpu_baseline:

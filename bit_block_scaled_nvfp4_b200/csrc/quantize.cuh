@@ -30,6 +30,15 @@ __device__ __forceinline__ float e4m3_code_to_float(uint32_t code) {
   return __low2float(e4m3x2_to_half2(code & 0xFFu));
 }
 
+// Markstein's correctly rounded division (round to nearest): with y = RN(1/b) and
+// q = RN(a y), which is within one ulp of a/b, the residual r = a - b q is exact as one FMA
+// and RN(q + r y) is RN(a/b), provided nothing under- or overflows.
+__device__ __forceinline__ float div_markstein(float a, float b, float y) {
+  const float q = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-b, q, a);
+  return __fmaf_rn(r, y, q);
+}
+
 // Element offset of 16-element block i (row i / bpr, block i % bpr of that row); a dense
 // tensor needs no division.
 __device__ __forceinline__ int64_t block_offset(int64_t i, uint32_t bpr, int64_t row_stride,
@@ -137,9 +146,16 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
     uint32_t w[2] = {0u, 0u};
     if (sbv != 0.f) {
       const float den = __fmul_rn(sbv, s_t);
+      // x / den correctly rounded, by Markstein's theorem where its conditions hold (the
+      // reciprocal correctly rounded, no intermediate over- or underflow: den within
+      // [2^-90, 2^90], and the quotients that decide a code are at most 8), else by IEEE
+      // division. The test is false for NaN and infinities.
+      const bool fast = (den >= 0x1p-90f && den <= 0x1p90f);
+      const float y = __frcp_rn(den);
 #pragma unroll
       for (int k = 0; k < 16; k += 2) {
-        const float q0 = __fdiv_rn(f[k], den), q1 = __fdiv_rn(f[k + 1], den);
+        const float q0 = fast ? div_markstein(f[k], den, y) : __fdiv_rn(f[k], den);
+        const float q1 = fast ? div_markstein(f[k + 1], den, y) : __fdiv_rn(f[k + 1], den);
         uint32_t byte = cvt_e2m1x2(q0, q1) & 0x77u;
         byte |= (__float_as_uint(f[k]) >> 31) << 3;
         byte |= (__float_as_uint(f[k + 1]) >> 31) << 7;

@@ -42,6 +42,19 @@ def test_nvfp4_ragged_shapes(shape, dtype):
     _nvfp4_equal(x, tensor_scale=0.0625)
 
 
+@pytest.mark.parametrize("ts", [None, 2.0 ** -120, 2.0 ** -95, 0.3, 1.7e5, 2.0 ** 85, 2.0 ** 100])
+def test_nvfp4_division_across_scale_ranges(ts):
+    """Element quotients x / (s_b s_t) with the divisor on both sides of the bounds of the
+    kernel's fast division (2^-90, 2^90) and far inside them, non-power-of-two scales, block
+    magnitudes spread over 24 octaves around the scale: codes bit-exact against the oracle."""
+    g = torch.Generator().manual_seed(17)
+    base = 1.0 if ts is None else ts
+    x = torch.randn(8192, 64, generator=g, dtype=torch.float64)
+    octave = torch.randint(-12, 13, (8192, 1), generator=g).double()
+    x = (x * base * 1.37 * torch.pow(2.0, octave)).to(torch.bfloat16)
+    _nvfp4_equal(x, tensor_scale=ts)
+
+
 def test_nvfp4_zero_tensor():
     g = api.quantize_nvfp4(torch.zeros(4, 64, dtype=torch.bfloat16, device=DEV))
     assert g.tensor_scale.item() == 1.0 and not g.codes.any() and not g.scales.any()
