@@ -758,6 +758,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_wait_ld();
         const float m_run = red_fin[(it & 1) * 128 + row];
         const float l_run = __uint_as_float(lr[0]);
+        const float inv_l = __frcp_rn(l_run);     // O / l by Markstein's division (ptx.cuh)
         const bool store = qi < a.Nq;
         const int64_t orow = static_cast<int64_t>(w.bhq) * a.Nq + qi;
 #pragma unroll
@@ -769,7 +770,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (store) {
             float v[32];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] = __fdiv_rn(__uint_as_float(o[k]), l_run);
+            for (int k = 0; k < 32; ++k) v[k] = div_markstein(__uint_as_float(o[k]), l_run, inv_l);
             if (a.out_kind == 2) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c);
 #pragma unroll

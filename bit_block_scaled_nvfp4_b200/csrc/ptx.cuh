@@ -331,6 +331,15 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Markstein's correctly rounded division (round to nearest): with y = RN(1/b) and
+// q = RN(a y), which is within one ulp of a/b, the residual r = a - b q is exact as one FMA
+// and RN(q + r y) is RN(a/b), provided nothing under- or overflows.
+__device__ __forceinline__ float div_markstein(float a, float b, float y) {
+  const float q = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-b, q, a);
+  return __fmaf_rn(r, y, q);
+}
+
 // Two E4M3 codes (low byte, high byte) -> half2 (exact).
 __device__ __forceinline__ __half2 e4m3x2_to_half2(uint32_t codes16) {
   uint32_t r;

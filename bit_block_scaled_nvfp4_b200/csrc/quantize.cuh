@@ -30,15 +30,6 @@ __device__ __forceinline__ float e4m3_code_to_float(uint32_t code) {
   return __low2float(e4m3x2_to_half2(code & 0xFFu));
 }
 
-// Markstein's correctly rounded division (round to nearest): with y = RN(1/b) and
-// q = RN(a y), which is within one ulp of a/b, the residual r = a - b q is exact as one FMA
-// and RN(q + r y) is RN(a/b), provided nothing under- or overflows.
-__device__ __forceinline__ float div_markstein(float a, float b, float y) {
-  const float q = __fmul_rn(a, y);
-  const float r = __fmaf_rn(-b, q, a);
-  return __fmaf_rn(r, y, q);
-}
-
 // Element offset of 16-element block i (row i / bpr, block i % bpr of that row); a dense
 // tensor needs no division.
 __device__ __forceinline__ int64_t block_offset(int64_t i, uint32_t bpr, int64_t row_stride,
