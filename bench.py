@@ -169,9 +169,22 @@ def make_prefill_step(name):
     mixed = cfg.get("frac_bp", 0) > 0
     scale = 1.0 / math.sqrt(cfg["d"])
 
+    side = (torch.cuda.Stream(), torch.cuda.Stream())
+
     def quant(q=q, k=k, v=v):
-        return (api.quantize_nvfp4(q, want_fp16=mixed), api.quantize_nvfp4(k, want_fp16=mixed),
-                api.quantize_mxfp8_v(v, want_fp16=mixed))
+        # Q, K and V are quantized on three streams (independent kernels that each leave most
+        # of the GPU idle when run alone); the caller's stream waits for all three.
+        main = torch.cuda.current_stream()
+        for s_ in side:
+            s_.wait_stream(main)
+        q4 = api.quantize_nvfp4(q, want_fp16=mixed)
+        with torch.cuda.stream(side[0]):
+            k4 = api.quantize_nvfp4(k, want_fp16=mixed)
+        with torch.cuda.stream(side[1]):
+            v8 = api.quantize_mxfp8_v(v, want_fp16=mixed)
+        for s_ in side:
+            main.wait_stream(s_)
+        return q4, k4, v8
 
     def step(q=q, k=k, v=v):
         q4, k4, v8 = quant(q, k, v)
