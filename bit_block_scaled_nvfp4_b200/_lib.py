@@ -55,6 +55,17 @@ class DecodeParams(C.Structure):
     ]
 
 
+class AppendParams(C.Structure):
+    _fields_ = [
+        ("k_new", vp), ("v_new", vp), ("dtype", i32),
+        ("cu_new", vp), ("lens", vp), ("page_table", vp),
+        ("k_pages", vp), ("k_page_scales", vp), ("k_tensor_scale", vp),
+        ("v_pages", vp), ("v_page_scales", vp), ("v_tail", vp),
+        ("num_seqs", i32), ("num_pages", i32), ("max_pages", i32), ("kv_heads", i32),
+        ("head_dim", i32), ("max_new", i32),
+    ]
+
+
 #: name -> (restype, argtypes); exactly the functions include/qk4v8.h declares.
 SIGNATURES = {
     "qk4v8_version": (C.c_int, []),
@@ -74,6 +85,7 @@ SIGNATURES = {
     "attn_qk4v8_decode_workspace_size": (sz, [C.POINTER(DecodeParams)]),
     "attn_qk4v8_decode_paged": (i32, [C.POINTER(DecodeParams), vp, sz, vp]),
     "attn_qk4v8_decode_paged_noalloc": (i32, [C.POINTER(DecodeParams), vp]),
+    "kv_append_paged": (i32, [C.POINTER(AppendParams), vp]),
 }
 
 _LIB = None

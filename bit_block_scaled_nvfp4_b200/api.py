@@ -250,6 +250,31 @@ def attn_qk4v8_decode_paged_noalloc(q: NVFP4Tensor, cache: PagedKV, page_table: 
     return (out, lse) if want_lse else out
 
 
+def kv_append_paged(cache: PagedKV, k_new: torch.Tensor, v_new: torch.Tensor,
+                    cu_new: torch.Tensor, lens: torch.Tensor, page_table: torch.Tensor,
+                    v_tail: torch.Tensor, max_new: int) -> None:
+    """Quantize new tokens into the paged cache in place. k_new, v_new [total_new, Hkv, D]
+    (fp16/bf16); cu_new [S + 1] int32 offsets of each sequence's new rows; lens [S] int32
+    lengths before the call (the caller adds the new counts); page_table [S, max_pages];
+    v_tail [S, Hkv, D, 32] of k_new's dtype, each sequence's incomplete V group, updated."""
+    lib = _lib.load()
+    for t in (k_new, v_new, cu_new, lens, page_table, v_tail):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("kv_append_paged needs contiguous CUDA tensors")
+    if v_new.dtype != k_new.dtype or v_tail.dtype != k_new.dtype:
+        raise ValueError("k_new, v_new and v_tail must share a dtype")
+    _, hkv, d = k_new.shape
+    p = _lib.AppendParams(
+        k_new=_ptr(k_new), v_new=_ptr(v_new), dtype=_dtype(k_new), cu_new=_ptr(cu_new),
+        lens=_ptr(lens), page_table=_ptr(page_table), k_pages=_ptr(cache.k_pages),
+        k_page_scales=_ptr(cache.k_scales), k_tensor_scale=_ptr(cache.k_tensor_scale),
+        v_pages=_ptr(cache.v_pages), v_page_scales=_ptr(cache.v_scales), v_tail=_ptr(v_tail),
+        num_seqs=lens.numel(), num_pages=cache.k_pages.shape[0], max_pages=page_table.shape[1],
+        kv_heads=hkv, head_dim=d, max_new=int(max_new))
+    st = lib.kv_append_paged(C.byref(p), _stream())
+    _lib.check(st, "kv_append_paged")
+
+
 def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool,
                     softmax_scale: float | None = None, fp16_frac_bp: int = 0,
                     out_dtype=None, want_lse: bool = False):

@@ -11,6 +11,7 @@
 #include "tilescore.cuh"
 #include "attn_fwd.cuh"
 #include "decode.cuh"
+#include "append.cuh"
 
 using namespace qk4v8;
 
@@ -83,7 +84,10 @@ extern "C" {
 int qk4v8_version(void) { return 100; }
 
 size_t qk4v8_struct_size(int32_t which) {
-  return which == 0 ? sizeof(qk4v8_fwd_params) : which == 1 ? sizeof(qk4v8_decode_params) : 0;
+  return which == 0   ? sizeof(qk4v8_fwd_params)
+         : which == 1 ? sizeof(qk4v8_decode_params)
+         : which == 2 ? sizeof(qk4v8_append_params)
+                      : 0;
 }
 
 const char* qk4v8_status_string(qk4v8_status s) {
@@ -469,4 +473,33 @@ extern "C" qk4v8_status attn_qk4v8_decode_paged_noalloc(const qk4v8_decode_param
     ptr = g_noalloc_ptr[dev];
   }
   return attn_qk4v8_decode_paged(p, ptr, QK4V8_NOALLOC_DECODE_SCRATCH_BYTES, stream);
+}
+
+// ------------------------------------------------------------------------------------------
+extern "C" qk4v8_status kv_append_paged(const qk4v8_append_params* p, cudaStream_t stream) {
+  if (p == nullptr || p->k_new == nullptr || p->v_new == nullptr || p->cu_new == nullptr ||
+      p->lens == nullptr || p->page_table == nullptr || p->k_pages == nullptr ||
+      p->k_page_scales == nullptr || p->k_tensor_scale == nullptr || p->v_pages == nullptr ||
+      p->v_page_scales == nullptr || p->v_tail == nullptr)
+    return QK4V8_ERR_INVALID_ARG;
+  if (p->dtype != QK4V8_F16 && p->dtype != QK4V8_BF16) return QK4V8_ERR_INVALID_ARG;
+  if (p->num_seqs <= 0 || p->kv_heads <= 0 || p->num_pages <= 0 || p->max_pages <= 0 ||
+      p->max_new < 0)
+    return QK4V8_ERR_INVALID_ARG;
+  if (p->head_dim != 128) return QK4V8_ERR_UNSUPPORTED;
+  if (p->num_seqs > 65535 || p->kv_heads > 65535) return QK4V8_ERR_UNSUPPORTED;
+  if (!aligned(p->k_new, 16) || !aligned(p->v_new, 16) || !aligned(p->k_pages, 8) ||
+      !aligned(p->v_pages, 16) || !aligned(p->v_tail, 2))
+    return QK4V8_ERR_INVALID_ARG;
+  AppendArgs a;
+  a.k_new = p->k_new; a.v_new = p->v_new; a.cu_new = p->cu_new; a.lens = p->lens;
+  a.page_table = p->page_table;
+  a.k_pages = p->k_pages; a.k_scales = p->k_page_scales; a.k_ts = p->k_tensor_scale;
+  a.v_pages = p->v_pages; a.v_scales = p->v_page_scales; a.v_tail = p->v_tail;
+  a.S = p->num_seqs; a.num_pages = p->num_pages; a.max_pages = p->max_pages;
+  a.Hkv = p->kv_heads; a.max_new = p->max_new;
+  const dim3 grid(p->kv_heads, p->num_seqs);
+  if (p->dtype == QK4V8_BF16) kv_append_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(a);
+  else kv_append_kernel<__half><<<grid, 128, 0, stream>>>(a);
+  return launch_status();
 }

@@ -101,6 +101,37 @@ __device__ __forceinline__ float reduce_partials(const float* __restrict__ parti
   return t;
 }
 
+// One 16-element NVFP4 block with tensor scale s_t: returns the E4M3 scale code and writes
+// the 8 code bytes (element 2i in the low nibble of byte i) to w[0..1].
+__device__ __forceinline__ uint32_t nvfp4_encode16(const float* f, float s_t, uint32_t* w) {
+  float amax_b = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(f[k]));
+  const float sbf = __fdiv_rn(__fdiv_rn(amax_b, 6.f), s_t);
+  const uint32_t sc = cvt_e4m3x2(sbf, 0.f) & 0xFFu;
+  const float sbv = e4m3_code_to_float(sc);
+  w[0] = w[1] = 0u;
+  if (sbv != 0.f) {
+    const float den = __fmul_rn(sbv, s_t);
+    // x / den correctly rounded, by Markstein's theorem where its conditions hold (the
+    // reciprocal correctly rounded, no intermediate over- or underflow: den within
+    // [2^-90, 2^90], and the quotients that decide a code are at most 8), else by IEEE
+    // division. The test is false for NaN and infinities.
+    const bool fast = (den >= 0x1p-90f && den <= 0x1p90f);
+    const float y = __frcp_rn(den);
+#pragma unroll
+    for (int k = 0; k < 16; k += 2) {
+      const float q0 = fast ? div_markstein(f[k], den, y) : __fdiv_rn(f[k], den);
+      const float q1 = fast ? div_markstein(f[k + 1], den, y) : __fdiv_rn(f[k + 1], den);
+      uint32_t byte = cvt_e2m1x2(q0, q1) & 0x77u;
+      byte |= (__float_as_uint(f[k]) >> 31) << 3;
+      byte |= (__float_as_uint(f[k + 1]) >> 31) << 7;
+      w[k >> 3] |= byte << ((k & 7) * 4);
+    }
+  }
+  return sc;
+}
+
 // ---------------------------------------------------------------------------------------
 // Pass 2: encode. One thread per 16-element block.
 // ---------------------------------------------------------------------------------------
@@ -128,31 +159,8 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
     float f[16];
     unpack8<T>(a, f);
     unpack8<T>(b, f + 8);
-    float amax_b = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(f[k]));
-    const float sbf = __fdiv_rn(__fdiv_rn(amax_b, 6.f), s_t);
-    const uint32_t sc = cvt_e4m3x2(sbf, 0.f) & 0xFFu;
-    const float sbv = e4m3_code_to_float(sc);
-    uint32_t w[2] = {0u, 0u};
-    if (sbv != 0.f) {
-      const float den = __fmul_rn(sbv, s_t);
-      // x / den correctly rounded, by Markstein's theorem where its conditions hold (the
-      // reciprocal correctly rounded, no intermediate over- or underflow: den within
-      // [2^-90, 2^90], and the quotients that decide a code are at most 8), else by IEEE
-      // division. The test is false for NaN and infinities.
-      const bool fast = (den >= 0x1p-90f && den <= 0x1p90f);
-      const float y = __frcp_rn(den);
-#pragma unroll
-      for (int k = 0; k < 16; k += 2) {
-        const float q0 = fast ? div_markstein(f[k], den, y) : __fdiv_rn(f[k], den);
-        const float q1 = fast ? div_markstein(f[k + 1], den, y) : __fdiv_rn(f[k + 1], den);
-        uint32_t byte = cvt_e2m1x2(q0, q1) & 0x77u;
-        byte |= (__float_as_uint(f[k]) >> 31) << 3;
-        byte |= (__float_as_uint(f[k + 1]) >> 31) << 7;
-        w[k >> 3] |= byte << ((k & 7) * 4);
-      }
-    }
+    uint32_t w[2];
+    const uint32_t sc = nvfp4_encode16(f, s_t, w);
     const int64_t blk = i;                        // outputs are dense: block i of row i / bpr
     *reinterpret_cast<uint2*>(codes + blk * 8) = make_uint2(w[0], w[1]);
     scales[blk] = static_cast<uint8_t>(sc);
@@ -180,6 +188,26 @@ __device__ __forceinline__ int floor_log2_pos(float a) {   // a > 0, finite
   const int ef = static_cast<int>(bits >> 23);
   if (ef > 0) return ef - 127;
   return (31 - __clz(bits & 0x7FFFFFu)) - 149;              // subnormal
+}
+
+// One MXFP8 group of 32 values: returns the shared exponent e (scale code e + 127) and writes
+// the 32 E4M3 codes of v * 2^-e to cb.
+__device__ __forceinline__ int mxfp8_encode32(const float* f, uint8_t* cb) {
+  float amax = 0.f;
+#pragma unroll
+  for (int t = 0; t < 32; ++t) amax = fmaxf(amax, fabsf(f[t]));
+  int e = 0;
+  if (amax > 0.f) e = max(-127, min(127, floor_log2_pos(amax) - 8));
+  const float mul = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+#pragma unroll
+  for (int t = 0; t < 32; t += 2) {
+    uint32_t two = cvt_e4m3x2(__fmul_rn(f[t], mul), __fmul_rn(f[t + 1], mul)) & 0x7F7Fu;
+    two |= (__float_as_uint(f[t]) >> 31) << 7;
+    two |= (__float_as_uint(f[t + 1]) >> 31) << 15;
+    cb[t] = static_cast<uint8_t>(two & 0xFF);
+    cb[t + 1] = static_cast<uint8_t>(two >> 8);
+  }
+  return e;
 }
 
 template <typename T, int D, bool kWrite16>
@@ -212,24 +240,10 @@ __global__ void __launch_bounds__(256) mxfp8_v_kernel(const T* __restrict__ v, i
   for (int task = threadIdx.x; task < D * 4; task += blockDim.x) {
     const int c = task % D, g = task / D;
     float f[32];
-    float amax = 0.f;
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      f[t] = to_float<T>(tile[(g * 32 + t) * LD + c]);
-      amax = fmaxf(amax, fabsf(f[t]));
-    }
-    int e = 0;
-    if (amax > 0.f) e = max(-127, min(127, floor_log2_pos(amax) - 8));
-    const float mul = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);   // 2^-e
+    for (int t = 0; t < 32; ++t) f[t] = to_float<T>(tile[(g * 32 + t) * LD + c]);
     __align__(16) uint8_t cb[32];
-#pragma unroll
-    for (int t = 0; t < 32; t += 2) {
-      uint32_t two = cvt_e4m3x2(__fmul_rn(f[t], mul), __fmul_rn(f[t + 1], mul)) & 0x7F7Fu;
-      two |= (__float_as_uint(f[t]) >> 31) << 7;
-      two |= (__float_as_uint(f[t + 1]) >> 31) << 15;
-      cb[t] = static_cast<uint8_t>(two & 0xFF);
-      cb[t + 1] = static_cast<uint8_t>(two >> 8);
-    }
+    const int e = mxfp8_encode32(f, cb);
     const int64_t rowc = bh * D + c;
     uint4* dst = reinterpret_cast<uint4*>(codes + rowc * Npad + tok0 + g * 32);
     dst[0] = *reinterpret_cast<uint4*>(cb);

@@ -25,6 +25,11 @@ def empty_cache(num_pages: int, kv_heads: int, head_dim: int, k_tensor_scale: fl
     )
 
 
+def empty_tail(num_seqs: int, kv_heads: int, head_dim: int, dtype, device) -> torch.Tensor:
+    """The per-sequence incomplete-V-group state that kv_append_paged reads and updates."""
+    return torch.zeros(num_seqs, kv_heads, head_dim, 32, dtype=dtype, device=device)
+
+
 def write_sequence(cache: PagedKV, k: torch.Tensor, v: torch.Tensor, pages: torch.Tensor) -> None:
     """Quantize one sequence's K, V ([len, Hkv, D] on the cache's device) into the physical
     pages ``pages`` (int tensor of ceil(len/64) ids)."""

@@ -47,7 +47,8 @@ typedef enum { QK4V8_F16 = 0, QK4V8_BF16 = 1, QK4V8_F32 = 2 } qk4v8_dtype;
 int qk4v8_version(void);
 
 /* sizeof the parameter structs, for bindings that mirror them: which = 0 gives
- * sizeof(qk4v8_fwd_params), 1 gives sizeof(qk4v8_decode_params), anything else 0. */
+ * sizeof(qk4v8_fwd_params), 1 sizeof(qk4v8_decode_params), 2 sizeof(qk4v8_append_params),
+ * anything else 0. */
 size_t qk4v8_struct_size(int32_t which);
 
 /* Human-readable name of a status code (static string). */
@@ -239,6 +240,48 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* params, void* wo
 #define QK4V8_NOALLOC_DECODE_SCRATCH_BYTES (16u * 1024u * 1024u)
 qk4v8_status attn_qk4v8_decode_paged_noalloc(const qk4v8_decode_params* params,
                                              cudaStream_t stream);
+
+/*
+ * kv_append_paged — quantize new tokens' K and V into the paged NVFP4-K / MXFP8-V cache that
+ * attn_qk4v8_decode_paged reads (hotelren.com MpFA article §6: QK4V8 combined with paged KV
+ * management; sns.style BitDecoding-FP4 summary: a native FP4 paged KV cache, filled as the
+ * sequence grows). For sequence s the new tokens are rows cu_new[s] .. cu_new[s+1]-1 of
+ * k_new / v_new and take positions lens[s] .. lens[s] + n_s - 1 (n_s = cu_new[s+1] -
+ * cu_new[s] >= 0); position t lives in physical page page_table[s][t / 64], slot t % 64.
+ *   K: NVFP4 per 16 channels with the cache's fixed tensor scale (the quantize_nvfp4
+ *      arithmetic with tensor_scale_in = *k_tensor_scale), per token.
+ *   V: MXFP8 per channel and 32-token group (groups aligned at position 0). Every group the
+ *      new tokens fall in is encoded again from all of its tokens so far, the earlier ones
+ *      taken from v_tail, so after the call the sequence's pages hold exactly what
+ *      quantize_mxfp8_v gives for the whole prefix (codes past the new length are 0).
+ * k_new, v_new  [total_new, Hkv, D] fp16/bf16 (dtype), token-major, 16-byte aligned.
+ * cu_new        [S + 1] int32, cu_new[0] = 0, nondecreasing, cu_new[S] = total_new.
+ * lens          [S] int32 lengths before the call (not modified; the caller adds n_s).
+ * v_tail        [S, Hkv, D, 32] of dtype, caller-owned state: for each sequence the tokens of
+ *               its last, incomplete V group in the input precision (position 32*(len/32) + i
+ *               at index i). Read and rewritten by every call; zero it for a new sequence.
+ * max_new       host-side bound on n_s (sizes nothing on the device; n_s above it is an
+ *               error). head_dim must be 128.
+ * Device checks: a page id outside [0, num_pages) or a position at or past 64 * max_pages
+ * sets QK4V8_ERR_BOUNDS (reported by qk4v8_check_status) and that token is not written.
+ */
+typedef struct {
+  const void* k_new;           /* [total_new, Hkv, D] */
+  const void* v_new;           /* [total_new, Hkv, D] */
+  qk4v8_dtype dtype;
+  const int32_t* cu_new;       /* [S + 1] */
+  const int32_t* lens;         /* [S] */
+  const int32_t* page_table;   /* [S, max_pages] */
+  uint8_t* k_pages;            /* [num_pages, Hkv, 64, D/2] */
+  uint8_t* k_page_scales;      /* [num_pages, Hkv, 64, D/16] */
+  const float* k_tensor_scale;
+  uint8_t* v_pages;            /* [num_pages, Hkv, D, 64] */
+  uint8_t* v_page_scales;      /* [num_pages, Hkv, D, 2] */
+  void* v_tail;                /* [S, Hkv, D, 32] of dtype */
+  int32_t num_seqs, num_pages, max_pages, kv_heads, head_dim, max_new;
+} qk4v8_append_params;
+
+qk4v8_status kv_append_paged(const qk4v8_append_params* params, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -144,3 +144,27 @@ def test_decode_validation_and_workspace(lib):
     assert f(_dec(q_heads=64, kv_heads=2)) == _lib.QK4V8_ERR_UNSUPPORTED  # g = 32 > 16
     assert f(_dec(), wsb=16) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(_dec(page_table=None)) == _lib.QK4V8_ERR_INVALID_ARG
+
+
+def _app(**kw):
+    p = _lib.AppendParams(k_new=FAKE, v_new=FAKE, dtype=_lib.QK4V8_BF16, cu_new=FAKE, lens=FAKE,
+                          page_table=FAKE, k_pages=FAKE, k_page_scales=FAKE, k_tensor_scale=FAKE,
+                          v_pages=FAKE, v_page_scales=FAKE, v_tail=FAKE, num_seqs=4,
+                          num_pages=64, max_pages=16, kv_heads=8, head_dim=128, max_new=32)
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_append_validation(lib):
+    f = lambda p: lib.kv_append_paged(C.byref(p), None)
+    assert lib.qk4v8_struct_size(2) == C.sizeof(_lib.AppendParams)
+    assert f(_app(v_tail=None)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_app(cu_new=None)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_app(dtype=_lib.QK4V8_F32)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_app(num_seqs=0)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_app(max_new=-1)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_app(head_dim=64)) == _lib.QK4V8_ERR_UNSUPPORTED
+    assert f(_app(num_seqs=70000)) == _lib.QK4V8_ERR_UNSUPPORTED
+    assert f(_app(k_new=FAKE + 8)) == _lib.QK4V8_ERR_INVALID_ARG    # not 16-byte aligned
+    assert f(_app(v_pages=FAKE + 4)) == _lib.QK4V8_ERR_INVALID_ARG
