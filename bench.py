@@ -251,6 +251,51 @@ def make_decode_step(name):
                 quant_bytes=q.numel() * (2 + 0.5 + 1 / 16))
 
 
+def make_append(cfg, chunk=512, seed=7):
+    """The KV producer side of decode: quantize-on-append into a paged cache of the decode
+    workload's shape (its sequences, KV heads and head_dim), one token per sequence (a decode
+    step) and a chunk of ``chunk`` tokens per sequence (a prompt chunk). Each call appends at
+    fixed positions (the lengths are not advanced), so repeated calls rewrite the same bytes.
+    Algorithmic bytes: the new K/V read (2 x Hkv x d x 2 B per token), K codes + scales written
+    (Hkv x (d/2 + d/16) B per token) and the V codes + scale of every touched 32-token group
+    (Hkv x d x (32 + 1) B per group)."""
+    from bit_block_scaled_nvfp4_b200 import api, paged
+    S, hkv, d = cfg["S"], cfg["Hkv"], cfg["d"]
+    g = torch.Generator().manual_seed(seed)
+    lens0 = torch.randint(0, 64, (S,), generator=g, dtype=torch.int32)
+    per = (64 + chunk + 63) // 64 + 1
+    cache = paged.empty_cache(S * per, hkv, d, workloads.DECODE_K_TENSOR_SCALE, "cuda")
+    table = torch.randperm(S * per, generator=g).view(S, per).to(torch.int32).cuda()
+    tail = paged.empty_tail(S, hkv, d, torch.bfloat16, "cuda")
+    lens = lens0.cuda()
+    out = {}
+    for name, n in (("step", 1), ("chunk", chunk)):
+        k = torch.randn(S * n, hkv, d, generator=g).to(torch.bfloat16).cuda()
+        v = torch.randn(S * n, hkv, d, generator=g).to(torch.bfloat16).cuda()
+        cu = (torch.arange(S + 1, dtype=torch.int32) * n).cuda()
+        groups = sum(((int(l) + n + 31) // 32 - int(l) // 32) for l in lens0)
+        nbytes = S * n * hkv * (2 * d * 2 + d // 2 + d // 16) + groups * hkv * d * 33
+
+        def fn(k=k, v=v, cu=cu, n=n):
+            api.kv_append_paged(cache, k, v, cu, lens, table, tail, max_new=n)
+        out[name] = (fn, nbytes, S * n)
+    return out
+
+
+def time_graph(fn, K):
+    """Mean time (ms) of ``fn`` captured as a CUDA graph and replayed K times after an L2 flush."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    graph, _ = capture_step(fn)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        graph.replay()
+        b.record()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / K
+
+
 def capture_step(step):
     """The whole step (quantize + attention, or quantize + decode + merge) as one CUDA graph, so
     that a timed step is the device work alone, without host launch gaps between kernels."""
@@ -511,6 +556,16 @@ def main():
                          "ms": st["quant_ms"], "bytes": st["quant_bytes"]},
             "device_status": status,
             "clocks": clk.summary()}
+    if st["kind"] == "decode":
+        # the producer side of the decode path: quantize-on-append into the paged cache
+        app = {}
+        for nm, (fn, nbytes, ntok) in make_append(cfg).items():
+            ms = max_over_ranks(time_graph(fn, max(3, args.steps // 3)), world)
+            app[nm] = {"ms": ms, "tokens": ntok, "bytes": nbytes,
+                       "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                       "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+        line["append"] = {"kernel": "kv_append_kernel", "timing": KERNEL_TIMING,
+                          "peak_gbs": pk["hbm_gbs"], **app}
     if rank == 0 and not args.no_cpu_baseline:
         dt, u, desc = oracle_sample(name, rows=64 if st["kind"] == "prefill" else 64, heads=1)
         cv = u / dt / (1e12 if st["kind"] == "prefill" else 1e9)

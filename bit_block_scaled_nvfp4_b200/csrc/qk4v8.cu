@@ -489,7 +489,7 @@ extern "C" qk4v8_status kv_append_paged(const qk4v8_append_params* p, cudaStream
   if (p->head_dim != 128) return QK4V8_ERR_UNSUPPORTED;
   if (p->num_seqs > 65535 || p->kv_heads > 65535) return QK4V8_ERR_UNSUPPORTED;
   if (!aligned(p->k_new, 16) || !aligned(p->v_new, 16) || !aligned(p->k_pages, 8) ||
-      !aligned(p->v_pages, 16) || !aligned(p->v_tail, 2))
+      !aligned(p->v_pages, 16) || !aligned(p->v_tail, 16))
     return QK4V8_ERR_INVALID_ARG;
   AppendArgs a;
   a.k_new = p->k_new; a.v_new = p->v_new; a.cu_new = p->cu_new; a.lens = p->lens;
@@ -498,7 +498,8 @@ extern "C" qk4v8_status kv_append_paged(const qk4v8_append_params* p, cudaStream
   a.v_pages = p->v_pages; a.v_scales = p->v_page_scales; a.v_tail = p->v_tail;
   a.S = p->num_seqs; a.num_pages = p->num_pages; a.max_pages = p->max_pages;
   a.Hkv = p->kv_heads; a.max_new = p->max_new;
-  const dim3 grid(p->kv_heads, p->num_seqs);
+  // one CTA per (32-token group the new tokens touch, KV head, sequence)
+  const dim3 grid((p->max_new + 31) / 32 + 1, p->kv_heads, p->num_seqs);
   if (p->dtype == QK4V8_BF16) kv_append_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(a);
   else kv_append_kernel<__half><<<grid, 128, 0, stream>>>(a);
   return launch_status();

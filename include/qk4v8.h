@@ -257,9 +257,10 @@ qk4v8_status attn_qk4v8_decode_paged_noalloc(const qk4v8_decode_params* params,
  * k_new, v_new  [total_new, Hkv, D] fp16/bf16 (dtype), token-major, 16-byte aligned.
  * cu_new        [S + 1] int32, cu_new[0] = 0, nondecreasing, cu_new[S] = total_new.
  * lens          [S] int32 lengths before the call (not modified; the caller adds n_s).
- * v_tail        [S, Hkv, D, 32] of dtype, caller-owned state: for each sequence the tokens of
- *               its last, incomplete V group in the input precision (position 32*(len/32) + i
- *               at index i). Read and rewritten by every call; zero it for a new sequence.
+ * v_tail        [S, Hkv, D, 32] of dtype, 16-byte aligned, caller-owned state: for each
+ *               sequence the tokens of its last, incomplete V group in the input precision
+ *               (position 32*(len/32) + i at index i; later entries are don't-care). Read and
+ *               rewritten by every call that appends to the sequence; zero it for a new one.
  * max_new       host-side bound on n_s (sizes nothing on the device; n_s above it is an
  *               error). head_dim must be 128.
  * Device checks: a page id outside [0, num_pages) or a position at or past 64 * max_pages

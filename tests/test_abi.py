@@ -168,3 +168,4 @@ def test_append_validation(lib):
     assert f(_app(num_seqs=70000)) == _lib.QK4V8_ERR_UNSUPPORTED
     assert f(_app(k_new=FAKE + 8)) == _lib.QK4V8_ERR_INVALID_ARG    # not 16-byte aligned
     assert f(_app(v_pages=FAKE + 4)) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(_app(v_tail=FAKE + 2)) == _lib.QK4V8_ERR_INVALID_ARG
