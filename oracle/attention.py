@@ -35,6 +35,17 @@ FP16 tile (a tile marked in the selection): s_j from the FP16-rounded inputs, an
 p_j = fp16(448 p~_j) / 448 (the FP16 branch works in the same P*448 units as the E4M3
 branch, so both accumulate into one O); V from its FP16-rounded copy.
 
+Underflow-aware probability scaling (sns.style BitDecoding-FP4 summary, the second algorithm
+item: long-context probabilities are tiny, the E4M3 encoding of P can round whole blocks to
+zero, so the probability scaling is adjusted to avoid it). Reading (the page gives no formula):
+each 32-key block b of a tile row gets its own power-of-two scale 2^e_b, e_b = ceil(log2 of
+the block's largest p~) clipped to [-127, 0] (0 for an all-zero block), and
+
+    p_j = decode_E4M3(E4M3(448 p~_j 2^-e_b)) 2^e_b / 448
+
+so every block's largest value lands in (224, 448] before rounding. This is the E8M0 block
+scale the FP8 MMA applies to its P operand; l and O see the same p_j.
+
 Split-K decode: the key range of a sequence is cut into splits of ``split_tokens`` keys
 (a multiple of 128; 0 means one split). Each split runs the loop above from m = -inf, and the
 splits merge exactly: M = max_s m_s, O = sum_s e^(m_s - M) O_s / sum_s e^(m_s - M) l_s.
@@ -57,9 +68,23 @@ def _p_fp16(p_tilde: np.ndarray) -> np.ndarray:
     return fp16_round(p_tilde * P_SCALE) / P_SCALE
 
 
+def _p_e4m3_block_scaled(p_tilde: np.ndarray) -> np.ndarray:
+    """Underflow-aware P: per row and 32-key block, scale by 2^-e_b before the E4M3 encode."""
+    p = np.zeros_like(p_tilde)
+    for b in range(0, p_tilde.shape[1], 32):
+        blk = p_tilde[:, b:b + 32]
+        mx = blk.max(axis=1)
+        e = np.zeros(mx.shape)
+        pos = mx > 0
+        e[pos] = np.clip(np.ceil(np.log2(mx[pos])), -127, 0)
+        sc = np.ldexp(1.0, e.astype(np.int64))[:, None]
+        p[:, b:b + 32] = e4m3_round(blk * P_SCALE / sc) * sc / P_SCALE
+    return p
+
+
 def attention_rows(q: np.ndarray, row_pos: np.ndarray, k: np.ndarray, v: np.ndarray,
                    causal: bool, softmax_scale: float, *,
-                   quantize_p: bool = True,
+                   quantize_p: bool = True, p_underflow_aware: bool = False,
                    fp16_select=None, q16=None, k16=None, v16=None,
                    key_begin: int = 0, key_end: int | None = None):
     """Online-softmax attention of query rows ``q`` [R, d] at positions ``row_pos`` over keys
@@ -101,7 +126,7 @@ def attention_rows(q: np.ndarray, row_pos: np.ndarray, k: np.ndarray, v: np.ndar
         m_new = np.maximum(m_old, s.max(axis=1))
         p_tilde = np.where(valid, np.exp(s - m_new[:, None]), 0.0)
         if quantize_p:
-            p = _p_e4m3(p_tilde)
+            p = _p_e4m3_block_scaled(p_tilde) if p_underflow_aware else _p_e4m3(p_tilde)
             if sel.any():
                 p[sel] = _p_fp16(p_tilde[sel])
         else:
@@ -158,7 +183,7 @@ def exact_attention(q, k, v, causal, softmax_scale):
 
 
 def decode_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, length: int,
-                softmax_scale: float, split_tokens: int):
+                softmax_scale: float, split_tokens: int, p_underflow_aware: bool = False):
     """One decode step for the query rows ``q`` [R, d] of one sequence over its first
     ``length`` keys, in splits of ``split_tokens`` keys (0: one split). Returns (O, lse)."""
     if split_tokens <= 0:
@@ -168,5 +193,6 @@ def decode_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, length: int,
     parts = []
     for b in range(0, length, split_tokens):
         parts.append(attention_rows(q, rows, k, v, False, softmax_scale,
+                                    p_underflow_aware=p_underflow_aware,
                                     key_begin=b, key_end=min(b + split_tokens, length)))
     return finish(*merge_splits(parts))

@@ -165,3 +165,55 @@ def test_decode_context_length_one_is_v0():
     q, k, v = _rand(14, 4, 10, 64)
     o, _ = A.decode_rows(q, k, v, 1, 0.125, split_tokens=128)
     assert np.array_equal(o, np.repeat(v[:1], 4, axis=0))
+
+
+# ---- underflow-aware probability scaling (per 32-key block power-of-two scale) ----
+
+def test_block_scaled_p_relative_error_and_no_block_underflow():
+    """Closed form: after the per-block scale every value at or above 2^-6 of its block's
+    largest lies in the normal E4M3 range, so its relative error is at most 2^-4; a block
+    whose values are all below 2^-10 / 448 encodes to zero with the fixed 448 scale but not
+    with the block scale."""
+    rng = np.random.default_rng(3)
+    p = np.exp2(rng.uniform(-40, 0, (64, 128)))
+    p[:, 32:64] *= 2.0 ** -30                            # a whole block far below the row max
+    got = A._p_e4m3_block_scaled(p)
+    for b in range(0, 128, 32):
+        blk, g = p[:, b:b + 32], got[:, b:b + 32]
+        big = blk >= blk.max(axis=1, keepdims=True) * 2.0 ** -6
+        assert np.all(np.abs(g[big] - blk[big]) <= blk[big] * 2.0 ** -4)
+        assert np.all(g.max(axis=1) > 0)
+    tiny = p[:, 32:64].max(axis=1) < 2.0 ** -10 / 448
+    assert tiny.any()
+    assert np.all(A._p_e4m3(p[tiny, 32:64]) == 0)
+    assert np.all(got[tiny, 32:64].max(axis=1) > 0)
+
+
+def test_block_scaled_p_equals_fixed_when_every_block_holds_a_top_value():
+    """A block whose largest p~ is above 1/2 gets e_b = 0: the encoding is the fixed one."""
+    rng = np.random.default_rng(4)
+    p = rng.uniform(0, 1, (16, 128))
+    p[:, ::32] = rng.uniform(0.51, 1.0, (16, 4))
+    assert np.array_equal(A._p_e4m3_block_scaled(p), A._p_e4m3(p))
+
+
+def test_underflow_aware_constant_v_and_closer_to_exact():
+    """Constant V still gives exactly that constant (l and O see the same p). One key 14 nats
+    above 4095 others: each of those has p~ = e^-14 < 2^-10 / 448, so the fixed scale drops
+    them all (O = the top key's v) although together they hold 4095 e^-14 = 0.34 % of the
+    weight; the block scale keeps them and lands within E4M3 precision of the exact result."""
+    d, n, scale = 16, 4096, 0.25
+    q = np.zeros((1, d)); q[0, 0] = 1.0
+    k = np.zeros((n, d)); k[:, 0] = 6.0 / scale; k[5, 0] = 20.0 / scale
+    v = np.full((n, d), 0.75)
+    o, _ = A.decode_rows(q, k, v, n, scale, 0, p_underflow_aware=True)
+    assert np.allclose(o, 0.75, rtol=0, atol=1e-12)
+    rng = np.random.default_rng(5)
+    v = rng.standard_normal((n, d)) + 3.0
+    ref = A.exact_attention(q, k, v, False, scale)
+    o_fix, _ = A.decode_rows(q, k, v, n, scale, 0)
+    o_ua, _ = A.decode_rows(q, k, v, n, scale, 0, p_underflow_aware=True)
+    assert np.array_equal(o_fix[0], v[5])                      # every other key dropped
+    err_fix = np.abs(o_fix - ref).max()
+    err_ua = np.abs(o_ua - ref).max()
+    assert err_fix > 5e-3 and err_ua < err_fix / 20
