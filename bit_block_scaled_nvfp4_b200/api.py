@@ -192,7 +192,8 @@ class PagedKV:
 
 def decode_params(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
                   context_lens: torch.Tensor, max_context: int, split_tokens: int,
-                  out: torch.Tensor, softmax_scale: float | None = None, lse=None):
+                  out: torch.Tensor, softmax_scale: float | None = None, lse=None,
+                  underflow_aware: bool = False):
     S, Hq, dh = q.codes.shape
     P, Hkv = cache.k_pages.shape[0], cache.k_pages.shape[1]
     d = dh * 2
@@ -209,20 +210,23 @@ def decode_params(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
     p.out_dtype = _OUT_DT[out.dtype]
     p.out = out.data_ptr()
     p.lse = lse.data_ptr() if lse is not None else None
+    p.p_underflow_aware = int(bool(underflow_aware))
     return p
 
 
 def attn_qk4v8_decode_paged(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
                             context_lens: torch.Tensor, max_context: int, split_tokens: int,
                             softmax_scale: float | None = None, out_dtype=torch.bfloat16,
-                            want_lse: bool = False, workspace: torch.Tensor | None = None):
-    """One decode step. q.codes [S, Hq, D/2]; returns out [S, Hq, D] (and lse [S, Hq])."""
+                            want_lse: bool = False, workspace: torch.Tensor | None = None,
+                            underflow_aware: bool = False):
+    """One decode step. q.codes [S, Hq, D/2]; returns out [S, Hq, D] (and lse [S, Hq]).
+    ``underflow_aware`` scales P per 32-key block by a power of two before its E4M3 encode."""
     lib = _lib.load()
     S, Hq, dh = q.codes.shape
     out = torch.empty(S, Hq, dh * 2, dtype=out_dtype, device=q.codes.device)
     lse = torch.empty(S, Hq, dtype=torch.float32, device=q.codes.device) if want_lse else None
     p = decode_params(q, cache, page_table, context_lens, max_context, split_tokens, out,
-                      softmax_scale, lse)
+                      softmax_scale, lse, underflow_aware)
     need = lib.attn_qk4v8_decode_workspace_size(C.byref(p))
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.codes.device)

@@ -50,10 +50,13 @@ struct DecLayout {
   static constexpr int NK = GM <= 4 ? 2 : 3, NVS = NK;
   static constexpr int OFF_Q = 0;                 // 16 rows x 64 B (SW64)
   static constexpr int OFF_QSF = 1024;            // 2 chunks
-  static constexpr int OFF_PSF = 2048;            // 1 chunk
-  static constexpr int OFF_P = 3072;              // 2 x [16 rows x 128 B] (SW128), 1024-aligned
+  // P^T scale factors: two chunks by block parity (query row n, 32-key block b at byte
+  // n*16 + b; E8M0 127 = 1.0 unless underflow-aware scaling lowers it), then a constant chunk of
+  // 1.0 for the ones operand
+  static constexpr int OFF_PSF = 2048;
+  static constexpr int OFF_P = 4096;              // 2 x [16 rows x 128 B] (SW128), 1024-aligned
   static constexpr int OFF_ONES = OFF_P + 2 * 2048;       // 128 x 32 B of E4M3 1.0 (SW32)
-  static constexpr int OFF_KST = OFF_ONES + 4096;         // 11264, 1024-aligned
+  static constexpr int OFF_KST = OFF_ONES + 4096;         // 12288, 1024-aligned
   static constexpr int ST_K = 0;                  // 128 keys x 64 B (SW64)
   static constexpr int ST_KSF = 8192;             // 2 chunks
   static constexpr int KST_BYTES = 9216;
@@ -71,7 +74,8 @@ struct DecLayout {
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   // S^T x2 [0,32), O^T [32,48), L^T [48,64) (every row: l), Q / P scales, K and V scales by
   // stage
-  static constexpr uint32_t T_S = 0, T_O = 32, T_L = 48, T_QSF = 64, T_PSF = 72, T_KSF = 76,
+  static constexpr uint32_t T_S = 0, T_O = 32, T_L = 48, T_QSF = 64, T_PSF = 72, T_ONESF = 80,
+                            T_KSF = 84,
                             T_VSF = T_KSF + 8 * NK;
   static_assert(T_VSF + 4 * NVS <= 128, "TMEM columns");
   static constexpr int NQ = 16;                   // MMA N (query heads, padded)
@@ -80,7 +84,9 @@ struct DecLayout {
   static constexpr int THREADS = 256;
 };
 
-template <int GM>
+// kUA: underflow-aware P scaling (a separate instance, so that the default path carries none
+// of its work).
+template <int GM, bool kUA>
 __global__ void __launch_bounds__(256, DecLayout<GM>::CTAS_PER_SM)
 decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
               const __grid_constant__ CUtensorMap tm_vp, DecArgs a) {
@@ -143,6 +149,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   }
   for (int i = threadIdx.x; i < 128; i += blockDim.x)
     reinterpret_cast<uint32_t*>(sm + L::OFF_PSF)[i] = 0x7F7F7F7Fu;
+  for (int i = threadIdx.x; i < 128; i += blockDim.x) {
+    reinterpret_cast<uint32_t*>(sm + L::OFF_PSF + 512)[i] = 0x7F7F7F7Fu;
+    reinterpret_cast<uint32_t*>(sm + L::OFF_PSF + 1024)[i] = 0x7F7F7F7Fu;
+  }
   for (int i = threadIdx.x; i < 2 * 16 * 128 / 16; i += blockDim.x)   // zero both P^T buffers
     reinterpret_cast<uint4*>(sm + L::OFF_P)[i] = make_uint4(0, 0, 0, 0);
   for (int i = threadIdx.x; i < 4096 / 16; i += blockDim.x)            // the ones operand
@@ -316,7 +326,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t sP = smem_u32(sm + L::OFF_P);
     if (lane == 0) {
       tc_fence_after();
-      tmem_cp_sf(tbase + L::T_PSF, sm + L::OFF_PSF);
+      tmem_cp_sf(tbase + L::T_ONESF, sm + L::OFF_PSF + 1024);
     }
     bool ok = true;
     for (int bb = 0; ok && bb < nblk; ++bb) {
@@ -340,7 +350,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       if (lane == 0) {
         tc_fence_after();
         const uint32_t tv = tbase + L::T_VSF + 4 * st_i;
+        // P^T scales: this block's (slot b2) with underflow-aware scaling, else the 1.0 chunk
+        const uint32_t tp = kUA ? tbase + L::T_PSF + 4 * b2 : tbase + L::T_ONESF;
         tmem_cp_sf(tv, st + L::ST_VSF);
+        if (kUA) tmem_cp_sf(tp, sm + L::OFF_PSF + 512 * b2);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t sV = smem_u32(st + ((kk >> 1) ? L::ST_V1 : L::ST_V0));
@@ -348,19 +361,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const uint64_t db = make_sdesc(sP + b2 * 2048 + kk * 32, 16, 1024, kSw128);
           mma_mxf8(tbase + L::T_O, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
                    tv | (static_cast<uint32_t>(kk) << 30),
-                   (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                   tp | (static_cast<uint32_t>(kk) << 30),
                    (bb > 0 || kk > 0) ? 1u : 0u);
         }
         // l on the tensor core: L^T += 1 P^T (A = 128 rows of E4M3 1.0, the same 32-key slice
-        // for every step), so every row of L^T holds the row sums of the quantized P, rescaled
-        // with O^T.
+        // for every step, scale 1.0; B with the P^T scales), so every row of L^T holds the row
+        // sums of the quantized P, rescaled with O^T.
         const uint64_t d1 = make_sdesc(smem_u32(sm + L::OFF_ONES), 16, 256, kSw32);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t db = make_sdesc(sP + b2 * 2048 + kk * 32, 16, 1024, kSw128);
           mma_mxf8(tbase + L::T_L, d1, db, idesc_with_sf_ids(idesc_pv, kk, kk),
-                   (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
-                   (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                   (tbase + L::T_ONESF) | (static_cast<uint32_t>(kk) << 30),
+                   tp | (static_cast<uint32_t>(kk) << 30),
                    (bb > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(pv_done + b2);
@@ -401,12 +414,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // four warps through shared memory (slots alternate by block parity, so a fast warp's
       // next write cannot land before the others have read).
       float* rm = red_max + b2 * 64;
+      float own[GM];                                       // this warp's 32-key block max
 #pragma unroll
       for (int q = 0; q < GM; ++q) {
         x[q] = (valid && q < g) ? x[q] : -INFINITY;        // raw MMA units
-        float mm;
-        asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(mm) : "f"(x[q]));
-        if (lane == 0) rm[wq * 16 + q] = mm;
+        asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(own[q]) : "f"(x[q]));
+        if (lane == 0) rm[wq * 16 + q] = own[q];
       }
       if (failed && lane == 0) *soft_flag = 1;
       named_bar_sync(1, 128);
@@ -423,18 +436,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         all_one = all_one && (alpha[q] == 1.f);
         m_run[q] = m_new;
       }
+      // Underflow-aware P scaling: this warp's 32 keys are one block of the P^T operand; with
+      // mu = log2 of the block's largest p~ (<= 0), P is encoded as 448 p~ 2^-e, e = ceil(mu)
+      // clipped to [-127, 0], and the MMA's E8M0 scale of that block is 2^e.
+      float pe[GM];
+#pragma unroll
+      for (int q = 0; q < GM; ++q) {
+        const float mu = (own[q] - moff[q]) * C;
+        pe[q] = (kUA && mu > -1.0e30f) ? fminf(fmaxf(ceilf(mu), -127.f), 0.f) : 0.f;
+      }
       uint32_t codes[GM / 4];
 #pragma unroll
       for (int q = 0; q < GM; q += 4) {
         float p[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) p[i] = ex2_approx((x[q + i] - moff[q + i]) * C) * 448.f;
+        for (int i = 0; i < 4; ++i) p[i] = ex2_approx((x[q + i] - moff[q + i]) * C - pe[q + i]) * 448.f;
         codes[q >> 2] = cvt_e4m3x2(p[0], p[1]) | (cvt_e4m3x2(p[2], p[3]) << 16);
       }
       // P^T buffer b2 was read by PV(blk-2); O^T and L^T are rescaled below after PV(blk-1).
       if (blk >= 1) {
         if (!waits(pv_done + ((blk - 1) & 1), ((blk - 1) >> 1) & 1, blk)) failed = true;
         tc_fence_after();
+      }
+      // P^T scales of this warp's block (row q, byte wq of the block-parity chunk)
+      if (kUA && lane == 0) {
+#pragma unroll
+        for (int q = 0; q < GM; ++q)
+          if (q < g) sm[L::OFF_PSF + 512 * b2 + q * 16 + wq] = static_cast<unsigned char>(127 + static_cast<int>(pe[q]));
       }
       // P^T row q (query), column r (key), 128-byte swizzle.
       unsigned char* pb = sP + b2 * 2048;

@@ -388,6 +388,7 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   if (p->out_dtype != QK4V8_F16 && p->out_dtype != QK4V8_BF16 && p->out_dtype != QK4V8_F32)
     return QK4V8_ERR_INVALID_ARG;
   if (!(p->softmax_scale > 0.f)) return QK4V8_ERR_INVALID_ARG;
+  if (p->p_underflow_aware != 0 && p->p_underflow_aware != 1) return QK4V8_ERR_INVALID_ARG;
   if (p->head_dim != 128 || p->q_heads / p->kv_heads > 16) return QK4V8_ERR_UNSUPPORTED;
   if (!aligned(p->q_codes, 16) || !aligned(p->k_pages, 16) || !aligned(p->v_pages, 16) ||
       !aligned(p->q_scales, 8) || !aligned(p->k_page_scales, 8) || !aligned(p->v_page_scales, 4) ||
@@ -413,8 +414,12 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   }
   static bool attr = false;
   if (!attr) {
-    if (!set_smem(decode_kernel<4>, DecLayout<4>::SMEM_ALLOC) || !set_smem(decode_kernel<8>, DecLayout<8>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<16>, DecLayout<16>::SMEM_ALLOC))
+    if (!set_smem(decode_kernel<4, false>, DecLayout<4>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<8, false>, DecLayout<8>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<16, false>, DecLayout<16>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<4, true>, DecLayout<4>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<8, true>, DecLayout<8>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<16, true>, DecLayout<16>::SMEM_ALLOC))
       return QK4V8_ERR_CUDA;
     attr = true;
   }
@@ -429,9 +434,14 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   dim3 grid(n_splits, p->kv_heads, p->num_seqs);
   // the softmax handles the g = Hq / Hkv real query columns: an instance per bound on g
   const int g = p->q_heads / p->kv_heads;
-  if (g <= 4) decode_kernel<4><<<grid, DecLayout<4>::THREADS, DecLayout<4>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
-  else if (g <= 8) decode_kernel<8><<<grid, DecLayout<8>::THREADS, DecLayout<8>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
-  else decode_kernel<16><<<grid, DecLayout<16>::THREADS, DecLayout<16>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a);
+  const bool ua = p->p_underflow_aware != 0;
+#define QK4V8_DEC(GM)                                                                          \
+  (ua ? decode_kernel<GM, true><<<grid, DecLayout<GM>::THREADS, DecLayout<GM>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a) \
+      : decode_kernel<GM, false><<<grid, DecLayout<GM>::THREADS, DecLayout<GM>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a))
+  if (g <= 4) QK4V8_DEC(4);
+  else if (g <= 8) QK4V8_DEC(8);
+  else QK4V8_DEC(16);
+#undef QK4V8_DEC
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   decode_merge_kernel<<<p->num_seqs * p->q_heads, 128, 0, stream>>>(
       a.ws, n_splits, static_cast<int32_t>(p->out_dtype), p->out, p->lse);

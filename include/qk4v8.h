@@ -215,6 +215,11 @@ typedef struct {
   qk4v8_dtype out_dtype;
   void* out;                   /* [S, Hq, D] out (out_dtype) */
   float* lse;                  /* optional [S, Hq] out; or NULL */
+  int32_t p_underflow_aware;   /* 0: P encoded as E4M3(448 p~) per 128-key block; 1: each
+                                  32-key block of a query row as E4M3(448 p~ 2^-e) with
+                                  e = ceil(log2 max p~) clipped to [-127, 0] and the MMA's E8M0
+                                  scale 2^e (sns.style BitDecoding-FP4 summary, underflow-aware
+                                  probability scaling: long-context P must not round to zero) */
 } qk4v8_decode_params;
 
 size_t attn_qk4v8_decode_workspace_size(const qk4v8_decode_params* params);
