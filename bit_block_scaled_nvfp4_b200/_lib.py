@@ -39,7 +39,7 @@ class FwdParams(C.Structure):
         ("batch", i32), ("q_heads", i32), ("kv_heads", i32), ("n_q", i32), ("n_k", i32),
         ("head_dim", i32), ("causal", i32), ("softmax_scale", f32),
         ("fp16_bitmap", vp), ("q16", vp), ("k16", vp), ("v16", vp),
-        ("out_dtype", i32), ("out", vp), ("lse", vp),
+        ("out_dtype", i32), ("out", vp), ("lse", vp), ("p_underflow_aware", i32),
     ]
 
 

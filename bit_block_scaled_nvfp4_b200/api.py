@@ -153,7 +153,8 @@ def tile_score_select(q: NVFP4Tensor, k: NVFP4Tensor, causal: bool, frac_bp: int
 
 def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
                    softmax_scale: float | None = None, out_dtype=torch.bfloat16,
-                   fp16_bitmap: torch.Tensor | None = None, want_lse: bool = False):
+                   fp16_bitmap: torch.Tensor | None = None, want_lse: bool = False,
+                   underflow_aware: bool = False):
     """QK4V8 attention forward. q.codes [B, Hq, Nq, D/2], k.codes [B, Hkv, Nk, D/2],
     v.codes [B, Hkv, D, Nk_pad]. With ``fp16_bitmap`` the FP16 copies (q.fp16, k.fp16,
     v.fp16) must be present. Returns out [B, Hq, Nq, D] (and lse [B, Hq, Nq])."""
@@ -176,6 +177,7 @@ def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
     p.out_dtype = _OUT_DT[out_dtype]
     p.out = out.data_ptr()
     p.lse = lse.data_ptr() if lse is not None else None
+    p.p_underflow_aware = int(bool(underflow_aware))
     _lib.check(lib.attn_qk4v8_fwd(C.byref(p), _stream()), "attn_qk4v8_fwd")
     return (out, lse) if want_lse else out
 
@@ -281,7 +283,7 @@ def kv_append_paged(cache: PagedKV, k_new: torch.Tensor, v_new: torch.Tensor,
 
 def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool,
                     softmax_scale: float | None = None, fp16_frac_bp: int = 0,
-                    out_dtype=None, want_lse: bool = False):
+                    out_dtype=None, want_lse: bool = False, underflow_aware: bool = False):
     """The whole prefill path on bf16/fp16 CUDA tensors q [B, Hq, N, D], k/v [B, Hkv, N, D]:
     quantize Q, K (NVFP4) and V (MXFP8), optionally score tiles and recompute the top
     ``fp16_frac_bp`` basis points of them in FP16, then attention."""
@@ -293,4 +295,4 @@ def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: b
     if mixed:
         _, _, bitmap = tile_score_select(q4, k4, causal, fp16_frac_bp)
     return attn_qk4v8_fwd(q4, k4, v8, causal, softmax_scale, out_dtype or q.dtype,
-                          fp16_bitmap=bitmap, want_lse=want_lse)
+                          fp16_bitmap=bitmap, want_lse=want_lse, underflow_aware=underflow_aware)

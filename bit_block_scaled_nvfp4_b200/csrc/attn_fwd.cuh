@@ -114,7 +114,10 @@ struct FwdLayout {
   // | V scales] per s (measured faster than two separate arrays); otherwise K blocks
   // [K | K scales] followed by V blocks [V | V scales].
   static constexpr bool kInterleaved = (NK == NVS);
-  static constexpr int OFF_STG = OFF_PSF + 1024;
+  // P scale factors of the underflow-aware variant, two chunks by tile parity (row r's four
+  // 32-key block scales in the word at (r % 32) * 16 + (r / 32) * 4)
+  static constexpr int OFF_PSFU = OFF_PSF + 1024;
+  static constexpr int OFF_STG = OFF_PSFU + 1024;
   static constexpr int STG_BYTES = K_BYTES + V_BYTES + 2048;
   static constexpr int OFF_VSTG = OFF_STG + NK * (K_BYTES + 1024);
   __device__ static constexpr int k_off(int s) {
@@ -147,15 +150,18 @@ struct FwdLayout {
   // scale factors in two slots by tile parity (8 columns each: a slot is rewritten only after
   // the MMA two items / tiles back that read it has completed).
   static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_PSF = 416, T_KSF = 420,
-                            T_VSF = 436;
-  static_assert(T_O + NV <= T_QSF && T_VSF + 16 <= 512, "TMEM columns");
+                            T_VSF = 436, T_PSFU = 452;    // T_PSFU: 2 slots by tile parity
+  static_assert(T_O + NV <= T_QSF && T_PSFU + 8 <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
   static constexpr int PV_WARP = 2;
   static constexpr int THREADS = 384;
 };
 
-template <int D, bool kMixed>
+// kUA: underflow-aware P scaling — each 32-key block of a tile row encoded as
+// E4M3(448 p~ 2^-e), e = ceil(log2 of the block's largest p~) clipped to [-127, 0], with the
+// block's E8M0 P scale 2^e in the PV MMA (FP4 tiles only).
+template <int D, bool kMixed, bool kUA = false>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q16,
@@ -542,13 +548,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (!f16) {
             const uint32_t tv = tbase + L::T_VSF + 8 * b2;   // PV(g-2), its last reader, is done
             tmem_cp_sf(tv, sm + L::v_sf_off(s));
+            // P scales: the tile's own (slot b2, written by the softmax) in the underflow-aware
+            // variant, else the constant 1.0 chunk
+            const uint32_t tp = kUA ? tbase + L::T_PSFU + 4 * b2 : tbase + L::T_PSF;
+            if constexpr (kUA) tmem_cp_sf(tp, sm + L::OFF_PSFU + 512 * b2);
             const uint32_t sV = smem_u32(sm + L::v_off(s));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t da = make_sdesc(sP + pb * 16384 + kk * 32, 16, 1024, kSw128);
               const uint64_t db = make_sdesc(sV + kk * 32, 16, 1024, kSw128);
               mma_mxf8(tO, da, db, idesc_with_sf_ids(idesc_pv, kk, kk),
-                       (tbase + L::T_PSF) | (static_cast<uint32_t>(kk) << 30),
+                       tp | (static_cast<uint32_t>(kk) << 30),
                        tv | (static_cast<uint32_t>(kk) << 30), (j > 0 || kk > 0) ? 1u : 0u);
             }
           } else {
@@ -631,7 +641,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int c = 0; c < 128; ++c) x[c] = (c <= lim) ? x[c] : -INFINITY;
         }
         float mt;
-        {
+        float bm[4];                         // 32-key block maxima (underflow-aware variant)
+        if constexpr (kUA) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            bm[b] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) bm[b] = fmax3(bm[b], x[32 * b + c], x[32 * b + c + 1]);
+          }
+          mt = fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3]));
+        } else {
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c = 0; c < 128; c += 8) {
@@ -656,6 +675,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const bool dead = (m_new == -INFINITY);
         const float bias = kLog2_448 - (dead ? 0.f : m_new) * C;
         const float2 B2 = make_float2(bias, bias);
+        float2 Bb[4];                        // per-block bias (underflow-aware variant)
+        uint32_t psf_word = 0u;
+        if constexpr (kUA) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const float mu = (bm[b] - m_new) * C;       // log2 of the block's largest p~ (<= 0)
+            const float e = (!dead && mu > -1.0e30f) ? fminf(fmaxf(ceilf(mu), -127.f), 0.f) : 0.f;
+            Bb[b] = make_float2(bias - e, bias - e);
+            psf_word |= static_cast<uint32_t>(127 + static_cast<int>(e)) << (8 * b);
+          }
+        }
         // P buffer pb was last used by PV(gg-NP), the last phase of its barrier that can have
         // completed. An FP16 tile's P fills both buffers (NP = 2 in that kernel): writing one
         // needs PV(gg-1) done as well, and the tile after an FP16 tile too. The waits come
@@ -668,14 +698,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           // kPolyOf8 of every 8 groups of 4 scores take the FMA-pipe exponential, the rest the
           // special-function unit.
           unsigned char* prow = sP + pb * 16384 + row * 128;
+          if constexpr (kUA)
+            *reinterpret_cast<uint32_t*>(sm + L::OFF_PSFU + b2 * 512 + (row & 31) * 16 + (row >> 5) * 4) = psf_word;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {               // 16 keys per 16-byte chunk
             uint32_t w4[4];
+            const float2 Bc = kUA ? Bb[ch >> 1] : B2;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int c = ch * 16 + q * 4;
-              const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
-              const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), C2, B2);
+              const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, Bc);
+              const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), C2, Bc);
               float2 e0, e1;
               if (((c >> 2) & 7) < kPolyOf8) {
                 e0 = exp2_poly2(t0);

@@ -275,7 +275,7 @@ qk4v8_status tile_score_select(const uint8_t* q_codes, const uint8_t* q_scales,
 
 // ------------------------------------------------------------------------------------------
 }  // extern "C"
-template <int D, bool kMixed>
+template <int D, bool kMixed, bool kUA = false>
 static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   using L = FwdLayout<D, kMixed>;
   const int32_t B = p->batch, Hq = p->q_heads, Hkv = p->kv_heads;
@@ -313,7 +313,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   }
   static bool attr = false;
   if (!attr) {
-    if (!set_smem(attn_fwd_kernel<D, kMixed>, L::SMEM_ALLOC)) return QK4V8_ERR_CUDA;
+    if (!set_smem(attn_fwd_kernel<D, kMixed, kUA>, L::SMEM_ALLOC)) return QK4V8_ERR_CUDA;
     attr = true;
   }
   FwdArgs a;
@@ -329,7 +329,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   const int64_t items = static_cast<int64_t>(a.Tq) * B * Hq;
   if (items > INT32_MAX / 2) return QK4V8_ERR_UNSUPPORTED;
   const int64_t grid = items < sm_count() ? items : sm_count();
-  attn_fwd_kernel<D, kMixed><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
+  attn_fwd_kernel<D, kMixed, kUA><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
   return launch_status();
 }
 
@@ -358,6 +358,11 @@ qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
     return QK4V8_ERR_INVALID_ARG;
   const int64_t tiles = static_cast<int64_t>((p->n_q + 127) / 128) * p->batch * p->q_heads;
   if (tiles > 0x7fffffffLL) return QK4V8_ERR_UNSUPPORTED;
+  if (p->p_underflow_aware != 0 && p->p_underflow_aware != 1) return QK4V8_ERR_INVALID_ARG;
+  if (p->p_underflow_aware) {
+    if (mixed) return QK4V8_ERR_UNSUPPORTED;
+    return p->head_dim == 128 ? launch_fwd<128, false, true>(p, stream) : launch_fwd<64, false, true>(p, stream);
+  }
   if (p->head_dim == 128) return mixed ? launch_fwd<128, true>(p, stream) : launch_fwd<128, false>(p, stream);
   return mixed ? launch_fwd<64, true>(p, stream) : launch_fwd<64, false>(p, stream);
 }

@@ -180,6 +180,9 @@ typedef struct {
   qk4v8_dtype out_dtype;
   void* out;                   /* [B, Hq, Nq, D] out (out_dtype), 16-byte aligned */
   float* lse;                  /* optional [B, Hq, Nq] natural-log sum-exp out; or NULL */
+  int32_t p_underflow_aware;   /* 0 or 1 as in qk4v8_decode_params (each 32-key block of a
+                                  tile row scaled by its own power of two before the E4M3
+                                  encode); not with fp16_bitmap */
 } qk4v8_fwd_params;
 
 qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* params, cudaStream_t stream);

@@ -17,12 +17,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _run(q, k, v, causal, scale=None, frac_bp=0, out_dtype=torch.float32):
+def _run(q, k, v, causal, scale=None, frac_bp=0, out_dtype=torch.float32, ua=False):
     return api.qk4v8_attention(q.to(DEV), k.to(DEV), v.to(DEV), causal, scale,
-                               fp16_frac_bp=frac_bp, out_dtype=out_dtype)
+                               fp16_frac_bp=frac_bp, out_dtype=out_dtype, underflow_aware=ua)
 
 
-def _full_oracle(q, k, v, causal, scale):
+def _full_oracle(q, k, v, causal, scale, ua=False, exact=False):
     B, Hq, N, D = q.shape
     out = np.zeros((B, Hq, q.shape[2], D))
     Hkv = k.shape[1]
@@ -34,7 +34,11 @@ def _full_oracle(q, k, v, causal, scale):
             vh = OQ.mxfp8_dequantize_v(vc, vs, v.shape[2])
             for hq in range(hk * (Hq // Hkv), (hk + 1) * (Hq // Hkv)):
                 qh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(f32(q[b, hq]), tensor_scale=sq))
-                out[b, hq] = OA.attention_head(qh, kh, vh, causal, scale)[0]
+                if exact:
+                    out[b, hq] = OA.exact_attention(qh, kh, vh, causal, scale)
+                else:
+                    out[b, hq] = OA.attention_head(qh, kh, vh, causal, scale,
+                                                   p_underflow_aware=ua)[0]
     return out
 
 
@@ -121,3 +125,34 @@ def test_bf16_output_workload_long_rows():
     out = _run(q, k, v, True, out_dtype=torch.bfloat16)
     ref = _full_oracle(q, k, v, True, 1 / math.sqrt(128))
     assert_rounded_output_close(f32(out), ref, torch.bfloat16, "bf16 output")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,D,causal", [
+    (1, 4, 2, 700, 700, 128, True),
+    (1, 2, 1, 300, 900, 64, False),
+])
+def test_underflow_aware_parity(B, Hq, Hkv, Nq, Nk, D, causal):
+    """Peaky scores (K x 6), so most 32-key blocks take a scale below 1: the underflow-aware
+    kernel matches the oracle's underflow-aware attention."""
+    g = torch.Generator().manual_seed(Nq + Nk + D)
+    q = torch.randn(B, Hq, Nq, D, generator=g).to(torch.bfloat16)
+    k = (torch.randn(B, Hkv, Nk, D, generator=g) * 6).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Nk, D, generator=g).to(torch.bfloat16)
+    out = _run(q, k, v, causal, ua=True)
+    ref = _full_oracle(q, k, v, causal, 1 / math.sqrt(D), ua=True)
+    assert_attention_close(f32(out), ref, "underflow-aware")
+
+
+def test_underflow_aware_keeps_the_small_keys():
+    """One key about 14 nats above 2047 others: the fixed P scale rounds all of those to zero,
+    the underflow-aware one keeps them and is several times closer to exact attention."""
+    n, d = 2048, 128
+    q = torch.ones(1, 2, n, d).to(torch.bfloat16)
+    k = torch.full((1, 1, n, d), 0.5) + 0.01 * torch.randn(1, 1, n, d, generator=torch.Generator().manual_seed(2))
+    k[0, 0, 7] = 1.75
+    k = k.to(torch.bfloat16)
+    v = (torch.randn(1, 1, n, d, generator=torch.Generator().manual_seed(3)) + 2.0).to(torch.bfloat16)
+    scale = 1 / math.sqrt(d)
+    exact = _full_oracle(q, k, v, False, scale, exact=True)
+    err = {ua: np.abs(f32(_run(q, k, v, False, scale, ua=ua)) - exact).max() for ua in (False, True)}
+    assert err[False] > 1e-3 and err[False] > 5 * err[True], err
