@@ -89,6 +89,29 @@ def nvfp4_dequantize(packed: np.ndarray, scales: np.ndarray, s_t: float) -> np.n
     return (vals * sb[..., None] * np.float64(s_t)).reshape(codes.shape)
 
 
+def nvfp4_residual(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, s_t) -> np.ndarray:
+    """The part of ``x`` its NVFP4 encoding (packed, scales, s_t) misses, in FP32 steps:
+    den = fl32(decode(s_b) * s_t), d_i = fl32(decode(code_i) * den), r_i = fl32(x_i - d_i)."""
+    x = np.asarray(x, dtype=F32)
+    cols = x.shape[-1]
+    vals = e2m1_decode(nvfp4_unpack(packed)).astype(F32)            # exact small values
+    vals = vals.reshape(vals.shape[:-1] + (cols // NVFP4_BLOCK, NVFP4_BLOCK))
+    den = (e4m3_decode(scales).astype(F32) * F32(s_t)).astype(F32)
+    d = (vals * den[..., None]).astype(F32)
+    blocks = x.reshape(vals.shape)
+    return (blocks - d).astype(F32).reshape(x.shape)
+
+
+def nvfp4_dual_quantize(x: np.ndarray, tensor_scale: float | None = None):
+    """Dual-residual NVFP4 (sns.style BitDecoding-FP4 summary, first algorithm item: the query
+    is split into two FP4 tensors, the second carrying what the first leaves over). Reading:
+    Q1 = NVFP4(x); Q2 = NVFP4(x - x_hat1) with the same tensor scale s_t, so that Q1 K^T and
+    Q2 K^T share one accumulator. Returns (codes1, scales1, codes2, scales2, s_t)."""
+    c1, s1, s_t = nvfp4_quantize(x, tensor_scale)
+    c2, s2, _ = nvfp4_quantize(nvfp4_residual(x, c1, s1, s_t), tensor_scale=s_t)
+    return c1, s1, c2, s2, s_t
+
+
 def mxfp8_round_up_tokens(n: int) -> int:
     """Token extent of the stored V codes: whole 128-token tiles."""
     return (n + 127) // 128 * 128

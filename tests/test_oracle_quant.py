@@ -174,3 +174,62 @@ def test_mxfp8_dequant_layout_round_trip():
     err = np.abs(vh - vv)
     assert np.all(err[~sat] <= bound[~sat])
     assert np.all(np.abs(vh[sat]) == 448.0 * step[sat])
+
+
+# ---- dual-residual NVFP4 (Q = Q1 + Q2) ----
+
+def test_dual_residual_hand_worked_block():
+    """Fixed s_t = 1, block [6, 1.3, 0, ...]: Q1 keeps 6 and rounds 1.3 to 1.5 (s_b = 1).
+    The residual fl32(1.3 - 1.5) = -0.2 has amax/6 = 0.0333, which E4M3 rounds to
+    1.125 * 2^-5 = 0.03515625 (its neighbours 0.03125 and 0.03515625); -0.2 / 0.03515625 =
+    -5.69 rounds to E2M1 -6, so Q2 holds -0.2109375 and Q1 + Q2 = 1.2890625."""
+    x = np.zeros((1, 16), dtype=np.float32)
+    x[0, 0], x[0, 1] = 6.0, 1.3
+    c1, s1, c2, s2, s_t = Q.nvfp4_dual_quantize(x, tensor_scale=1.0)
+    x1 = Q.nvfp4_dequantize(c1, s1, s_t)
+    x2 = Q.nvfp4_dequantize(c2, s2, s_t)
+    assert x1[0, 0] == 6.0 and x1[0, 1] == 1.5
+    assert F.e4m3_decode(s2)[0, 0] == 0.03515625
+    assert x2[0, 1] == -0.2109375 and x2[0, 0] == 0.0
+    assert x1[0, 1] + x2[0, 1] == 1.2890625
+
+
+def test_dual_residual_is_zero_on_the_grid():
+    """Values exactly on the NVFP4 grid leave no residual: every Q2 code and scale is 0."""
+    rng = np.random.default_rng(1)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float32)
+    x = rng.choice(grid, (64, 32)) * rng.choice([-1, 1], (64, 32)).astype(np.float32)
+    x[:, 0] = 6.0                                       # every block's scale is exactly 1
+    x[:, 16] = 6.0
+    c1, s1, c2, s2, _ = Q.nvfp4_dual_quantize(x, tensor_scale=1.0 / 448)
+    assert not (Q.nvfp4_unpack(c2) & 7).any() and not s2.any()
+
+
+def test_residual_brute_force_fp32_steps():
+    """The residual, element by element with numpy float32 scalars."""
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((3, 32)) * 5).astype(np.float32)
+    c1, s1, s_t = Q.nvfp4_quantize(x)
+    r = Q.nvfp4_residual(x, c1, s1, s_t)
+    codes = Q.nvfp4_unpack(c1)
+    for i in range(3):
+        for j in range(32):
+            den = np.float32(np.float32(F.e4m3_decode(s1[i, j // 16])) * s_t)
+            d = np.float32(np.float32(F.e2m1_decode(codes[i, j])) * den)
+            assert r[i, j] == np.float32(x[i, j] - d)
+
+
+def test_dual_residual_cuts_logit_error():
+    """Relative logit error |(q - q_hat) . k| / |q . k| over many query/key pairs: the second
+    FP4 tensor cuts it several fold (the page reports 60 % -> 1 % on real queries)."""
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((256, 128)).astype(np.float32)
+    q[:, :4] *= 10.0                                   # outlier channels
+    k = rng.standard_normal((256, 128))
+    c1, s1, c2, s2, s_t = Q.nvfp4_dual_quantize(q)
+    q1 = Q.nvfp4_dequantize(c1, s1, s_t)
+    q12 = q1 + Q.nvfp4_dequantize(c2, s2, s_t)
+    ref = q.astype(np.float64) @ k.T
+    e1 = np.linalg.norm((q1 - q) @ k.T) / np.linalg.norm(ref)
+    e2 = np.linalg.norm((q12 - q) @ k.T) / np.linalg.norm(ref)
+    assert e2 < e1 / 5, (e1, e2)
