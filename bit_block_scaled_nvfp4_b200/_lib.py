@@ -40,6 +40,7 @@ class FwdParams(C.Structure):
         ("head_dim", i32), ("causal", i32), ("softmax_scale", f32),
         ("fp16_bitmap", vp), ("q16", vp), ("k16", vp), ("v16", vp),
         ("out_dtype", i32), ("out", vp), ("lse", vp), ("p_underflow_aware", i32),
+        ("q2_codes", vp), ("q2_scales", vp),
     ]
 
 
@@ -79,6 +80,7 @@ SIGNATURES = {
     "quantize_nvfp4_workspace_size": (sz, []),
     "quantize_nvfp4": (i32, [vp, i32, i64, i32, i64, f32, vp, vp, vp, vp, vp, sz, vp]),
     "quantize_mxfp8_v": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),
+    "quantize_nvfp4_residual": (i32, [vp, i32, i64, i32, i64, vp, vp, vp, vp, vp, vp]),
     "tile_score_select_workspace_size": (sz, [i32, i32, i32, i32]),
     "tile_score_select": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                 vp, vp, vp, vp, sz, vp]),

@@ -107,6 +107,20 @@ def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16
     return NVFP4Tensor(codes, scales, ts, x16)
 
 
+def quantize_nvfp4_dual(x: torch.Tensor, tensor_scale: float | None = None):
+    """Dual-residual NVFP4: (Q1, Q2) with Q1 = quantize_nvfp4(x) and Q2 the encoding of
+    x - Q1's values under Q1's tensor scale (shared tensor-scale tensor)."""
+    q1 = quantize_nvfp4(x, tensor_scale)
+    cols = x.shape[-1]
+    codes2, scales2 = torch.empty_like(q1.codes), torch.empty_like(q1.scales)
+    st = _lib.load().quantize_nvfp4_residual(_ptr(x), _dtype(x), x.numel() // cols, cols, cols,
+                                             _ptr(q1.codes), _ptr(q1.scales),
+                                             _ptr(q1.tensor_scale), _ptr(codes2), _ptr(scales2),
+                                             _stream())
+    _lib.check(st, "quantize_nvfp4_residual")
+    return q1, NVFP4Tensor(codes2, scales2, q1.tensor_scale)
+
+
 def quantize_mxfp8_v(v: torch.Tensor, want_fp16: bool = False) -> MXFP8V:
     """MXFP8-quantize V laid out (..., N, D) along the token axis."""
     lib = _lib.load()
@@ -154,7 +168,7 @@ def tile_score_select(q: NVFP4Tensor, k: NVFP4Tensor, causal: bool, frac_bp: int
 def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
                    softmax_scale: float | None = None, out_dtype=torch.bfloat16,
                    fp16_bitmap: torch.Tensor | None = None, want_lse: bool = False,
-                   underflow_aware: bool = False):
+                   underflow_aware: bool = False, q2: NVFP4Tensor | None = None):
     """QK4V8 attention forward. q.codes [B, Hq, Nq, D/2], k.codes [B, Hkv, Nk, D/2],
     v.codes [B, Hkv, D, Nk_pad]. With ``fp16_bitmap`` the FP16 copies (q.fp16, k.fp16,
     v.fp16) must be present. Returns out [B, Hq, Nq, D] (and lse [B, Hq, Nq])."""
@@ -178,6 +192,8 @@ def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
     p.out = out.data_ptr()
     p.lse = lse.data_ptr() if lse is not None else None
     p.p_underflow_aware = int(bool(underflow_aware))
+    if q2 is not None:                      # dual-residual Q: S = (Q1 + Q2) K^T
+        p.q2_codes, p.q2_scales = q2.codes.data_ptr(), q2.scales.data_ptr()
     _lib.check(lib.attn_qk4v8_fwd(C.byref(p), _stream()), "attn_qk4v8_fwd")
     return (out, lse) if want_lse else out
 
@@ -283,16 +299,23 @@ def kv_append_paged(cache: PagedKV, k_new: torch.Tensor, v_new: torch.Tensor,
 
 def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool,
                     softmax_scale: float | None = None, fp16_frac_bp: int = 0,
-                    out_dtype=None, want_lse: bool = False, underflow_aware: bool = False):
+                    out_dtype=None, want_lse: bool = False, underflow_aware: bool = False,
+                    dual_q: bool = False):
     """The whole prefill path on bf16/fp16 CUDA tensors q [B, Hq, N, D], k/v [B, Hkv, N, D]:
     quantize Q, K (NVFP4) and V (MXFP8), optionally score tiles and recompute the top
-    ``fp16_frac_bp`` basis points of them in FP16, then attention."""
+    ``fp16_frac_bp`` basis points of them in FP16, then attention. ``dual_q`` adds the
+    residual second Q tensor; ``underflow_aware`` scales P per 32-key block."""
     mixed = fp16_frac_bp > 0
-    q4 = quantize_nvfp4(q, want_fp16=mixed)
+    q2 = None
+    if dual_q:
+        q4, q2 = quantize_nvfp4_dual(q)
+    else:
+        q4 = quantize_nvfp4(q, want_fp16=mixed)
     k4 = quantize_nvfp4(k, want_fp16=mixed)
     v8 = quantize_mxfp8_v(v, want_fp16=mixed)
     bitmap = None
     if mixed:
         _, _, bitmap = tile_score_select(q4, k4, causal, fp16_frac_bp)
     return attn_qk4v8_fwd(q4, k4, v8, causal, softmax_scale, out_dtype or q.dtype,
-                          fp16_bitmap=bitmap, want_lse=want_lse, underflow_aware=underflow_aware)
+                          fp16_bitmap=bitmap, want_lse=want_lse, underflow_aware=underflow_aware,
+                          q2=q2)

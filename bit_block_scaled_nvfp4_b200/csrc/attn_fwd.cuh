@@ -54,6 +54,7 @@ constexpr int kPolyOf8 = 0;
 
 struct FwdArgs {
   const uint8_t* q_scales;
+  const uint8_t* q2_scales;   // dual-residual second Q tensor's scales, or null (no second Q)
   const uint8_t* k_scales;
   const uint8_t* v_scales;
   const float* q_ts;
@@ -140,7 +141,11 @@ struct FwdLayout {
   static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
-  static constexpr int OFF_BAR = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
+  // second Q tensor of dual-residual query quantization (FP4-tile kernel only): two buffers by
+  // item parity and their scale factors
+  static constexpr int OFF_Q2 = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
+  static constexpr int OFF_Q2SF = OFF_Q2 + (kMixed ? 0 : 2 * Q_BYTES);
+  static constexpr int OFF_BAR = OFF_Q2SF + (kMixed ? 0 : 2048);
   static constexpr int N_BARS = 2 * NK + 2 * NVS + 2 * NP + 17;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
@@ -150,8 +155,9 @@ struct FwdLayout {
   // scale factors in two slots by tile parity (8 columns each: a slot is rewritten only after
   // the MMA two items / tiles back that read it has completed).
   static constexpr uint32_t T_S = 0, T_O = 256, T_QSF = 400, T_PSF = 416, T_KSF = 420,
-                            T_VSF = 436, T_PSFU = 452;    // T_PSFU: 2 slots by tile parity
-  static_assert(T_O + NV <= T_QSF && T_PSFU + 8 <= 512, "TMEM columns");
+                            T_VSF = 436, T_PSFU = 452,    // T_PSFU: 2 slots by tile parity
+                            T_Q2SF = 460;                 // 2 slots by item parity
+  static_assert(T_O + NV <= T_QSF && T_Q2SF + 16 <= 512, "TMEM columns");
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
   static constexpr int PV_WARP = 2;
@@ -376,12 +382,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < L::KSTEPS; ++kk)
             cp_async4(sm + L::OFF_QSF + qb * 1024 + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
+          if (!kMixed && a.q2_scales != nullptr) {       // the second Q tensor's scales
+            const uint8_t* src2 = a.q2_scales + (valid ? (row0 + r) * (D / 16) : 0);
+#pragma unroll
+            for (int kk = 0; kk < L::KSTEPS; ++kk)
+              cp_async4(sm + L::OFF_Q2SF + qb * 1024 + kk * 512 + lane * 16 + r1 * 4, src2 + kk * 4, valid);
+          }
         }
         cp_async_arrive_noinc(q_full + qb);
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_expect_tx(q_full + qb, L::Q_BYTES);
+          const bool dual = !kMixed && a.q2_scales != nullptr;
+          mbar_arrive_expect_tx(q_full + qb, L::Q_BYTES * (dual ? 2 : 1));
           tma_load_3d(sm + L::OFF_Q + qb * L::Q_BYTES, &tm_q, q_full + qb, 0, w.qt * 128, w.bhq);
+          // (without FP16 tiles the FP16-Q map slot carries the second Q tensor's map)
+          if (dual) tma_load_3d(sm + L::OFF_Q2 + qb * L::Q_BYTES, &tm_q16, q_full + qb, 0, w.qt * 128, w.bhq);
         }
         q_issued = it + 1;
       }
@@ -469,6 +484,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < L::KSTEPS; ++kk)
           tmem_cp_sf(tq + 4 * kk, sm + L::OFF_QSF + qb * 1024 + kk * 512);
         const uint32_t sQ = smem_u32(sm + L::OFF_Q + qb * L::Q_BYTES);
+        const bool dual = !kMixed && a.q2_scales != nullptr;
+        const uint32_t tq2 = tbase + L::T_Q2SF + 8 * qb;
+        if (dual)
+          for (int kk = 0; kk < L::KSTEPS; ++kk)
+            tmem_cp_sf(tq2 + 4 * kk, sm + L::OFF_Q2SF + qb * 1024 + kk * 512);
+        const uint32_t sQ2 = smem_u32(sm + L::OFF_Q2 + qb * L::Q_BYTES);
         bool q16_ready = false, had16 = false;
         for (int j = 0; j < w.nt; ++j, ++g) {
           const int s = g % L::NK;
@@ -487,6 +508,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               const uint64_t da = make_sdesc(sQ + kk * 32, 16, L::QK_SBO, L::QK_SW);
               const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
               mma_nvf4(tS, da, db, idesc_qk, tq + 4 * kk, tk + 4 * kk, kk > 0 ? 1u : 0u);
+            }
+            if (dual) {                              // S += Q2 K^T (same tensor scales)
+              for (int kk = 0; kk < L::KSTEPS; ++kk) {
+                const uint64_t da = make_sdesc(sQ2 + kk * 32, 16, L::QK_SBO, L::QK_SW);
+                const uint64_t db = make_sdesc(sK + kk * 32, 16, L::QK_SBO, L::QK_SW);
+                mma_nvf4(tS, da, db, idesc_qk, tq2 + 4 * kk, tk + 4 * kk, 1u);
+              }
             }
           } else {
             if (!q16_ready) {

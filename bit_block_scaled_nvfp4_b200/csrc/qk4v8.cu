@@ -187,6 +187,30 @@ qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int3
 
 // ------------------------------------------------------------------------------------------
 }  // extern "C"
+static qk4v8_status quantize_nvfp4_residual_impl(const void* x, qk4v8_dtype dtype, int64_t rows,
+                                          int32_t cols, int64_t row_stride, const uint8_t* codes,
+                                          const uint8_t* scales, const float* tensor_scale,
+                                          uint8_t* codes2, uint8_t* scales2, cudaStream_t stream) {
+  if (x == nullptr || codes == nullptr || scales == nullptr || tensor_scale == nullptr ||
+      codes2 == nullptr || scales2 == nullptr)
+    return QK4V8_ERR_INVALID_ARG;
+  if (dtype != QK4V8_F16 && dtype != QK4V8_BF16) return QK4V8_ERR_INVALID_ARG;
+  if (rows < 0 || cols <= 0 || cols % 16 != 0 || row_stride < cols || row_stride % 8 != 0)
+    return QK4V8_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 8) || !aligned(codes2, 8)) return QK4V8_ERR_INVALID_ARG;
+  const int64_t blocks = rows * (cols / 16);
+  const int grid = grid_for(blocks, 256);
+  if (dtype == QK4V8_BF16)
+    nvfp4_residual_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), rows, cols, row_stride, codes, scales, tensor_scale,
+        codes2, scales2);
+  else
+    nvfp4_residual_kernel<__half><<<grid, 256, 0, stream>>>(
+        static_cast<const __half*>(x), rows, cols, row_stride, codes, scales, tensor_scale,
+        codes2, scales2);
+  return launch_status();
+}
+
 template <typename T, int D>
 static void launch_mxfp8(const void* v, int32_t bh, int32_t n, int32_t npad, uint8_t* codes,
                          uint8_t* scales, void* v16, cudaStream_t stream) {
@@ -296,7 +320,14 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
     const uint32_t bv[2] = {128, D};
     if (!make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->v_codes, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
   }
-  if (kMixed) {
+  const bool dual = !kMixed && p->q2_codes != nullptr;
+  if (dual) {                                   // the FP16-Q map slot carries the second Q
+    tk16 = tk; tv16 = tv;
+    const uint64_t dq[3] = {D / 2, static_cast<uint64_t>(Nq), static_cast<uint64_t>(B) * Hq};
+    const uint64_t sq[2] = {D / 2, static_cast<uint64_t>(Nq) * (D / 2)};
+    const uint32_t bq[3] = {D / 2, 128, 1};
+    if (!make_map(&tq16, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p->q2_codes, dq, sq, bq, qk_sw)) return QK4V8_ERR_CUDA;
+  } else if (kMixed) {
     const uint64_t dq[3] = {D, static_cast<uint64_t>(Nq), static_cast<uint64_t>(B) * Hq};
     const uint64_t sq[2] = {D * 2, static_cast<uint64_t>(Nq) * D * 2};
     const uint32_t bq[3] = {64, 128, 1};
@@ -318,6 +349,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   }
   FwdArgs a;
   a.q_scales = p->q_scales; a.k_scales = p->k_scales; a.v_scales = p->v_scales;
+  a.q2_scales = dual ? p->q2_scales : nullptr;
   a.q_ts = p->q_tensor_scale; a.k_ts = p->k_tensor_scale;
   a.bitmap = p->fp16_bitmap; a.out = p->out; a.lse = p->lse;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.Npad = npad;
@@ -359,6 +391,10 @@ qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   const int64_t tiles = static_cast<int64_t>((p->n_q + 127) / 128) * p->batch * p->q_heads;
   if (tiles > 0x7fffffffLL) return QK4V8_ERR_UNSUPPORTED;
   if (p->p_underflow_aware != 0 && p->p_underflow_aware != 1) return QK4V8_ERR_INVALID_ARG;
+  if ((p->q2_codes == nullptr) != (p->q2_scales == nullptr)) return QK4V8_ERR_INVALID_ARG;
+  if (p->q2_codes != nullptr && (!aligned(p->q2_codes, 16) || !aligned(p->q2_scales, sa)))
+    return QK4V8_ERR_INVALID_ARG;
+  if (p->q2_codes != nullptr && mixed) return QK4V8_ERR_UNSUPPORTED;
   if (p->p_underflow_aware) {
     if (mixed) return QK4V8_ERR_UNSUPPORTED;
     return p->head_dim == 128 ? launch_fwd<128, false, true>(p, stream) : launch_fwd<64, false, true>(p, stream);
@@ -518,4 +554,13 @@ extern "C" qk4v8_status kv_append_paged(const qk4v8_append_params* p, cudaStream
   if (p->dtype == QK4V8_BF16) kv_append_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(a);
   else kv_append_kernel<__half><<<grid, 128, 0, stream>>>(a);
   return launch_status();
+}
+
+extern "C" qk4v8_status quantize_nvfp4_residual(const void* x, qk4v8_dtype dtype, int64_t rows,
+                                                int32_t cols, int64_t row_stride,
+                                                const uint8_t* codes, const uint8_t* scales,
+                                                const float* tensor_scale, uint8_t* codes2,
+                                                uint8_t* scales2, cudaStream_t stream) {
+  return quantize_nvfp4_residual_impl(x, dtype, rows, cols, row_stride, codes, scales,
+                                      tensor_scale, codes2, scales2, stream);
 }

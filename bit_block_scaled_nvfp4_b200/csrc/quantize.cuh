@@ -176,6 +176,49 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
+// Residual of an NVFP4 encoding, encoded again with the same tensor scale (dual-residual
+// quantization: x ~ x_hat1 + x_hat2). Per element, in FP32 steps: den = fl32(s_b * s_t),
+// d = fl32(value(code) * den), r = fl32(x - d); then r is NVFP4-encoded with s_t.
+// ---------------------------------------------------------------------------------------
+// E2M1 code (magnitude in bits 0-2, sign in bit 3) -> its value, exactly.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const float v = (m < 2u) ? 0.5f * static_cast<float>(m)
+                           : __uint_as_float((((m >> 1) + 126u) << 23) | ((m & 1u) << 22));
+  return (c & 8u) ? -v : v;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) nvfp4_residual_kernel(
+    const T* __restrict__ x, int64_t rows, int32_t cols, int64_t row_stride,
+    const uint8_t* __restrict__ codes1, const uint8_t* __restrict__ scales1,
+    const float* __restrict__ ts, uint8_t* __restrict__ codes2, uint8_t* __restrict__ scales2) {
+  const float s_t = *ts;
+  const uint32_t blocks_per_row = static_cast<uint32_t>(cols / 16);
+  const int64_t total = rows * blocks_per_row;
+  const bool contiguous = (row_stride == cols);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4* p = reinterpret_cast<const uint4*>(x + block_offset(i, blocks_per_row, row_stride, contiguous));
+    const uint4 a = __ldg(p), b = __ldg(p + 1);
+    const uint2 c1 = __ldg(reinterpret_cast<const uint2*>(codes1 + i * 8));
+    const float den = __fmul_rn(e4m3_code_to_float(scales1[i]), s_t);
+    float f[16];
+    unpack8<T>(a, f);
+    unpack8<T>(b, f + 8);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t code = ((k < 8 ? c1.x : c1.y) >> (4 * (k & 7))) & 0xFu;
+      f[k] = __fsub_rn(f[k], __fmul_rn(e2m1_value(code), den));
+    }
+    uint32_t w[2];
+    const uint32_t sc = nvfp4_encode16(f, s_t, w);
+    *reinterpret_cast<uint2*>(codes2 + i * 8) = make_uint2(w[0], w[1]);
+    scales2[i] = static_cast<uint8_t>(sc);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // MXFP8 for V. v: [BH, N, D] token-major. codes: [BH, D, Npad] token-contiguous; scales:
 // [BH, D, Npad/32] E8M0. Npad = N rounded up to 128; padding tokens read as 0.
 // Shared exponent (OCP MX rule): e = floor(log2 amax) - 8 clamped to [-127, 127]; code

@@ -108,6 +108,22 @@ qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int3
                             size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * quantize_nvfp4_residual — the second tensor of dual-residual query quantization
+ * (sns.style BitDecoding-FP4 summary, first algorithm item: the query as two FP4 tensors, the
+ * second compensating the residual the first leaves). Given x and its NVFP4 encoding (codes,
+ * scales, *tensor_scale) from quantize_nvfp4, per element in FP32 steps
+ *   den = fl32(s_b * s_t),  d = fl32(value(code) * den),  r = fl32(x - d),
+ * and r is NVFP4-encoded with the SAME tensor scale s_t (so Q1 K^T and Q2 K^T share one
+ * accumulator): codes2 [rows, cols/2], scales2 [rows, cols/16]. Shapes and alignment as for
+ * quantize_nvfp4 (codes2 8-byte aligned). attn_qk4v8_fwd and attn_qk4v8_decode_paged take the
+ * result as q2_codes / q2_scales.
+ */
+qk4v8_status quantize_nvfp4_residual(const void* x, qk4v8_dtype dtype, int64_t rows,
+                                     int32_t cols, int64_t row_stride, const uint8_t* codes,
+                                     const uint8_t* scales, const float* tensor_scale,
+                                     uint8_t* codes2, uint8_t* scales2, cudaStream_t stream);
+
+/*
  * quantize_mxfp8_v — MXFP8 quantization of V along the token axis (tqpw.cn article §2.1:
  * E8M0 scale per 32 elements; here the 32 elements are consecutive tokens of one channel,
  * the contraction axis of P V). Shared exponent e = floor(log2 amax) - 8 clamped to
@@ -183,6 +199,11 @@ typedef struct {
   int32_t p_underflow_aware;   /* 0 or 1 as in qk4v8_decode_params (each 32-key block of a
                                   tile row scaled by its own power of two before the E4M3
                                   encode); not with fp16_bitmap */
+  const uint8_t* q2_codes;     /* optional second Q tensor (quantize_nvfp4_residual, same
+                                  layout and tensor scale as q): S = (Q1 + Q2) K^T, two FP4
+                                  MMAs into one accumulator; NULL for one Q tensor; not with
+                                  fp16_bitmap */
+  const uint8_t* q2_scales;
 } qk4v8_fwd_params;
 
 qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* params, cudaStream_t stream);

@@ -169,3 +169,17 @@ def test_append_validation(lib):
     assert f(_app(k_new=FAKE + 8)) == _lib.QK4V8_ERR_INVALID_ARG    # not 16-byte aligned
     assert f(_app(v_pages=FAKE + 4)) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(_app(v_tail=FAKE + 2)) == _lib.QK4V8_ERR_INVALID_ARG
+
+
+def test_quantize_residual_validation(lib):
+    f = lambda **kw: lib.quantize_nvfp4_residual(*[dict(x=FAKE, dt=_lib.QK4V8_BF16, rows=4,
+                                                        cols=64, stride=64, c=FAKE, s=FAKE,
+                                                        ts=FAKE, c2=FAKE, s2=FAKE, st=None,
+                                                        **{})[k] if k not in kw else kw[k]
+                                                   for k in ("x", "dt", "rows", "cols", "stride",
+                                                             "c", "s", "ts", "c2", "s2", "st")])
+    assert f(x=None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(ts=None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(cols=40) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(c2=FAKE + 4) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(dt=_lib.QK4V8_F32) == _lib.QK4V8_ERR_INVALID_ARG

@@ -17,12 +17,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _run(q, k, v, causal, scale=None, frac_bp=0, out_dtype=torch.float32, ua=False):
+def _run(q, k, v, causal, scale=None, frac_bp=0, out_dtype=torch.float32, ua=False, dual=False):
     return api.qk4v8_attention(q.to(DEV), k.to(DEV), v.to(DEV), causal, scale,
-                               fp16_frac_bp=frac_bp, out_dtype=out_dtype, underflow_aware=ua)
+                               fp16_frac_bp=frac_bp, out_dtype=out_dtype, underflow_aware=ua,
+                               dual_q=dual)
 
 
-def _full_oracle(q, k, v, causal, scale, ua=False, exact=False):
+def _full_oracle(q, k, v, causal, scale, ua=False, exact=False, dual=False, q_exact=False):
     B, Hq, N, D = q.shape
     out = np.zeros((B, Hq, q.shape[2], D))
     Hkv = k.shape[1]
@@ -33,7 +34,13 @@ def _full_oracle(q, k, v, causal, scale, ua=False, exact=False):
             vc, vs = OQ.mxfp8_quantize_v(f32(v[b, hk]))
             vh = OQ.mxfp8_dequantize_v(vc, vs, v.shape[2])
             for hq in range(hk * (Hq // Hkv), (hk + 1) * (Hq // Hkv)):
-                qh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(f32(q[b, hq]), tensor_scale=sq))
+                if q_exact:                            # the unquantized query
+                    qh = f32(q[b, hq]).astype(np.float64)
+                elif dual:                             # Q1 + Q2
+                    c1, s1, c2, s2, t = OQ.nvfp4_dual_quantize(f32(q[b, hq]), tensor_scale=sq)
+                    qh = OQ.nvfp4_dequantize(c1, s1, t) + OQ.nvfp4_dequantize(c2, s2, t)
+                else:
+                    qh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(f32(q[b, hq]), tensor_scale=sq))
                 if exact:
                     out[b, hq] = OA.exact_attention(qh, kh, vh, causal, scale)
                 else:
@@ -156,3 +163,25 @@ def test_underflow_aware_keeps_the_small_keys():
     exact = _full_oracle(q, k, v, False, scale, exact=True)
     err = {ua: np.abs(f32(_run(q, k, v, False, scale, ua=ua)) - exact).max() for ua in (False, True)}
     assert err[False] > 1e-3 and err[False] > 5 * err[True], err
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,D,causal", [
+    (1, 4, 2, 700, 700, 128, True),
+    (1, 2, 1, 300, 900, 64, False),
+])
+def test_dual_q_parity_and_quality(B, Hq, Hkv, Nq, Nk, D, causal):
+    """Dual-residual Q: the kernel matches the oracle's attention with Q1 + Q2, and it is closer
+    than the single-Q kernel to the attention whose query is not quantized at all."""
+    g = torch.Generator().manual_seed(Nq * 3 + D)
+    q = torch.randn(B, Hq, Nq, D, generator=g)
+    q[..., :4] *= 8                                      # outlier channels make Q1 coarse
+    q = q.to(torch.bfloat16)
+    k = (torch.randn(B, Hkv, Nk, D, generator=g) * 2).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Nk, D, generator=g).to(torch.bfloat16)
+    scale = 1 / math.sqrt(D)
+    out2 = f32(_run(q, k, v, causal, scale, dual=True))
+    assert_attention_close(out2, _full_oracle(q, k, v, causal, scale, dual=True), "dual Q")
+    ref = _full_oracle(q, k, v, causal, scale, q_exact=True)
+    out1 = f32(_run(q, k, v, causal, scale))
+    e1, e2 = np.abs(out1 - ref).mean(), np.abs(out2 - ref).mean()
+    assert e2 < e1 / 2, (e1, e2)

@@ -134,3 +134,18 @@ def test_e4m3_element_conversion_exhaustive_fp16():
     v[0, :, 5] = tokens
     v[0, :, 60] = -tokens
     _mxfp8_equal(v)
+
+
+@pytest.mark.parametrize("shape,dtype", [((16, 4096, 128), torch.bfloat16), ((3, 37, 64), torch.float16),
+                                         ((1, 16), torch.bfloat16)])
+def test_nvfp4_residual_bit_exact(shape, dtype):
+    """The second tensor of dual-residual quantization: codes and scales bit-exact."""
+    g = torch.Generator().manual_seed(sum(shape))
+    x = (torch.randn(shape, generator=g) * torch.rand(shape[:-1] + (1,), generator=g) * 7).to(dtype)
+    q1, q2 = api.quantize_nvfp4_dual(x.to(DEV))
+    c1, s1, c2, s2, t = OQ.nvfp4_dual_quantize(f32(x))
+    assert np.array_equal(q1.codes.cpu().numpy(), c1) and np.array_equal(q1.scales.cpu().numpy(), s1)
+    gs, gc = q2.scales.cpu().numpy(), q2.codes.cpu().numpy()
+    assert np.array_equal(gs, s2), f"scales differ at {np.argwhere(gs != s2)[:5]}"
+    assert np.array_equal(gc, c2), f"codes differ at {np.argwhere(gc != c2)[:5]}"
+    assert q2.tensor_scale is q1.tensor_scale and np.float32(q1.tensor_scale.item()) == t
