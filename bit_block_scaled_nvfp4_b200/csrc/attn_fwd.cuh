@@ -89,7 +89,7 @@ __device__ __forceinline__ int fwd_item_index(int it, int G, int c) {
   return it * G + ((it & 1) ? (G - 1 - c) : c);
 }
 
-template <int D, bool kMixed>
+template <int D, bool kMixed, bool kDQ = false>
 struct FwdLayout {
   // K and V stages. In the FP16-tile kernel, whose FP16 operands take 100 KB, K and V form
   // rings of their own (three K, two V stages): a K stage is free once QK^T of its tile is
@@ -141,11 +141,11 @@ struct FwdLayout {
   static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
   static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
   static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
-  // second Q tensor of dual-residual query quantization (FP4-tile kernel only): two buffers by
+  // second Q tensor of dual-residual query quantization (its own instance): two buffers by
   // item parity and their scale factors
   static constexpr int OFF_Q2 = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
-  static constexpr int OFF_Q2SF = OFF_Q2 + (kMixed ? 0 : 2 * Q_BYTES);
-  static constexpr int OFF_BAR = OFF_Q2SF + (kMixed ? 0 : 2048);
+  static constexpr int OFF_Q2SF = OFF_Q2 + (kDQ ? 2 * Q_BYTES : 0);
+  static constexpr int OFF_BAR = OFF_Q2SF + (kDQ ? 2048 : 0);
   static constexpr int N_BARS = 2 * NK + 2 * NVS + 2 * NP + 17;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
@@ -167,13 +167,16 @@ struct FwdLayout {
 // kUA: underflow-aware P scaling — each 32-key block of a tile row encoded as
 // E4M3(448 p~ 2^-e), e = ceil(log2 of the block's largest p~) clipped to [-127, 0], with the
 // block's E8M0 P scale 2^e in the PV MMA (FP4 tiles only).
-template <int D, bool kMixed, bool kUA = false>
+// kDQ: dual-residual query quantization — a second Q tensor (same layout and tensor scale)
+// whose QK^T MMAs accumulate into the same S (FP4 tiles only).
+template <int D, bool kMixed, bool kUA = false, bool kDQ = false>
 __global__ void __launch_bounds__(384, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q16,
                 const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
                 FwdArgs a) {
-  using L = FwdLayout<D, kMixed>;
+  using L = FwdLayout<D, kMixed, kDQ>;
+  static_assert(!(kMixed && kDQ), "no second Q tensor with FP16 tiles");
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte aligned base, kept as an offset from the shared array so that the compiler
   // still sees shared-memory accesses (not generic ones)
@@ -382,7 +385,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < L::KSTEPS; ++kk)
             cp_async4(sm + L::OFF_QSF + qb * 1024 + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
-          if (!kMixed && a.q2_scales != nullptr) {       // the second Q tensor's scales
+          if constexpr (kDQ) {                           // the second Q tensor's scales
             const uint8_t* src2 = a.q2_scales + (valid ? (row0 + r) * (D / 16) : 0);
 #pragma unroll
             for (int kk = 0; kk < L::KSTEPS; ++kk)
@@ -392,7 +395,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         cp_async_arrive_noinc(q_full + qb);
         __syncwarp();
         if (lane == 0) {
-          const bool dual = !kMixed && a.q2_scales != nullptr;
+          constexpr bool dual = kDQ;
           mbar_arrive_expect_tx(q_full + qb, L::Q_BYTES * (dual ? 2 : 1));
           tma_load_3d(sm + L::OFF_Q + qb * L::Q_BYTES, &tm_q, q_full + qb, 0, w.qt * 128, w.bhq);
           // (without FP16 tiles the FP16-Q map slot carries the second Q tensor's map)
@@ -484,7 +487,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int kk = 0; kk < L::KSTEPS; ++kk)
           tmem_cp_sf(tq + 4 * kk, sm + L::OFF_QSF + qb * 1024 + kk * 512);
         const uint32_t sQ = smem_u32(sm + L::OFF_Q + qb * L::Q_BYTES);
-        const bool dual = !kMixed && a.q2_scales != nullptr;
+        constexpr bool dual = kDQ;
         const uint32_t tq2 = tbase + L::T_Q2SF + 8 * qb;
         if (dual)
           for (int kk = 0; kk < L::KSTEPS; ++kk)

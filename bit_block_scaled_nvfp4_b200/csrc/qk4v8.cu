@@ -299,9 +299,9 @@ qk4v8_status tile_score_select(const uint8_t* q_codes, const uint8_t* q_scales,
 
 // ------------------------------------------------------------------------------------------
 }  // extern "C"
-template <int D, bool kMixed, bool kUA = false>
+template <int D, bool kMixed, bool kUA = false, bool kDQ = false>
 static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
-  using L = FwdLayout<D, kMixed>;
+  using L = FwdLayout<D, kMixed, kDQ>;
   const int32_t B = p->batch, Hq = p->q_heads, Hkv = p->kv_heads;
   const int32_t Nq = p->n_q, Nk = p->n_k;
   const int32_t npad = (Nk + 127) / 128 * 128;
@@ -320,7 +320,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
     const uint32_t bv[2] = {128, D};
     if (!make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->v_codes, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
   }
-  const bool dual = !kMixed && p->q2_codes != nullptr;
+  constexpr bool dual = kDQ;
   if (dual) {                                   // the FP16-Q map slot carries the second Q
     tk16 = tk; tv16 = tv;
     const uint64_t dq[3] = {D / 2, static_cast<uint64_t>(Nq), static_cast<uint64_t>(B) * Hq};
@@ -344,7 +344,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   }
   static bool attr = false;
   if (!attr) {
-    if (!set_smem(attn_fwd_kernel<D, kMixed, kUA>, L::SMEM_ALLOC)) return QK4V8_ERR_CUDA;
+    if (!set_smem(attn_fwd_kernel<D, kMixed, kUA, kDQ>, L::SMEM_ALLOC)) return QK4V8_ERR_CUDA;
     attr = true;
   }
   FwdArgs a;
@@ -361,7 +361,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   const int64_t items = static_cast<int64_t>(a.Tq) * B * Hq;
   if (items > INT32_MAX / 2) return QK4V8_ERR_UNSUPPORTED;
   const int64_t grid = items < sm_count() ? items : sm_count();
-  attn_fwd_kernel<D, kMixed, kUA><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
+  attn_fwd_kernel<D, kMixed, kUA, kDQ><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(tq, tk, tv, tq16, tk16, tv16, a);
   return launch_status();
 }
 
@@ -395,9 +395,15 @@ qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   if (p->q2_codes != nullptr && (!aligned(p->q2_codes, 16) || !aligned(p->q2_scales, sa)))
     return QK4V8_ERR_INVALID_ARG;
   if (p->q2_codes != nullptr && mixed) return QK4V8_ERR_UNSUPPORTED;
-  if (p->p_underflow_aware) {
+  const bool dq = p->q2_codes != nullptr;
+  if (p->p_underflow_aware || dq) {
     if (mixed) return QK4V8_ERR_UNSUPPORTED;
-    return p->head_dim == 128 ? launch_fwd<128, false, true>(p, stream) : launch_fwd<64, false, true>(p, stream);
+    if (p->head_dim == 128) {
+      if (p->p_underflow_aware) return dq ? launch_fwd<128, false, true, true>(p, stream) : launch_fwd<128, false, true>(p, stream);
+      return launch_fwd<128, false, false, true>(p, stream);
+    }
+    if (p->p_underflow_aware) return dq ? launch_fwd<64, false, true, true>(p, stream) : launch_fwd<64, false, true>(p, stream);
+    return launch_fwd<64, false, false, true>(p, stream);
   }
   if (p->head_dim == 128) return mixed ? launch_fwd<128, true>(p, stream) : launch_fwd<128, false>(p, stream);
   return mixed ? launch_fwd<64, true>(p, stream) : launch_fwd<64, false>(p, stream);
