@@ -53,7 +53,7 @@ class DecodeParams(C.Structure):
         ("num_seqs", i32), ("num_pages", i32), ("max_pages", i32), ("q_heads", i32),
         ("kv_heads", i32), ("head_dim", i32), ("max_context", i32), ("split_tokens", i32),
         ("softmax_scale", f32), ("out_dtype", i32), ("out", vp), ("lse", vp),
-        ("p_underflow_aware", i32),
+        ("p_underflow_aware", i32), ("q2_codes", vp), ("q2_scales", vp),
     ]
 
 

@@ -211,7 +211,7 @@ class PagedKV:
 def decode_params(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
                   context_lens: torch.Tensor, max_context: int, split_tokens: int,
                   out: torch.Tensor, softmax_scale: float | None = None, lse=None,
-                  underflow_aware: bool = False):
+                  underflow_aware: bool = False, q2: NVFP4Tensor | None = None):
     S, Hq, dh = q.codes.shape
     P, Hkv = cache.k_pages.shape[0], cache.k_pages.shape[1]
     d = dh * 2
@@ -229,6 +229,8 @@ def decode_params(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
     p.out = out.data_ptr()
     p.lse = lse.data_ptr() if lse is not None else None
     p.p_underflow_aware = int(bool(underflow_aware))
+    if q2 is not None:                      # dual-residual Q
+        p.q2_codes, p.q2_scales = q2.codes.data_ptr(), q2.scales.data_ptr()
     return p
 
 
@@ -236,7 +238,7 @@ def attn_qk4v8_decode_paged(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Te
                             context_lens: torch.Tensor, max_context: int, split_tokens: int,
                             softmax_scale: float | None = None, out_dtype=torch.bfloat16,
                             want_lse: bool = False, workspace: torch.Tensor | None = None,
-                            underflow_aware: bool = False):
+                            underflow_aware: bool = False, q2: NVFP4Tensor | None = None):
     """One decode step. q.codes [S, Hq, D/2]; returns out [S, Hq, D] (and lse [S, Hq]).
     ``underflow_aware`` scales P per 32-key block by a power of two before its E4M3 encode."""
     lib = _lib.load()
@@ -244,7 +246,7 @@ def attn_qk4v8_decode_paged(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Te
     out = torch.empty(S, Hq, dh * 2, dtype=out_dtype, device=q.codes.device)
     lse = torch.empty(S, Hq, dtype=torch.float32, device=q.codes.device) if want_lse else None
     p = decode_params(q, cache, page_table, context_lens, max_context, split_tokens, out,
-                      softmax_scale, lse, underflow_aware)
+                      softmax_scale, lse, underflow_aware, q2)
     need = lib.attn_qk4v8_decode_workspace_size(C.byref(p))
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.codes.device)

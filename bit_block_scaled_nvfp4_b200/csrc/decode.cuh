@@ -26,6 +26,7 @@ namespace qk4v8 {
 
 struct DecArgs {
   const uint8_t* q_scales;       // [S*Hq, D/16]
+  const uint8_t* q2_scales;      // the second Q tensor's, or null
   const float* q_ts;
   const uint8_t* k_page_scales;  // [P, Hkv, 64, D/16]
   const float* k_ts;
@@ -41,7 +42,7 @@ struct DecArgs {
 // the first GM query columns of the N = 16 MMA operand (rows >= g of Q^T and P^T are zero).
 // With GM = 4 the kernel fits three CTAs per SM (80 registers, two stages per ring); the
 // wider instances keep two CTAs per SM and three stages.
-template <int GM>
+template <int GM, bool kDQ = false>
 struct DecLayout {
   static constexpr int CTAS_PER_SM = GM <= 4 ? 3 : 2;
   static constexpr int D = 128;
@@ -54,7 +55,9 @@ struct DecLayout {
   // n*16 + b; E8M0 127 = 1.0 unless underflow-aware scaling lowers it), then a constant chunk of
   // 1.0 for the ones operand
   static constexpr int OFF_PSF = 2048;
-  static constexpr int OFF_P = 4096;              // 2 x [16 rows x 128 B] (SW128), 1024-aligned
+  // second Q tensor of dual-residual query quantization (its own instance): operand + scales
+  static constexpr int OFF_Q2 = 4096, OFF_Q2SF = 5120;
+  static constexpr int OFF_P = kDQ ? 6144 : 4096; // 2 x [16 rows x 128 B] (SW128), 1024-aligned
   static constexpr int OFF_ONES = OFF_P + 2 * 2048;       // 128 x 32 B of E4M3 1.0 (SW32)
   static constexpr int OFF_KST = OFF_ONES + 4096;         // 12288, 1024-aligned
   static constexpr int ST_K = 0;                  // 128 keys x 64 B (SW64)
@@ -77,7 +80,8 @@ struct DecLayout {
   static constexpr uint32_t T_S = 0, T_O = 32, T_L = 48, T_QSF = 64, T_PSF = 72, T_ONESF = 80,
                             T_KSF = 84,
                             T_VSF = T_KSF + 8 * NK;
-  static_assert(T_VSF + 4 * NVS <= 128, "TMEM columns");
+  static constexpr uint32_t T_Q2SF = T_VSF + 4 * NVS;          // 2 chunks (kDQ only)
+  static_assert(T_Q2SF + (kDQ ? 8 : 0) <= 128, "TMEM columns");
   static constexpr int NQ = 16;                   // MMA N (query heads, padded)
   static constexpr int PV_WARP = 6;
   static constexpr int VLOAD_WARP = 7;
@@ -86,11 +90,14 @@ struct DecLayout {
 
 // kUA: underflow-aware P scaling (a separate instance, so that the default path carries none
 // of its work).
-template <int GM, bool kUA>
+// kDQ: a second Q tensor (dual-residual query quantization, same tensor scale) whose QK^T
+// MMAs accumulate into the same S^T; tm_q2 maps it (unused otherwise).
+template <int GM, bool kUA, bool kDQ = false>
 __global__ void __launch_bounds__(256, DecLayout<GM>::CTAS_PER_SM)
 decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
-              const __grid_constant__ CUtensorMap tm_vp, DecArgs a) {
-  using L = DecLayout<GM>;
+              const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_q2,
+              DecArgs a) {
+  using L = DecLayout<GM, kDQ>;
   constexpr int D = L::D;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -212,11 +219,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       *reinterpret_cast<uint4*>(sm + L::OFF_QSF + lane * 16) = make_uint4(w0, 0, 0, 0);
       *reinterpret_cast<uint4*>(sm + L::OFF_QSF + 512 + lane * 16) = make_uint4(w1, 0, 0, 0);
+      if constexpr (kDQ) {                             // the second Q tensor's scales
+        uint32_t u0 = 0, u1 = 0;
+        if (lane < g) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.q2_scales + (qrow0 + lane) * (D / 16)));
+          u0 = v.x; u1 = v.y;
+        }
+        *reinterpret_cast<uint4*>(sm + L::OFF_Q2SF + lane * 16) = make_uint4(u0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sm + L::OFF_Q2SF + 512 + lane * 16) = make_uint4(u1, 0, 0, 0);
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, 16 * 64);
+        mbar_arrive_expect_tx(q_full, 16 * 64 * (kDQ ? 2 : 1));
         tma_load_2d(sm + L::OFF_Q, &tm_q, q_full, 0, static_cast<int>(qrow0));
+        if constexpr (kDQ) tma_load_2d(sm + L::OFF_Q2, &tm_q2, q_full, 0, static_cast<int>(qrow0));
       }
     }
     int issued = 0;
@@ -289,6 +306,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_after();
         tmem_cp_sf(tbase + L::T_QSF, sm + L::OFF_QSF);
         tmem_cp_sf(tbase + L::T_QSF + 4, sm + L::OFF_QSF + 512);
+        if constexpr (kDQ) {
+          tmem_cp_sf(tbase + L::T_Q2SF, sm + L::OFF_Q2SF);
+          tmem_cp_sf(tbase + L::T_Q2SF + 4, sm + L::OFF_Q2SF + 512);
+        }
       }
       for (int blk = 0; ok && blk < nblk; ++blk) {
         const int st_i = blk % L::NK, b2 = blk & 1;
@@ -309,6 +330,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           const uint64_t db = make_sdesc(sQ + kk * 32, 16, 512, kSw64);
           mma_nvf4(tbase + L::T_S + b2 * 16, da, db, idesc_qk, tk + 4 * kk,
                    tbase + L::T_QSF + 4 * kk, kk > 0 ? 1u : 0u);
+        }
+        if constexpr (kDQ) {                           // S^T += K Q2^T
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint64_t da = make_sdesc(sK + kk * 32, 16, 512, kSw64);
+            const uint64_t db = make_sdesc(smem_u32(sm + L::OFF_Q2) + kk * 32, 16, 512, kSw64);
+            mma_nvf4(tbase + L::T_S + b2 * 16, da, db, idesc_qk, tk + 4 * kk,
+                     tbase + L::T_Q2SF + 4 * kk, 1u);
+          }
         }
         mma_commit(s_full + b2);
         mma_commit(k_empty + st_i);

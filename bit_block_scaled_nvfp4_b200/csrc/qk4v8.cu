@@ -436,6 +436,9 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
     return QK4V8_ERR_INVALID_ARG;
   if (!(p->softmax_scale > 0.f)) return QK4V8_ERR_INVALID_ARG;
   if (p->p_underflow_aware != 0 && p->p_underflow_aware != 1) return QK4V8_ERR_INVALID_ARG;
+  if ((p->q2_codes == nullptr) != (p->q2_scales == nullptr)) return QK4V8_ERR_INVALID_ARG;
+  if (p->q2_codes != nullptr && (!aligned(p->q2_codes, 16) || !aligned(p->q2_scales, 8)))
+    return QK4V8_ERR_INVALID_ARG;
   if (p->head_dim != 128 || p->q_heads / p->kv_heads > 16) return QK4V8_ERR_UNSUPPORTED;
   if (!aligned(p->q_codes, 16) || !aligned(p->k_pages, 16) || !aligned(p->v_pages, 16) ||
       !aligned(p->q_scales, 8) || !aligned(p->k_page_scales, 8) || !aligned(p->v_page_scales, 4) ||
@@ -445,12 +448,16 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   const int32_t n_splits = decode_splits(p);
   if (n_splits > 65535 || p->num_seqs > 65535 || p->kv_heads > 65535) return QK4V8_ERR_UNSUPPORTED;
   constexpr int D = 128;
-  CUtensorMap tq, tkp, tvp;
+  CUtensorMap tq, tq2, tkp, tvp;
   {
     const uint64_t dq[2] = {D / 2, static_cast<uint64_t>(p->num_seqs) * p->q_heads};
     const uint64_t sq[1] = {D / 2};
     const uint32_t bq[2] = {D / 2, 16};
     if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->q_codes, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_64B)) return QK4V8_ERR_CUDA;
+    tq2 = tq;                                    // the second Q tensor's map (dual-residual Q)
+    if (p->q2_codes != nullptr &&
+        !make_map(&tq2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->q2_codes, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_64B))
+      return QK4V8_ERR_CUDA;
     const uint64_t dk[2] = {D / 2, static_cast<uint64_t>(p->num_pages) * p->kv_heads * 64};
     const uint32_t bk[2] = {D / 2, 64};
     if (!make_map(&tkp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->k_pages, dk, sq, bk, CU_TENSOR_MAP_SWIZZLE_64B)) return QK4V8_ERR_CUDA;
@@ -466,12 +473,18 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
         !set_smem(decode_kernel<16, false>, DecLayout<16>::SMEM_ALLOC) ||
         !set_smem(decode_kernel<4, true>, DecLayout<4>::SMEM_ALLOC) ||
         !set_smem(decode_kernel<8, true>, DecLayout<8>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<16, true>, DecLayout<16>::SMEM_ALLOC))
+        !set_smem(decode_kernel<16, true>, DecLayout<16>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<4, false, true>, DecLayout<4, true>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<8, false, true>, DecLayout<8, true>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<16, false, true>, DecLayout<16, true>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<4, true, true>, DecLayout<4, true>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<8, true, true>, DecLayout<8, true>::SMEM_ALLOC) ||
+        !set_smem(decode_kernel<16, true, true>, DecLayout<16, true>::SMEM_ALLOC))
       return QK4V8_ERR_CUDA;
     attr = true;
   }
   DecArgs a;
-  a.q_scales = p->q_scales; a.q_ts = p->q_tensor_scale;
+  a.q_scales = p->q_scales; a.q2_scales = p->q2_scales; a.q_ts = p->q_tensor_scale;
   a.k_page_scales = p->k_page_scales; a.k_ts = p->k_tensor_scale;
   a.v_page_scales = p->v_page_scales; a.page_table = p->page_table; a.lens = p->context_lens;
   a.ws = static_cast<float*>(workspace);
@@ -482,12 +495,16 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   // the softmax handles the g = Hq / Hkv real query columns: an instance per bound on g
   const int g = p->q_heads / p->kv_heads;
   const bool ua = p->p_underflow_aware != 0;
-#define QK4V8_DEC(GM)                                                                          \
-  (ua ? decode_kernel<GM, true><<<grid, DecLayout<GM>::THREADS, DecLayout<GM>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a) \
-      : decode_kernel<GM, false><<<grid, DecLayout<GM>::THREADS, DecLayout<GM>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, a))
+  const bool dq = p->q2_codes != nullptr;
+#define QK4V8_DEC1(GM, UA, DQ) \
+  decode_kernel<GM, UA, DQ><<<grid, DecLayout<GM, DQ>::THREADS, DecLayout<GM, DQ>::SMEM_ALLOC, stream>>>(tq, tkp, tvp, tq2, a)
+#define QK4V8_DEC(GM)                                                                              \
+  (ua ? (dq ? QK4V8_DEC1(GM, true, true) : QK4V8_DEC1(GM, true, false))                            \
+      : (dq ? QK4V8_DEC1(GM, false, true) : QK4V8_DEC1(GM, false, false)))
   if (g <= 4) QK4V8_DEC(4);
   else if (g <= 8) QK4V8_DEC(8);
   else QK4V8_DEC(16);
+#undef QK4V8_DEC1
 #undef QK4V8_DEC
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   decode_merge_kernel<<<p->num_seqs * p->q_heads, 128, 0, stream>>>(

@@ -244,6 +244,10 @@ typedef struct {
                                   e = ceil(log2 max p~) clipped to [-127, 0] and the MMA's E8M0
                                   scale 2^e (sns.style BitDecoding-FP4 summary, underflow-aware
                                   probability scaling: long-context P must not round to zero) */
+  const uint8_t* q2_codes;     /* optional second Q tensor [S, Hq, D/2] from
+                                  quantize_nvfp4_residual (same tensor scale as q): S^T = K
+                                  (Q1 + Q2)^T, two FP4 MMAs into one accumulator; or NULL */
+  const uint8_t* q2_scales;    /* [S, Hq, D/16] with q2_codes */
 } qk4v8_decode_params;
 
 size_t attn_qk4v8_decode_workspace_size(const qk4v8_decode_params* params);

@@ -37,12 +37,16 @@ def _build(lens, hkv, d, seed, shuffle=True):
     return cache, table, seqs
 
 
-def _oracle_decode(q, seqs, lens, hq, hkv, split, scale, ua=False, exact=False):
+def _oracle_decode(q, seqs, lens, hq, hkv, split, scale, ua=False, exact=False, dual=False):
     """Oracle outputs [S, Hq, D] from the dense per-sequence K/V and the step's q."""
     S, _, d = q.shape
     sq = oracle_tensor_scale(q)
-    qc, qs, qt = OQ.nvfp4_quantize(f32(q), tensor_scale=sq)
-    qh = OQ.nvfp4_dequantize(qc, qs, qt)
+    if dual:                                             # Q1 + Q2
+        c1, s1, c2, s2, t = OQ.nvfp4_dual_quantize(f32(q), tensor_scale=sq)
+        qh = OQ.nvfp4_dequantize(c1, s1, t) + OQ.nvfp4_dequantize(c2, s2, t)
+    else:
+        qc, qs, qt = OQ.nvfp4_quantize(f32(q), tensor_scale=sq)
+        qh = OQ.nvfp4_dequantize(qc, qs, qt)
     g = hq // hkv
     out = np.zeros((S, hq, d))
     lse = np.zeros((S, hq))
@@ -183,3 +187,22 @@ def test_decode_underflow_aware_parity_and_quality():
     err_fix = np.abs(out_fix - exact).max()
     err_ua = np.abs(out_ua - exact).max()
     assert err_fix > 1e-3 and err_fix > 5 * err_ua, (err_fix, err_ua)
+
+
+@pytest.mark.parametrize("ua", [False, True])
+def test_decode_dual_q_parity(ua):
+    """Dual-residual Q (and with underflow-aware P): the kernel matches the oracle's decode
+    with Q1 + Q2."""
+    lens, hq, hkv, d, split = [5000, 333, 1], 32, 8, 128, 1024
+    cache, table, seqs = _build(lens, hkv, d, seed=77)
+    g = torch.Generator().manual_seed(12)
+    q = torch.randn(len(lens), hq, d, generator=g)
+    q[..., :4] *= 8
+    q = q.to(torch.bfloat16)
+    q1, q2 = api.quantize_nvfp4_dual(q.to(DEV))
+    ctx = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    out = api.attn_qk4v8_decode_paged(q1, cache, table.to(DEV), ctx, max(lens), split,
+                                      out_dtype=torch.float32, underflow_aware=ua, q2=q2)
+    assert api.check_status() == 0
+    want, _ = _oracle_decode(q, seqs, lens, hq, hkv, split, 1 / math.sqrt(d), ua=ua, dual=True)
+    assert_attention_close(f32(out), want, "decode dual Q")
