@@ -81,6 +81,8 @@ SIGNATURES = {
     "quantize_nvfp4": (i32, [vp, i32, i64, i32, i64, f32, vp, vp, vp, vp, vp, sz, vp]),
     "quantize_mxfp8_v": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),
     "quantize_nvfp4_residual": (i32, [vp, i32, i64, i32, i64, vp, vp, vp, vp, vp, vp]),
+    "quantize_nvfp4_searched": (i32, [vp, i32, i64, i32, i64, f32, vp, vp, vp, vp, vp, sz, vp]),
+    "qk_smooth_rotate": (i32, [vp, i32, i64, i32, vp, i32, vp, vp]),
     "tile_score_select_workspace_size": (sz, [i32, i32, i32, i32]),
     "tile_score_select": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                 vp, vp, vp, vp, sz, vp]),

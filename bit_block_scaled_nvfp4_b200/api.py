@@ -85,8 +85,9 @@ def selftest_wait_timeout() -> None:
 
 
 def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16: bool = False,
-                   workspace: torch.Tensor | None = None) -> NVFP4Tensor:
-    """NVFP4-quantize ``x`` (..., D) along its last axis (contiguous fp16/bf16 CUDA tensor)."""
+                   workspace: torch.Tensor | None = None, scale_search: bool = False) -> NVFP4Tensor:
+    """NVFP4-quantize ``x`` (..., D) along its last axis (contiguous fp16/bf16 CUDA tensor);
+    ``scale_search`` picks each block's scale among four candidates by squared error."""
     lib = _lib.load()
     if not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA tensor")
@@ -99,12 +100,28 @@ def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16
     x16 = torch.empty(x.shape, dtype=torch.float16, device=dev) if want_fp16 else None
     if workspace is None:
         workspace = torch.empty(lib.quantize_nvfp4_workspace_size(), dtype=torch.uint8, device=dev)
-    st = lib.quantize_nvfp4(_ptr(x), _dtype(x), rows, cols, cols,
+    fn = lib.quantize_nvfp4_searched if scale_search else lib.quantize_nvfp4
+    st = fn(_ptr(x), _dtype(x), rows, cols, cols,
                             float(tensor_scale) if tensor_scale else 0.0, _ptr(codes),
                             _ptr(scales), _ptr(ts), _ptr(x16), _ptr(workspace),
                             workspace.numel(), _stream())
     _lib.check(st, "quantize_nvfp4")
     return NVFP4Tensor(codes, scales, ts, x16)
+
+
+def qk_smooth_rotate(x: torch.Tensor, role: str, lam: torch.Tensor | None = None) -> torch.Tensor:
+    """Outlier-aware transform of queries (role 'q': x * lam) or keys ('k': x / lam) along the
+    last axis (128): per-channel smoothing, the 128-point Hadamard rotation and 2^-3 / 2^-4,
+    so that transformed queries and keys keep their dot products. Returns a new tensor."""
+    if not x.is_cuda or not x.is_contiguous() or x.shape[-1] != 128:
+        raise ValueError("x must be a contiguous CUDA tensor with last dimension 128")
+    if lam is not None and (not lam.is_cuda or lam.dtype != torch.float32 or lam.numel() != 128):
+        raise ValueError("lam must be 128 float32 values on the GPU")
+    out = torch.empty_like(x)
+    st = _lib.load().qk_smooth_rotate(_ptr(x), _dtype(x), x.numel() // 128, 128, _ptr(lam),
+                                      0 if role == "q" else 1, _ptr(out), _stream())
+    _lib.check(st, "qk_smooth_rotate")
+    return out
 
 
 def quantize_nvfp4_dual(x: torch.Tensor, tensor_scale: float | None = None):

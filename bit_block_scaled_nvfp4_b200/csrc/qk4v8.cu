@@ -141,10 +141,14 @@ qk4v8_status qk4v8_selftest_wait_timeout(cudaStream_t stream) {
 constexpr int kAmaxPartials = 1024;
 size_t quantize_nvfp4_workspace_size(void) { return 4 * kAmaxPartials; }
 
-qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,
-                            int64_t row_stride, float tensor_scale_in, uint8_t* codes,
-                            uint8_t* scales, float* tensor_scale, void* x16, void* workspace,
-                            size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+// NVFP4 quantize; kSearch: per-block scale search (outlier-aware keys).
+template <bool kSearch>
+static qk4v8_status quantize_nvfp4_impl(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,
+                                        int64_t row_stride, float tensor_scale_in, uint8_t* codes,
+                                        uint8_t* scales, float* tensor_scale, void* x16, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream) {
   if (x == nullptr || codes == nullptr || scales == nullptr || tensor_scale == nullptr)
     return QK4V8_ERR_INVALID_ARG;
   if (dtype != QK4V8_F16 && dtype != QK4V8_BF16) return QK4V8_ERR_INVALID_ARG;
@@ -175,13 +179,50 @@ qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int3
   __half* h = static_cast<__half*>(x16);
   if (dtype == QK4V8_BF16) {
     auto xb = static_cast<const __nv_bfloat16*>(x);
-    if (h) nvfp4_encode_kernel<__nv_bfloat16, true><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
-    else nvfp4_encode_kernel<__nv_bfloat16, false><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
+    if (h) nvfp4_encode_kernel<__nv_bfloat16, true, kSearch><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
+    else nvfp4_encode_kernel<__nv_bfloat16, false, kSearch><<<grid, 256, 0, stream>>>(xb, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
   } else {
     auto xh = static_cast<const __half*>(x);
-    if (h) nvfp4_encode_kernel<__half, true><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
-    else nvfp4_encode_kernel<__half, false><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
+    if (h) nvfp4_encode_kernel<__half, true, kSearch><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
+    else nvfp4_encode_kernel<__half, false, kSearch><<<grid, 256, 0, stream>>>(xh, rows, cols, row_stride, amax, agrid, tensor_scale_in, codes, scales, tensor_scale, h);
   }
+  return launch_status();
+}
+
+extern "C" {
+qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,
+                            int64_t row_stride, float tensor_scale_in, uint8_t* codes,
+                            uint8_t* scales, float* tensor_scale, void* x16, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
+  return quantize_nvfp4_impl<false>(x, dtype, rows, cols, row_stride, tensor_scale_in, codes,
+                                    scales, tensor_scale, x16, workspace, workspace_bytes, stream);
+}
+
+qk4v8_status quantize_nvfp4_searched(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,
+                                     int64_t row_stride, float tensor_scale_in, uint8_t* codes,
+                                     uint8_t* scales, float* tensor_scale, void* x16,
+                                     void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return quantize_nvfp4_impl<true>(x, dtype, rows, cols, row_stride, tensor_scale_in, codes,
+                                   scales, tensor_scale, x16, workspace, workspace_bytes, stream);
+}
+
+qk4v8_status qk_smooth_rotate(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t head_dim,
+                              const float* lam, int32_t role, void* out, cudaStream_t stream) {
+  if (x == nullptr || out == nullptr || rows < 0) return QK4V8_ERR_INVALID_ARG;
+  if (dtype != QK4V8_F16 && dtype != QK4V8_BF16) return QK4V8_ERR_INVALID_ARG;
+  if (role != 0 && role != 1) return QK4V8_ERR_INVALID_ARG;
+  if (head_dim != 128) return QK4V8_ERR_UNSUPPORTED;
+  if (!aligned(x, 8) || !aligned(out, 8) || (lam != nullptr && !aligned(lam, 4)))
+    return QK4V8_ERR_INVALID_ARG;
+  if (rows == 0) return QK4V8_OK;
+  const int64_t grid = (rows + 7) / 8;                 // 8 rows (warps) per CTA
+  if (grid > 0x7fffffffLL) return QK4V8_ERR_UNSUPPORTED;
+  if (dtype == QK4V8_BF16)
+    smooth_rotate_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), rows, lam, role, static_cast<__nv_bfloat16*>(out));
+  else
+    smooth_rotate_kernel<__half><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        static_cast<const __half*>(x), rows, lam, role, static_cast<__half*>(out));
   return launch_status();
 }
 

@@ -103,6 +103,7 @@ __device__ __forceinline__ float reduce_partials(const float* __restrict__ parti
 
 // One 16-element NVFP4 block with tensor scale s_t: returns the E4M3 scale code and writes
 // the 8 code bytes (element 2i in the low nibble of byte i) to w[0..1].
+__device__ __forceinline__ void e2m1_encode16(const float* f, float den, uint32_t* w);
 __device__ __forceinline__ uint32_t nvfp4_encode16(const float* f, float s_t, uint32_t* w) {
   float amax_b = 0.f;
 #pragma unroll
@@ -111,31 +112,75 @@ __device__ __forceinline__ uint32_t nvfp4_encode16(const float* f, float s_t, ui
   const uint32_t sc = cvt_e4m3x2(sbf, 0.f) & 0xFFu;
   const float sbv = e4m3_code_to_float(sc);
   w[0] = w[1] = 0u;
-  if (sbv != 0.f) {
-    const float den = __fmul_rn(sbv, s_t);
-    // x / den correctly rounded, by Markstein's theorem where its conditions hold (the
-    // reciprocal correctly rounded, no intermediate over- or underflow: den within
-    // [2^-90, 2^90], and the quotients that decide a code are at most 8), else by IEEE
-    // division. The test is false for NaN and infinities.
-    const bool fast = (den >= 0x1p-90f && den <= 0x1p90f);
-    const float y = __frcp_rn(den);
+  if (sbv != 0.f) e2m1_encode16(f, __fmul_rn(sbv, s_t), w);
+  return sc;
+}
+
+// The 16 E2M1 codes of a block under divisor den (> 0): code_i = E2M1(fl32(x_i / den)), the
+// quotient correctly rounded (Markstein's division inside its safe range, else IEEE).
+__device__ __forceinline__ void e2m1_encode16(const float* f, float den, uint32_t* w) {
+  w[0] = w[1] = 0u;
+  const bool fast = (den >= 0x1p-90f && den <= 0x1p90f);
+  const float y = __frcp_rn(den);
 #pragma unroll
-    for (int k = 0; k < 16; k += 2) {
-      const float q0 = fast ? div_markstein(f[k], den, y) : __fdiv_rn(f[k], den);
-      const float q1 = fast ? div_markstein(f[k + 1], den, y) : __fdiv_rn(f[k + 1], den);
-      uint32_t byte = cvt_e2m1x2(q0, q1) & 0x77u;
-      byte |= (__float_as_uint(f[k]) >> 31) << 3;
-      byte |= (__float_as_uint(f[k + 1]) >> 31) << 7;
-      w[k >> 3] |= byte << ((k & 7) * 4);
+  for (int k = 0; k < 16; k += 2) {
+    const float q0 = fast ? div_markstein(f[k], den, y) : __fdiv_rn(f[k], den);
+    const float q1 = fast ? div_markstein(f[k + 1], den, y) : __fdiv_rn(f[k + 1], den);
+    uint32_t byte = cvt_e2m1x2(q0, q1) & 0x77u;
+    byte |= (__float_as_uint(f[k]) >> 31) << 3;
+    byte |= (__float_as_uint(f[k + 1]) >> 31) << 7;
+    w[k >> 3] |= byte << ((k & 7) * 4);
+  }
+}
+
+// E2M1 code (magnitude in bits 0-2, sign in bit 3) -> its value, exactly.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const float v = (m < 2u) ? 0.5f * static_cast<float>(m)
+                           : __uint_as_float((((m >> 1) + 126u) << 23) | ((m & 1u) << 22));
+  return (c & 8u) ? -v : v;
+}
+
+// NVFP4 block with a scale search (outlier-aware keys): the E4M3 scale codes c0, c0 - 1,
+// c0 - 2, c0 + 1 (c0 the usual choice; codes outside 1..126 skipped) each encode the block, and
+// the one with the smallest squared error sum_i fl32(d_i^2), d_i = fl32(x_i - fl32(v_i den)),
+// accumulated in order with float32 adds, wins (ties to the earlier candidate).
+__device__ __forceinline__ uint32_t nvfp4_encode16_searched(const float* f, float s_t, uint32_t* w) {
+  float amax_b = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(f[k]));
+  const int c0 = static_cast<int>(cvt_e4m3x2(__fdiv_rn(__fdiv_rn(amax_b, 6.f), s_t), 0.f) & 0xFFu);
+  w[0] = w[1] = 0u;
+  if (c0 == 0) return 0u;
+  float best = INFINITY;
+  int best_c = c0;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int c = c0 + (t == 3 ? 1 : -t);
+    if (c < 1 || c > 126) continue;
+    const float den = __fmul_rn(e4m3_code_to_float(static_cast<uint32_t>(c)), s_t);
+    uint32_t wc[2];
+    e2m1_encode16(f, den, wc);
+    float err = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float d = __fsub_rn(f[i], __fmul_rn(e2m1_value((wc[i >> 3] >> (4 * (i & 7))) & 0xFu), den));
+      err = __fadd_rn(err, __fmul_rn(d, d));
+    }
+    if (err < best) {
+      best = err;
+      best_c = c;
+      w[0] = wc[0];
+      w[1] = wc[1];
     }
   }
-  return sc;
+  return static_cast<uint32_t>(best_c);
 }
 
 // ---------------------------------------------------------------------------------------
 // Pass 2: encode. One thread per 16-element block.
 // ---------------------------------------------------------------------------------------
-template <typename T, bool kWrite16>
+template <typename T, bool kWrite16, bool kSearch = false>
 __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
     const T* __restrict__ x, int64_t rows, int32_t cols, int64_t row_stride,
     const float* __restrict__ amax_partial, int32_t n_partial, float tensor_scale_in,
@@ -160,7 +205,7 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
     unpack8<T>(a, f);
     unpack8<T>(b, f + 8);
     uint32_t w[2];
-    const uint32_t sc = nvfp4_encode16(f, s_t, w);
+    const uint32_t sc = kSearch ? nvfp4_encode16_searched(f, s_t, w) : nvfp4_encode16(f, s_t, w);
     const int64_t blk = i;                        // outputs are dense: block i of row i / bpr
     *reinterpret_cast<uint2*>(codes + blk * 8) = make_uint2(w[0], w[1]);
     scales[blk] = static_cast<uint8_t>(sc);
@@ -180,14 +225,6 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
 // quantization: x ~ x_hat1 + x_hat2). Per element, in FP32 steps: den = fl32(s_b * s_t),
 // d = fl32(value(code) * den), r = fl32(x - d); then r is NVFP4-encoded with s_t.
 // ---------------------------------------------------------------------------------------
-// E2M1 code (magnitude in bits 0-2, sign in bit 3) -> its value, exactly.
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-  const uint32_t m = c & 7u;
-  const float v = (m < 2u) ? 0.5f * static_cast<float>(m)
-                           : __uint_as_float((((m >> 1) + 126u) << 23) | ((m & 1u) << 22));
-  return (c & 8u) ? -v : v;
-}
-
 template <typename T>
 __global__ void __launch_bounds__(256) nvfp4_residual_kernel(
     const T* __restrict__ x, int64_t rows, int32_t cols, int64_t row_stride,
@@ -216,6 +253,64 @@ __global__ void __launch_bounds__(256) nvfp4_residual_kernel(
     *reinterpret_cast<uint2*>(codes2 + i * 8) = make_uint2(w[0], w[1]);
     scales2[i] = static_cast<uint8_t>(sc);
   }
+}
+
+// ---------------------------------------------------------------------------------------
+// Smoothing and Hadamard rotation of 128-wide rows (outlier-aware key quantization): per
+// channel x * lam (queries, role 0) or x / lam (keys, role 1), then x H by seven butterfly
+// stages — stage s replaces the pair (i, i + 2^s) by (a + b, a - b) — then 2^-3 (queries) or
+// 2^-4 (keys), so that logits are unchanged, and one rounding to the 16-bit type. One warp per
+// row; lane l holds elements 4l .. 4l+3, so stages 0-1 stay in the lane and stages 2-6 pair
+// lanes l and l ^ 2^(s-2).
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ T from_float(float v);
+template <> __device__ __forceinline__ __half from_float<__half>(float v) { return __float2half_rn(v); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) smooth_rotate_kernel(const T* __restrict__ x, int64_t rows,
+                                                            const float* __restrict__ lam,
+                                                            int32_t role, T* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const T* src = x + row * 128 + lane * 4;
+  float v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = to_float<T>(src[k]);
+  if (lam != nullptr) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      v[k] = role == 0 ? __fmul_rn(v[k], lam[lane * 4 + k]) : __fdiv_rn(v[k], lam[lane * 4 + k]);
+  }
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {                        // pairs inside the lane
+    const int h = 1 << s;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i & h) continue;
+      const float a = v[i], b = v[i + h];
+      v[i] = __fadd_rn(a, b);
+      v[i + h] = __fsub_rn(a, b);
+    }
+  }
+#pragma unroll
+  for (int s = 2; s < 7; ++s) {                        // pairs across lanes
+    const int h = 1 << (s - 2);
+    const bool upper = (lane & h) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[i], h);
+      v[i] = upper ? __fsub_rn(p, v[i]) : __fadd_rn(v[i], p);
+    }
+  }
+  const float post = role == 0 ? 0.125f : 0.0625f;
+  T* dst = out + row * 128 + lane * 4;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) dst[k] = from_float<T>(__fmul_rn(v[k], post));
 }
 
 // ---------------------------------------------------------------------------------------

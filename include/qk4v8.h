@@ -108,6 +108,29 @@ qk4v8_status quantize_nvfp4(const void* x, qk4v8_dtype dtype, int64_t rows, int3
                             size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Outlier-aware key quantization (sns.style BitDecoding-FP4 summary, third algorithm item:
+ * static smoothing, Hadamard rotation and scale search against outlier key channels).
+ *
+ * qk_smooth_rotate — rows of 128 (x [rows, 128] fp16/bf16, 8-byte aligned) -> out, same shape
+ * and type: per channel x * lam[c] (role 0, queries) or x / lam[c] (role 1, keys; lam [128]
+ * float, a fixed calibration vector, or NULL for none), then x H with H the 128-point Sylvester
+ * Walsh-Hadamard matrix (seven float32 butterfly stages, stage s turning each pair
+ * (i, i + 2^s) into (a + b, a - b)), then 2^-3 (queries) or 2^-4 (keys), rounded once to the
+ * type. Since H H^T = 128 I, a query and a key treated this way have the same dot product.
+ *
+ * quantize_nvfp4_searched — quantize_nvfp4 with a per-block scale search: the E4M3 scale codes
+ * c0, c0 - 1, c0 - 2, c0 + 1 (c0 quantize_nvfp4's choice; codes outside 1..126 skipped) each
+ * encode the block and the one with the smallest squared error (float32, accumulated over the
+ * 16 elements in order) is kept, ties to the earlier candidate. Arguments as quantize_nvfp4.
+ */
+qk4v8_status qk_smooth_rotate(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t head_dim,
+                              const float* lam, int32_t role, void* out, cudaStream_t stream);
+qk4v8_status quantize_nvfp4_searched(const void* x, qk4v8_dtype dtype, int64_t rows, int32_t cols,
+                                     int64_t row_stride, float tensor_scale_in, uint8_t* codes,
+                                     uint8_t* scales, float* tensor_scale, void* x16,
+                                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * quantize_nvfp4_residual — the second tensor of dual-residual query quantization
  * (sns.style BitDecoding-FP4 summary, first algorithm item: the query as two FP4 tensors, the
  * second compensating the residual the first leaves). Given x and its NVFP4 encoding (codes,

@@ -183,3 +183,14 @@ def test_quantize_residual_validation(lib):
     assert f(cols=40) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(c2=FAKE + 4) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(dt=_lib.QK4V8_F32) == _lib.QK4V8_ERR_INVALID_ARG
+
+
+def test_smooth_rotate_validation(lib):
+    f = lambda x=FAKE, dt=_lib.QK4V8_BF16, rows=4, hd=128, lam=None, role=0, out=FAKE: \
+        lib.qk_smooth_rotate(x, dt, rows, hd, lam, role, out, None)
+    assert f(x=None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(role=2) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(hd=64) == _lib.QK4V8_ERR_UNSUPPORTED
+    assert f(out=FAKE + 4) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(dt=_lib.QK4V8_F32) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(rows=0) == _lib.QK4V8_OK                     # nothing to do, nothing launched
