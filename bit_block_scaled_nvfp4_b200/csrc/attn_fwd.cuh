@@ -47,10 +47,9 @@ namespace qk4v8 {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
-// Share of the exponentials taken on the FMA pipe, in eighths. 0: all on the special-function
-// unit, the fastest setting measured on B200 for this kernel's instruction mix (2/8 ran 2%
-// slower: the extra FMA-pipe instructions cost more issue slots than the exp unit saved).
-constexpr int kPolyOf8 = 0;
+// The exponentials all run on the special-function unit: moving a share to the FMA pipe
+// (exp2_poly2) measured slower on B200 for this kernel's instruction mix (2/8 of them: 2 to
+// 10 % slower) — the extra FMA-pipe instructions cost more issue slots than the unit saves.
 
 struct FwdArgs {
   const uint8_t* q_scales;
@@ -726,29 +725,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if ((f16 || prev_f16) && gg >= 1 &&
             !waitw(pv_done + (gg - 1) % L::NP, ((gg - 1) / L::NP) & 1, gg)) { ok = false; continue; }
         if (!f16) {
-          // kPolyOf8 of every 8 groups of 4 scores take the FMA-pipe exponential, the rest the
-          // special-function unit.
           unsigned char* prow = sP + pb * 16384 + row * 128;
           if constexpr (kUA)
             *reinterpret_cast<uint32_t*>(sm + L::OFF_PSFU + b2 * 512 + (row & 31) * 16 + (row >> 5) * 4) = psf_word;
+          // All 128 exponentials first (in place), then the E4M3 conversions and the stores: one
+          // long run of independent special-function instructions (measured 1 % faster than
+          // converting and storing chunk by chunk).
+#pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            const float2 Bc = kUA ? Bb[c >> 5] : B2;
+            const float2 t = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, Bc);
+            x[c] = ex2_approx(t.x);
+            x[c + 1] = ex2_approx(t.y);
+          }
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {               // 16 keys per 16-byte chunk
             uint32_t w4[4];
-            const float2 Bc = kUA ? Bb[ch >> 1] : B2;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int c = ch * 16 + q * 4;
-              const float2 t0 = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, Bc);
-              const float2 t1 = __ffma2_rn(make_float2(x[c + 2], x[c + 3]), C2, Bc);
-              float2 e0, e1;
-              if (((c >> 2) & 7) < kPolyOf8) {
-                e0 = exp2_poly2(t0);
-                e1 = exp2_poly2(t1);
-              } else {
-                e0 = make_float2(ex2_approx(t0.x), ex2_approx(t0.y));
-                e1 = make_float2(ex2_approx(t1.x), ex2_approx(t1.y));
-              }
-              w4[q] = cvt_e4m3x2(e0.x, e0.y) | (cvt_e4m3x2(e1.x, e1.y) << 16);
+              w4[q] = cvt_e4m3x2(x[c], x[c + 1]) | (cvt_e4m3x2(x[c + 2], x[c + 3]) << 16);
             }
             *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
