@@ -161,11 +161,11 @@ static qk4v8_status quantize_nvfp4_impl(const void* x, qk4v8_dtype dtype, int64_
     return QK4V8_ERR_INVALID_ARG;
   const int64_t blocks = rows * (cols / 16);
   const int grid = grid_for(blocks, 256);
-  // amax pass: two CTAs per SM (at most kAmaxPartials), each writing one partial maximum
+  // amax pass: four CTAs per SM (at most kAmaxPartials), each writing one partial maximum
   int64_t ag = (blocks + 255) / 256;
-  if (ag > 2 * kNumSMs) ag = 2 * kNumSMs;
+  if (ag > 4 * kNumSMs) ag = 4 * kNumSMs;
   const int agrid = static_cast<int>(ag < 1 ? 1 : ag);
-  static_assert(2 * kNumSMs <= kAmaxPartials, "amax partials");
+  static_assert(4 * kNumSMs <= kAmaxPartials, "amax partials");
   float* amax = static_cast<float*>(workspace);
   if (!(tensor_scale_in > 0.f)) {
     if (dtype == QK4V8_BF16)

@@ -40,7 +40,7 @@ __device__ __forceinline__ int64_t block_offset(int64_t i, uint32_t bpr, int64_t
 }
 
 // ---------------------------------------------------------------------------------------
-// Pass 1: tensor amax. A grid of a few CTAs per SM; CTA c writes the maximum of |x| over its
+// Pass 1: tensor amax. A grid of four CTAs per SM; CTA c writes the maximum of |x| over its
 // share to partial[c] (no atomics, nothing to clear), and the encode pass reduces the
 // partials. Four blocks of 16 per thread are loaded before any is reduced.
 // ---------------------------------------------------------------------------------------
