@@ -39,9 +39,9 @@ METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of H
 # decode_paged_decode_s64.md). Only workloads with
 # a capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
-    "prefill_h16_n4096": 18_165_760 + 1_024,
-    "prefill_gqa_n32768": 167_058_944 + 216_239_616,
-    "paged_decode_s64": 2_170_641_000 + 11_350_272,
+    "prefill_h16_n4096": 18_158_336 + 4_608,
+    "prefill_gqa_n32768": 158_131_456 + 218_139_648,
+    "paged_decode_s64": 2_170_382_000 + 13_552_384,
 }
 KERNEL_TIMING = "CUDA graph of the kernel(s) alone, replayed after a 256 MB L2 flush, CUDA events"
 FP4_OVER_BF16 = 4.0          # nominal dense ratio 9 PF / 2.25 PF
