@@ -194,3 +194,15 @@ def test_smooth_rotate_validation(lib):
     assert f(out=FAKE + 4) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(dt=_lib.QK4V8_F32) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(rows=0) == _lib.QK4V8_OK                     # nothing to do, nothing launched
+
+
+def test_product_path_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    """No CPU fallback: with the library absent every entry point raises instead of computing."""
+    import torch
+    from bit_block_scaled_nvfp4_b200 import api
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(_lib, "_LIB", None)
+    with pytest.raises(ImportError):
+        _lib.load()
+    with pytest.raises(ImportError):
+        api.quantize_nvfp4(torch.zeros(4, 16, dtype=torch.bfloat16))
