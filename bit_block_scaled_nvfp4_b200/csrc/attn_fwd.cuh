@@ -33,12 +33,18 @@
 //
 // Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
-//              tcgen05 scale layout with 4-byte asynchronous copies, FP16 tiles when selected
+//              tcgen05 scale layout with 4-byte asynchronous copies
 //   warp 1     TMEM owner and QK^T issuer (one thread)
 //   warp 2     PV issuer (one thread)
 //   warp 3     FP16 operand producer (FP16-tile kernel only)
 //   warps 4-11 softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
 // TMEM (512 columns): S_0, S_1 [0,256), O (D + 16 columns) from 256, scale factors from 400.
+//
+// Variants, each its own instance so the default one carries none of their work: kUA,
+// underflow-aware P scaling (sns.style BitDecoding-FP4 summary: each 32-key block of a row
+// encoded against its own power of two, applied back as the P operand's E8M0 block scale), and
+// kDQ, a second Q tensor (the same summary's dual-residual query quantization: its QK^T MMAs
+// accumulate into the same S).
 #pragma once
 #include "ptx.cuh"
 
