@@ -14,10 +14,15 @@
 // Partials (O unnormalised, m, l) go to the workspace; the merge kernel combines the splits:
 // M = max m_s, O = sum e^(m_s - M) O_s / sum e^(m_s - M) l_s.
 //
-// Warp roles (two or three CTAs per SM): warp 0 K producer (TMA of the two pages' K codes, K scale
-// factors by 4-byte asynchronous copies into the tcgen05 layout), warp 7 V producer (TMA of V
-// codes, bulk copy of the pages' V scales), warp 1 QK^T issuer, warp 6 PV issuer (and the V
-// scale rearrangement), warps 2-5 softmax. K and V stages form separate rings.
+// Warp roles (two or three CTAs per SM): warp 0 K producer (TMA of the two pages' K codes,
+// K scale factors by 4-byte asynchronous copies into the tcgen05 layout), warp 7 V producer
+// (TMA of V codes, bulk copy of the pages' V scales), warp 1 QK^T issuer, warp 6 PV issuer (and
+// the V scale rearrangement), warps 2-5 softmax. K and V stages form separate rings.
+//
+// Instances: GM (a bound on g: 4, 8 or 16 query columns reduced and exponentiated), kUA
+// (underflow-aware P scaling: each warp's 32 keys are one block of P^T, encoded against its own
+// power of two, which the PV MMA applies back as the block's E8M0 scale) and kDQ (a second Q
+// tensor from dual-residual query quantization, two more FP4 MMAs into S^T).
 #pragma once
 #include "ptx.cuh"
 #include "attn_fwd.cuh"
