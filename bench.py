@@ -486,6 +486,9 @@ def main():
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         run_reference(args, world, rank)
+        if world > 1:                   # no collective was used; release the group
+            import torch.distributed as dist
+            dist.destroy_process_group()
         return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device for --impl ours")
