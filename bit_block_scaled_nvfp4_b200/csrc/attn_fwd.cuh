@@ -666,10 +666,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free + b2);
-        if (f16) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c) x[c] *= R16;
-        }
         const int kbase = j * 128;
         if ((a.causal && kbase + 127 > qi) || (kbase + 128 > a.Nk)) {
           const int lim = min(a.Nk - 1, a.causal ? qi : a.Nk - 1) - kbase;   // last valid column
@@ -695,6 +691,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         }
+        // An FP16 tile's scores are true dot products: its max is brought into raw units here
+        // (exact: a positive factor commutes with the max) and its exponent takes the factor
+        // in its multiplier, so both kinds of tile share one exponential loop.
+        if (kMixed && f16) mt *= R16;
         // Running max before this tile: handed on by the group that processed tile gg - 1 of
         // the same item (the first tile of an item starts from -inf).
         float m_prev = -INFINITY;
@@ -730,20 +730,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (gg >= L::NP && !waitw(pv_done + pb, ((gg - L::NP) / L::NP) & 1, gg)) { ok = false; continue; }
         if ((f16 || prev_f16) && gg >= 1 &&
             !waitw(pv_done + (gg - 1) % L::NP, ((gg - 1) / L::NP) & 1, gg)) { ok = false; continue; }
+        // All 128 exponentials first (in place), then the conversions and the stores: one long
+        // run of independent special-function instructions (measured 1 % faster than converting
+        // and storing chunk by chunk).
+        const float Cs = (kMixed && f16) ? C * R16 : C;
+        const float2 Ct = make_float2(Cs, Cs);
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float2 Bc = kUA ? Bb[c >> 5] : B2;
+          const float2 t = __ffma2_rn(make_float2(x[c], x[c + 1]), Ct, Bc);
+          x[c] = ex2_approx(t.x);
+          x[c + 1] = ex2_approx(t.y);
+        }
         if (!f16) {
           unsigned char* prow = sP + pb * 16384 + row * 128;
           if constexpr (kUA)
             *reinterpret_cast<uint32_t*>(sm + L::OFF_PSFU + b2 * 512 + (row & 31) * 16 + (row >> 5) * 4) = psf_word;
-          // All 128 exponentials first (in place), then the E4M3 conversions and the stores: one
-          // long run of independent special-function instructions (measured 1 % faster than
-          // converting and storing chunk by chunk).
-#pragma unroll
-          for (int c = 0; c < 128; c += 2) {
-            const float2 Bc = kUA ? Bb[c >> 5] : B2;
-            const float2 t = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, Bc);
-            x[c] = ex2_approx(t.x);
-            x[c + 1] = ex2_approx(t.y);
-          }
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {               // 16 keys per 16-byte chunk
             uint32_t w4[4];
@@ -764,8 +766,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const int c = h * 64 + ch * 8 + q * 2;
-                const float2 t = __ffma2_rn(make_float2(x[c], x[c + 1]), C2, B2);
-                const __half2 hv = __floats2half2_rn(ex2_approx(t.x), ex2_approx(t.y));
+                const __half2 hv = __floats2half2_rn(x[c], x[c + 1]);
                 w4[q] = *reinterpret_cast<const uint32_t*>(&hv);
               }
               *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
