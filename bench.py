@@ -39,7 +39,7 @@ METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of H
 # attn_fwd_mixed_prefill_n16384.md, decode_paged_decode_s64.md). Only workloads with
 # a capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
-    "prefill_h16_n4096": 18_158_336 + 4_608,
+    "prefill_h16_n4096": 18_156_800 + 4_096,
     "prefill_gqa_n32768": 158_131_456 + 218_139_648,
     "mixed_prefill_n16384": 186_571_264 + 95_679_232,
     "paged_decode_s64": 2_170_382_000 + 13_552_384,
