@@ -626,8 +626,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* red_fin = red_m + 256;                                     // [2 items][128]
     // Scores stay in the FP4 MMA's raw units (S = sum codes*scales); the running max m is
     // kept in those units and 448 p = 2^(s C + (log2 448 - m C)) with
-    // C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true dot products and are
-    // brought into raw units by 1 / (s_tQ s_tK).
+    // C = s_tQ s_tK softmax_scale log2(e). FP16 tiles produce true dot products: their max is
+    // brought into raw units by R16 = 1 / (s_tQ s_tK) and their exponent multiplier is C R16.
     const float C = (*a.q_ts) * (*a.k_ts) * a.softmax_scale * kLog2e;
     const float R16 = 1.f / ((*a.q_ts) * (*a.k_ts));
     const float2 C2 = make_float2(C, C);
