@@ -32,6 +32,54 @@ def _dtype(t: torch.Tensor) -> int:
     return _DT[t.dtype]
 
 
+# The library derives every buffer's extent from the sizes it is given and takes plain device
+# pointers, so a host tensor, a strided view or a buffer of the wrong shape would be read (or
+# written) as if it had the dense layout those sizes imply. These checks run before any call.
+def _expect(t, name: str, shape, dtype) -> None:
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+
+
+def _expect_dims(t, name: str, ndim: int, layout: str) -> None:
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {layout}, got shape {tuple(t.shape)}")
+
+
+def _expect_scalar(t, name: str) -> None:
+    if t is None or t.numel() != 1 or t.dtype != torch.float32:
+        raise ValueError(f"{name} must be a one-element float32 tensor")
+
+
+def _on_one_gpu(*ts) -> None:
+    ts = [t for t in ts if t is not None]
+    dev = ts[0].get_device()
+    for t in ts:
+        if not t.is_cuda or t.get_device() != dev or not t.is_contiguous():
+            raise ValueError("the library takes contiguous tensors on one CUDA device")
+
+
+def _nvfp4_empty(shape, device, want_fp16: bool = False) -> NVFP4Tensor:
+    """Uninitialised NVFP4 output for an input of ``shape`` (..., D)."""
+    lead, cols = tuple(shape[:-1]), shape[-1]
+    return NVFP4Tensor(torch.empty(*lead, cols // 2, dtype=torch.uint8, device=device),
+                       torch.empty(*lead, cols // 16, dtype=torch.uint8, device=device),
+                       torch.empty(1, dtype=torch.float32, device=device),
+                       torch.empty(tuple(shape), dtype=torch.float16, device=device) if want_fp16 else None)
+
+
+def _mxfp8_empty(shape, device, want_fp16: bool = False) -> MXFP8V:
+    """Uninitialised MXFP8 output for V of ``shape`` (..., N, D): [..., D, N_pad128]."""
+    lead, n, d = tuple(shape[:-2]), shape[-2], shape[-1]
+    npad = (n + 127) // 128 * 128
+    return MXFP8V(torch.empty(*lead, d, npad, dtype=torch.uint8, device=device),
+                  torch.empty(*lead, d, npad // 32, dtype=torch.uint8, device=device), n,
+                  torch.empty(*lead, d, npad, dtype=torch.float16, device=device) if want_fp16 else None)
+
+
 @dataclass
 class NVFP4Tensor:
     """NVFP4 codes [..., D/2], E4M3 scales [..., D/16], FP32 tensor scale (1-element device
@@ -93,20 +141,19 @@ def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16
         raise ValueError("x must be a contiguous CUDA tensor")
     cols = x.shape[-1]
     rows = x.numel() // cols
-    dev = x.device
-    codes = torch.empty(*x.shape[:-1], cols // 2, dtype=torch.uint8, device=dev)
-    scales = torch.empty(*x.shape[:-1], cols // 16, dtype=torch.uint8, device=dev)
-    ts = torch.empty(1, dtype=torch.float32, device=dev)
-    x16 = torch.empty(x.shape, dtype=torch.float16, device=dev) if want_fp16 else None
+    r = _nvfp4_empty(x.shape, x.device, want_fp16)
+    need = lib.quantize_nvfp4_workspace_size()
     if workspace is None:
-        workspace = torch.empty(lib.quantize_nvfp4_workspace_size(), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    elif workspace.numel() < need or workspace.dtype != torch.uint8:
+        raise ValueError(f"workspace must hold {need} bytes (uint8)")
+    _on_one_gpu(x, workspace)
     fn = lib.quantize_nvfp4_searched if scale_search else lib.quantize_nvfp4
     st = fn(_ptr(x), _dtype(x), rows, cols, cols,
-                            float(tensor_scale) if tensor_scale else 0.0, _ptr(codes),
-                            _ptr(scales), _ptr(ts), _ptr(x16), _ptr(workspace),
-                            workspace.numel(), _stream())
+            float(tensor_scale) if tensor_scale else 0.0, _ptr(r.codes), _ptr(r.scales),
+            _ptr(r.tensor_scale), _ptr(r.fp16), _ptr(workspace), workspace.numel(), _stream())
     _lib.check(st, "quantize_nvfp4")
-    return NVFP4Tensor(codes, scales, ts, x16)
+    return r
 
 
 def qk_smooth_rotate(x: torch.Tensor, role: str, lam: torch.Tensor | None = None) -> torch.Tensor:
@@ -115,8 +162,9 @@ def qk_smooth_rotate(x: torch.Tensor, role: str, lam: torch.Tensor | None = None
     so that transformed queries and keys keep their dot products. Returns a new tensor."""
     if not x.is_cuda or not x.is_contiguous() or x.shape[-1] != 128:
         raise ValueError("x must be a contiguous CUDA tensor with last dimension 128")
-    if lam is not None and (not lam.is_cuda or lam.dtype != torch.float32 or lam.numel() != 128):
-        raise ValueError("lam must be 128 float32 values on the GPU")
+    if lam is not None and (lam.dtype != torch.float32 or lam.numel() != 128):
+        raise ValueError("lam must be 128 float32 values")
+    _on_one_gpu(x, lam)
     out = torch.empty_like(x)
     st = _lib.load().qk_smooth_rotate(_ptr(x), _dtype(x), x.numel() // 128, 128, _ptr(lam),
                                       0 if role == "q" else 1, _ptr(out), _stream())
@@ -127,7 +175,7 @@ def qk_smooth_rotate(x: torch.Tensor, role: str, lam: torch.Tensor | None = None
 def quantize_nvfp4_dual(x: torch.Tensor, tensor_scale: float | None = None):
     """Dual-residual NVFP4: (Q1, Q2) with Q1 = quantize_nvfp4(x) and Q2 the encoding of
     x - Q1's values under Q1's tensor scale (shared tensor-scale tensor)."""
-    q1 = quantize_nvfp4(x, tensor_scale)
+    q1 = quantize_nvfp4(x, tensor_scale)             # checks x
     cols = x.shape[-1]
     codes2, scales2 = torch.empty_like(q1.codes), torch.empty_like(q1.scales)
     st = _lib.load().quantize_nvfp4_residual(_ptr(x), _dtype(x), x.numel() // cols, cols, cols,
@@ -145,25 +193,28 @@ def quantize_mxfp8_v(v: torch.Tensor, want_fp16: bool = False) -> MXFP8V:
         raise ValueError("v must be a contiguous CUDA tensor")
     n, d = v.shape[-2], v.shape[-1]
     bh = v.numel() // (n * d)
-    npad = (n + 127) // 128 * 128
-    lead = v.shape[:-2]
-    codes = torch.empty(*lead, d, npad, dtype=torch.uint8, device=v.device)
-    scales = torch.empty(*lead, d, npad // 32, dtype=torch.uint8, device=v.device)
-    v16 = torch.empty(*lead, d, npad, dtype=torch.float16, device=v.device) if want_fp16 else None
-    st = lib.quantize_mxfp8_v(_ptr(v), _dtype(v), bh, n, d, _ptr(codes), _ptr(scales),
-                              _ptr(v16), _stream())
+    r = _mxfp8_empty(v.shape, v.device, want_fp16)
+    st = lib.quantize_mxfp8_v(_ptr(v), _dtype(v), bh, n, d, _ptr(r.codes), _ptr(r.scales),
+                              _ptr(r.fp16), _stream())
     _lib.check(st, "quantize_mxfp8_v")
-    return MXFP8V(codes, scales, n, v16)
+    return r
 
 
 def tile_score_select(q: NVFP4Tensor, k: NVFP4Tensor, causal: bool, frac_bp: int,
                       k_max: int | None = None):
     """Top-fraction tile selection. q.codes [B, Hq, N, D/2], k.codes [B, Hkv, N, D/2].
     Returns (idx [B*Hq, k_max] rank-ordered, n_sel [B*Hq], bitmap [B*Hq, T, T])."""
-    lib = _lib.load()
+    _expect_dims(q.codes, "q.codes", 4, "[B, Hq, N, D/2]")
+    _expect_dims(k.codes, "k.codes", 4, "[B, Hkv, N, D/2]")
     B, Hq, N, dh = q.codes.shape
     Hkv = k.codes.shape[1]
     d = dh * 2
+    _expect(q.codes, "q.codes", (B, Hq, N, d // 2), torch.uint8)
+    _expect(q.scales, "q.scales", (B, Hq, N, d // 16), torch.uint8)
+    _expect(k.codes, "k.codes", (B, Hkv, N, d // 2), torch.uint8)
+    _expect(k.scales, "k.scales", (B, Hkv, N, d // 16), torch.uint8)
+    _on_one_gpu(q.codes, q.scales, k.codes, k.scales)
+    lib = _lib.load()
     T = (N + 127) // 128
     n_cand = T * (T + 1) // 2 if causal else T * T
     need = (n_cand * frac_bp + 9999) // 10000
@@ -189,10 +240,37 @@ def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
     """QK4V8 attention forward. q.codes [B, Hq, Nq, D/2], k.codes [B, Hkv, Nk, D/2],
     v.codes [B, Hkv, D, Nk_pad]. With ``fp16_bitmap`` the FP16 copies (q.fp16, k.fp16,
     v.fp16) must be present. Returns out [B, Hq, Nq, D] (and lse [B, Hq, Nq])."""
-    lib = _lib.load()
+    _expect_dims(q.codes, "q.codes", 4, "[B, Hq, Nq, D/2]")
+    _expect_dims(k.codes, "k.codes", 4, "[B, Hkv, Nk, D/2]")
     B, Hq, Nq, dh = q.codes.shape
     Hkv, Nk = k.codes.shape[1], k.codes.shape[2]
     d = dh * 2
+    npad = (Nk + 127) // 128 * 128
+    _expect(q.codes, "q.codes", (B, Hq, Nq, d // 2), torch.uint8)
+    _expect(q.scales, "q.scales", (B, Hq, Nq, d // 16), torch.uint8)
+    _expect_scalar(q.tensor_scale, "q.tensor_scale")
+    _expect(k.codes, "k.codes", (B, Hkv, Nk, d // 2), torch.uint8)
+    _expect(k.scales, "k.scales", (B, Hkv, Nk, d // 16), torch.uint8)
+    _expect_scalar(k.tensor_scale, "k.tensor_scale")
+    _expect(v.codes, "v.codes", (B, Hkv, d, npad), torch.uint8)
+    _expect(v.scales, "v.scales", (B, Hkv, d, npad // 32), torch.uint8)
+    bufs = [q.codes, q.scales, q.tensor_scale, k.codes, k.scales, k.tensor_scale, v.codes, v.scales]
+    if fp16_bitmap is not None:
+        if q2 is not None:
+            raise ValueError("the second Q tensor is not combined with FP16 tiles")
+        tiles = B * Hq * ((Nq + 127) // 128) * ((Nk + 127) // 128)
+        if fp16_bitmap.dtype != torch.uint8 or fp16_bitmap.numel() != tiles:
+            raise ValueError(f"fp16_bitmap must hold {tiles} uint8 tile flags")
+        _expect(q.fp16, "q.fp16 (quantize with want_fp16=True)", (B, Hq, Nq, d), torch.float16)
+        _expect(k.fp16, "k.fp16 (quantize with want_fp16=True)", (B, Hkv, Nk, d), torch.float16)
+        _expect(v.fp16, "v.fp16 (quantize with want_fp16=True)", (B, Hkv, d, npad), torch.float16)
+        bufs += [fp16_bitmap, q.fp16, k.fp16, v.fp16]
+    if q2 is not None:
+        _expect(q2.codes, "q2.codes", (B, Hq, Nq, d // 2), torch.uint8)
+        _expect(q2.scales, "q2.scales", (B, Hq, Nq, d // 16), torch.uint8)
+        bufs += [q2.codes, q2.scales]
+    _on_one_gpu(*bufs)
+    lib = _lib.load()
     out = torch.empty(B, Hq, Nq, d, dtype=out_dtype, device=q.codes.device)
     lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.codes.device) if want_lse else None
     p = _lib.FwdParams()
@@ -229,9 +307,33 @@ def decode_params(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,
                   context_lens: torch.Tensor, max_context: int, split_tokens: int,
                   out: torch.Tensor, softmax_scale: float | None = None, lse=None,
                   underflow_aware: bool = False, q2: NVFP4Tensor | None = None):
+    """The decode parameter struct, after checking every buffer against the sizes it states."""
+    _expect_dims(q.codes, "q.codes", 3, "[S, Hq, D/2]")
+    _expect_dims(cache.k_pages, "cache.k_pages", 4, "[P, Hkv, 64, D/2]")
+    _expect_dims(page_table, "page_table", 2, "[S, max_pages]")
     S, Hq, dh = q.codes.shape
     P, Hkv = cache.k_pages.shape[0], cache.k_pages.shape[1]
     d = dh * 2
+    _expect(q.scales, "q.scales", (S, Hq, d // 16), torch.uint8)
+    _expect_scalar(q.tensor_scale, "q.tensor_scale")
+    _expect(cache.k_pages, "cache.k_pages", (P, Hkv, 64, d // 2), torch.uint8)
+    _expect(cache.k_scales, "cache.k_scales", (P, Hkv, 64, d // 16), torch.uint8)
+    _expect_scalar(cache.k_tensor_scale, "cache.k_tensor_scale")
+    _expect(cache.v_pages, "cache.v_pages", (P, Hkv, d, 64), torch.uint8)
+    _expect(cache.v_scales, "cache.v_scales", (P, Hkv, d, 2), torch.uint8)
+    _expect(page_table, "page_table", (S, page_table.shape[1]), torch.int32)
+    _expect(context_lens, "context_lens", (S,), torch.int32)
+    _expect(out, "out", (S, Hq, d), out.dtype)
+    bufs = [q.codes, q.scales, q.tensor_scale, cache.k_pages, cache.k_scales, cache.k_tensor_scale,
+            cache.v_pages, cache.v_scales, page_table, context_lens, out]
+    if lse is not None:
+        _expect(lse, "lse", (S, Hq), torch.float32)
+        bufs.append(lse)
+    if q2 is not None:
+        _expect(q2.codes, "q2.codes", (S, Hq, d // 2), torch.uint8)
+        _expect(q2.scales, "q2.scales", (S, Hq, d // 16), torch.uint8)
+        bufs += [q2.codes, q2.scales]
+    _on_one_gpu(*bufs)
     p = _lib.DecodeParams()
     p.q_codes, p.q_scales, p.q_tensor_scale = q.codes.data_ptr(), q.scales.data_ptr(), q.tensor_scale.data_ptr()
     p.k_pages, p.k_page_scales, p.k_tensor_scale = (cache.k_pages.data_ptr(), cache.k_scales.data_ptr(),
@@ -258,15 +360,19 @@ def attn_qk4v8_decode_paged(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Te
                             underflow_aware: bool = False, q2: NVFP4Tensor | None = None):
     """One decode step. q.codes [S, Hq, D/2]; returns out [S, Hq, D] (and lse [S, Hq]).
     ``underflow_aware`` scales P per 32-key block by a power of two before its E4M3 encode."""
-    lib = _lib.load()
     S, Hq, dh = q.codes.shape
     out = torch.empty(S, Hq, dh * 2, dtype=out_dtype, device=q.codes.device)
     lse = torch.empty(S, Hq, dtype=torch.float32, device=q.codes.device) if want_lse else None
     p = decode_params(q, cache, page_table, context_lens, max_context, split_tokens, out,
                       softmax_scale, lse, underflow_aware, q2)
+    lib = _lib.load()
     need = lib.attn_qk4v8_decode_workspace_size(C.byref(p))
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.codes.device)
+    elif workspace.dtype != torch.uint8:
+        raise TypeError("workspace must be a uint8 tensor")
+    else:
+        _on_one_gpu(q.codes, workspace)
     st = lib.attn_qk4v8_decode_paged(C.byref(p), _ptr(workspace), workspace.numel(), _stream())
     _lib.check(st, "attn_qk4v8_decode_paged")
     return (out, lse) if want_lse else out
@@ -280,12 +386,12 @@ def attn_qk4v8_decode_paged_noalloc(q: NVFP4Tensor, cache: PagedKV, page_table: 
     the split partials in its own fixed 16 MiB device buffer instead of a caller workspace,
     for callers that cannot provide device memory. Only the output (and lse) are allocated
     here, as for every other entry point of this binding."""
-    lib = _lib.load()
     S, Hq, dh = q.codes.shape
     out = torch.empty(S, Hq, dh * 2, dtype=out_dtype, device=q.codes.device)
     lse = torch.empty(S, Hq, dtype=torch.float32, device=q.codes.device) if want_lse else None
     p = decode_params(q, cache, page_table, context_lens, max_context, split_tokens, out,
                       softmax_scale, lse)
+    lib = _lib.load()
     st = lib.attn_qk4v8_decode_paged_noalloc(C.byref(p), _stream())
     _lib.check(st, "attn_qk4v8_decode_paged_noalloc")
     return (out, lse) if want_lse else out
@@ -298,13 +404,26 @@ def kv_append_paged(cache: PagedKV, k_new: torch.Tensor, v_new: torch.Tensor,
     (fp16/bf16); cu_new [S + 1] int32 offsets of each sequence's new rows; lens [S] int32
     lengths before the call (the caller adds the new counts); page_table [S, max_pages];
     v_tail [S, Hkv, D, 32] of k_new's dtype, each sequence's incomplete V group, updated."""
-    lib = _lib.load()
-    for t in (k_new, v_new, cu_new, lens, page_table, v_tail):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("kv_append_paged needs contiguous CUDA tensors")
+    _expect_dims(k_new, "k_new", 3, "[total_new, Hkv, D]")
+    _expect_dims(cache.k_pages, "cache.k_pages", 4, "[P, Hkv, 64, D/2]")
+    _expect_dims(page_table, "page_table", 2, "[S, max_pages]")
     if v_new.dtype != k_new.dtype or v_tail.dtype != k_new.dtype:
         raise ValueError("k_new, v_new and v_tail must share a dtype")
     _, hkv, d = k_new.shape
+    S, P = lens.numel(), cache.k_pages.shape[0]
+    _expect(v_new, "v_new", tuple(k_new.shape), k_new.dtype)
+    _expect(cu_new, "cu_new", (S + 1,), torch.int32)
+    _expect(lens, "lens", (S,), torch.int32)
+    _expect(page_table, "page_table", (S, page_table.shape[1]), torch.int32)
+    _expect(v_tail, "v_tail", (S, hkv, d, 32), k_new.dtype)
+    _expect(cache.k_pages, "cache.k_pages", (P, hkv, 64, d // 2), torch.uint8)
+    _expect(cache.k_scales, "cache.k_scales", (P, hkv, 64, d // 16), torch.uint8)
+    _expect_scalar(cache.k_tensor_scale, "cache.k_tensor_scale")
+    _expect(cache.v_pages, "cache.v_pages", (P, hkv, d, 64), torch.uint8)
+    _expect(cache.v_scales, "cache.v_scales", (P, hkv, d, 2), torch.uint8)
+    _on_one_gpu(k_new, v_new, cu_new, lens, page_table, v_tail, cache.k_pages, cache.k_scales,
+                cache.k_tensor_scale, cache.v_pages, cache.v_scales)
+    lib = _lib.load()
     p = _lib.AppendParams(
         k_new=_ptr(k_new), v_new=_ptr(v_new), dtype=_dtype(k_new), cu_new=_ptr(cu_new),
         lens=_ptr(lens), page_table=_ptr(page_table), k_pages=_ptr(cache.k_pages),

@@ -43,7 +43,7 @@ def _rank(rank, world, port, out):
 
 def test_dist_setup_and_max_over_ranks_gloo():
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:      # no fork of a threaded process
         out = m.dict()
         mp.spawn(_rank, args=(2, port, out), nprocs=2, join=True)
         assert dict(out) == {0: 2.5, 1: 2.5}
