@@ -196,14 +196,23 @@ def make_prefill_step(name):
 
     prep = {}
 
-    def attn_only():
-        # the attention kernel alone, on inputs quantized (and scored) once beforehand
+    def prepared():
+        # inputs quantized (and scored) once, outside the graphs that time single kernels
         if not prep:
             prep["in"] = quant()
             prep["bm"] = (api.tile_score_select(prep["in"][0], prep["in"][1], cfg["causal"],
                                                 cfg["frac_bp"])[2] if mixed else None)
-        q4, k4, v8 = prep["in"]
+        return prep
+
+    def attn_only():
+        # the attention kernel alone
+        q4, k4, v8 = prepared()["in"]
         return api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=prep["bm"])
+
+    def score_only():
+        # tile scoring and top-fraction selection alone
+        q4, k4, _ = prepared()["in"]
+        return api.tile_score_select(q4, k4, cfg["causal"], cfg["frac_bp"])
 
     launches = 6 + (3 if mixed else 0)
     host = [w.q.pin_memory(), w.k.pin_memory(), w.v.pin_memory()]
@@ -211,8 +220,11 @@ def make_prefill_step(name):
     # codes + E8M0 scales (V) written, plus the fp16 copies the FP16 tiles read
     nq, nk, nv = q.numel(), k.numel(), v.numel()
     qbytes = (nq + nk) * (2 + 0.5 + 1 / 16) + nv * (2 + 1 + 1 / 32) + (2 * (nq + nk + nv) if mixed else 0)
+    # algorithmic scoring bytes: the Q and K codes and E4M3 scales read once
+    sbytes = (nq + nk) * (0.5 + 1 / 16)
     return dict(cfg=cfg, step=step, inputs=(q, k, v), host=host, launches=launches,
                 flops=prefill_flops(cfg), kind="prefill", quant=quant, quant_bytes=qbytes,
+                score=(score_only, sbytes) if mixed else None,
                 attn_only=attn_only)
 
 
@@ -570,6 +582,14 @@ def main():
                        "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
         line["append"] = {"kernel": "kv_append_kernel", "timing": KERNEL_TIMING,
                           "peak_gbs": pk["hbm_gbs"], **app}
+    if st.get("score") is not None:
+        # tile scoring and selection of the FP16-tile workload, against the HBM peak
+        fn, nbytes = st["score"]
+        ms = max_over_ranks(time_graph(fn, max(3, args.steps // 3)), world)
+        line["score"] = {"kernel": "row_norm_tile_max_kernel + tile_select_kernel",
+                         "timing": KERNEL_TIMING, "ms": ms, "bytes": nbytes,
+                         "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
+                         "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
     if rank == 0 and not args.no_cpu_baseline:
         dt, u, desc = oracle_sample(name, rows=64 if st["kind"] == "prefill" else 64, heads=1)
         cv = u / dt / (1e12 if st["kind"] == "prefill" else 1e9)
