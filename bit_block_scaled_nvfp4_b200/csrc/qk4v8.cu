@@ -488,6 +488,8 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
   if (workspace_bytes < attn_qk4v8_decode_workspace_size(p)) return QK4V8_ERR_INVALID_ARG;
   const int32_t n_splits = decode_splits(p);
   if (n_splits > 65535 || p->num_seqs > 65535 || p->kv_heads > 65535) return QK4V8_ERR_UNSUPPORTED;
+  // the page maps' rows (page, KV head, channel) are addressed by 32-bit TMA coordinates
+  if (static_cast<int64_t>(p->num_pages) * p->kv_heads * 128 > 0x7fffffffLL) return QK4V8_ERR_UNSUPPORTED;
   constexpr int D = 128;
   CUtensorMap tq, tq2, tkp, tvp;
   {

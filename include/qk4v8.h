@@ -255,7 +255,9 @@ typedef struct {
   const uint8_t* v_page_scales;/* [num_pages, Hkv, D, 2] */
   const int32_t* page_table;   /* [S, max_pages] physical page of each logical page */
   const int32_t* context_lens; /* [S], 1 <= len <= min(max_context, 64 * max_pages) */
-  int32_t num_seqs, num_pages, max_pages, q_heads, kv_heads, head_dim; /* head_dim 128 */
+  int32_t num_seqs, num_pages, max_pages, q_heads, kv_heads, head_dim; /* head_dim 128;
+                                  num_pages * kv_heads * head_dim < 2^31 (32-bit tensor-map
+                                  row coordinates), else QK4V8_ERR_UNSUPPORTED */
   int32_t max_context;         /* host-side bound on context_lens (sizes grid and workspace) */
   int32_t split_tokens;        /* keys per split, a positive multiple of 128, at most 16384 */
   float softmax_scale;

@@ -144,6 +144,8 @@ def test_decode_validation_and_workspace(lib):
     assert f(_dec(q_heads=64, kv_heads=2)) == _lib.QK4V8_ERR_UNSUPPORTED  # g = 32 > 16
     assert f(_dec(), wsb=16) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(_dec(page_table=None)) == _lib.QK4V8_ERR_INVALID_ARG
+    # page rows beyond 32-bit tensor-map coordinates: refused before any map is built
+    assert f(_dec(num_pages=(1 << 31) // (8 * 128))) == _lib.QK4V8_ERR_UNSUPPORTED
 
 
 def _app(**kw):
