@@ -444,6 +444,8 @@ def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: b
     ``fp16_frac_bp`` basis points of them in FP16, then attention. ``dual_q`` adds the
     residual second Q tensor; ``underflow_aware`` scales P per 32-key block."""
     mixed = fp16_frac_bp > 0
+    if mixed and dual_q:
+        raise ValueError("dual_q is not combined with FP16 tiles")
     q2 = None
     if dual_q:
         q4, q2 = quantize_nvfp4_dual(q)

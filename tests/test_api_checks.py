@@ -151,3 +151,9 @@ def test_append_refuses_mismatched_buffers():
     with pytest.raises(ValueError, match="cache.k_pages"):
         api.kv_append_paged(paged.empty_cache(40, 3, 64, 0.0625, "cpu"), k, v, cu, lens, table,
                             tail, max_new=1)
+
+
+def test_dual_q_with_fp16_tiles_is_refused_before_any_work():
+    x = torch.zeros(1, 2, 128, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="dual_q"):
+        api.qk4v8_attention(x, x, x, True, fp16_frac_bp=500, dual_q=True)
