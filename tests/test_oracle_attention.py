@@ -46,6 +46,25 @@ def test_hand_worked_examples():
     assert np.allclose(o[0, :3], want, rtol=0, atol=1e-15)
 
 
+def test_hand_worked_fp16_tile_examples():
+    g = keyed("attention_examples.txt")
+    d = 64
+    q = np.zeros((1, d)); q[0, 0] = 8.0
+    # example C: example A's single tile in FP16 (operands exact in fp16)
+    k = np.zeros((2, d)); k[1, 0] = -1.0
+    v = np.zeros((2, d)); v[0, 0] = 1.0; v[1, 1] = 1.0
+    every = lambda qt, t: np.ones(qt.shape, dtype=bool)
+    o, _ = A.attention_head(q, k, v, False, 1 / 8, fp16_select=every, q16=q, k16=k, v16=v)
+    assert np.allclose(o[0, :3], [float(t) for t in g["C"]], rtol=0, atol=1e-15)
+    # example D: tile 0 in E4M3, tile 1 in FP16 with a rise of the running max
+    k = np.zeros((130, d)); k[1:128, 0] = -100.0; k[128, 0] = 2.0; k[129, 0] = 1.0
+    v = np.zeros((130, d)); v[:, 2] = 1.0
+    v[0] = 0; v[0, 0] = 1.0; v[128] = 0; v[128, 1] = 1.0; v[129] = 0; v[129, 3] = 1.0
+    second = lambda qt, t: np.full(qt.shape, t == 1)
+    o, _ = A.attention_head(q, k, v, False, 1 / 8, fp16_select=second, q16=q, k16=k, v16=v)
+    assert np.allclose(o[0, :4], [float(t) for t in g["D"]], rtol=0, atol=1e-15)
+
+
 @pytest.mark.parametrize("c", [1.0, 0.375, -2.5])
 def test_constant_v_gives_constant_output(c):
     q, k, _ = _rand(4, 200, 200, 64, scale_k=3.0)
