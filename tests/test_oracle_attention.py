@@ -46,6 +46,19 @@ def test_hand_worked_examples():
     assert np.allclose(o[0, :3], want, rtol=0, atol=1e-15)
 
 
+def test_hand_worked_underflow_aware_example():
+    g = keyed("attention_examples.txt")
+    d = 64
+    q = np.zeros((1, d)); q[0, 0] = 8.0
+    k = np.zeros((64, d)); k[:, 0] = -100.0; k[0, 0] = 0.0; k[32, 0] = -12.0
+    v = np.zeros((64, d)); v[:, 2] = 1.0
+    v[0] = 0; v[0, 0] = 1.0; v[32] = 0; v[32, 1] = 1.0
+    o, _ = A.attention_head(q, k, v, False, 1 / 8, p_underflow_aware=True)
+    assert np.allclose(o[0, :3], [float(t) for t in g["E"]], rtol=0, atol=1e-15)
+    o_fixed, _ = A.attention_head(q, k, v, False, 1 / 8)
+    assert abs(o_fixed[0, 1] - float(g["E"][1])) > 1e-6       # the fixed encoding differs
+
+
 def test_hand_worked_fp16_tile_examples():
     g = keyed("attention_examples.txt")
     d = 64
