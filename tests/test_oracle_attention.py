@@ -59,6 +59,19 @@ def test_hand_worked_underflow_aware_example():
     assert abs(o_fixed[0, 1] - float(g["E"][1])) > 1e-6       # the fixed encoding differs
 
 
+def test_hand_worked_split_decode_examples():
+    g = keyed("attention_examples.txt")
+    d = 64
+    q = np.zeros((1, d)); q[0, 0] = 8.0
+    k = np.zeros((256, d)); k[:, 0] = -100.0; k[0, 0] = 2.0; k[128, 0] = 0.0; k[129, 0] = -1.0
+    v = np.zeros((256, d)); v[:, 2] = 1.0
+    for j, c in ((0, 0), (128, 1), (129, 3)):
+        v[j] = 0; v[j, c] = 1.0
+    for key, split in (("F", 128), ("G", 256)):
+        o, _ = A.decode_rows(q, k, v, 256, 1 / 8, split)
+        assert np.allclose(o[0, :4], [float(t) for t in g[key]], rtol=0, atol=1e-15), key
+
+
 def test_hand_worked_fp16_tile_examples():
     g = keyed("attention_examples.txt")
     d = 64
