@@ -590,8 +590,8 @@ def main():
                          "timing": KERNEL_TIMING, "ms": ms, "bytes": nbytes,
                          "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                          "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
-    if rank == 0 and not args.no_cpu_baseline:
-        dt, u, desc = oracle_sample(name, rows=64 if st["kind"] == "prefill" else 64, heads=1)
+    if world == 1 and not args.no_cpu_baseline:          # the oracle is timed at N = 1 only
+        dt, u, desc = oracle_sample(name, rows=64, heads=1)
         cv = u / dt / (1e12 if st["kind"] == "prefill" else 1e9)
         line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
                                 "sample": desc, "seconds": dt}
