@@ -521,11 +521,16 @@ def main():
             step_ms, kern_ms = time_steps(st, args.steps, args.warmup, world)
         e2e_ms, h2d, d2h = time_e2e(st, max(3, args.steps // 3), world)
         status = api.check_status()
-        if status == 0:
+        # every rank takes the same decision, so that all of them run the same collectives
+        agreed = max_over_ranks(float(status), world)
+        if agreed == 0:
             break
-        print(f"bench: device status {status}, first timed-out wait {api.timeout_site()}"
-              f" (attempt {attempt + 1})", file=sys.stderr)
-    if status != 0:
+        print(f"bench: device status {status} (worst over ranks {agreed:g}), first timed-out"
+              f" wait {api.timeout_site()} (attempt {attempt + 1})", file=sys.stderr)
+    if agreed != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
         raise SystemExit(3)
     step_ms = max_over_ranks(step_ms, world)
     kern_ms = max_over_ranks(kern_ms, world)
