@@ -535,6 +535,7 @@ def main():
     step_ms = max_over_ranks(step_ms, world)
     kern_ms = max_over_ranks(kern_ms, world)
     e2e_ms = max_over_ranks(e2e_ms, world)
+    st["quant_ms"] = max_over_ranks(st["quant_ms"], world)
     pk, src = peaks()
     cfg = st["cfg"]
     if st["kind"] == "prefill":
