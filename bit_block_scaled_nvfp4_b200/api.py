@@ -134,8 +134,13 @@ def selftest_wait_timeout() -> None:
 
 def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16: bool = False,
                    workspace: torch.Tensor | None = None, scale_search: bool = False) -> NVFP4Tensor:
-    """NVFP4-quantize ``x`` (..., D) along its last axis (contiguous fp16/bf16 CUDA tensor);
-    ``scale_search`` picks each block's scale among four candidates by squared error."""
+    """NVFP4-quantize ``x`` (..., D) along its last axis (contiguous fp16/bf16 CUDA tensor).
+
+    ``tensor_scale``: a fixed FP32 tensor scale (a paged cache's, for instance); None or a
+    value <= 0 computes it from the tensor's amax (amax / (6 * 448)). ``want_fp16`` also
+    writes an fp16 copy of ``x`` for the FP16-tile attention path. ``workspace``: optional
+    uint8 scratch of ``quantize_nvfp4_workspace_size()`` bytes. ``scale_search`` picks each
+    block's scale among four candidates by squared error."""
     lib = _lib.load()
     if not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA tensor")
