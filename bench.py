@@ -1,10 +1,14 @@
 #!/usr/bin/env python
 """Benchmark of the QK4V8 hot path on B200; prints ONE JSON line (rank 0).
 
-Default workload: causal prefill, batch 1, 16 heads, 4096 tokens, head_dim 128, bf16 inputs.
-A step = quantize Q and K (NVFP4), quantize V (MXFP8), QK4V8 attention forward. Other
-workloads (--workload): prefill_gqa_n32768, mixed_prefill_n16384 (tile scoring + FP16 tiles
-in the step), paged_decode_s64 (one decode step: quantize the step's Q, paged split-K decode).
+Default: both halves of the metric in one line. The headline workload is the long-context
+causal prefill with GQA (batch 1, 32 query / 8 KV heads, 32768 tokens, head_dim 128, bf16
+inputs); a step = quantize Q and K (NVFP4), quantize V (MXFP8), QK4V8 attention forward. The
+``decode`` object of the same line measures the paged decode workload (64 sequences of
+8192-32768 tokens, 32 / 8 heads, 64-token pages): a step = quantize the step's Q, paged
+split-K decode, split merge; with it, the quantize-on-append kernel. Other workloads
+(--workload): prefill_h16_n4096, mixed_prefill_n16384 (tile scoring + FP16 tiles in the
+step), paged_decode_s64 alone.
 
 Timing: inputs resident in HBM; W warm-up steps; then K steps, each bracketed by CUDA events
 on the launching stream, with a 256 MB L2 flush between steps (outside the events); barrier +
@@ -34,10 +38,9 @@ from bit_block_scaled_nvfp4_b200 import workloads  # noqa: E402
 
 METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of HBM peak"
 
-# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu capture summarised
-# in profiles/ (attn_fwd_prefill_h16_n4096.md, attn_fwd_prefill_gqa_n32768.md,
-# attn_fwd_mixed_prefill_n16384.md, decode_paged_decode_s64.md). Only workloads with
-# a capture of the current kernel have an entry; the others report null.
+# DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture of that
+# kernel on the workload (dram__bytes_read.sum + dram__bytes_write.sum). Only workloads with a
+# capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
     "prefill_h16_n4096": 18_156_800 + 4_096,
     "prefill_gqa_n32768": 158_131_456 + 218_139_648,
@@ -402,6 +405,18 @@ def time_e2e(st, K, world):
 # ---------------------------------------------------------------------------------------
 # CPU oracle (the reference arm and the cpu_baseline leg)
 # ---------------------------------------------------------------------------------------
+_INPUTS = {}
+
+
+def _inputs(name):
+    """The workload's seeded inputs (CPU), drawn once per process: drawing them is set-up, not
+    part of a timed oracle sample."""
+    if name not in _INPUTS:
+        _INPUTS[name] = (workloads.make_decode_layout(name) if name == "paged_decode_s64"
+                         else workloads.make_prefill(name))
+    return _INPUTS[name]
+
+
 def oracle_sample(name, rows=256, heads=1):
     """Time the oracle, as it stands, on a bounded sample of the workload: ``heads`` query
     heads x ``rows`` query rows spread over the sequence (prefill; the whole-tensor scales
@@ -411,7 +426,7 @@ def oracle_sample(name, rows=256, heads=1):
     from oracle import quant as OQ
     from oracle import paged as OP
     if name == "paged_decode_s64":
-        lay = workloads.make_decode_layout(name)
+        lay = _inputs(name)
         cfg = lay.cfg
         q = workloads.make_decode_query(lay).float().numpy()
         t0 = time.perf_counter()
@@ -431,7 +446,7 @@ def oracle_sample(name, rows=256, heads=1):
         per_tok = cfg["d"] // 2 + cfg["d"] // 16 + cfg["d"] + cfg["d"] // 32
         units = ((n + 63) // 64) * 64 * cfg["Hkv"] * per_tok
         return dt, float(units), f"1 sequence ({n} tokens) x {cfg['Hkv']} KV heads of one decode step"
-    w = workloads.make_prefill(name)
+    w = _inputs(name)
     cfg = w.cfg
     N, d = cfg["N"], cfg["d"]
     rng = np.random.default_rng(0)
@@ -463,6 +478,11 @@ def cpu_cores():
         return os.cpu_count()
 
 
+def config_of(name):
+    """The workload as both arms name it: its name and its sizes."""
+    return {"workload": name, **dict(workloads.WORKLOADS[name])}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -479,40 +499,18 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": name, **{k: v_ for k, v_ in workloads.WORKLOADS[name].items()}},
+            "config": config_of(name),
             "cpu_baseline": {"value": v, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="prefill_h16_n4096",
-                    choices=[n for n in workloads.WORKLOADS if n != "tiny_prefill"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-    world, rank, local = dist_setup(args)
-    if args.impl == "reference":
-        run_reference(args, world, rank)
-        if world > 1:                   # no collective was used; release the group
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+def measure(name, args, world):
+    """Time one workload: the step, its dominant kernel alone, its quantize kernels alone and the
+    step end to end from host buffers (all max over ranks). Returns the pieces of a line, or
+    None when a device wait timed out twice."""
     from bit_block_scaled_nvfp4_b200 import api
-    name = args.workload
-    try:
-        apps = subprocess.run(["nvidia-smi", "--query-compute-apps=pid,process_name,used_memory",
-                               "--format=csv,noheader"], capture_output=True, text=True, timeout=20).stdout
-        print(f"bench: compute apps on the GPUs before the run: {apps.strip() or 'none'}", file=sys.stderr)
-    except (OSError, subprocess.TimeoutExpired):
-        pass
     st = make_decode_step(name) if name == "paged_decode_s64" else make_prefill_step(name)
     # A run in which a device wait timed out (status != 0) produced no valid result: report
     # where, take the measurement once more, and give up without a number if it repeats.
@@ -525,19 +523,15 @@ def main():
         agreed = max_over_ranks(float(status), world)
         if agreed == 0:
             break
-        print(f"bench: device status {status} (worst over ranks {agreed:g}), first timed-out"
-              f" wait {api.timeout_site()} (attempt {attempt + 1})", file=sys.stderr)
+        print(f"bench: {name}: device status {status} (worst over ranks {agreed:g}), first "
+              f"timed-out wait {api.timeout_site()} (attempt {attempt + 1})", file=sys.stderr)
     if agreed != 0:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        raise SystemExit(3)
+        return None
     step_ms = max_over_ranks(step_ms, world)
     kern_ms = max_over_ranks(kern_ms, world)
     e2e_ms = max_over_ranks(e2e_ms, world)
-    st["quant_ms"] = max_over_ranks(st["quant_ms"], world)
+    quant_ms = max_over_ranks(st["quant_ms"], world)
     pk, src = peaks()
-    cfg = st["cfg"]
     if st["kind"] == "prefill":
         units = st["flops"]
         value = units * world / (step_ms * 1e-3) / 1e12
@@ -547,7 +541,8 @@ def main():
         peak = pk["bf16_tflops"] * FP4_OVER_BF16
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": NCU_TRAFFIC_BYTES.get(name),
-                "kernel": "attn_fwd_kernel", "timing": KERNEL_TIMING, "peak_source": f"{src} bf16 x {FP4_OVER_BF16:g} (FP4 dense)",
+                "kernel": "attn_fwd_kernel", "kernel_ms": kern_ms, "timing": KERNEL_TIMING,
+                "peak_source": f"{src} bf16 x {FP4_OVER_BF16:g} (FP4 dense)",
                 "mixed_fp4_fp8_bound_tflops": peak / 1.5}
     else:
         units = st["bytes"]
@@ -558,49 +553,97 @@ def main():
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "traffic": NCU_TRAFFIC_BYTES.get(name), "traffic_kernel": "decode_kernel",
-                "kernel": "decode_kernel + decode_merge_kernel", "timing": KERNEL_TIMING,
-                "peak_source": f"{src} hbm_gbs"}
-    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4/mxfp8 (fp32 accumulate)",
-            "data": "synthetic",
-            "config": {"workload": name, **{k: v_ for k, v_ in workloads.WORKLOADS[name].items()},
-                       "l2": "256 MB flush between timed steps",
-                       "step": "one CUDA graph replay (all kernels of the step)", "parallelism": f"replicas x{world}"},
-            "roofline": roof,
-            "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": st["launches"] * args.steps,
-            # the quantize kernels of the step, timed as a graph of their own after an L2 flush
-            # (algorithmic bytes: the amax pass's second read of each input is not counted)
-            "quantize": {"achieved_gbs": st["quant_bytes"] / (st["quant_ms"] * 1e-3) / 1e9,
-                         "peak_gbs": pk["hbm_gbs"],
-                         "frac": st["quant_bytes"] / (st["quant_ms"] * 1e-3) / 1e9 / pk["hbm_gbs"],
-                         "ms": st["quant_ms"], "bytes": st["quant_bytes"]},
-            "device_status": status,
-            "clocks": clk.summary()}
+                "kernel": "decode_kernel + decode_merge_kernel", "kernel_ms": kern_ms,
+                "timing": KERNEL_TIMING, "peak_source": f"{src} hbm_gbs"}
+    out = {"value": value, "unit": unit, "ms_per_step": step_ms, "config": config_of(name),
+           "roofline": roof,
+           "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "gpu_launches": st["launches"] * args.steps,
+           # the quantize kernels of the step, timed as a graph of their own after an L2 flush
+           # (algorithmic bytes: the amax pass's second read of each input is not counted)
+           "quantize": {"achieved_gbs": st["quant_bytes"] / (quant_ms * 1e-3) / 1e9,
+                        "peak_gbs": pk["hbm_gbs"],
+                        "frac": st["quant_bytes"] / (quant_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                        "ms": quant_ms, "bytes": st["quant_bytes"]},
+           "device_status": status, "clocks": clk.summary()}
     if st["kind"] == "decode":
         # the producer side of the decode path: quantize-on-append into the paged cache
         app = {}
-        for nm, (fn, nbytes, ntok) in make_append(cfg).items():
+        for nm, (fn, nbytes, ntok) in make_append(st["cfg"]).items():
             ms = max_over_ranks(time_graph(fn, max(3, args.steps // 3)), world)
             app[nm] = {"ms": ms, "tokens": ntok, "bytes": nbytes,
                        "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
                        "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
-        line["append"] = {"kernel": "kv_append_kernel", "timing": KERNEL_TIMING,
-                          "peak_gbs": pk["hbm_gbs"], **app}
+        out["append"] = {"kernel": "kv_append_kernel", "timing": KERNEL_TIMING,
+                         "peak_gbs": pk["hbm_gbs"], **app}
     if st.get("score") is not None:
         # tile scoring and selection of the FP16-tile workload, against the HBM peak
         fn, nbytes = st["score"]
         ms = max_over_ranks(time_graph(fn, max(3, args.steps // 3)), world)
-        line["score"] = {"kernel": "row_norm_tile_max_kernel + tile_select_kernel",
-                         "timing": KERNEL_TIMING, "ms": ms, "bytes": nbytes,
-                         "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
-                         "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+        out["score"] = {"kernel": "row_norm_tile_max_kernel + tile_select_kernel",
+                        "timing": KERNEL_TIMING, "ms": ms, "bytes": nbytes,
+                        "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
+                        "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
     if world == 1 and not args.no_cpu_baseline:          # the oracle is timed at N = 1 only
         dt, u, desc = oracle_sample(name, rows=64, heads=1)
         cv = u / dt / (1e12 if st["kind"] == "prefill" else 1e9)
-        line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
-                                "sample": desc, "seconds": dt}
+        out["cpu_baseline"] = {"value": cv, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
+                               "sample": desc, "seconds": dt}
+    del st
+    torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill_gqa_n32768",
+                    choices=[n for n in workloads.WORKLOADS if n != "tiny_prefill"])
+    ap.add_argument("--no-decode", action="store_true",
+                    help="leave out the decode object (paged_decode_s64) of a prefill line")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:                   # no collective was used; release the group
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    name = args.workload
+    try:
+        apps = subprocess.run(["nvidia-smi", "--query-compute-apps=pid,process_name,used_memory",
+                               "--format=csv,noheader"], capture_output=True, text=True, timeout=20).stdout
+        print(f"bench: compute apps on the GPUs before the run: {apps.strip() or 'none'}", file=sys.stderr)
+    except (OSError, subprocess.TimeoutExpired):
+        pass
+    head = measure(name, args, world)
+    dec = None
+    if head is not None and name != "paged_decode_s64" and not args.no_decode:
+        dec = measure("paged_decode_s64", args, world)
+    if head is None or (dec is None and name != "paged_decode_s64" and not args.no_decode):
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        raise SystemExit(3)
+    line = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4/mxfp8 (fp32 accumulate)", "data": "synthetic",
+            "config": head["config"],
+            "parallelism": f"replicas x{world}",
+            "timing": {"l2": "256 MB flush between timed steps",
+                       "step": "one CUDA graph replay (all kernels of the step)"},
+            **{k: v for k, v in head.items() if k not in ("value", "unit", "ms_per_step", "config")}}
+    if dec is not None:
+        # the other half of the metric: decode KV GB/s against the HBM peak, timed the same way
+        line["decode"] = dec
+        line["gpu_launches"] += dec["gpu_launches"]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

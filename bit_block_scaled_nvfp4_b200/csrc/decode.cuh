@@ -564,11 +564,14 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float* __restri
     Lsum += w * p[i * (D + 2) + D + 1];
     acc += w * p[i * (D + 2) + threadIdx.x];
   }
-  const float v = acc / Lsum;
+  // A row with no key (its context length failed the bounds check, so every split is empty)
+  // gets O = 0 and lse = -inf rather than 0/0; the status word reports the error.
+  const bool empty = !(Lsum > 0.f);
+  const float v = empty ? 0.f : acc / Lsum;
   if (out_kind == 2) static_cast<float*>(out)[row * D + threadIdx.x] = v;
   else if (out_kind == 1) static_cast<__nv_bfloat16*>(out)[row * D + threadIdx.x] = __float2bfloat16_rn(v);
   else static_cast<__half*>(out)[row * D + threadIdx.x] = __float2half_rn(v);
-  if (lse != nullptr && threadIdx.x == 0) lse[row] = M * kLn2 + logf(Lsum * (1.f / 448.f));
+  if (lse != nullptr && threadIdx.x == 0) lse[row] = empty ? -INFINITY : M * kLn2 + logf(Lsum * (1.f / 448.f));
 }
 
 }  // namespace qk4v8

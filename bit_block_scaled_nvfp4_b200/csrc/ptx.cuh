@@ -387,7 +387,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // 2^t for a pair on the FMA pipe, so that part of the softmax's exponentials leave the
 // special-function unit (its throughput bounds the prefill kernel): 2^t = 2^n p(t - n) with
 // n = round(t) (by the 1.5 * 2^23 rounding constant) and p a degree-5 polynomial for 2^f on
-// [-1/2, 1/2] fitted for relative error (fit_exp2.py: 1.5e-7 with fp32 coefficients). The
+// [-1/2, 1/2] fitted for relative error (a Lawson-weighted least-squares fit made for this kernel: 1.5e-7 with fp32 coefficients). The
 // scale 2^n is added to the exponent field. t is clamped below at -30 (2^-30 is below every
 // E4M3 and FP16 code this feeds); t must not exceed 127.
 __device__ __forceinline__ float2 exp2_poly2(float2 t) {

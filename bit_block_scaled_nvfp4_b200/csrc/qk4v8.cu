@@ -77,6 +77,33 @@ bool set_smem(K kernel, int bytes) {
          cudaSuccess;
 }
 
+// A set-up step that must run once per device: CUDA keeps a kernel's shared-memory opt-in
+// (cudaFuncAttributeMaxDynamicSharedMemorySize) per device context, so a process that drives
+// several GPUs opts each kernel in on each of them. Thread-safe; a failed step is retried on
+// the next call. Devices beyond kMaxDevices run the step on every call.
+constexpr int kMaxDevices = 64;
+class PerDeviceOnce {
+ public:
+  template <typename F>
+  bool run(int dev, F&& step) {
+    if (dev < 0 || dev >= kMaxDevices) return step();
+    std::lock_guard<std::mutex> lock(mu_);
+    if (done_[dev]) return true;
+    if (!step()) return false;
+    done_[dev] = true;
+    return true;
+  }
+
+ private:
+  std::mutex mu_;
+  bool done_[kMaxDevices] = {};
+};
+
+int current_device() {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -129,6 +156,14 @@ qk4v8_status qk4v8_selftest_exp2(const float* t, float* out, int32_t n, cudaStre
   if (n == 0) return QK4V8_OK;
   exp2_selftest_kernel<<<(n / 2 + 255) / 256, 256, 0, stream>>>(t, out, n);
   return launch_status();
+}
+
+int32_t qk4v8_selftest_device_once(int32_t dev) {
+  static PerDeviceOnce latch;
+  static int32_t runs[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return -1;
+  latch.run(dev, [dev] { ++runs[dev]; return true; });
+  return runs[dev];
 }
 
 qk4v8_status qk4v8_selftest_wait_timeout(cudaStream_t stream) {
@@ -328,11 +363,11 @@ qk4v8_status tile_score_select(const uint8_t* q_codes, const uint8_t* q_scales,
   }
   if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
   const int smem = (2 * T + 2) * 8 + kSelectMax * (16 + 4);
-  static bool attr = false;
-  if (!attr) {
-    if (!set_smem(tile_select_kernel, (2 * 4096 + 2) * 8 + kSelectMax * 20)) return QK4V8_ERR_CUDA;
-    attr = true;
-  }
+  static PerDeviceOnce opt_in;
+  if (!opt_in.run(current_device(), [] {
+        return set_smem(tile_select_kernel, (2 * 4096 + 2) * 8 + kSelectMax * 20);
+      }))
+    return QK4V8_ERR_CUDA;
   tile_select_kernel<<<batch * q_heads, kSelectThreads, smem, stream>>>(
       qmax, kmax, q_heads, kv_heads, T, T, causal, frac_bp, k_max, idx, n_sel, bitmap);
   return launch_status();
@@ -383,11 +418,9 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   } else {
     tq16 = tq; tk16 = tk; tv16 = tv;
   }
-  static bool attr = false;
-  if (!attr) {
-    if (!set_smem(attn_fwd_kernel<D, kMixed, kUA, kDQ>, L::SMEM_ALLOC)) return QK4V8_ERR_CUDA;
-    attr = true;
-  }
+  static PerDeviceOnce opt_in;                  // one per kernel instance
+  if (!opt_in.run(current_device(), [] { return set_smem(attn_fwd_kernel<D, kMixed, kUA, kDQ>, L::SMEM_ALLOC); }))
+    return QK4V8_ERR_CUDA;
   FwdArgs a;
   a.q_scales = p->q_scales; a.k_scales = p->k_scales; a.v_scales = p->v_scales;
   a.q2_scales = dual ? p->q2_scales : nullptr;
@@ -509,23 +542,22 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
     const uint32_t bv[2] = {64, D};
     if (!make_map(&tvp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->v_pages, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_64B)) return QK4V8_ERR_CUDA;
   }
-  static bool attr = false;
-  if (!attr) {
-    if (!set_smem(decode_kernel<4, false>, DecLayout<4>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<8, false>, DecLayout<8>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<16, false>, DecLayout<16>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<4, true>, DecLayout<4>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<8, true>, DecLayout<8>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<16, true>, DecLayout<16>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<4, false, true>, DecLayout<4, true>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<8, false, true>, DecLayout<8, true>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<16, false, true>, DecLayout<16, true>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<4, true, true>, DecLayout<4, true>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<8, true, true>, DecLayout<8, true>::SMEM_ALLOC) ||
-        !set_smem(decode_kernel<16, true, true>, DecLayout<16, true>::SMEM_ALLOC))
-      return QK4V8_ERR_CUDA;
-    attr = true;
-  }
+  static PerDeviceOnce opt_in;
+  if (!opt_in.run(current_device(), [] {
+        return set_smem(decode_kernel<4, false>, DecLayout<4>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<8, false>, DecLayout<8>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<16, false>, DecLayout<16>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<4, true>, DecLayout<4>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<8, true>, DecLayout<8>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<16, true>, DecLayout<16>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<4, false, true>, DecLayout<4, true>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<8, false, true>, DecLayout<8, true>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<16, false, true>, DecLayout<16, true>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<4, true, true>, DecLayout<4, true>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<8, true, true>, DecLayout<8, true>::SMEM_ALLOC) &&
+               set_smem(decode_kernel<16, true, true>, DecLayout<16, true>::SMEM_ALLOC);
+      }))
+    return QK4V8_ERR_CUDA;
   DecArgs a;
   a.q_scales = p->q_scales; a.q2_scales = p->q2_scales; a.q_ts = p->q_tensor_scale;
   a.k_page_scales = p->k_page_scales; a.k_ts = p->k_tensor_scale;
@@ -565,7 +597,6 @@ qk4v8_status attn_qk4v8_decode_paged(const qk4v8_decode_params* p, void* workspa
 static __device__ __align__(256) unsigned char g_noalloc_decode_scratch[QK4V8_NOALLOC_DECODE_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 }  // namespace

@@ -70,6 +70,16 @@ qk4v8_status qk4v8_check_status(cudaStream_t stream);
 uint64_t qk4v8_timeout_site(void);
 
 /*
+ * Host-side self-test (no GPU needed) of the once-per-device latch that guards each kernel's
+ * one-time set-up, its opt-in to more than 48 KB of dynamic shared memory, which CUDA keeps
+ * per device: a process driving several GPUs opts every kernel in on each device it uses.
+ * Runs a counting set-up step through a test instance of that latch for device `dev` and
+ * returns how many times the step has run for `dev` so far (1 after any number of calls), or
+ * -1 when dev is outside [0, 64).
+ */
+int32_t qk4v8_selftest_device_once(int32_t dev);
+
+/*
  * Failure-path self-test: launches one warp that waits on a barrier nothing arrives at. Its
  * bounded wait gives up after about a second and the kernel returns; the following
  * qk4v8_check_status() reports QK4V8_ERR_TIMEOUT and qk4v8_timeout_site() names kernel 3.
@@ -254,7 +264,10 @@ typedef struct {
   const uint8_t* v_pages;      /* [num_pages, Hkv, D, 64] */
   const uint8_t* v_page_scales;/* [num_pages, Hkv, D, 2] */
   const int32_t* page_table;   /* [S, max_pages] physical page of each logical page */
-  const int32_t* context_lens; /* [S], 1 <= len <= min(max_context, 64 * max_pages) */
+  const int32_t* context_lens; /* [S], 1 <= len <= min(max_context, 64 * max_pages); a
+                                  length outside that range sets QK4V8_ERR_BOUNDS (reported by
+                                  qk4v8_check_status) and that sequence's rows get O = 0 and
+                                  lse = -inf */
   int32_t num_seqs, num_pages, max_pages, q_heads, kv_heads, head_dim; /* head_dim 128;
                                   num_pages * kv_heads * head_dim < 2^31 (32-bit tensor-map
                                   row coordinates), else QK4V8_ERR_UNSUPPORTED */

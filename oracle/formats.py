@@ -158,7 +158,7 @@ def e8m0_decode(codes: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------------------
-# IEEE half precision (used only by the FP16 tile path)
+# IEEE half precision (the FP16 tile path; fp16 outputs) and bfloat16 (bf16 outputs)
 # ---------------------------------------------------------------------------------------
 
 def fp16_round(x: np.ndarray) -> np.ndarray:
@@ -167,3 +167,22 @@ def fp16_round(x: np.ndarray) -> np.ndarray:
     numpy's float64 -> float16 cast rounds once, to nearest even.
     """
     return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to bfloat16 (8-bit significand, float32's exponent range) once,
+    to nearest with ties to even, returned as float64. An attention output requested in bf16
+    is the float64 result rounded this way (a single rounding: no float32 step in between).
+
+    Each finite value is split as m 2^e with m in [0.5, 1); m 2^8 is then an exact float64 and
+    np.rint rounds it to the nearest integer, ties to even. Below bfloat16's smallest normal
+    (2^-126) the step is the subnormal quantum 2^-133; beyond the largest finite value
+    (2^128 (1 - 2^-8)) the result is infinite, as IEEE rounding to nearest gives.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    step_exp = np.maximum(e - 8, -133)                       # exponent of one unit in the last place
+    out = np.rint(np.ldexp(x, -step_exp)) * np.ldexp(1.0, step_exp)
+    big = np.abs(out) >= 2.0 ** 128
+    out = np.where(big, np.copysign(np.inf, x), out)
+    return np.where(np.isfinite(x), out, x)

@@ -1,8 +1,8 @@
 """Oracle — NVFP4 and MXFP8 quantizers (TEST INFRASTRUCTURE ONLY; see oracle/formats.py).
 
 NVFP4 (Q and K). Structure from the tqpw.cn "块缩放数值格式" article §2.2: E2M1 elements,
-one E4M3 scale per 16 consecutive elements, one FP32 scale per tensor ("分级缩放体系 …
-张量级全局FP32缩放系数, 紧凑块设计16元素/块"). The article's own listing has the wrong
+one E4M3 scale per 16 consecutive elements, one FP32 scale per tensor (the article describes
+a two-level scaling: a tensor-wide FP32 factor above small 16-element blocks). The article's own listing has the wrong
 arithmetic (raw amax as global scale, no division by 6, an integer grid); the reading used
 here is the plainest one that keeps every block scale representable in E4M3:
 
@@ -18,8 +18,8 @@ All FP32 steps are single IEEE operations rounded to nearest (numpy float32 arit
 subnormals are kept. A caller-supplied tensor scale replaces s_t (used for a KV cache whose
 scale is fixed in advance). Packing: element 2i in the low nibble, 2i+1 in the high nibble.
 
-MXFP8 (V). The tqpw.cn article §2.1 and the zdszero primer ("mxfp8: e8m0 scale, block quant
-1x32") fix E4M3 elements with one E8M0 scale per 32 elements. The shared-exponent rule is not
+MXFP8 (V). The tqpw.cn article §2.1 and the zdszero primer (MXFP8 section: an E8M0 scale for
+each 1x32 block) fix E4M3 elements with one E8M0 scale per 32 elements. The shared-exponent rule is not
 on the pages; the OCP MX rule is used: e = floor(log2 amax) - 8 (8 is the exponent of E4M3's
 largest normal, 448 = 1.75 * 2^8), clamped to [-127, 127]; scale code e + 127; elements
 E4M3(v / 2^e); an all-zero group gets scale code 127 and zero codes. Groups run along the

@@ -32,16 +32,47 @@ def assert_attention_close(out_gpu, out_oracle, what=""):
     return mx, mean
 
 
-def assert_rounded_output_close(out_gpu, out_oracle, dtype, what=""):
-    """Parity of a 16-bit output: the bar above plus half a unit in the last place of the
-    output format at each element (the output's own rounding)."""
+def oracle_output(out_oracle, dtype):
+    """The oracle's O as the method defines a 16-bit output: the float64 O / l rounded once to
+    the output dtype (fp32 outputs are compared with the float64 values)."""
+    if dtype == torch.bfloat16:
+        return OF.bf16_round(out_oracle)
+    if dtype == torch.float16:
+        return OF.fp16_round(out_oracle)
+    return out_oracle
+
+
+def round_to_output(x, dtype):
+    """float values rounded once to a 16-bit output dtype (float64 in, float64 out)."""
+    return OF.bf16_round(x) if dtype == torch.bfloat16 else OF.fp16_round(x)
+
+
+def assert_rounded_output_close(out16, out32, out_oracle, dtype, what=""):
+    """Parity of a 16-bit output, with no allowance added to the bar:
+
+    * the 16-bit output is the same kernel's fp32 output rounded once to that dtype, bit for
+      bit (the fp32 output itself is held to the plain bar by the caller);
+    * against the oracle's O rounded once to that dtype, the mean error is within the plain
+      bar, and every element over the plain max bar is exactly one unit in the last place of
+      the output format away (the two unrounded values straddle a rounding boundary; one bf16
+      unit at |O| > 2.56 rms is already more than 2e-2 rms, so no kernel could meet the max bar
+      there), on at most one element in 10^4.
+    """
+    ref16 = round_to_output(out_oracle, dtype)
+    assert np.array_equal(out16, round_to_output(out32.astype(np.float64), dtype)), \
+        f"{what}: the 16-bit output is not the fp32 output rounded once"
     rms = float(np.sqrt(np.mean(out_oracle.astype(np.float64) ** 2)))
-    mant = {torch.bfloat16: 8, torch.float16: 11}[dtype]
-    half_ulp = np.ldexp(1.0, np.frexp(np.abs(out_oracle))[1] - mant - 1)
-    d = np.abs(out_gpu.astype(np.float64) - out_oracle)
-    assert np.all(np.isfinite(out_gpu)), what
-    assert np.all(d <= MAX_TOL * rms + half_ulp), f"{what}: worst excess {np.max(d - half_ulp) / rms:.3e}"
-    assert d.mean() <= MEAN_TOL * rms + half_ulp.mean(), what
+    d = np.abs(out16.astype(np.float64) - ref16)
+    assert np.all(np.isfinite(out16)), what
+    assert d.mean() <= MEAN_TOL * rms, f"{what}: mean {d.mean() / rms:.3e} (x rms)"
+    over = d > MAX_TOL * rms
+    if over.any():
+        mant = {torch.bfloat16: 8, torch.float16: 11}[dtype]
+        mag = np.maximum(np.abs(out16[over]).astype(np.float64), np.abs(ref16[over]))
+        ulp = np.ldexp(1.0, np.frexp(mag)[1] - mant)           # one unit at the larger one
+        lower = np.ldexp(1.0, np.frexp(np.minimum(np.abs(out16[over]), np.abs(ref16[over])))[1] - mant)
+        assert np.all((d[over] == ulp) | (d[over] == lower)), f"{what}: an element off by more than one unit"
+        assert over.sum() <= max(1, d.size // 10000), f"{what}: {over.sum()} elements one unit apart"
 
 
 def oracle_tensor_scale(x: torch.Tensor) -> np.float32:

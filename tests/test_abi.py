@@ -55,6 +55,17 @@ def test_version_and_status_strings(lib):
 FAKE = 1 << 20          # aligned fake device addresses: never dereferenced on these paths
 
 
+def test_per_device_set_up_runs_once_per_device(lib):
+    """The latch behind each kernel's shared-memory opt-in keeps one flag per device: the set-up
+    step runs once for device 0 however often it is asked, and once more, on its own, for each
+    other device; an out-of-range index is refused."""
+    f = lib.qk4v8_selftest_device_once
+    assert f(0) == 1 and f(0) == 1
+    assert f(3) == 1 and f(3) == 1 and f(0) == 1
+    assert f(63) == 1
+    assert f(64) == -1 and f(-1) == -1
+
+
 def test_quantize_nvfp4_validation(lib):
     f = lib.quantize_nvfp4
     ok = dict(x=FAKE, dt=1, rows=4, cols=64, stride=64, ts=0.0, codes=FAKE, scales=FAKE,

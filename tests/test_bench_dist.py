@@ -61,3 +61,7 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    sys.path.insert(0, ROOT)
+    import bench
+    # the config both arms print is the workload's name and sizes, nothing else
+    assert d["config"] == bench.config_of("prefill_gqa_n32768")

@@ -59,7 +59,7 @@ def test_workload_full_parity(name):
     assert_attention_close(f32(out), ref, name)
     out16 = _run(w.q, w.k, w.v, w.cfg["causal"], scale, out_dtype=w.q.dtype)
     assert out16.dtype == w.q.dtype
-    assert_rounded_output_close(f32(out16), ref, w.q.dtype, name + " 16-bit output")
+    assert_rounded_output_close(f32(out16), f32(out), ref, w.q.dtype, name + " 16-bit output")
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,D,causal", [
@@ -124,14 +124,16 @@ def test_lse_matches_oracle():
 
 
 def test_bf16_output_workload_long_rows():
-    """bf16 output of the 32k GQA workload stays within the bar plus its own rounding."""
+    """A bf16 output (2000 causal rows, g = 2) matches the oracle's O rounded once to bf16."""
     g = torch.Generator().manual_seed(4)
     q = torch.randn(1, 2, 2000, 128, generator=g).to(torch.bfloat16)
     k = (torch.randn(1, 1, 2000, 128, generator=g) * 2).to(torch.bfloat16)
     v = torch.randn(1, 1, 2000, 128, generator=g).to(torch.bfloat16)
     out = _run(q, k, v, True, out_dtype=torch.bfloat16)
+    out32 = _run(q, k, v, True, out_dtype=torch.float32)
     ref = _full_oracle(q, k, v, True, 1 / math.sqrt(128))
-    assert_rounded_output_close(f32(out), ref, torch.bfloat16, "bf16 output")
+    assert_attention_close(f32(out32), ref, "fp32 output")
+    assert_rounded_output_close(f32(out), f32(out32), ref, torch.bfloat16, "bf16 output")
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,D,causal", [

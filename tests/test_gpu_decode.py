@@ -115,9 +115,12 @@ def test_bad_page_id_reports_bounds_error():
     assert api.check_status() == 0                          # cleared
 
 
-def test_paged_workload_sampled_sequences():
-    """64 sequences, lengths U[8192, 32768], 32/8 heads, shuffled pages; oracle on the
-    shortest, the longest and two seeded sequences (all heads)."""
+@pytest.fixture(scope="module")
+def paged_workload():
+    """The 64-sequence workload (lengths U[8192, 32768], 32/8 heads, shuffled pages) decoded
+    once at the benchmark's split of 4096 tokens, fp32 output; the oracle on the shortest, the
+    longest and two seeded sequences (all heads) with that split, in one pass (split 0), and
+    exact attention on the same quantized operands."""
     lay = workloads.make_decode_layout()
     cfg = lay.cfg
     cache = paged.empty_cache(lay.num_pages, cfg["Hkv"], cfg["d"], KTS, DEV)
@@ -135,21 +138,54 @@ def test_paged_workload_sampled_sequences():
     split = 4096
     out = api.attn_qk4v8_decode_paged(q4, cache, lay.page_table.to(DEV), lay.lens.to(DEV),
                                       max(lens), split, out_dtype=torch.float32)
+    assert api.check_status() == 0
     sq = oracle_tensor_scale(q)
     qc, qs, qt = OQ.nvfp4_quantize(f32(q), tensor_scale=sq)
     qh = OQ.nvfp4_dequantize(qc, qs, qt)
     g = cfg["Hq"] // cfg["Hkv"]
-    got, want = [], []
+    r = {"gpu": [], "split": [], "one_pass": [], "exact": []}
     for s, (k, v) in sorted(seqs.items()):
         kc, ks, vc, vs = OP.quantize_sequence(f32(k), f32(v), KTS)
         kh = OQ.nvfp4_dequantize(kc, ks, np.float32(KTS))
         vh = OQ.mxfp8_dequantize_v(vc, vs, lens[s])
         for h in range(cfg["Hkv"]):
-            o, _ = OA.decode_rows(qh[s, h * g:(h + 1) * g], kh[h], vh[h], lens[s],
-                                  1 / math.sqrt(128), split)
-            want.append(o)
-            got.append(f32(out[s, h * g:(h + 1) * g]))
-    assert_attention_close(np.concatenate(got), np.concatenate(want), "paged decode workload")
+            qq = qh[s, h * g:(h + 1) * g]
+            r["split"].append(OA.decode_rows(qq, kh[h], vh[h], lens[s], 1 / math.sqrt(128), split)[0])
+            r["one_pass"].append(OA.decode_rows(qq, kh[h], vh[h], lens[s], 1 / math.sqrt(128), 0)[0])
+            r["exact"].append(OA.exact_attention(qq, kh[h, :lens[s]], vh[h, :lens[s]], False,
+                                                 1 / math.sqrt(128)))
+            r["gpu"].append(f32(out[s, h * g:(h + 1) * g]))
+    return {k_: np.concatenate(v_) for k_, v_ in r.items()}
+
+
+def test_paged_workload_sampled_sequences(paged_workload):
+    """Parity with the oracle's split-K decode at the kernel's split (4096 tokens)."""
+    r = paged_workload
+    assert_attention_close(r["gpu"], r["split"], "paged decode workload")
+
+
+@pytest.mark.xfail(strict=True, reason="split-K reading: each 4096-token split encodes P against "
+                   "its own running max, which moves O by E4M3-rounding-level noise (oracle vs "
+                   "oracle: 9.3e-2 max, 6.5e-3 mean x rms) -- above the bar against the one-pass method")
+def test_split_decode_against_one_pass_method(paged_workload):
+    """The benchmark's split-K decode against the sequential one-pass method at the parity
+    bar. It does not meet it, by the reading of split-K decode, not by a kernel error: the
+    oracle's own split and one-pass decodes differ by the same amount."""
+    r = paged_workload
+    assert_attention_close(r["gpu"], r["one_pass"], "split 4096 vs one pass")
+
+
+def test_split_decode_is_no_less_accurate_than_one_pass(paged_workload):
+    """The split reading costs no accuracy: against exact attention on the same quantized
+    operands, the GPU's split-K decode is at least as close as the one-pass method (measured
+    on the oracle: 6.9e-3 against 8.0e-3 mean x rms; the smaller per-split maxima put the
+    encoded P values higher in the E4M3 range)."""
+    r = paged_workload
+    rms = float(np.sqrt(np.mean(r["exact"] ** 2)))
+    e_gpu = np.abs(r["gpu"] - r["exact"])
+    e_one = np.abs(r["one_pass"] - r["exact"])
+    assert e_gpu.mean() <= 1.05 * e_one.mean(), (e_gpu.mean() / rms, e_one.mean() / rms)
+    assert e_gpu.max() <= 1.10 * e_one.max(), (e_gpu.max() / rms, e_one.max() / rms)
 
 
 def test_decode_underflow_aware_parity_and_quality():

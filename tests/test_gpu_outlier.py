@@ -12,7 +12,7 @@ from bit_block_scaled_nvfp4_b200 import api, workloads
 from oracle import attention as OA
 from oracle import outlier as OO
 from oracle import quant as OQ
-from helpers import assert_attention_close, f32, oracle_tensor_scale
+from helpers import assert_attention_close, f32
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -67,10 +67,14 @@ def test_outlier_aware_attention_parity_and_quality():
     assert api.check_status() == 0
     ref = np.zeros_like(out_t)
     exact = np.zeros_like(out_t)
-    qr_h, kr_h = f32(qr), f32(kr)
+    # the oracle's own transform of the CPU inputs (bit-exact with the kernel's, tested above)
+    lam_np = lam.cpu().numpy()
+    qr_o = OO.smooth_rotate(f32(q), lam_np, "q", "bf16")
+    kr_o = OO.smooth_rotate(f32(k), lam_np, "k", "bf16")
+    sq, sk = OQ.nvfp4_tensor_scale(qr_o), OQ.nvfp4_tensor_scale(kr_o)
     for h in range(2):
-        qh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(qr_h[0, h], tensor_scale=oracle_tensor_scale(qr)))
-        kh = OQ.nvfp4_dequantize(*OO.nvfp4_quantize_searched(kr_h[0, h], tensor_scale=oracle_tensor_scale(kr)))
+        qh = OQ.nvfp4_dequantize(*OQ.nvfp4_quantize(qr_o[0, h], tensor_scale=sq))
+        kh = OQ.nvfp4_dequantize(*OO.nvfp4_quantize_searched(kr_o[0, h], tensor_scale=sk))
         vc, vs = OQ.mxfp8_quantize_v(f32(v[0, h]))
         vh = OQ.mxfp8_dequantize_v(vc, vs, 1024)
         ref[0, h] = OA.attention_head(qh, kh, vh, True, scale)[0]

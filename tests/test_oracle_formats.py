@@ -117,3 +117,42 @@ def test_fp16_round_is_ieee_half():
     ref = torch.tensor(x, dtype=torch.float64).to(torch.float16).double().numpy()
     assert (F.fp16_round(x) == ref).all()
     assert F.fp16_round(np.array([1.0 + 2.0 ** -11]))[0] == 1.0          # tie to even
+
+
+def test_bf16_round_matches_torch_cast_of_float32_values():
+    """Values exactly representable in float32 (so torch's float32 -> bfloat16 cast, which
+    rounds to nearest even, rounds them once too): the two agree everywhere, subnormals
+    included."""
+    g = torch.Generator().manual_seed(1)
+    x = torch.cat([torch.randn(200000, generator=g) * s for s in (1e-40, 1e-30, 1e-3, 1.0, 3e4, 1e30)])
+    ref = x.to(torch.bfloat16).double().numpy()
+    assert (F.bf16_round(x.double().numpy()) == ref).all()
+
+
+def test_bf16_round_hand_worked():
+    """Ties to even on both sides, a value just above a tie, and one rounding from float64:
+    1 + 2^-8 + 2^-40 rounds up to 1 + 2^-7, while a float32 step first would land on the tie
+    1 + 2^-8 and then round down to 1."""
+    cases = [(1.0 + 2.0 ** -8, 1.0), (1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -6),
+             (-(1.0 + 2.0 ** -8), -1.0), (1.0 + 2.0 ** -8 + 2.0 ** -40, 1.0 + 2.0 ** -7),
+             (0.0, 0.0), (2.0 ** -133 * 0.75, 2.0 ** -133), (2.0 ** -133 * 0.5, 0.0),
+             (3.0 * 2.0 ** 126 + 2.0 ** 118, 3.0 * 2.0 ** 126)]
+    for x, want in cases:
+        assert F.bf16_round(np.array([x]))[0] == want, x
+    assert np.float32(1.0 + 2.0 ** -8 + 2.0 ** -40) == np.float32(1.0 + 2.0 ** -8)
+
+
+def test_bf16_round_is_nearest_brute_force():
+    """Against the two bracketing bfloat16 values, enumerated from the float32 bit patterns
+    around each input: the result is the nearer one, the even one on a tie."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(3000) * np.exp2(rng.integers(-20, 20, 3000))
+    got = F.bf16_round(x)
+    for xi, gi in zip(x, got):
+        b = int(np.array(abs(xi), dtype=np.float32).view(np.uint32)) & ~0xFFFF
+        lo = float(np.array(b, dtype=np.uint32).view(np.float32))
+        hi = float(np.array(b + 0x10000, dtype=np.uint32).view(np.float32))
+        assert lo <= abs(xi) <= hi
+        dl, dh = abs(xi) - lo, hi - abs(xi)
+        want = lo if (dl < dh or (dl == dh and (b >> 16) % 2 == 0)) else hi
+        assert gi == np.copysign(want, xi), xi
