@@ -173,22 +173,9 @@ def make_prefill_step(name):
     mixed = cfg.get("frac_bp", 0) > 0
     scale = 1.0 / math.sqrt(cfg["d"])
 
-    side = (torch.cuda.Stream(), torch.cuda.Stream())
-
     def quant(q=q, k=k, v=v):
-        # Q, K and V are quantized on three streams (independent kernels that each leave most
-        # of the GPU idle when run alone); the caller's stream waits for all three.
-        main = torch.cuda.current_stream()
-        for s_ in side:
-            s_.wait_stream(main)
-        q4 = api.quantize_nvfp4(q, want_fp16=mixed)
-        with torch.cuda.stream(side[0]):
-            k4 = api.quantize_nvfp4(k, want_fp16=mixed)
-        with torch.cuda.stream(side[1]):
-            v8 = api.quantize_mxfp8_v(v, want_fp16=mixed)
-        for s_ in side:
-            main.wait_stream(s_)
-        return q4, k4, v8
+        # Q, K (NVFP4) and V (MXFP8) in two launches: the amax pass of Q and K, then one encode
+        return api.quantize_qkv(q, k, v, want_fp16=mixed)
 
     def step(q=q, k=k, v=v):
         q4, k4, v8 = quant(q, k, v)
@@ -217,7 +204,7 @@ def make_prefill_step(name):
         q4, k4, _ = prepared()["in"]
         return api.tile_score_select(q4, k4, cfg["causal"], cfg["frac_bp"])
 
-    launches = 6 + (3 if mixed else 0)
+    launches = 3 + (3 if mixed else 0)
     host = [w.q.pin_memory(), w.k.pin_memory(), w.v.pin_memory()]
     # algorithmic quantize bytes: bf16 read once, NVFP4 codes + E4M3 scales (Q, K) and MXFP8
     # codes + E8M0 scales (V) written, plus the fp16 copies the FP16 tiles read

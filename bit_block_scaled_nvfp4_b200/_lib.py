@@ -68,6 +68,17 @@ class AppendParams(C.Structure):
     ]
 
 
+class QkvParams(C.Structure):
+    _fields_ = [
+        ("q", vp), ("k", vp), ("v", vp), ("dtype", i32), ("head_dim", i32),
+        ("q_rows", i64), ("k_rows", i64), ("v_bh", i32), ("v_tokens", i32),
+        ("q_codes", vp), ("q_scales", vp), ("q_tensor_scale", vp),
+        ("k_codes", vp), ("k_scales", vp), ("k_tensor_scale", vp),
+        ("v_codes", vp), ("v_scales", vp),
+        ("q16", vp), ("k16", vp), ("v16", vp),
+    ]
+
+
 #: name -> (restype, argtypes); exactly the functions include/qk4v8.h declares.
 SIGNATURES = {
     "qk4v8_version": (C.c_int, []),
@@ -81,6 +92,8 @@ SIGNATURES = {
     "quantize_nvfp4_workspace_size": (sz, []),
     "quantize_nvfp4": (i32, [vp, i32, i64, i32, i64, f32, vp, vp, vp, vp, vp, sz, vp]),
     "quantize_mxfp8_v": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),
+    "quantize_qkv_workspace_size": (sz, []),
+    "quantize_qkv": (i32, [C.POINTER(QkvParams), vp, sz, vp]),
     "quantize_nvfp4_residual": (i32, [vp, i32, i64, i32, i64, vp, vp, vp, vp, vp, vp]),
     "quantize_nvfp4_searched": (i32, [vp, i32, i64, i32, i64, f32, vp, vp, vp, vp, vp, sz, vp]),
     "qk_smooth_rotate": (i32, [vp, i32, i64, i32, vp, i32, vp, vp]),

@@ -191,6 +191,42 @@ def quantize_nvfp4_dual(x: torch.Tensor, tensor_scale: float | None = None):
     return q1, NVFP4Tensor(codes2, scales2, q1.tensor_scale)
 
 
+def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, want_fp16: bool = False,
+                 workspace: torch.Tensor | None = None):
+    """Q and K (..., D) to NVFP4 with their own tensor scales and V (..., N, D) to MXFP8, in two
+    launches (quantize_qkv); the same outputs as quantize_nvfp4(q), quantize_nvfp4(k) and
+    quantize_mxfp8_v(v). Returns (q4, k4, v8)."""
+    lib = _lib.load()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k and v must share a dtype")
+    d = q.shape[-1]
+    if k.shape[-1] != d or v.shape[-1] != d or v.dim() < 2:
+        raise ValueError("q, k and v must share the last (head) dimension; v is (..., N, D)")
+    need = lib.quantize_qkv_workspace_size()
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    elif workspace.numel() < need or workspace.dtype != torch.uint8:
+        raise ValueError(f"workspace must hold {need} bytes (uint8)")
+    _on_one_gpu(q, k, v, workspace)
+    q4 = _nvfp4_empty(q.shape, q.device, want_fp16)
+    k4 = _nvfp4_empty(k.shape, k.device, want_fp16)
+    v8 = _mxfp8_empty(v.shape, v.device, want_fp16)
+    n = v.shape[-2]
+    p = _lib.QkvParams(
+        q=_ptr(q), k=_ptr(k), v=_ptr(v), dtype=_dtype(q), head_dim=d,
+        q_rows=q.numel() // d, k_rows=k.numel() // d, v_bh=v.numel() // (n * d), v_tokens=n,
+        q_codes=_ptr(q4.codes), q_scales=_ptr(q4.scales), q_tensor_scale=_ptr(q4.tensor_scale),
+        k_codes=_ptr(k4.codes), k_scales=_ptr(k4.scales), k_tensor_scale=_ptr(k4.tensor_scale),
+        v_codes=_ptr(v8.codes), v_scales=_ptr(v8.scales), q16=_ptr(q4.fp16), k16=_ptr(k4.fp16),
+        v16=_ptr(v8.fp16))
+    _lib.check(lib.quantize_qkv(C.byref(p), _ptr(workspace), workspace.numel(), _stream()),
+               "quantize_qkv")
+    return q4, k4, v8
+
+
 def quantize_mxfp8_v(v: torch.Tensor, want_fp16: bool = False) -> MXFP8V:
     """MXFP8-quantize V laid out (..., N, D) along the token axis."""
     lib = _lib.load()
@@ -454,10 +490,10 @@ def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: b
     q2 = None
     if dual_q:
         q4, q2 = quantize_nvfp4_dual(q)
+        k4 = quantize_nvfp4(k)
+        v8 = quantize_mxfp8_v(v)
     else:
-        q4 = quantize_nvfp4(q, want_fp16=mixed)
-    k4 = quantize_nvfp4(k, want_fp16=mixed)
-    v8 = quantize_mxfp8_v(v, want_fp16=mixed)
+        q4, k4, v8 = quantize_qkv(q, k, v, want_fp16=mixed)
     bitmap = None
     if mixed:
         _, _, bitmap = tile_score_select(q4, k4, causal, fp16_frac_bp)

@@ -114,6 +114,7 @@ size_t qk4v8_struct_size(int32_t which) {
   return which == 0   ? sizeof(qk4v8_fwd_params)
          : which == 1 ? sizeof(qk4v8_decode_params)
          : which == 2 ? sizeof(qk4v8_append_params)
+         : which == 3 ? sizeof(qk4v8_qkv_params)
                       : 0;
 }
 
@@ -315,6 +316,79 @@ qk4v8_status quantize_mxfp8_v(const void* v, qk4v8_dtype dtype, int32_t batch_he
     else launch_mxfp8<__half, 64>(v, batch_heads, n_tokens, npad, codes, scales, v16, stream);
   }
   return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------
+size_t quantize_qkv_workspace_size(void) { return 2 * 4 * kAmaxPartials; }
+}  // extern "C"
+
+template <typename T, int D>
+static qk4v8_status launch_qkv(const qk4v8_qkv_params* p, float* q_part, float* k_part,
+                               cudaStream_t stream) {
+  // first launch: the amax pass (four CTAs per SM, split between Q and K in proportion to their
+  // sizes) and V's MXFP8 encode; second launch: the NVFP4 encode of Q and K
+  const int64_t qb = p->q_rows * (D / 16), kb = p->k_rows * (D / 16);
+  const int total = 4 * kNumSMs;
+  int gq = static_cast<int>((static_cast<double>(total) * qb) / static_cast<double>(qb + kb) + 0.5);
+  gq = gq < 1 ? 1 : (gq > total - 1 ? total - 1 : gq);
+  const int gk = total - gq;
+  static_assert(4 * kNumSMs <= kAmaxPartials, "amax partials");
+  QkvEncodeArgs a;
+  a.q = p->q; a.k = p->k; a.v = p->v;
+  a.q_blocks = qb; a.k_blocks = kb;
+  a.q_partial = q_part; a.k_partial = k_part; a.q_nparts = gq; a.k_nparts = gk;
+  a.q_codes = p->q_codes; a.q_scales = p->q_scales; a.q_ts = p->q_tensor_scale;
+  a.k_codes = p->k_codes; a.k_scales = p->k_scales; a.k_ts = p->k_tensor_scale;
+  a.v_codes = p->v_codes; a.v_scales = p->v_scales;
+  a.q16 = static_cast<__half*>(p->q16); a.k16 = static_cast<__half*>(p->k16);
+  a.v16 = static_cast<__half*>(p->v16);
+  a.q_chunks = static_cast<int32_t>((qb + kChunkBlocks - 1) / kChunkBlocks);
+  a.k_chunks = static_cast<int32_t>((kb + kChunkBlocks - 1) / kChunkBlocks);
+  a.nv_ctas = (a.q_chunks + a.k_chunks + kChunksPerCta - 1) / kChunksPerCta;
+  a.v_npad = (p->v_tokens + 127) / 128 * 128;
+  a.v_tiles = a.v_npad / 128;
+  a.v_n = p->v_tokens;
+  const int64_t grid1 = total + static_cast<int64_t>(a.v_tiles) * p->v_bh;
+  if (grid1 > 0x7fffffffLL) return QK4V8_ERR_UNSUPPORTED;
+  if (p->q16 != nullptr)
+    qk_amax_v_kernel<T, D, true><<<static_cast<unsigned>(grid1), 256, 0, stream>>>(a, p->q_rows, p->k_rows, gq, gk);
+  else
+    qk_amax_v_kernel<T, D, false><<<static_cast<unsigned>(grid1), 256, 0, stream>>>(a, p->q_rows, p->k_rows, gq, gk);
+  if (launch_status() != QK4V8_OK) return QK4V8_ERR_CUDA;
+  if (p->q16 != nullptr)
+    qk_encode_kernel<T, true><<<static_cast<unsigned>(a.nv_ctas), 256, 0, stream>>>(a);
+  else
+    qk_encode_kernel<T, false><<<static_cast<unsigned>(a.nv_ctas), 256, 0, stream>>>(a);
+  return launch_status();
+}
+
+extern "C" {
+qk4v8_status quantize_qkv(const qk4v8_qkv_params* p, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+  if (p == nullptr || !p->q || !p->k || !p->v || !p->q_codes || !p->q_scales ||
+      !p->q_tensor_scale || !p->k_codes || !p->k_scales || !p->k_tensor_scale || !p->v_codes ||
+      !p->v_scales || workspace == nullptr)
+    return QK4V8_ERR_INVALID_ARG;
+  if (p->dtype != QK4V8_F16 && p->dtype != QK4V8_BF16) return QK4V8_ERR_INVALID_ARG;
+  if (p->q_rows <= 0 || p->k_rows <= 0 || p->v_bh <= 0 || p->v_tokens <= 0)
+    return QK4V8_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return QK4V8_ERR_UNSUPPORTED;
+  const bool f16 = p->q16 != nullptr;
+  if ((p->k16 != nullptr) != f16 || (p->v16 != nullptr) != f16) return QK4V8_ERR_INVALID_ARG;
+  if (!aligned(p->q, 16) || !aligned(p->k, 16) || !aligned(p->v, 16) || !aligned(p->q_codes, 8) ||
+      !aligned(p->k_codes, 8) || !aligned(p->v_codes, 16) || !aligned(workspace, 4) ||
+      (f16 && (!aligned(p->q16, 16) || !aligned(p->k16, 16) || !aligned(p->v16, 16))))
+    return QK4V8_ERR_INVALID_ARG;
+  if (workspace_bytes < quantize_qkv_workspace_size()) return QK4V8_ERR_INVALID_ARG;
+  if (p->v_bh > 0x7fffffff / ((p->v_tokens + 127) / 128)) return QK4V8_ERR_UNSUPPORTED;
+  if ((p->q_rows + p->k_rows) * (p->head_dim / 16) / kChunkBlocks > 0x3fffffffLL) return QK4V8_ERR_UNSUPPORTED;
+  float* q_part = static_cast<float*>(workspace);
+  float* k_part = q_part + kAmaxPartials;
+  if (p->dtype == QK4V8_BF16)
+    return p->head_dim == 128 ? launch_qkv<__nv_bfloat16, 128>(p, q_part, k_part, stream)
+                              : launch_qkv<__nv_bfloat16, 64>(p, q_part, k_part, stream);
+  return p->head_dim == 128 ? launch_qkv<__half, 128>(p, q_part, k_part, stream)
+                            : launch_qkv<__half, 64>(p, q_part, k_part, stream);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -44,16 +44,17 @@ __device__ __forceinline__ int64_t block_offset(int64_t i, uint32_t bpr, int64_t
 // share to partial[c] (no atomics, nothing to clear), and the encode pass reduces the
 // partials. Four blocks of 16 per thread are loaded before any is reduced.
 // ---------------------------------------------------------------------------------------
+// The maximum of |x| over CTA `cta`'s share (of `nctas`) of a tensor's 16-element blocks,
+// valid in thread 0 of the CTA (256 threads).
 template <typename T>
-__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const T* __restrict__ x, int64_t rows,
-                                                         int32_t cols, int64_t row_stride,
-                                                         float* __restrict__ partial) {
+__device__ __forceinline__ float amax_share(const T* __restrict__ x, int64_t rows, int32_t cols,
+                                            int64_t row_stride, int cta, int nctas) {
   const uint32_t blocks_per_row = static_cast<uint32_t>(cols / 16);
   const int64_t total = rows * blocks_per_row;
   const bool contiguous = (row_stride == cols);
-  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t step = static_cast<int64_t>(nctas) * blockDim.x;
   float m = 0.f;
-  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < total;
+  for (int64_t i0 = cta * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < total;
        i0 += 4 * step) {
     uint4 u[8];
 #pragma unroll
@@ -79,11 +80,18 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const T* __restrict__ x
   __shared__ float wm[8];
   if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float t = 0.f;
+  float t = 0.f;
+  if (threadIdx.x == 0)
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t = fmaxf(t, wm[w]);
-    partial[blockIdx.x] = t;
-  }
+  return t;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const T* __restrict__ x, int64_t rows,
+                                                         int32_t cols, int64_t row_stride,
+                                                         float* __restrict__ partial) {
+  const float t = amax_share(x, rows, cols, row_stride, blockIdx.x, gridDim.x);
+  if (threadIdx.x == 0) partial[blockIdx.x] = t;
 }
 
 // Maximum of n (<= 1024) partial maxima, by every thread of a 256-thread CTA.
@@ -131,6 +139,117 @@ __device__ __forceinline__ void e2m1_encode16(const float* f, float den, uint32_
     byte |= (__float_as_uint(f[k + 1]) >> 31) << 7;
     w[k >> 3] |= byte << ((k & 7) * 4);
   }
+}
+
+// ---------------------------------------------------------------------------------------
+// The same block encoding on sixteen 16-bit inputs held packed (u[0], u[1]: element 2j in the
+// low half of 32-bit word j), with the same FP32 results step for step:
+//   amax_b  max of the magnitudes, taken in the 16-bit format (exact);
+//   s_b     E4M3(fl32(fl32(amax_b / 6) / s_t)), each quotient correctly rounded: Markstein's
+//           correction q' = RN(q + (a - b q) y) with q = RN(a y), y = RN(1/b) (RN(1/6) a
+//           constant, y_t = RN(1/s_t) from the caller), which is RN(a / b) while nothing
+//           under- or overflows; IEEE division outside [2^-60, 2^60];
+//   codes   E2M1(fl32(x / den)) as in e2m1_encode16, two elements per packed FP32 operation;
+//           each code's sign bit taken from its input's sign bit.
+// ---------------------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float2 to_float2(uint32_t w);
+template <> __device__ __forceinline__ float2 to_float2<__nv_bfloat16>(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+template <> __device__ __forceinline__ float2 to_float2<__half>(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+template <typename T> __device__ __forceinline__ float amax16_packed(const uint4* u);
+template <> __device__ __forceinline__ float amax16_packed<__nv_bfloat16>(const uint4* u) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(u);
+  __nv_bfloat162 m;
+  *reinterpret_cast<uint32_t*>(&m) = w[0] & 0x7FFF7FFFu;
+#pragma unroll
+  for (int j = 1; j < 8; ++j) {
+    const uint32_t a = w[j] & 0x7FFF7FFFu;
+    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&a));
+  }
+  return fmaxf(__low2float(m), __high2float(m));
+}
+template <> __device__ __forceinline__ float amax16_packed<__half>(const uint4* u) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(u);
+  __half2 m;
+  *reinterpret_cast<uint32_t*>(&m) = w[0] & 0x7FFF7FFFu;
+#pragma unroll
+  for (int j = 1; j < 8; ++j) {
+    const uint32_t a = w[j] & 0x7FFF7FFFu;
+    m = __hmax2(m, *reinterpret_cast<const __half2*>(&a));
+  }
+  return fmaxf(__low2float(m), __high2float(m));
+}
+// RN(a / b) with y = RN(1 / b): Markstein's correction inside [2^-60, 2^60] for a and b (a > 0
+// or 0), IEEE division outside it.
+__device__ __forceinline__ float div_rn_with(float a, float b, float y) {
+  const bool fast = (a >= 0x1p-60f && a <= 0x1p60f && b >= 0x1p-60f && b <= 0x1p60f) || a == 0.f;
+  return fast ? div_markstein(a, b, y) : __fdiv_rn(a, b);
+}
+// Per tensor scale s_t, for every E4M3 block-scale code c: den = fl32(decode(c) * s_t) and
+// y = RN(1 / den) (0 when den is 0 or outside Markstein's safe range [2^-90, 2^90]), built by
+// a CTA's threads into shared memory once, so a block looks both up instead of computing them.
+__device__ __forceinline__ void nvfp4_den_table(float s_t, float2* tab) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float den = __fmul_rn(e4m3_code_to_float(static_cast<uint32_t>(c)), s_t);
+    const bool fast = den >= 0x1p-90f && den <= 0x1p90f;
+    tab[c] = make_float2(den, fast ? __frcp_rn(den) : 0.f);
+  }
+}
+// Four E2M1 pair bytes (each in the low byte of c[0..3]) and the input words they came from ->
+// one code word: magnitudes from the conversion, each sign bit from its input's sign bit.
+__device__ __forceinline__ uint32_t e2m1_word(const uint32_t* c, const uint32_t* w) {
+  const uint32_t codes = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+  const uint32_t a = __byte_perm(w[0], w[1], 0x7531), b = __byte_perm(w[2], w[3], 0x7531);
+  const uint32_t lo = __byte_perm(a, b, 0x6420), hi = __byte_perm(a, b, 0x7531);   // sign bytes
+  return (codes & 0x77777777u) | ((lo >> 4) & 0x08080808u) | (hi & 0x80808080u);
+}
+template <typename T, bool kWrite16>
+__device__ __forceinline__ uint32_t nvfp4_encode16_packed(const uint4* u, float s_t, float y_t,
+                                                          const float2* tab, uint32_t* out,
+                                                          uint4* h16) {
+  constexpr float kInv6 = 0x1.555556p-3f;             // RN(1/6)
+  const float amax_b = amax16_packed<T>(u);
+  const float sbf = div_rn_with(div_rn_with(amax_b, 6.f, kInv6), s_t, y_t);
+  const uint32_t sc = cvt_e4m3x2(sbf, 0.f) & 0xFFu;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(u);
+  out[0] = out[1] = 0u;
+  if constexpr (kWrite16) {
+    uint32_t hw[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const __half2 h = __float22half2_rn(to_float2<T>(w[j]));
+      hw[j] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    h16[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    h16[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+  }
+  if (sc == 0u) return sc;                            // s_b = 0: every code 0
+  const float2 dy = tab[sc];
+  const float den = dy.x;
+  uint32_t cb[8];
+  if (dy.y != 0.f) {
+    const float2 y2 = make_float2(dy.y, dy.y), nd2 = make_float2(-den, -den);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 x = to_float2<T>(w[j]);
+      const float2 q = __fmul2_rn(x, y2);
+      const float2 r = __ffma2_rn(nd2, q, x);
+      const float2 qq = __ffma2_rn(r, y2, q);
+      cb[j] = cvt_e2m1x2(qq.x, qq.y);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 x = to_float2<T>(w[j]);
+      cb[j] = cvt_e2m1x2(__fdiv_rn(x.x, den), __fdiv_rn(x.y, den));
+    }
+  }
+  out[0] = e2m1_word(cb, w);
+  out[1] = e2m1_word(cb + 4, w + 4);
+  return sc;
 }
 
 // E2M1 code (magnitude in bits 0-2, sign in bit 3) -> its value, exactly.
@@ -194,29 +313,46 @@ __global__ void __launch_bounds__(256) nvfp4_encode_kernel(
     s_t = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 2688.f);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *ts_out = s_t;
+  const float y_t = __frcp_rn(s_t);
+  __shared__ float2 tab[128];
+  if constexpr (!kSearch) {
+    nvfp4_den_table(s_t, tab);
+    __syncthreads();
+  }
   const uint32_t blocks_per_row = static_cast<uint32_t>(cols / 16);
   const int64_t total = rows * blocks_per_row;
   const bool contiguous = (row_stride == cols);
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const uint4* p = reinterpret_cast<const uint4*>(x + block_offset(i, blocks_per_row, row_stride, contiguous));
-    const uint4 a = __ldg(p), b = __ldg(p + 1);
-    float f[16];
-    unpack8<T>(a, f);
-    unpack8<T>(b, f + 8);
-    uint32_t w[2];
-    const uint32_t sc = kSearch ? nvfp4_encode16_searched(f, s_t, w) : nvfp4_encode16(f, s_t, w);
+    uint4 u[2] = {__ldg(p), __ldg(p + 1)};
     const int64_t blk = i;                        // outputs are dense: block i of row i / bpr
+    uint32_t w[2];
+    uint32_t sc;
+    if constexpr (kSearch) {
+      float f[16];
+      unpack8<T>(u[0], f);
+      unpack8<T>(u[1], f + 8);
+      sc = nvfp4_encode16_searched(f, s_t, w);
+      if constexpr (kWrite16) {
+        __align__(16) __half h[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) h[k] = __float2half_rn(f[k]);
+        uint4* o = reinterpret_cast<uint4*>(x16 + blk * 16);
+        o[0] = *reinterpret_cast<uint4*>(h);
+        o[1] = *reinterpret_cast<uint4*>(h + 8);
+      }
+    } else {
+      uint4 h[2];
+      sc = nvfp4_encode16_packed<T, kWrite16>(u, s_t, y_t, tab, w, h);
+      if constexpr (kWrite16) {
+        uint4* o = reinterpret_cast<uint4*>(x16 + blk * 16);
+        o[0] = h[0];
+        o[1] = h[1];
+      }
+    }
     *reinterpret_cast<uint2*>(codes + blk * 8) = make_uint2(w[0], w[1]);
     scales[blk] = static_cast<uint8_t>(sc);
-    if constexpr (kWrite16) {
-      __align__(16) __half h[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) h[k] = __float2half_rn(f[k]);
-      uint4* o = reinterpret_cast<uint4*>(x16 + blk * 16);
-      o[0] = *reinterpret_cast<uint4*>(h);
-      o[1] = *reinterpret_cast<uint4*>(h + 8);
-    }
   }
 }
 
@@ -348,15 +484,14 @@ __device__ __forceinline__ int mxfp8_encode32(const float* f, uint8_t* cb) {
   return e;
 }
 
+// One 128-token x D tile (tile_id) of batch-head bh, staged through `tile` (128 x (D + 8)).
 template <typename T, int D, bool kWrite16>
-__global__ void __launch_bounds__(256) mxfp8_v_kernel(const T* __restrict__ v, int32_t N,
-                                                      int32_t Npad, uint8_t* __restrict__ codes,
-                                                      uint8_t* __restrict__ scales,
-                                                      __half* __restrict__ v16t) {
+__device__ __forceinline__ void mxfp8_v_tile(const T* __restrict__ v, int32_t N, int32_t Npad,
+                                             uint8_t* __restrict__ codes,
+                                             uint8_t* __restrict__ scales,
+                                             __half* __restrict__ v16t, int tile_id, int64_t bh,
+                                             T* tile) {
   constexpr int LD = D + 8;                       // padded row (elements)
-  __shared__ __align__(16) T tile[128 * LD];
-  const int tile_id = blockIdx.x;
-  const int64_t bh = blockIdx.y;
   const int tok0 = tile_id * 128;
   // Load 128 tokens x D (16-byte chunks), zero past N.
   // (256 threads: every load of the tile is in flight before the first shared store)
@@ -395,6 +530,162 @@ __global__ void __launch_bounds__(256) mxfp8_v_kernel(const T* __restrict__ v, i
 #pragma unroll
       for (int k = 0; k < 4; ++k) o[k] = reinterpret_cast<uint4*>(h)[k];
     }
+  }
+}
+
+template <typename T, int D, bool kWrite16>
+__global__ void __launch_bounds__(256) mxfp8_v_kernel(const T* __restrict__ v, int32_t N,
+                                                      int32_t Npad, uint8_t* __restrict__ codes,
+                                                      uint8_t* __restrict__ scales,
+                                                      __half* __restrict__ v16t) {
+  __shared__ __align__(16) T tile[128 * (D + 8)];
+  mxfp8_v_tile<T, D, kWrite16>(v, N, Npad, codes, scales, v16t, blockIdx.x, blockIdx.y, tile);
+}
+
+// ---------------------------------------------------------------------------------------
+// Q, K and V of one attention call: after qk_amax_kernel, one launch encodes everything.
+// ---------------------------------------------------------------------------------------
+constexpr int kChunkBlocks = 1024;                // 16-element blocks per chunk (4 per thread)
+constexpr int kChunksPerCta = 4;                  // chunks one NVFP4 CTA of the fused encode takes
+
+// The eight 16-byte loads of a thread's four blocks t, t + 256, t + 512, t + 768 of chunk
+// `chunk` of a dense tensor of `total` blocks (zero past the end).
+template <typename T>
+__device__ __forceinline__ void nvfp4_chunk_load(const T* __restrict__ x, int64_t total,
+                                                 int64_t chunk, uint4* u) {
+  const int64_t b0 = chunk * kChunkBlocks + threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t i = b0 + k * 256;
+    u[2 * k] = u[2 * k + 1] = make_uint4(0, 0, 0, 0);
+    if (i < total) {
+      const uint4* p = reinterpret_cast<const uint4*>(x + i * 16);
+      u[2 * k] = __ldg(p);
+      u[2 * k + 1] = __ldg(p + 1);
+    }
+  }
+}
+
+// NVFP4 encode of a thread's four blocks of chunk `chunk` (loaded by nvfp4_chunk_load);
+// consecutive threads write consecutive code words and scale bytes.
+template <typename T, bool kWrite16>
+__device__ __forceinline__ void nvfp4_chunk_encode(const uint4* u, int64_t total, int64_t chunk,
+                                                   float s_t, float y_t, const float2* tab,
+                                                   uint8_t* __restrict__ codes,
+                                                   uint8_t* __restrict__ scales,
+                                                   __half* __restrict__ x16) {
+  const int64_t b0 = chunk * kChunkBlocks + threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t i = b0 + k * 256;
+    if (i >= total) break;
+    uint32_t w[2];
+    uint4 h[2];
+    const uint32_t sc = nvfp4_encode16_packed<T, kWrite16>(u + 2 * k, s_t, y_t, tab, w, h);
+    *reinterpret_cast<uint2*>(codes + i * 8) = make_uint2(w[0], w[1]);
+    scales[i] = static_cast<uint8_t>(sc);
+    if constexpr (kWrite16) {
+      uint4* o = reinterpret_cast<uint4*>(x16 + i * 16);
+      o[0] = h[0];
+      o[1] = h[1];
+    }
+  }
+}
+
+struct QkvEncodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t q_blocks, k_blocks;                     // 16-element blocks of Q and K
+  const float* q_partial;
+  const float* k_partial;
+  int32_t q_nparts, k_nparts;                     // per-CTA maxima of the amax pass
+  uint8_t* q_codes;
+  uint8_t* q_scales;
+  float* q_ts;
+  uint8_t* k_codes;
+  uint8_t* k_scales;
+  float* k_ts;
+  uint8_t* v_codes;
+  uint8_t* v_scales;
+  __half* q16;
+  __half* k16;
+  __half* v16;
+  int32_t q_chunks, k_chunks;                     // chunks of kChunkBlocks blocks per tensor
+  int32_t nv_ctas;                                // NVFP4 CTAs (kChunksPerCta positions each)
+  int32_t v_tiles, v_n, v_npad;                   // 128-token V tiles per batch-head, tokens
+};
+
+// Position p of the Q/K chunk order: the K chunks spread among the Q chunks in proportion to
+// the sizes (p is a K chunk when the count of K chunks before it, floor(p k / n), steps at p),
+// each tensor from its last chunk to its first.
+__device__ __forceinline__ void qk_position(const QkvEncodeArgs& a, int64_t p, bool& k_role,
+                                            int64_t& chunk) {
+  const int64_t n = static_cast<int64_t>(a.q_chunks) + a.k_chunks;
+  const int64_t kc0 = p * a.k_chunks / n, kc1 = (p + 1) * a.k_chunks / n;
+  k_role = kc1 > kc0;
+  chunk = k_role ? (a.k_chunks - 1 - kc0) : (a.q_chunks - 1 - (p - kc0));
+}
+
+// First launch: the amax pass of Q and K and the whole MXFP8 encode of V (which needs no
+// tensor scale, so its traffic overlaps the read-only amax pass). CTAs [0, gq) take Q's
+// share of the amax pass and [gq, gq + gk) K's, each writing its maximum to its tensor's
+// partials; the rest encode V tiles.
+template <typename T, int D, bool kWrite16>
+__global__ void __launch_bounds__(256) qk_amax_v_kernel(QkvEncodeArgs a, int64_t q_rows,
+                                                        int64_t k_rows, int32_t gq, int32_t gk) {
+  __shared__ __align__(16) T tile[128 * (D + 8)];
+  const int c = blockIdx.x;
+  if (c < gq) {
+    const float t = amax_share(static_cast<const T*>(a.q), q_rows, D, D, c, gq);
+    if (threadIdx.x == 0) const_cast<float*>(a.q_partial)[c] = t;
+  } else if (c < gq + gk) {
+    const float t = amax_share(static_cast<const T*>(a.k), k_rows, D, D, c - gq, gk);
+    if (threadIdx.x == 0) const_cast<float*>(a.k_partial)[c - gq] = t;
+  } else {
+    const int t = c - gq - gk;
+    mxfp8_v_tile<T, D, kWrite16>(static_cast<const T*>(a.v), a.v_n, a.v_npad, a.v_codes, a.v_scales,
+                                 a.v16, t % a.v_tiles, t / a.v_tiles, tile);
+  }
+}
+
+// Second launch: the NVFP4 encode of Q and K. Each CTA encodes kChunksPerCta consecutive
+// positions of the Q/K chunk order, so the tails the amax pass read last, still in L2, are
+// encoded first. A CTA issues its first chunk's loads before it reduces the amax partials and
+// builds the two tensors' scale tables. Four CTAs per SM (at most 64 registers a thread): the
+// per-block arithmetic is long, and other warps hide its latency better than a second register
+// buffer would.
+template <typename T, bool kWrite16>
+__global__ void __launch_bounds__(256, 4) qk_encode_kernel(QkvEncodeArgs a) {
+  __shared__ float2 tabq[128], tabk[128];
+  const int c = blockIdx.x;
+  const int64_t n = static_cast<int64_t>(a.q_chunks) + a.k_chunks;
+  const int64_t p0 = static_cast<int64_t>(c) * kChunksPerCta;
+  const int np = static_cast<int>(min(static_cast<int64_t>(kChunksPerCta), n - p0));
+  bool kr;
+  int64_t ch;
+  qk_position(a, p0, kr, ch);
+  uint4 u[8];
+  nvfp4_chunk_load<T>(static_cast<const T*>(kr ? a.k : a.q), kr ? a.k_blocks : a.q_blocks, ch, u);
+  const float amq = reduce_partials(a.q_partial, a.q_nparts);
+  __syncthreads();                                 // the reduction's scratch is reused
+  const float amk = reduce_partials(a.k_partial, a.k_nparts);
+  const float stq = (amq == 0.f) ? 1.f : __fdiv_rn(amq, 2688.f);
+  const float stk = (amk == 0.f) ? 1.f : __fdiv_rn(amk, 2688.f);
+  const float ytq = __frcp_rn(stq), ytk = __frcp_rn(stk);
+  nvfp4_den_table(stq, tabq);
+  nvfp4_den_table(stk, tabk);
+  __syncthreads();
+  for (int i = 0; i < np; ++i) {
+    if (i > 0) {
+      qk_position(a, p0 + i, kr, ch);
+      nvfp4_chunk_load<T>(static_cast<const T*>(kr ? a.k : a.q), kr ? a.k_blocks : a.q_blocks, ch, u);
+    }
+    if (ch == 0 && threadIdx.x == 0) *(kr ? a.k_ts : a.q_ts) = kr ? stk : stq;
+    if (kr)
+      nvfp4_chunk_encode<T, kWrite16>(u, a.k_blocks, ch, stk, ytk, tabk, a.k_codes, a.k_scales, a.k16);
+    else
+      nvfp4_chunk_encode<T, kWrite16>(u, a.q_blocks, ch, stq, ytq, tabq, a.q_codes, a.q_scales, a.q16);
   }
 }
 

@@ -48,7 +48,7 @@ int qk4v8_version(void);
 
 /* sizeof the parameter structs, for bindings that mirror them: which = 0 gives
  * sizeof(qk4v8_fwd_params), 1 sizeof(qk4v8_decode_params), 2 sizeof(qk4v8_append_params),
- * anything else 0. */
+ * 3 sizeof(qk4v8_qkv_params), anything else 0. */
 size_t qk4v8_struct_size(int32_t which);
 
 /* Human-readable name of a status code (static string). */
@@ -172,6 +172,48 @@ qk4v8_status quantize_nvfp4_residual(const void* x, qk4v8_dtype dtype, int64_t r
 qk4v8_status quantize_mxfp8_v(const void* v, qk4v8_dtype dtype, int32_t batch_heads,
                               int32_t n_tokens, int32_t head_dim, uint8_t* codes,
                               uint8_t* scales, void* v16, cudaStream_t stream);
+
+/*
+ * quantize_qkv — Q and K to NVFP4 (each with its own dynamic tensor scale, exactly as
+ * quantize_nvfp4 with tensor_scale_in <= 0) and V to MXFP8 (exactly as quantize_mxfp8_v), for
+ * one attention call, in two launches: the amax pass of Q and K (per-CTA maxima, no grid-wide
+ * wait), then one launch that encodes all three. The encode launch takes Q and K from their
+ * last 16-element blocks to their first, so the parts the amax pass read last, still cached in
+ * L2, are read again first. Same formats and arithmetic as the per-tensor calls (the tqpw.cn
+ * article §2.2 for NVFP4, §2.1 for MXFP8); outputs are bit-identical to theirs.
+ * q [q_rows, head_dim], k [k_rows, head_dim], v [v_bh, v_tokens, head_dim]: dense fp16/bf16
+ * (one dtype), 16-byte aligned; head_dim 64 or 128.
+ * q_codes/q_scales/q_tensor_scale, k_...: as quantize_nvfp4's outputs (codes 8-byte aligned).
+ * v_codes/v_scales: as quantize_mxfp8_v's outputs (codes 16-byte aligned).
+ * q16/k16/v16: optional fp16 copies (all three or none), as those calls' x16 / v16.
+ * workspace >= quantize_qkv_workspace_size() bytes, 4-byte aligned (the amax partials).
+ * Errors: QK4V8_ERR_INVALID_ARG for null pointers, bad sizes or alignment, a short workspace;
+ * QK4V8_ERR_UNSUPPORTED for another head_dim.
+ */
+typedef struct {
+  const void* q;
+  const void* k;
+  const void* v;
+  qk4v8_dtype dtype;
+  int32_t head_dim;
+  int64_t q_rows, k_rows;
+  int32_t v_bh, v_tokens;
+  uint8_t* q_codes;
+  uint8_t* q_scales;
+  float* q_tensor_scale;
+  uint8_t* k_codes;
+  uint8_t* k_scales;
+  float* k_tensor_scale;
+  uint8_t* v_codes;
+  uint8_t* v_scales;
+  void* q16;
+  void* k16;
+  void* v16;
+} qk4v8_qkv_params;
+
+size_t quantize_qkv_workspace_size(void);
+qk4v8_status quantize_qkv(const qk4v8_qkv_params* params, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
 
 /*
  * tile_score_select — ThriftAttention-style tile importance (ai-feeds.com ThriftAttention

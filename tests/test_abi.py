@@ -85,6 +85,31 @@ def test_quantize_nvfp4_validation(lib):
     assert call(dt=7) == _lib.QK4V8_ERR_INVALID_ARG
 
 
+def test_quantize_qkv_validation(lib):
+    """The fused Q/K/V quantize rejects bad calls on the host, before any launch."""
+    assert lib.qk4v8_struct_size(3) == C.sizeof(_lib.QkvParams)
+    f = lib.quantize_qkv
+    wsb = lib.quantize_qkv_workspace_size()
+    assert wsb >= 8
+
+    def p(**kw):
+        d = dict(q=FAKE, k=FAKE, v=FAKE, dtype=1, head_dim=128, q_rows=64, k_rows=16, v_bh=1,
+                 v_tokens=16, q_codes=FAKE, q_scales=FAKE, q_tensor_scale=FAKE, k_codes=FAKE,
+                 k_scales=FAKE, k_tensor_scale=FAKE, v_codes=FAKE, v_scales=FAKE)
+        d.update(kw)
+        return C.byref(_lib.QkvParams(**d))
+    assert f(None, FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(p(v=None), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(p(k_tensor_scale=None), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(p(), None, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(p(), FAKE, wsb - 4, None) == _lib.QK4V8_ERR_INVALID_ARG     # short workspace
+    assert f(p(dtype=2), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG   # fp32 input
+    assert f(p(q_rows=0), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG
+    assert f(p(head_dim=96), FAKE, wsb, None) == _lib.QK4V8_ERR_UNSUPPORTED
+    assert f(p(q=FAKE + 8), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG   # misaligned
+    assert f(p(q16=FAKE), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG     # copies: all or none
+
+
 def test_quantize_mxfp8_validation(lib):
     f = lib.quantize_mxfp8_v
     assert f(None, 1, 1, 128, 128, FAKE, FAKE, None, None) == _lib.QK4V8_ERR_INVALID_ARG

@@ -89,6 +89,38 @@ def test_e4m3_block_scale_exhaustive_fp16():
     _nvfp4_equal(x, tensor_scale=2.0 ** -4)
 
 
+def _all_bf16_values(lo_bits, hi_bits):
+    return torch.arange(lo_bits, hi_bits, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("ts", [None, 0.37, 2.0 ** -70, 3.1e17])
+def test_block_scale_and_codes_exhaustive_bf16(ts):
+    """Every positive finite bf16 value (subnormals included) as a block's largest magnitude,
+    with the other elements of the block at -1/3, 5/7 and 1/11 of it: the block scale
+    E4M3(amax_b / 6 / s_t) and every element code, bit-exact against the oracle, for the
+    computed tensor scale and fixed scales with ordinary, tiny and huge values (both sides of
+    the exponent bounds of the kernels' fast division). Checked through the per-tensor kernel
+    and the fused Q/K/V kernel."""
+    amax = _all_bf16_values(0x0001, 0x7F80)
+    x = torch.zeros(amax.numel(), 16, dtype=torch.bfloat16)
+    x[:, 3] = amax
+    x[:, 7] = (-amax.double() / 3).to(torch.bfloat16)
+    x[:, 9] = (amax.double() * 5 / 7).to(torch.bfloat16)
+    x[:, 14] = (amax.double() / 11).to(torch.bfloat16)
+    assert torch.isfinite(x.float()).all()
+    _nvfp4_equal(x, tensor_scale=ts)
+    if ts is None:
+        # the same 16-element blocks, 128 to a row (the fused call's head dimension)
+        xq = torch.cat([x, torch.zeros(1, 16, dtype=torch.bfloat16)]).reshape(-1, 128)
+        xk = x[:4096].reshape(-1, 128)
+        v = torch.zeros(1, 128, 128, dtype=torch.bfloat16)
+        q4, k4, _ = api.quantize_qkv(xq.to(DEV), xk.to(DEV), v.to(DEV))
+        for g, xx in ((q4, xq), (k4, xk)):
+            c, sc, t = OQ.nvfp4_quantize(f32(xx))
+            assert np.array_equal(g.scales.cpu().numpy(), sc) and np.array_equal(g.codes.cpu().numpy(), c)
+            assert np.float32(g.tensor_scale.item()) == t
+
+
 def _mxfp8_equal(v_cpu, want_fp16=False):
     g = api.quantize_mxfp8_v(v_cpu.to(DEV), want_fp16=want_fp16)
     c, s = OQ.mxfp8_quantize_v(f32(v_cpu))
@@ -149,3 +181,52 @@ def test_nvfp4_residual_bit_exact(shape, dtype):
     assert np.array_equal(gs, s2), f"scales differ at {np.argwhere(gs != s2)[:5]}"
     assert np.array_equal(gc, c2), f"codes differ at {np.argwhere(gc != c2)[:5]}"
     assert q2.tensor_scale is q1.tensor_scale and np.float32(q1.tensor_scale.item()) == t
+
+
+def _check_qkv(q, k, v, want_fp16=False):
+    """quantize_qkv (two launches) against the oracle, bit for bit, and against the per-tensor
+    calls (identical outputs)."""
+    q4, k4, v8 = api.quantize_qkv(q.to(DEV), k.to(DEV), v.to(DEV), want_fp16=want_fp16)
+    for g, x in ((q4, q), (k4, k)):
+        c, s, t = OQ.nvfp4_quantize(f32(x))
+        gc, gs = g.codes.cpu().numpy(), g.scales.cpu().numpy()
+        assert np.array_equal(gs, s), f"scales differ at {np.argwhere(gs != s)[:5]}"
+        assert np.array_equal(gc, c), f"codes differ at {np.argwhere(gc != c)[:5]}"
+        assert np.float32(g.tensor_scale.item()) == t
+        if want_fp16:
+            assert np.array_equal(g.fp16.cpu().numpy(), OF.fp16_round(f32(x)).astype(np.float16))
+    n = v.shape[-2]
+    vc, vs = OQ.mxfp8_quantize_v(f32(v))
+    npad = v8.codes.shape[-1]
+    assert np.array_equal(v8.codes.cpu().numpy(), vc)
+    assert np.array_equal(v8.scales.cpu().numpy(), vs)
+    if want_fp16:
+        r16 = np.zeros(v8.fp16.shape, dtype=np.float16)
+        r16[..., :n] = np.swapaxes(OF.fp16_round(f32(v)), -1, -2)
+        assert np.array_equal(v8.fp16.cpu().numpy(), r16)
+    # the per-tensor entry points give the same bytes
+    sq, sk, sv = api.quantize_nvfp4(q.to(DEV)), api.quantize_nvfp4(k.to(DEV)), api.quantize_mxfp8_v(v.to(DEV))
+    assert torch.equal(sq.codes, q4.codes) and torch.equal(sq.scales, q4.scales)
+    assert torch.equal(sk.codes, k4.codes) and torch.equal(sk.tensor_scale, k4.tensor_scale)
+    assert torch.equal(sv.codes, v8.codes) and torch.equal(sv.scales, v8.scales)
+    assert npad == (n + 127) // 128 * 128
+
+
+@pytest.mark.parametrize("name", ["tiny_prefill", "prefill_h16_n4096"])
+def test_qkv_workload_bit_exact(name):
+    w = workloads.make_prefill(name)
+    _check_qkv(w.q, w.k, w.v)
+
+
+@pytest.mark.parametrize("hq,hkv,n,d,dtype,fp16", [(4, 1, 1000, 128, torch.bfloat16, False),
+                                                  (3, 3, 77, 64, torch.float16, True),
+                                                  (8, 2, 300, 128, torch.bfloat16, True)])
+def test_qkv_ragged_shapes(hq, hkv, n, d, dtype, fp16):
+    """Chunk tails (blocks not a multiple of the 1024-block chunk), V tails (tokens not a
+    multiple of 128), head_dim 64, fp16 inputs, the optional fp16 copies, and Q/K size ratios of
+    1, 3 and 4."""
+    g = torch.Generator().manual_seed(n + d)
+    q = (torch.randn(1, hq, n, d, generator=g) * 3).to(dtype)
+    k = (torch.randn(1, hkv, n, d, generator=g) * torch.rand(1, hkv, n, 1, generator=g) * 9).to(dtype)
+    v = torch.randn(1, hkv, n, d, generator=g).to(dtype)
+    _check_qkv(q, k, v, want_fp16=fp16)
