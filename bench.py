@@ -230,22 +230,25 @@ def make_decode_step(name):
     q = workloads.make_decode_query(lay).cuda()
     table, ctx = lay.page_table.cuda(), lay.lens.cuda()
     split = 4096
-    ws = torch.empty(cfg["S"] * cfg["Hq"] * ((max(lens) + split - 1) // split) * (cfg["d"] + 2) * 4,
-                     dtype=torch.uint8, device="cuda")
+    # a serving loop's shape: the fixed buffers checked and allocated once (the decode plan, the
+    # query's NVFP4 buffers and workspace), so a step is its launches
+    plan = api.DecodePlan(cache, table, ctx, max(lens), split, cfg["S"], cfg["Hq"])
+    q4buf = api.quantize_nvfp4(q)
+    qws = torch.empty(api._lib.load().quantize_nvfp4_workspace_size(), dtype=torch.uint8, device="cuda")
 
     def quant(q=q):
-        return api.quantize_nvfp4(q)
+        return api.quantize_nvfp4(q, workspace=qws, out=q4buf)
 
-    def step(q=q, table=table, ctx=ctx):
-        return api.attn_qk4v8_decode_paged(quant(q), cache, table, ctx, max(lens), split, workspace=ws)
+    def step(q=q):
+        return plan.run(quant(q))
 
     prep = {}
 
     def attn_only():
         # decode + merge alone, on a query quantized once beforehand
         if not prep:
-            prep["q4"] = quant()
-        return api.attn_qk4v8_decode_paged(prep["q4"], cache, table, ctx, max(lens), split, workspace=ws)
+            prep["q4"] = api.quantize_nvfp4(q)
+        return plan.run(prep["q4"])
 
     kv, total = decode_bytes(lay)
     host = [workloads.make_decode_query(lay).pin_memory(), lay.page_table.pin_memory(), lay.lens.pin_memory()]
@@ -360,9 +363,10 @@ def time_steps(st, K, W, world):
 
 
 def time_e2e(st, K, world):
-    """Same step through the public API with H2D of the inputs and D2H of the output."""
+    """Same step through the public API with H2D of the inputs (into the device tensors the
+    step reads) and D2H of the output."""
     host = st["host"]
-    dev = [torch.empty_like(h, device="cuda") for h in host]
+    dev = list(st["inputs"])
     out_host = None
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     h2d = sum(h.numel() * h.element_size() for h in host)
@@ -376,7 +380,7 @@ def time_e2e(st, K, world):
         a.record()
         for d_, h_ in zip(dev, host):
             d_.copy_(h_, non_blocking=True)
-        out = st["step"](*dev)
+        out = st["step"]()
         if out_host is None:
             out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         out_host.copy_(out, non_blocking=True)

@@ -133,20 +133,32 @@ def selftest_wait_timeout() -> None:
 
 
 def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16: bool = False,
-                   workspace: torch.Tensor | None = None, scale_search: bool = False) -> NVFP4Tensor:
+                   workspace: torch.Tensor | None = None, scale_search: bool = False,
+                   out: NVFP4Tensor | None = None) -> NVFP4Tensor:
     """NVFP4-quantize ``x`` (..., D) along its last axis (contiguous fp16/bf16 CUDA tensor).
 
     ``tensor_scale``: a fixed FP32 tensor scale (a paged cache's, for instance); None or a
     value <= 0 computes it from the tensor's amax (amax / (6 * 448)). ``want_fp16`` also
     writes an fp16 copy of ``x`` for the FP16-tile attention path. ``workspace``: optional
     uint8 scratch of ``quantize_nvfp4_workspace_size()`` bytes. ``scale_search`` picks each
-    block's scale among four candidates by squared error."""
+    block's scale among four candidates by squared error. ``out``: optional preallocated
+    result (from a previous call on the same shape), written in place instead of allocating."""
     lib = _lib.load()
     if not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA tensor")
     cols = x.shape[-1]
     rows = x.numel() // cols
-    r = _nvfp4_empty(x.shape, x.device, want_fp16)
+    if out is None:
+        r = _nvfp4_empty(x.shape, x.device, want_fp16)
+    else:
+        r = out
+        lead = tuple(x.shape[:-1])
+        _expect(r.codes, "out.codes", lead + (cols // 2,), torch.uint8)
+        _expect(r.scales, "out.scales", lead + (cols // 16,), torch.uint8)
+        _expect_scalar(r.tensor_scale, "out.tensor_scale")
+        if want_fp16:
+            _expect(r.fp16, "out.fp16", tuple(x.shape), torch.float16)
+        _on_one_gpu(x, r.codes, r.scales, r.tensor_scale, r.fp16 if want_fp16 else None)
     need = lib.quantize_nvfp4_workspace_size()
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
@@ -156,7 +168,8 @@ def quantize_nvfp4(x: torch.Tensor, tensor_scale: float | None = None, want_fp16
     fn = lib.quantize_nvfp4_searched if scale_search else lib.quantize_nvfp4
     st = fn(_ptr(x), _dtype(x), rows, cols, cols,
             float(tensor_scale) if tensor_scale else 0.0, _ptr(r.codes), _ptr(r.scales),
-            _ptr(r.tensor_scale), _ptr(r.fp16), _ptr(workspace), workspace.numel(), _stream())
+            _ptr(r.tensor_scale), _ptr(r.fp16) if want_fp16 else None, _ptr(workspace),
+            workspace.numel(), _stream())
     _lib.check(st, "quantize_nvfp4")
     return r
 
@@ -417,6 +430,58 @@ def attn_qk4v8_decode_paged(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Te
     st = lib.attn_qk4v8_decode_paged(C.byref(p), _ptr(workspace), workspace.numel(), _stream())
     _lib.check(st, "attn_qk4v8_decode_paged")
     return (out, lse) if want_lse else out
+
+
+class DecodePlan:
+    """A decode step whose fixed buffers are checked once: the paged cache, page table,
+    context lengths, split, output (and lse) buffers and workspace. ``run(q)`` then checks only
+    the step's query and launches through attn_qk4v8_decode_paged, writing into the plan's own
+    output buffer (read it before the next ``run``). For serving loops, where the per-step
+    host work of checking and allocating would otherwise show up between the launches."""
+
+    def __init__(self, cache: PagedKV, page_table: torch.Tensor, context_lens: torch.Tensor,
+                 max_context: int, split_tokens: int, num_seqs: int, q_heads: int,
+                 softmax_scale: float | None = None, out_dtype=torch.bfloat16,
+                 want_lse: bool = False, workspace: torch.Tensor | None = None,
+                 underflow_aware: bool = False):
+        d = cache.k_pages.shape[-1] * 2
+        dev = cache.k_pages.device
+        self.q_shape = (num_seqs, q_heads, d // 2)
+        self.out = torch.empty(num_seqs, q_heads, d, dtype=out_dtype, device=dev)
+        self.lse = torch.empty(num_seqs, q_heads, dtype=torch.float32, device=dev) if want_lse else None
+        # a stand-in query of the step's shape: checks every fixed buffer against it once
+        probe = NVFP4Tensor(torch.empty(self.q_shape, dtype=torch.uint8, device=dev),
+                            torch.empty(num_seqs, q_heads, d // 16, dtype=torch.uint8, device=dev),
+                            torch.empty(1, dtype=torch.float32, device=dev))
+        self.params = decode_params(probe, cache, page_table, context_lens, max_context,
+                                    split_tokens, self.out, softmax_scale, self.lse,
+                                    underflow_aware)
+        self._keep = (cache, page_table, context_lens)
+        lib = _lib.load()
+        need = lib.attn_qk4v8_decode_workspace_size(C.byref(self.params))
+        if workspace is None or workspace.numel() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        elif workspace.dtype != torch.uint8:
+            raise TypeError("workspace must be a uint8 tensor")
+        _on_one_gpu(self.out, workspace)
+        self.workspace = workspace
+        self._dev = dev.index if dev.index is not None else torch.cuda.current_device()
+
+    def run(self, q: NVFP4Tensor):
+        """One decode step for the quantized query ``q`` [S, Hq, D/2]; returns the plan's out
+        (and lse)."""
+        c, sc, ts = q.codes, q.scales, q.tensor_scale
+        if tuple(c.shape) != self.q_shape or c.dtype != torch.uint8 or not c.is_cuda or \
+                c.get_device() != self._dev or not c.is_contiguous() or not sc.is_contiguous() or \
+                sc.get_device() != self._dev or ts.get_device() != self._dev or \
+                sc.numel() * 8 != c.numel():
+            raise ValueError(f"q must be an NVFP4 query of shape {self.q_shape} on the plan's device")
+        p = self.params
+        p.q_codes, p.q_scales, p.q_tensor_scale = c.data_ptr(), sc.data_ptr(), ts.data_ptr()
+        st = _lib.load().attn_qk4v8_decode_paged(C.byref(p), _ptr(self.workspace),
+                                                 self.workspace.numel(), _stream())
+        _lib.check(st, "attn_qk4v8_decode_paged")
+        return (self.out, self.lse) if self.lse is not None else self.out
 
 
 def attn_qk4v8_decode_paged_noalloc(q: NVFP4Tensor, cache: PagedKV, page_table: torch.Tensor,

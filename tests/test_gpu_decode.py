@@ -242,3 +242,23 @@ def test_decode_dual_q_parity(ua):
     assert api.check_status() == 0
     want, _ = _oracle_decode(q, seqs, lens, hq, hkv, split, 1 / math.sqrt(d), ua=ua, dual=True)
     assert_attention_close(f32(out), want, "decode dual Q")
+
+
+def test_decode_plan_matches_the_call():
+    """DecodePlan (fixed buffers checked once, only the query changes per step) gives the same
+    bytes as attn_qk4v8_decode_paged on two steps in a row, and rejects a query of another
+    shape."""
+    lens, hq, hkv, d, split = [700, 64, 1500], 8, 2, 128, 512
+    cache, table, _ = _build(lens, hkv, d, seed=31)
+    ctx = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    table = table.to(DEV)
+    plan = api.DecodePlan(cache, table, ctx, max(lens), split, len(lens), hq, want_lse=True)
+    g = torch.Generator().manual_seed(3)
+    for _ in range(2):
+        q4 = api.quantize_nvfp4(torch.randn(len(lens), hq, d, generator=g).to(torch.bfloat16).to(DEV))
+        out, lse = plan.run(q4)
+        ref, rlse = api.attn_qk4v8_decode_paged(q4, cache, table, ctx, max(lens), split, want_lse=True)
+        assert torch.equal(out, ref) and torch.equal(lse, rlse)
+    bad = api.quantize_nvfp4(torch.randn(len(lens), hq // 2, d).to(torch.bfloat16).to(DEV))
+    with pytest.raises(ValueError):
+        plan.run(bad)
