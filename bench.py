@@ -42,9 +42,9 @@ METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of H
 # kernel on the workload (dram__bytes_read.sum + dram__bytes_write.sum). Only workloads with a
 # capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
-    "prefill_h16_n4096": 18_156_800 + 4_096,
-    "prefill_gqa_n32768": 158_131_456 + 218_139_648,
-    "mixed_prefill_n16384": 186_571_264 + 95_679_232,
+    "prefill_h16_n4096": None,
+    "prefill_gqa_n32768": 134_921_984 + 214_016_512,
+    "mixed_prefill_n16384": 186_574_080 + 80_747_008,
     "paged_decode_s64": 2_170_382_000 + 13_552_384,
 }
 KERNEL_TIMING = "CUDA graph of the kernel(s) alone, replayed after a 256 MB L2 flush, CUDA events"

@@ -371,6 +371,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 0) {
     // ================================ producer ================================
     if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); }
+    // Q is read once per item: its codes load evict-first, so that L2 keeps K and V, which
+    // every query tile of the head reads again.
+    const uint64_t once = kL2EvictFirst;
     int g = 0, q_issued = 0, k_issued = 0, v_issued = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
@@ -402,9 +405,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) {
           constexpr bool dual = kDQ;
           mbar_arrive_expect_tx(q_full + qb, L::Q_BYTES * (dual ? 2 : 1));
-          tma_load_3d(sm + L::OFF_Q + qb * L::Q_BYTES, &tm_q, q_full + qb, 0, w.qt * 128, w.bhq);
+          tma_load_3d_hint(sm + L::OFF_Q + qb * L::Q_BYTES, &tm_q, q_full + qb, 0, w.qt * 128, w.bhq, once);
           // (without FP16 tiles the FP16-Q map slot carries the second Q tensor's map)
-          if (dual) tma_load_3d(sm + L::OFF_Q2 + qb * L::Q_BYTES, &tm_q16, q_full + qb, 0, w.qt * 128, w.bhq);
+          if (dual) tma_load_3d_hint(sm + L::OFF_Q2 + qb * L::Q_BYTES, &tm_q16, q_full + qb, 0, w.qt * 128, w.bhq, once);
         }
         q_issued = it + 1;
       }
@@ -432,6 +435,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // The FP16 Q of an item and the FP16 K / V of each selected tile, on a warp of their own
     // so that the FP4 producer never waits for the single FP16 operand buffer to drain.
     if (lane == 0) { prefetch_tmap(&tm_q16); prefetch_tmap(&tm_k16); prefetch_tmap(&tm_v16); }
+    const uint64_t once = kL2EvictFirst;             // FP16 Q: read once per item
     int g = 0, n16 = 0, nq16 = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
@@ -448,7 +452,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (lane == 0) {
             mbar_arrive_expect_tx(q16_full, L::F16_TILE);
             for (int h = 0; h < D / 64; ++h)
-              tma_load_3d(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, w.qt * 128, w.bhq);
+              tma_load_3d_hint(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, w.qt * 128, w.bhq, once);
           }
           q16_loaded = true;
           ++nq16;
@@ -828,6 +832,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const float inv_l = __frcp_rn(l_run);     // O / l by Markstein's division (ptx.cuh)
         const bool store = qi < a.Nq;
         const int64_t orow = static_cast<int64_t>(w.bhq) * a.Nq + qi;
+        // O is written once: streaming (evict-first) stores keep K and V in L2
 #pragma unroll
         for (int cc = 0; cc < D / 2; cc += 32) {
           const int c = grp * (D / 2) + cc;
@@ -841,7 +846,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (a.out_kind == 2) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow * D + c);
 #pragma unroll
-              for (int k = 0; k < 8; ++k) dst[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+              for (int k = 0; k < 8; ++k) __stcs(dst + k, make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
             } else {
               __align__(16) uint32_t packed[16];
 #pragma unroll
@@ -856,7 +861,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               }
               uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow * D + c);
 #pragma unroll
-              for (int k = 0; k < 4; ++k) dst[k] = reinterpret_cast<uint4*>(packed)[k];
+              for (int k = 0; k < 4; ++k) __stcs(dst + k, reinterpret_cast<uint4*>(packed)[k]);
             }
           }
         }

@@ -156,6 +156,20 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
         "r"(x), "r"(y), "r"(z) : "memory");
 }
+// The same loads with an L2 eviction-priority policy (the .L2::cache_hint operand).
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(x), "r"(y), "r"(z), "l"(policy) : "memory");
+}
+// L2 eviction priority "evict first" as a cache-policy word (the value CUTLASS's SM90/SM100
+// TMA copies pass for it), for data that is read once: its lines leave L2 before any
+// others, so operands that are read again (K and V of a head, re-read by every query tile)
+// stay.
+constexpr uint64_t kL2EvictFirst = 0x12F0000000000000ull;
 // 4-byte asynchronous global -> shared copy (zero-filled when `valid` is false).
 __device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
