@@ -88,7 +88,6 @@ SIGNATURES = {
     "qk4v8_timeout_site": (C.c_uint64, []),
     "qk4v8_selftest_wait_timeout": (i32, [vp]),
     "qk4v8_selftest_device_once": (i32, [i32]),
-    "qk4v8_selftest_exp2": (i32, [vp, vp, i32, vp]),
     "quantize_nvfp4_workspace_size": (sz, []),
     "quantize_nvfp4": (i32, [vp, i32, i64, i32, i64, f32, vp, vp, vp, vp, vp, sz, vp]),
     "quantize_mxfp8_v": (i32, [vp, i32, i32, i32, i32, vp, vp, vp, vp]),

@@ -116,17 +116,6 @@ def timeout_site() -> dict | None:
             "barrier": (v >> 40) & 0xFF, "tile": (v >> 20) & 0xFFFFF, "block": v & 0xFFFFF}
 
 
-def selftest_exp2(t: torch.Tensor) -> torch.Tensor:
-    """2^t by the prefill kernel's FMA-pipe exponential (float32 CUDA tensor, even length)."""
-    t = t.contiguous()
-    if t.dtype != torch.float32 or not t.is_cuda or t.numel() % 2:
-        raise ValueError("t must be an even-length float32 CUDA tensor")
-    out = torch.empty_like(t)
-    _lib.check(_lib.load().qk4v8_selftest_exp2(t.data_ptr(), out.data_ptr(), t.numel(), _stream()),
-               "qk4v8_selftest_exp2")
-    return out
-
-
 def selftest_wait_timeout() -> None:
     """Launch the bounded-wait self-test kernel (times out after about a second)."""
     _lib.check(_lib.load().qk4v8_selftest_wait_timeout(_stream()), "qk4v8_selftest_wait_timeout")

@@ -53,9 +53,11 @@ namespace qk4v8 {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(448)
-// The exponentials all run on the special-function unit: moving a share to the FMA pipe
-// (exp2_poly2) measured slower on B200 for this kernel's instruction mix (2/8 of them: 2 to
-// 10 % slower) — the extra FMA-pipe instructions cost more issue slots than the unit saves.
+// The exponentials all run on the special-function unit. Evaluating a share of them as
+// 2^n p(t - n) on the FMA pipe measured slower on B200 for every share from 1/4 to 1/2 of
+// them (3 to 13 %): the extra FMA-pipe and ALU instructions cost more issue slots than the
+// unit saves, and a degree-3 p (7.5e-5) flips enough E4M3 codes to fail parity on short
+// causal rows. ex2.approx.f16x2 gives no more results per cycle than the f32 form.
 
 struct FwdArgs {
   const uint8_t* q_scales;

@@ -398,37 +398,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^t for a pair on the FMA pipe, so that part of the softmax's exponentials leave the
-// special-function unit (its throughput bounds the prefill kernel): 2^t = 2^n p(t - n) with
-// n = round(t) (by the 1.5 * 2^23 rounding constant) and p a degree-5 polynomial for 2^f on
-// [-1/2, 1/2] fitted for relative error (a Lawson-weighted least-squares fit made for this kernel: 1.5e-7 with fp32 coefficients). The
-// scale 2^n is added to the exponent field. t is clamped below at -30 (2^-30 is below every
-// E4M3 and FP16 code this feeds); t must not exceed 127.
-__device__ __forceinline__ float2 exp2_poly2(float2 t) {
-  t.x = fmaxf(t.x, -30.f);
-  t.y = fmaxf(t.y, -30.f);
-  const float2 y = __fadd2_rn(t, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(y, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), t);
-  float2 p = __ffma2_rn(make_float2(0.0013276470126584172f, 0.0013276470126584172f), f,
-                        make_float2(0.009675540961325169f, 0.009675540961325169f));
-  p = __ffma2_rn(p, f, make_float2(0.05550713464617729f, 0.05550713464617729f));
-  p = __ffma2_rn(p, f, make_float2(0.24022120237350464f, 0.24022120237350464f));
-  p = __ffma2_rn(p, f, make_float2(0.6931469440460205f, 0.6931469440460205f));
-  p = __ffma2_rn(p, f, make_float2(1.0000001192092896f, 1.0000001192092896f));
-  // y holds 1.5 * 2^23 + n: its low bits are n in two's complement, so y << 23 is n << 23.
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23)));
-}
-__global__ void exp2_selftest_kernel(const float* t, float* out, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    const float2 r = exp2_poly2(make_float2(t[i], t[i + 1]));
-    out[i] = r.x;
-    out[i + 1] = r.y;
-  }
-}
-
 // Self-test of the bounded-wait path: one warp waits on a barrier that nothing arrives at.
 // The wait gives up after its time limit, records its site and the timeout status, and the
 // kernel returns normally.

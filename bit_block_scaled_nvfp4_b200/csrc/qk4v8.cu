@@ -152,13 +152,6 @@ uint64_t qk4v8_timeout_site(void) {
   return site;
 }
 
-qk4v8_status qk4v8_selftest_exp2(const float* t, float* out, int32_t n, cudaStream_t stream) {
-  if (t == nullptr || out == nullptr || n < 0 || (n & 1)) return QK4V8_ERR_INVALID_ARG;
-  if (n == 0) return QK4V8_OK;
-  exp2_selftest_kernel<<<(n / 2 + 255) / 256, 256, 0, stream>>>(t, out, n);
-  return launch_status();
-}
-
 int32_t qk4v8_selftest_device_once(int32_t dev) {
   static PerDeviceOnce latch;
   static int32_t runs[kMaxDevices] = {};

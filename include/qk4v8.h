@@ -88,15 +88,6 @@ int32_t qk4v8_selftest_device_once(int32_t dev);
 qk4v8_status qk4v8_selftest_wait_timeout(cudaStream_t stream);
 
 /*
- * Accuracy self-test of the exponential the prefill kernel evaluates on the FMA pipe for part
- * of its scores (no counterpart in the method's description: an implementation detail of the
- * softmax step, 448 p = 2^t). t and out: device float arrays of n elements (n even); out[i]
- * = 2^t[i] (t clamped below at -30). Errors: QK4V8_ERR_INVALID_ARG for null pointers, n < 0 or
- * odd n. Asynchronous on `stream`.
- */
-qk4v8_status qk4v8_selftest_exp2(const float* t, float* out, int32_t n, cudaStream_t stream);
-
-/*
  * quantize_nvfp4 — NVFP4 quantization of Q or K (tqpw.cn article §2.2: E2M1 elements, E4M3
  * scale per 16 elements, FP32 tensor scale). Per call:
  *   s_t = fl32(amax / 2688) over all of x (2688 = 6 * 448; s_t = 1 when amax is 0), or
