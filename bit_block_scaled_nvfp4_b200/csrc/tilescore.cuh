@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kSelectThreads) tile_select_kernel(
   // --- radix select the k-th largest score (tau) -------------------------------------
   U128 pre{0, 0};
   uint32_t k_rem = static_cast<uint32_t>(k);
+  const int lane = tid & 31;
   // Row norms are below 2^51, so scores are below 2^102: bytes 13-15 are always zero.
   if (k > 0) {
     for (int p = 12; p >= 0; --p) {
@@ -146,7 +147,6 @@ __global__ void __launch_bounds__(kSelectThreads) tile_select_kernel(
       // Warp per query-tile row, lanes over key tiles (no index division). Lanes with the
       // same digit add once per warp (most scores share their high bytes, and one shared-
       // memory atomic per candidate would serialise on a few bins).
-      const int lane = tid & 31;
       for (int qt = tid >> 5; qt < Tq; qt += kSelectThreads / 32) {
         const uint64_t a = mq[qt];
         const int kt_end = causal ? min(qt + 1, Tk) : Tk;
@@ -162,15 +162,25 @@ __global__ void __launch_bounds__(kSelectThreads) tile_select_kernel(
         }
       }
       __syncthreads();
-      if (tid == 0) {
-        uint32_t above = 0;
-        int bin = 255;
-        for (; bin > 0; --bin) {
-          if (above + hist[bin] >= k_rem) break;
-          above += hist[bin];
+      // The digit of the k_rem-th largest: the first bin from the top whose running count
+      // reaches k_rem (bin 0 if none does). Thread t holds bin 255 - t; an inclusive scan over
+      // the 256 bins in that order gives each bin its count from the top.
+      if (tid < 256) {
+        const uint32_t h = hist[255 - tid];
+        uint32_t incl = h;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t up = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += up;
         }
-        s_bin = static_cast<uint32_t>(bin);
-        s_above = above;
+        if (lane == 31) warp_tot[tid >> 5] = incl;
+        named_bar_sync(1, 256);
+        for (int w2 = 0; w2 < (tid >> 5); ++w2) incl += warp_tot[w2];
+        const uint32_t before = incl - h;
+        if ((incl >= k_rem || tid == 255) && before < k_rem) {
+          s_bin = static_cast<uint32_t>(255 - tid);
+          s_above = before;
+        }
       }
       __syncthreads();
       const uint32_t bin = s_bin;
@@ -200,12 +210,18 @@ __global__ void __launch_bounds__(kSelectThreads) tile_select_kernel(
       }
       // ordered compaction of the ties (block-wide exclusive scan)
       const unsigned bal = __ballot_sync(0xffffffffu, eq);
-      const int lane = tid & 31, w = tid >> 5;
+      const int w = tid >> 5;
       if (lane == 0) warp_tot[w] = __popc(bal);
       __syncthreads();
-      if (tid == 0) {
-        uint32_t run = 0;
-        for (int i = 0; i < kSelectThreads / 32; ++i) { const uint32_t t = warp_tot[i]; warp_tot[i] = run; run += t; }
+      if (w == 0) {                    // exclusive scan of the 32 warp counts
+        const uint32_t t = warp_tot[lane];
+        uint32_t incl = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t up = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += up;
+        }
+        warp_tot[lane] = incl - t;
       }
       __syncthreads();
       const uint32_t eq_rank = s_cnt_eq + warp_tot[w] + __popc(bal & ((1u << lane) - 1u));
