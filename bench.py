@@ -42,7 +42,7 @@ METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of H
 # kernel on the workload (dram__bytes_read.sum + dram__bytes_write.sum). Only workloads with a
 # capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
-    "prefill_h16_n4096": None,
+    "prefill_h16_n4096": 18_159_616 + 6_656,
     "prefill_gqa_n32768": 134_921_984 + 214_016_512,
     "mixed_prefill_n16384": 186_574_080 + 80_747_008,
     "paged_decode_s64": 2_170_382_000 + 13_552_384,
