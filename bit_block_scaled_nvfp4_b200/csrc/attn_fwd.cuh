@@ -11,13 +11,15 @@
 //
 // l comes from the tensor core: every V tile in shared memory carries 16 extra rows of 1.0
 // after its D channel rows, so the PV MMA (N = D + 16) accumulates sum_j P_j into O column D,
-// with the same rescaling as O.
+// with the same rescaling as O (an FP16 tile's PV adds a second MMA of N = 16 over a constant
+// block of FP16 ones).
 //
 // Persistent: one CTA per SM walks a list of work items (128-query tile, batch, query head),
 // heaviest causal items first, dealt to the CTAs in a zigzag so their loads even out. All
-// pipelines run on across items (a CTA-wide key-tile counter g numbers the stages and
-// buffers), so the next item's Q, K and V loads and its first QK^T overlap the current
-// item's last tiles and epilogue; Q has two buffers.
+// pipelines run on across items (a CTA-wide key-tile counter g numbers the S, P and scale
+// buffers, and a stage counter the K/V ring, where a selected FP16 tile takes two stages), so
+// the next item's Q, K and V loads and its first QK^T overlap the current item's last tiles
+// and epilogue; Q has two buffers.
 //
 // Softmax in two groups by the parity of g. Group 0 (warps 4-7) and group 1 (warps 8-11);
 // each thread owns one query row and all 128 keys of its tile. The groups hand the running max
@@ -33,10 +35,11 @@
 //
 // Warp roles:
 //   warp 0     producer: TMA of Q/K/V code tiles (swizzled), scale factors gathered into the
-//              tcgen05 scale layout with 4-byte asynchronous copies
+//              tcgen05 scale layout with 4-byte asynchronous copies; a selected tile's FP16 K
+//              and V into two ring stages
 //   warp 1     TMEM owner and QK^T issuer (one thread)
 //   warp 2     PV issuer (one thread)
-//   warp 3     FP16 operand producer (FP16-tile kernel only)
+//   warp 3     FP16 Q producer (FP16-tile kernel only)
 //   warps 4-11 softmax (two groups of four; warp w reaches TMEM lane quadrant w % 4)
 // TMEM (512 columns): S_0, S_1 [0,256), O (D + 16 columns) from 256, scale factors from 400.
 //
@@ -98,15 +101,14 @@ __device__ __forceinline__ int fwd_item_index(int it, int G, int c) {
 
 template <int D, bool kMixed, bool kDQ = false>
 struct FwdLayout {
-  // K and V stages. In the FP16-tile kernel, whose FP16 operands take 100 KB, K and V form
-  // rings of their own (three K, two V stages): a K stage is free once QK^T of its tile is
-  // done, a V stage only once PV is, so K runs ahead. Otherwise stage s of both arrays is one
-  // stage of a single ring of four (one full and one empty barrier), which measured faster:
-  // with K running ahead the two softmax groups fall into step and contend for the
-  // exponential unit at the same time.
-  static constexpr bool kSplit = kMixed;
-  static constexpr int NK = kMixed ? 3 : 4;
-  static constexpr int NVS = kMixed ? 2 : 4;
+  // K and V stages: one ring of four, stage s holding key tile g's K and V (one full and one
+  // empty barrier). Separate K and V rings, which let K run ahead, measured slower: the two
+  // softmax groups fall into step and contend for the exponential unit at the same time. In
+  // the FP16-tile kernel a selected tile takes two consecutive stages, its FP16 K in the first
+  // and its FP16 V in the second, so a stage is large enough for either.
+  static constexpr bool kSplit = false;
+  static constexpr int NK = 4;
+  static constexpr int NVS = 4;
   // P buffers, one per tile parity: the exponentials of tile g wait for PV(g - 2).
   static constexpr int NP = 2;
   static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
@@ -118,15 +120,16 @@ struct FwdLayout {
   static constexpr int OFF_Q = 0;                                         // 2 buffers
   static constexpr int OFF_QSF = OFF_Q + 2 * Q_BYTES;                     // 2 x KSTEPS chunks
   static constexpr int OFF_PSF = OFF_QSF + 2048;                          // all 1.0 (E8M0 127)
-  // Stage s of K and of V: with rings of equal depth, one block [K | V (+ ones rows) | K scales
-  // | V scales] per s (measured faster than two separate arrays); otherwise K blocks
-  // [K | K scales] followed by V blocks [V | V scales].
-  static constexpr bool kInterleaved = (NK == NVS);
+  // Stage s: one block [K | V (+ ones rows) | K scales | V scales] (measured faster than
+  // separate K and V arrays).
+  static constexpr bool kInterleaved = true;
   // P scale factors of the underflow-aware variant, two chunks by tile parity (row r's four
   // 32-key block scales in the word at (r % 32) * 16 + (r / 32) * 4)
   static constexpr int OFF_PSFU = OFF_PSF + 1024;
   static constexpr int OFF_STG = OFF_PSFU + 1024;
-  static constexpr int STG_BYTES = K_BYTES + V_BYTES + 2048;
+  static constexpr int F16_TILE = 128 * D * 2;     // FP16 Q, K or V (no ones rows) of a tile
+  static constexpr int STG_FP4 = K_BYTES + V_BYTES + 2048;
+  static constexpr int STG_BYTES = (kMixed && F16_TILE > STG_FP4) ? F16_TILE : STG_FP4;
   static constexpr int OFF_VSTG = OFF_STG + NK * (K_BYTES + 1024);
   __device__ static constexpr int k_off(int s) {
     return kInterleaved ? OFF_STG + s * STG_BYTES : OFF_STG + s * (K_BYTES + 1024);
@@ -144,20 +147,22 @@ struct FwdLayout {
                                             : OFF_VSTG + NVS * (V_BYTES + 1024);  // NP x 16 KB
   static constexpr int OFF_RED = OFF_P + NP * 16384;   // running max hand-off [2][128], final [128]
   static constexpr int OFF_Q16 = OFF_RED + 2048;
-  static constexpr int F16_TILE = 128 * D * 2;
-  static constexpr int V16_ATOM = NV * 128;                                // 64 keys x NV rows
-  static constexpr int OFF_K16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
-  static constexpr int OFF_V16 = OFF_K16 + (kMixed ? F16_TILE : 0);
+  // The FP16 PV's ones rows (the row sum l in column D of O): 16 rows of 1.0 for each 64-key
+  // atom, read by a second MMA of N = 16 (an FP16 V in a ring stage has no ones rows).
+  static constexpr int OFF_ONES16 = OFF_Q16 + (kMixed ? F16_TILE : 0);
+  static constexpr int V16_ATOM = D * 128;                                 // 64 keys x D rows
   // second Q tensor of dual-residual query quantization (its own instance): two buffers by
   // item parity and their scale factors
-  static constexpr int OFF_Q2 = OFF_V16 + (kMixed ? 2 * V16_ATOM : 0);
+  static constexpr int OFF_Q2 = OFF_ONES16 + (kMixed ? 2 * 2048 : 0);
   static constexpr int OFF_Q2SF = OFF_Q2 + (kDQ ? 2 * Q_BYTES : 0);
   static constexpr int OFF_BAR = OFF_Q2SF + (kDQ ? 2048 : 0);
   static constexpr int N_BARS = 2 * NK + 2 * NVS + 2 * NP + 17;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
-  static_assert(kSplit || NK == NVS, "a single ring has one stage count");
+  static_assert(NK == NVS, "a single ring has one stage count");
+  static_assert(STG_BYTES % 1024 == 0 && OFF_STG % 1024 == 0 && OFF_Q16 % 1024 == 0 &&
+                OFF_ONES16 % 1024 == 0, "1024-byte aligned operand atoms");
   // TMEM columns. S_b at T_S + 128 b; Q scale factors in two slots by item parity, K and V
   // scale factors in two slots by tile parity (8 columns each: a slot is rewritten only after
   // the MMA two items / tiles back that read it has completed).
@@ -201,8 +206,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* s_free = s_full + 2;           // [2], by tile parity
   uint64_t* m_ready = s_full + 4;          // [2], by tile parity: running max handed on
   uint64_t* o_free = s_full + 6;           // the epilogue has read O
-  uint64_t* kv16_full = s_full + 7;
-  uint64_t* kv16_empty = s_full + 8;
   uint64_t* q16_full = s_full + 9;
   uint64_t* q16_empty = s_full + 10;
   uint64_t* mma_final = s_full + 11;       // [2]: QK issuer, PV issuer
@@ -233,7 +236,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int i = 0; i < L::NP; ++i) { mbar_init(p_full + i, 4); mbar_init(pv_done + i, 1); }
     mbar_init(o_free, 8);
-    mbar_init(kv16_full, 1); mbar_init(kv16_empty, 1);
     mbar_init(q16_full, 1); mbar_init(q16_empty, 1);
     mbar_init(mma_final, 1); mbar_init(mma_final + 1, 1);
     *abort_flag = 0;
@@ -255,10 +257,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           reinterpret_cast<uint32_t*>(sm + L::v_sf_off(s))[i] = 0x7F7F7F7Fu;
   }
   if constexpr (kMixed) {
-    for (int h = 0; h < 2; ++h)
-      for (int i = threadIdx.x; i < 16 * 128 / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(sm + L::OFF_V16 + h * L::V16_ATOM + D * 128)[i] =
-            make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+    for (int i = threadIdx.x; i < 2 * 2048 / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(sm + L::OFF_ONES16)[i] =
+          make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
   }
   fence_proxy_async_smem();
   if (warp == 1) {
@@ -289,55 +290,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // r0*16 + r1*4; one 4-byte word holds the 4 scales of one 64-element MMA step, or the 4
   // E8M0 scales of a V channel row), completing on the same barrier as the TMA of the codes,
   // so the producer never waits on their latency.
-  auto load_k = [&](int g, int j, const FwdItem& w) -> bool {
-    const int s = g % L::NK;
-    if (g >= L::NK && !waitw(k_empty + s, ((g / L::NK) - 1) & 1, g)) return false;
-    unsigned char* st = sm + L::k_off(s);
-    unsigned char* sf = sm + L::k_sf_off(s);
-    const int64_t krow0 = static_cast<int64_t>(w.bhk) * a.Nk + j * 128;
-#pragma unroll
-    for (int r1 = 0; r1 < 4; ++r1) {
-      const int r = r1 * 32 + lane;
-      const bool valid = j * 128 + r < a.Nk;             // rows past Nk read as zero
-      const uint8_t* src = a.k_scales + (valid ? (krow0 + r) * (D / 16) : 0);
-#pragma unroll
-      for (int kk = 0; kk < L::KSTEPS; ++kk)
-        cp_async4(sf + kk * 512 + lane * 16 + r1 * 4, src + kk * 4, valid);
-    }
-    cp_async_arrive_noinc(k_full + s);
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive_expect_tx(k_full + s, L::K_BYTES);
-      tma_load_3d(st, &tm_k, k_full + s, 0, j * 128, w.bhk);
-    }
-    return true;
-  };
-  auto load_v = [&](int g, int j, const FwdItem& w) -> bool {
-    const int s = g % L::NVS;
-    if (g >= L::NVS && !waitw(v_empty + s, ((g / L::NVS) - 1) & 1, g)) return false;
-    unsigned char* st = sm + L::v_off(s);
-    unsigned char* sf = sm + L::v_sf_off(s);
-    // rows from D on (the ones rows) hold 1.0 set once at start
-#pragma unroll
-    for (int r1 = 0; r1 < 4; ++r1) {
-      const int r = r1 * 32 + lane;
-      if (r < D)
-        cp_async4(sf + lane * 16 + r1 * 4,
-                  a.v_scales + (static_cast<int64_t>(w.bhk) * D + r) * (a.Npad / 32) + j * 4, true);
-    }
-    cp_async_arrive_noinc(v_full + s);
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive_expect_tx(v_full + s, L::V_TMA_BYTES);
-      tma_load_2d(st, &tm_v, v_full + s, j * 128, w.bhk * D);
-    }
-    return true;
-  };
   // Both halves of a single-ring stage with one arrival per lane and one TMA transaction count
   // (measured faster than two arrivals on the same barrier).
-  auto load_kv = [&](int g, int j, const FwdItem& w) -> bool {
-    const int s = g % L::NK;
-    if (g >= L::NK && !waitw(k_empty + s, ((g / L::NK) - 1) & 1, g)) return false;
+  // r is the stage counter (ring position), g the tile counter (for timeout reports).
+  // dirty: stages whose constant rows an FP16 tile's K or V overwrote.
+  uint32_t dirty = 0;
+  auto load_kv = [&](int r, int g, int j, const FwdItem& w) -> bool {
+    const int s = r % L::NK;
+    if (r >= L::NK && !waitw(k_empty + s, ((r / L::NK) - 1) & 1, g)) return false;
+    if (kMixed && ((dirty >> s) & 1u)) {
+      // the ones rows after V (E4M3 1.0) and, at D < 128, the unused V scale rows (1.0)
+      uint4* ones = reinterpret_cast<uint4*>(sm + L::v_off(s) + L::V_TMA_BYTES);
+      for (int i = lane; i < 16 * 128 / 16; i += 32)
+        ones[i] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+      if constexpr (D < 128)
+        for (int i = lane; i < 128; i += 32)
+          if (((i >> 2) & 31) + 32 * (i & 3) >= D)
+            reinterpret_cast<uint32_t*>(sm + L::v_sf_off(s))[i] = 0x7F7F7F7Fu;
+      fence_proxy_async_smem();
+      dirty &= ~(1u << s);
+    }
     unsigned char* ksf = sm + L::k_sf_off(s);
     unsigned char* vsf = sm + L::v_sf_off(s);
     const int64_t krow0 = static_cast<int64_t>(w.bhk) * a.Nk + j * 128;
@@ -362,7 +334,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     return true;
   };
-  // Drain of a ring: wait for the last copy issued into each stage (n = tiles issued).
+  // Half of a selected tile in the FP16-tile kernel: its FP16 K (two 64-channel atoms) or its
+  // FP16 V (two 64-key atoms of D rows) into stage r. Only one issuer reads each half, so the
+  // producer arrives on the stage's empty barrier for the other (after it saw the stage's
+  // previous use released, so the arrival counts toward this use).
+  auto load_f16 = [&](int r, int g, int j, const FwdItem& w, bool v) -> bool {
+    const int s = r % L::NK;
+    if (r >= L::NK && !waitw(k_empty + s, ((r / L::NK) - 1) & 1, g)) return false;
+    dirty |= 1u << s;
+    mbar_arrive(k_full + s);                     // the 32 lane arrivals of the full barrier
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(k_full + s, L::F16_TILE);
+      unsigned char* st = sm + L::k_off(s);
+      if (!v) {
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(st + h * 16384, &tm_k16, k_full + s, h * 64, j * 128, w.bhk);
+      } else {
+        for (int h = 0; h < 2; ++h)
+          tma_load_2d(st + h * L::V16_ATOM, &tm_v16, k_full + s, j * 128 + h * 64, w.bhk * D);
+      }
+      mbar_arrive(k_empty + s);
+    }
+    return true;
+  };
+  // Drain of a ring: wait for the last copy issued into each stage (n = stages issued).
   auto drain = [&](uint64_t* full, int n_stages, int n) {
     for (int s = 0; s < n_stages && s < n; ++s) {
       const int last = s + ((n - 1 - s) / n_stages) * n_stages;
@@ -376,12 +372,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // Q is read once per item: its codes load evict-first, so that L2 keeps K and V, which
     // every query tile of the head reads again.
     const uint64_t once = kL2EvictFirst;
-    int g = 0, q_issued = 0, k_issued = 0, v_issued = 0;
+    int g = 0, r = 0, q_issued = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const int idx = fwd_item_index(it, G, cta);
       if (idx >= n_items) break;
       const FwdItem w = fwd_item(a, idx);
+      const uint8_t* bm_row = kMixed ? a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk : nullptr;
       const int qb = it & 1;
       // Q buffer qb was last read by the QK^T MMAs of item it - 2.
       if (it >= 2 && !waitw(q_empty + qb, ((it - 2) >> 1) & 1, g)) { ok = false; break; }
@@ -414,31 +411,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         q_issued = it + 1;
       }
       for (int j = 0; j < w.nt; ++j, ++g) {
-        if constexpr (L::kSplit) {
-          if (!load_k(g, j, w)) { ok = false; break; }
-          k_issued = g + 1;
-          if (!load_v(g, j, w)) { ok = false; break; }
-          v_issued = g + 1;
+        if (kMixed && bm_row[j]) {
+          if (!load_f16(r, g, j, w, false)) { ok = false; break; }
+          ++r;
+          if (!load_f16(r, g, j, w, true)) { ok = false; break; }
+          ++r;
         } else {
-          if (!load_kv(g, j, w)) { ok = false; break; }
-          k_issued = g + 1;
+          if (!load_kv(r, g, j, w)) { ok = false; break; }
+          ++r;
         }
       }
     }
     // Drain: never leave a copy in flight into this CTA's shared memory.
-    drain(k_full, L::NK, k_issued);
-    drain(v_full, L::NVS, v_issued);
+    drain(k_full, L::NK, r);
     for (int qb = 0; qb < 2 && qb < q_issued; ++qb) {
       const int last = qb + ((q_issued - 1 - qb) / 2) * 2;
       mbar_wait(q_full + qb, (last >> 1) & 1);
     }
   } else if (kMixed && warp == 3) {
-    // ========================== FP16 operand producer ==========================
-    // The FP16 Q of an item and the FP16 K / V of each selected tile, on a warp of their own
-    // so that the FP4 producer never waits for the single FP16 operand buffer to drain.
+    // ============================== FP16 Q producer ==============================
+    // The FP16 Q of each item with a selected tile, on a warp of its own so that the producer
+    // never waits for the single FP16 Q buffer to drain (the selected tiles' FP16 K and V come
+    // through the ring).
     if (lane == 0) { prefetch_tmap(&tm_q16); prefetch_tmap(&tm_k16); prefetch_tmap(&tm_v16); }
     const uint64_t once = kL2EvictFirst;             // FP16 Q: read once per item
-    int g = 0, n16 = 0, nq16 = 0;
+    int g = 0, nq16 = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
       const int idx = fwd_item_index(it, G, cta);
@@ -446,32 +443,21 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const FwdItem w = fwd_item(a, idx);
       const uint8_t* bm_row = a.bitmap + (static_cast<int64_t>(w.bhq) * a.Tq + w.qt) * a.Tk;
       bool q16_loaded = false;
-      for (int j = 0; j < w.nt; ++j, ++g) {
+      for (int j = 0; j < w.nt && !q16_loaded; ++j) {
         if (!bm_row[j]) continue;
-        if (!q16_loaded) {
-          // the single FP16 Q buffer was last read by the FP16 QK^Ts of an earlier item
-          if (nq16 >= 1 && !waitw(q16_empty, (nq16 - 1) & 1, g)) { ok = false; break; }
-          if (lane == 0) {
-            mbar_arrive_expect_tx(q16_full, L::F16_TILE);
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_3d_hint(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, w.qt * 128, w.bhq, once);
-          }
-          q16_loaded = true;
-          ++nq16;
-        }
-        if (n16 >= 1 && !waitw(kv16_empty, (n16 - 1) & 1, g)) { ok = false; break; }
+        // the single FP16 Q buffer was last read by the FP16 QK^Ts of an earlier item
+        if (nq16 >= 1 && !waitw(q16_empty, (nq16 - 1) & 1, g + j)) { ok = false; break; }
         if (lane == 0) {
-          mbar_arrive_expect_tx(kv16_full, L::F16_TILE + 2 * D * 128);
+          mbar_arrive_expect_tx(q16_full, L::F16_TILE);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_3d(sm + L::OFF_K16 + h * 16384, &tm_k16, kv16_full, h * 64, j * 128, w.bhk);
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d(sm + L::OFF_V16 + h * L::V16_ATOM, &tm_v16, kv16_full, j * 128 + h * 64, w.bhk * D);
+            tma_load_3d_hint(sm + L::OFF_Q16 + h * 16384, &tm_q16, q16_full, h * 64, w.qt * 128, w.bhq, once);
         }
-        ++n16;
+        q16_loaded = true;
+        ++nq16;
       }
+      g += w.nt;
     }
     // Drain: never leave a copy in flight into this CTA's shared memory.
-    if (n16 > 0) mbar_wait(kv16_full, (n16 - 1) & 1);
     if (nq16 > 0) mbar_wait(q16_full, (nq16 - 1) & 1);
   } else if (warp == 1) {
     // ============================ QK^T issuer (one thread) ============================
@@ -479,7 +465,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, 128);
       const uint32_t idesc_qk16 = idesc_f16(128, 128);
       bool ok = true;
-      int g = 0, n16 = 0, nq16 = 0;
+      int g = 0, r = 0, nq16 = 0;
       for (int it = 0; ok; ++it) {
         const int idx = fwd_item_index(it, G, cta);
         if (idx >= n_items) break;
@@ -506,9 +492,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t sQ2 = smem_u32(sm + L::OFF_Q2 + qb * L::Q_BYTES);
         bool q16_ready = false, had16 = false;
         for (int j = 0; j < w.nt; ++j, ++g) {
-          const int s = g % L::NK;
+          // tile j's stage: its K and V, or (selected tile) its FP16 K; the FP16 V in the next
+          const int s = r % L::NK;
           const bool f16 = kMixed && bm_row[j];
-          if (!wait1(k_full + s, (g / L::NK) & 1, g)) { ok = false; break; }
+          if (!wait1(k_full + s, (r / L::NK) & 1, g)) { ok = false; break; }
+          r += f16 ? 2 : 1;
           fence_proxy_async_smem();
           // S_{g&1} (and K scale slot g&1) were last used by tile g - 2
           if (g >= 2 && !wait1(s_free + (g & 1), ((g - 2) >> 1) & 1, g)) { ok = false; break; }
@@ -536,11 +524,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
               ++nq16;
               q16_ready = true;
             }
-            if (!wait1(kv16_full, n16 & 1, g)) { ok = false; break; }
             tc_fence_after();
-            ++n16;
             had16 = true;
-            const uint32_t sQ16 = smem_u32(sm + L::OFF_Q16), sK16 = smem_u32(sm + L::OFF_K16);
+            const uint32_t sQ16 = smem_u32(sm + L::OFF_Q16), sK16 = smem_u32(sm + L::k_off(s));
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t da = make_sdesc(sQ16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
               const uint64_t db = make_sdesc(sK16 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
@@ -549,6 +535,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
           mma_commit(s_full + (g & 1));
           mma_commit(k_empty + s);
+          if (f16) {
+            // The FP16 V went into the next stage, which this thread does not read. Waiting for
+            // it to land keeps this thread's next wait on that stage one phase after it (a parity
+            // wait cannot tell a phase from the one two later). The PV issuer, which skips the
+            // FP16 K's stage, needs no such wait: it reaches a later tile only after this tile's
+            // P, which follows the FP16 K's arrival.
+            const int rv = r - 1;
+            if (!wait1(k_full + rv % L::NK, (rv / L::NK) & 1, g)) { ok = false; break; }
+          }
         }
         if (!ok) break;
         mma_commit(q_empty + qb);                    // Q buffer qb is free
@@ -563,7 +558,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ============================== PV issuer (one thread) ==============================
     if (lane == 0) {
       const uint32_t idesc_pv = idesc_block_scaled(kFmtE4M3, kFmtE4M3, 1, 128, L::NV);
-      const uint32_t idesc_pv16 = idesc_f16(128, L::NV);
+      const uint32_t idesc_pv16 = idesc_f16(128, D);
+      const uint32_t idesc_l16 = idesc_f16(128, 16);
+      const uint32_t sOnes16 = smem_u32(sm + L::OFF_ONES16);
       const uint32_t sP = smem_u32(sm + L::OFF_P);
       const uint32_t tO = tbase + L::T_O;
       tc_fence_after();
@@ -571,7 +568,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int b2 = 0; b2 < 2; ++b2)               // second V scale chunk (rows 128..): 1.0
         tmem_cp_sf(tbase + L::T_VSF + 8 * b2 + 4, sm + L::OFF_PSF);
       bool ok = true;
-      int g = 0, n16 = 0;
+      int g = 0, r = 0;
       for (int it = 0; ok; ++it) {
         const int idx = fwd_item_index(it, G, cta);
         if (idx >= n_items) break;
@@ -580,11 +577,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // the first PV of an item overwrites O: the previous item's epilogue must have read it
         if (it >= 1 && !wait1(o_free, (it - 1) & 1, g)) { ok = false; break; }
         for (int j = 0; j < w.nt; ++j, ++g) {
-          const int s = g % L::NVS, b2 = g & 1, pb = g % L::NP;
           const bool f16 = kMixed && bm_row[j];
+          const int rv = f16 ? r + 1 : r;            // the stage holding this tile's V
+          r += f16 ? 2 : 1;
+          const int s = rv % L::NVS, b2 = g & 1, pb = g % L::NP;
           if (!wait1(p_full + pb, (g / L::NP) & 1, g)) { ok = false; break; }
-          if (!wait1(v_full + s, (g / L::NVS) & 1, g)) { ok = false; break; }
-          if (f16 && !wait1(kv16_full, n16 & 1, g)) { ok = false; break; }
+          if (!wait1(v_full + s, (rv / L::NVS) & 1, g)) { ok = false; break; }
           fence_proxy_async_smem();
           tc_fence_after();
           if (!f16) {
@@ -604,15 +602,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                        tv | (static_cast<uint32_t>(kk) << 30), (j > 0 || kk > 0) ? 1u : 0u);
             }
           } else {
-            ++n16;
-            const uint32_t sV16 = smem_u32(sm + L::OFF_V16);
+            // O[:, 0:D) += P V over the FP16 V in the stage; O[:, D:D+16) += P 1 (l in column D)
+            const uint32_t sV16 = smem_u32(sm + L::k_off(s));
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t da = make_sdesc(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSw128);
               const uint64_t db = make_sdesc(sV16 + (kk >> 2) * L::V16_ATOM + (kk & 3) * 32, 16, 1024, kSw128);
               mma_f16(tO, da, db, idesc_pv16, (j > 0 || kk > 0) ? 1u : 0u);
+              const uint64_t d1 = make_sdesc(sOnes16 + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, kSw128);
+              mma_f16(tO + D, da, d1, idesc_l16, (j > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(kv16_empty);
           }
           mma_commit(pv_done + pb);
           mma_commit(v_empty + s);
