@@ -175,14 +175,16 @@ def make_prefill_step(name):
 
     def quant(q=q, k=k, v=v):
         # Q, K (NVFP4) and V (MXFP8) in two launches: the amax pass of Q and K, then one encode
-        return api.quantize_qkv(q, k, v, want_fp16=mixed)
+        # (with FP16 tiles also V's fp16 copy; their Q and K are the inputs themselves)
+        return api.quantize_qkv(q, k, v, want_fp16_v=mixed)
 
     def step(q=q, k=k, v=v):
         q4, k4, v8 = quant(q, k, v)
         bitmap = None
         if mixed:
             _, _, bitmap = api.tile_score_select(q4, k4, cfg["causal"], cfg["frac_bp"])
-        return api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=bitmap)
+        return api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=bitmap,
+                                  q16=q if mixed else None, k16=k if mixed else None)
 
     prep = {}
 
@@ -197,7 +199,8 @@ def make_prefill_step(name):
     def attn_only():
         # the attention kernel alone
         q4, k4, v8 = prepared()["in"]
-        return api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=prep["bm"])
+        return api.attn_qk4v8_fwd(q4, k4, v8, cfg["causal"], scale, q.dtype, fp16_bitmap=prep["bm"],
+                                  q16=q if mixed else None, k16=k if mixed else None)
 
     def score_only():
         # tile scoring and top-fraction selection alone
@@ -207,9 +210,9 @@ def make_prefill_step(name):
     launches = 3 + (3 if mixed else 0)
     host = [w.q.pin_memory(), w.k.pin_memory(), w.v.pin_memory()]
     # algorithmic quantize bytes: bf16 read once, NVFP4 codes + E4M3 scales (Q, K) and MXFP8
-    # codes + E8M0 scales (V) written, plus the fp16 copies the FP16 tiles read
+    # codes + E8M0 scales (V) written, plus V's fp16 copy that the FP16 tiles read
     nq, nk, nv = q.numel(), k.numel(), v.numel()
-    qbytes = (nq + nk) * (2 + 0.5 + 1 / 16) + nv * (2 + 1 + 1 / 32) + (2 * (nq + nk + nv) if mixed else 0)
+    qbytes = (nq + nk) * (2 + 0.5 + 1 / 16) + nv * (2 + 1 + 1 / 32) + (2 * nv if mixed else 0)
     # algorithmic scoring bytes: the Q and K codes and E4M3 scales read once
     sbytes = (nq + nk) * (0.5 + 1 / 16)
     return dict(cfg=cfg, step=step, inputs=(q, k, v), host=host, launches=launches,

@@ -40,7 +40,7 @@ class FwdParams(C.Structure):
         ("head_dim", i32), ("causal", i32), ("softmax_scale", f32),
         ("fp16_bitmap", vp), ("q16", vp), ("k16", vp), ("v16", vp),
         ("out_dtype", i32), ("out", vp), ("lse", vp), ("p_underflow_aware", i32),
-        ("q2_codes", vp), ("q2_scales", vp),
+        ("q2_codes", vp), ("q2_scales", vp), ("qk16_dtype", i32),
     ]
 
 

@@ -193,11 +193,12 @@ def quantize_nvfp4_dual(x: torch.Tensor, tensor_scale: float | None = None):
     return q1, NVFP4Tensor(codes2, scales2, q1.tensor_scale)
 
 
-def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, want_fp16: bool = False,
+def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, want_fp16_v: bool = False,
                  workspace: torch.Tensor | None = None):
     """Q and K (..., D) to NVFP4 with their own tensor scales and V (..., N, D) to MXFP8, in two
     launches (quantize_qkv); the same outputs as quantize_nvfp4(q), quantize_nvfp4(k) and
-    quantize_mxfp8_v(v). Returns (q4, k4, v8)."""
+    quantize_mxfp8_v(v). ``want_fp16_v`` also writes V's fp16 copy (v8.fp16), the one 16-bit
+    operand the FP16-tile attention needs besides the caller's Q and K. Returns (q4, k4, v8)."""
     lib = _lib.load()
     for name, t in (("q", q), ("k", k), ("v", v)):
         if not t.is_cuda or not t.is_contiguous():
@@ -213,17 +214,16 @@ def quantize_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, want_fp16: b
     elif workspace.numel() < need or workspace.dtype != torch.uint8:
         raise ValueError(f"workspace must hold {need} bytes (uint8)")
     _on_one_gpu(q, k, v, workspace)
-    q4 = _nvfp4_empty(q.shape, q.device, want_fp16)
-    k4 = _nvfp4_empty(k.shape, k.device, want_fp16)
-    v8 = _mxfp8_empty(v.shape, v.device, want_fp16)
+    q4 = _nvfp4_empty(q.shape, q.device)
+    k4 = _nvfp4_empty(k.shape, k.device)
+    v8 = _mxfp8_empty(v.shape, v.device, want_fp16_v)
     n = v.shape[-2]
     p = _lib.QkvParams(
         q=_ptr(q), k=_ptr(k), v=_ptr(v), dtype=_dtype(q), head_dim=d,
         q_rows=q.numel() // d, k_rows=k.numel() // d, v_bh=v.numel() // (n * d), v_tokens=n,
         q_codes=_ptr(q4.codes), q_scales=_ptr(q4.scales), q_tensor_scale=_ptr(q4.tensor_scale),
         k_codes=_ptr(k4.codes), k_scales=_ptr(k4.scales), k_tensor_scale=_ptr(k4.tensor_scale),
-        v_codes=_ptr(v8.codes), v_scales=_ptr(v8.scales), q16=_ptr(q4.fp16), k16=_ptr(k4.fp16),
-        v16=_ptr(v8.fp16))
+        v_codes=_ptr(v8.codes), v_scales=_ptr(v8.scales), q16=None, k16=None, v16=_ptr(v8.fp16))
     _lib.check(lib.quantize_qkv(C.byref(p), _ptr(workspace), workspace.numel(), _stream()),
                "quantize_qkv")
     return q4, k4, v8
@@ -279,10 +279,13 @@ def tile_score_select(q: NVFP4Tensor, k: NVFP4Tensor, causal: bool, frac_bp: int
 def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
                    softmax_scale: float | None = None, out_dtype=torch.bfloat16,
                    fp16_bitmap: torch.Tensor | None = None, want_lse: bool = False,
-                   underflow_aware: bool = False, q2: NVFP4Tensor | None = None):
+                   underflow_aware: bool = False, q2: NVFP4Tensor | None = None,
+                   q16: torch.Tensor | None = None, k16: torch.Tensor | None = None):
     """QK4V8 attention forward. q.codes [B, Hq, Nq, D/2], k.codes [B, Hkv, Nk, D/2],
-    v.codes [B, Hkv, D, Nk_pad]. With ``fp16_bitmap`` the FP16 copies (q.fp16, k.fp16,
-    v.fp16) must be present. Returns out [B, Hq, Nq, D] (and lse [B, Hq, Nq])."""
+    v.codes [B, Hkv, D, Nk_pad]. With ``fp16_bitmap`` the selected tiles read the 16-bit Q and
+    K the codes were quantized from (``q16`` [B, Hq, Nq, D], ``k16`` [B, Hkv, Nk, D], fp16 or
+    bf16, one type) and V's fp16 copy (v.fp16, from quantize_qkv(want_fp16_v=True)).
+    Returns out [B, Hq, Nq, D] (and lse [B, Hq, Nq])."""
     _expect_dims(q.codes, "q.codes", 4, "[B, Hq, Nq, D/2]")
     _expect_dims(k.codes, "k.codes", 4, "[B, Hkv, Nk, D/2]")
     B, Hq, Nq, dh = q.codes.shape
@@ -304,10 +307,14 @@ def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
         tiles = B * Hq * ((Nq + 127) // 128) * ((Nk + 127) // 128)
         if fp16_bitmap.dtype != torch.uint8 or fp16_bitmap.numel() != tiles:
             raise ValueError(f"fp16_bitmap must hold {tiles} uint8 tile flags")
-        _expect(q.fp16, "q.fp16 (quantize with want_fp16=True)", (B, Hq, Nq, d), torch.float16)
-        _expect(k.fp16, "k.fp16 (quantize with want_fp16=True)", (B, Hkv, Nk, d), torch.float16)
-        _expect(v.fp16, "v.fp16 (quantize with want_fp16=True)", (B, Hkv, d, npad), torch.float16)
-        bufs += [fp16_bitmap, q.fp16, k.fp16, v.fp16]
+        if q16 is None or k16 is None:
+            raise ValueError("FP16 tiles need q16 and k16 (the 16-bit Q and K)")
+        if q16.dtype not in (torch.float16, torch.bfloat16):
+            raise TypeError(f"q16: dtype {q16.dtype}, expected float16 or bfloat16")
+        _expect(q16, "q16", (B, Hq, Nq, d), q16.dtype)
+        _expect(k16, "k16", (B, Hkv, Nk, d), q16.dtype)
+        _expect(v.fp16, "v.fp16 (quantize with want_fp16_v=True)", (B, Hkv, d, npad), torch.float16)
+        bufs += [fp16_bitmap, q16, k16, v.fp16]
     if q2 is not None:
         _expect(q2.codes, "q2.codes", (B, Hq, Nq, d // 2), torch.uint8)
         _expect(q2.scales, "q2.scales", (B, Hq, Nq, d // 16), torch.uint8)
@@ -325,7 +332,8 @@ def attn_qk4v8_fwd(q: NVFP4Tensor, k: NVFP4Tensor, v: MXFP8V, causal: bool,
     p.softmax_scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
     if fp16_bitmap is not None:
         p.fp16_bitmap = fp16_bitmap.data_ptr()
-        p.q16, p.k16, p.v16 = q.fp16.data_ptr(), k.fp16.data_ptr(), v.fp16.data_ptr()
+        p.q16, p.k16, p.v16 = q16.data_ptr(), k16.data_ptr(), v.fp16.data_ptr()
+        p.qk16_dtype = _dtype(q16)
     p.out_dtype = _OUT_DT[out_dtype]
     p.out = out.data_ptr()
     p.lse = lse.data_ptr() if lse is not None else None
@@ -547,10 +555,10 @@ def qk4v8_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: b
         k4 = quantize_nvfp4(k)
         v8 = quantize_mxfp8_v(v)
     else:
-        q4, k4, v8 = quantize_qkv(q, k, v, want_fp16=mixed)
+        q4, k4, v8 = quantize_qkv(q, k, v, want_fp16_v=mixed)
     bitmap = None
     if mixed:
         _, _, bitmap = tile_score_select(q4, k4, causal, fp16_frac_bp)
     return attn_qk4v8_fwd(q4, k4, v8, causal, softmax_scale, out_dtype or q.dtype,
                           fp16_bitmap=bitmap, want_lse=want_lse, underflow_aware=underflow_aware,
-                          q2=q2)
+                          q2=q2, q16=q if mixed else None, k16=k if mixed else None)

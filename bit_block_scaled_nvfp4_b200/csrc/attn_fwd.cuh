@@ -6,8 +6,9 @@
 // E4M3 as P*448 against the running max after the tile; O += P V on block-scaled FP8 tensor
 // cores (kind::mxf8f6f4, E8M0 scale per 32 tokens; P's scale is 1); O / l at the end, where
 // l sums the quantized weights. Optional FP16 tiles (ai-feeds.com ThriftAttention summary,
-// "方法" step 3): a tile marked in the selection bitmap runs QK^T and PV with kind::f16 on
-// FP16 copies of Q, K, V, with P = fp16(448 exp(s - m)), into the same (m, l, O).
+// "方法" step 3): a tile marked in the selection bitmap runs QK^T with kind::f16 on the caller's
+// 16-bit Q and K (fp16 or bf16: both products are exact) and PV on an FP16 copy of V, with
+// P = fp16(448 exp(s - m)), into the same (m, l, O).
 //
 // l comes from the tensor core: every V tile in shared memory carries 16 extra rows of 1.0
 // after its D channel rows, so the PV MMA (N = D + 16) accumulates sum_j P_j into O column D,
@@ -76,6 +77,7 @@ struct FwdArgs {
   int32_t causal;
   float softmax_scale;
   int32_t out_kind;          // 0 fp16, 1 bf16, 2 fp32
+  int32_t qk16_bf16;         // FP16 tiles: Q and K are the caller's bf16 (else fp16) tensors
 };
 
 // A work item of the persistent prefill kernel: the 128-query tile, batch and query head it
@@ -463,7 +465,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // ============================ QK^T issuer (one thread) ============================
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_block_scaled(kFmtE2M1_mxf4, kFmtE2M1_mxf4, 0, 128, 128);
-      const uint32_t idesc_qk16 = idesc_f16(128, 128);
+      const uint32_t idesc_qk16 = idesc_f16(128, 128, a.qk16_bf16 != 0);
       bool ok = true;
       int g = 0, r = 0, nq16 = 0;
       for (int it = 0; ok; ++it) {

@@ -243,8 +243,9 @@ __device__ __forceinline__ uint32_t idesc_with_sf_ids(uint32_t idesc, uint32_t a
 }
 // kind::f16: bits 4-5 D format (1 = F32), 7-9 A format (0 F16, 1 BF16), 10-12 B format,
 // 15/16 majors, 17-22 N>>3, 24-28 M>>4.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
-  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16 = false) {
+  return (1u << 4) | (bf16 ? (1u << 7) | (1u << 10) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 constexpr uint32_t kFmtE2M1_mxf4 = 1;   // E2M1 in kind::mxf4nvf4
 constexpr uint32_t kFmtE4M3 = 0;        // E4M3 in kind::mxf8f6f4

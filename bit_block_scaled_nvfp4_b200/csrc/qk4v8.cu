@@ -343,7 +343,7 @@ static qk4v8_status launch_qkv(const qk4v8_qkv_params* p, float* q_part, float* 
   a.v_n = p->v_tokens;
   const int64_t grid1 = total + static_cast<int64_t>(a.v_tiles) * p->v_bh;
   if (grid1 > 0x7fffffffLL) return QK4V8_ERR_UNSUPPORTED;
-  if (p->q16 != nullptr)
+  if (p->v16 != nullptr)
     qk_amax_v_kernel<T, D, true><<<static_cast<unsigned>(grid1), 256, 0, stream>>>(a, p->q_rows, p->k_rows, gq, gk);
   else
     qk_amax_v_kernel<T, D, false><<<static_cast<unsigned>(grid1), 256, 0, stream>>>(a, p->q_rows, p->k_rows, gq, gk);
@@ -366,11 +366,11 @@ qk4v8_status quantize_qkv(const qk4v8_qkv_params* p, void* workspace, size_t wor
   if (p->q_rows <= 0 || p->k_rows <= 0 || p->v_bh <= 0 || p->v_tokens <= 0)
     return QK4V8_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return QK4V8_ERR_UNSUPPORTED;
-  const bool f16 = p->q16 != nullptr;
-  if ((p->k16 != nullptr) != f16 || (p->v16 != nullptr) != f16) return QK4V8_ERR_INVALID_ARG;
+  const bool qk16 = p->q16 != nullptr;
+  if ((p->k16 != nullptr) != qk16) return QK4V8_ERR_INVALID_ARG;
   if (!aligned(p->q, 16) || !aligned(p->k, 16) || !aligned(p->v, 16) || !aligned(p->q_codes, 8) ||
       !aligned(p->k_codes, 8) || !aligned(p->v_codes, 16) || !aligned(workspace, 4) ||
-      (f16 && (!aligned(p->q16, 16) || !aligned(p->k16, 16) || !aligned(p->v16, 16))))
+      (qk16 && (!aligned(p->q16, 16) || !aligned(p->k16, 16))) || !aligned(p->v16, 16))
     return QK4V8_ERR_INVALID_ARG;
   if (workspace_bytes < quantize_qkv_workspace_size()) return QK4V8_ERR_INVALID_ARG;
   if (p->v_bh > 0x7fffffff / ((p->v_tokens + 127) / 128)) return QK4V8_ERR_UNSUPPORTED;
@@ -474,10 +474,13 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
     const uint64_t dq[3] = {D, static_cast<uint64_t>(Nq), static_cast<uint64_t>(B) * Hq};
     const uint64_t sq[2] = {D * 2, static_cast<uint64_t>(Nq) * D * 2};
     const uint32_t bq[3] = {64, 128, 1};
-    if (!make_map(&tq16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, p->q16, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
+    // the caller's 16-bit Q and K, in their own type
+    const CUtensorMapDataType t16 = (p->qk16_dtype == QK4V8_BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&tq16, t16, 3, p->q16, dq, sq, bq, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
     const uint64_t dk[3] = {D, static_cast<uint64_t>(Nk), static_cast<uint64_t>(B) * Hkv};
     const uint64_t sk[2] = {D * 2, static_cast<uint64_t>(Nk) * D * 2};
-    if (!make_map(&tk16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, p->k16, dk, sk, bq, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
+    if (!make_map(&tk16, t16, 3, p->k16, dk, sk, bq, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
     const uint64_t dv[2] = {static_cast<uint64_t>(npad), static_cast<uint64_t>(B) * Hkv * D};
     const uint64_t sv[1] = {static_cast<uint64_t>(npad) * 2};
     const uint32_t bv[2] = {64, D};
@@ -498,6 +501,7 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   a.causal = p->causal ? 1 : 0;
   a.softmax_scale = p->softmax_scale;
   a.out_kind = static_cast<int32_t>(p->out_dtype);
+  a.qk16_bf16 = (kMixed && p->qk16_dtype == QK4V8_BF16) ? 1 : 0;
   // Persistent: one CTA per SM (or per work item when there are fewer items).
   const int64_t items = static_cast<int64_t>(a.Tq) * B * Hq;
   if (items > INT32_MAX / 2) return QK4V8_ERR_UNSUPPORTED;
@@ -527,7 +531,7 @@ qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
     return QK4V8_ERR_INVALID_ARG;
   const bool mixed = p->fp16_bitmap != nullptr;
   if (mixed && (!p->q16 || !p->k16 || !p->v16 || !aligned(p->q16, 16) || !aligned(p->k16, 16) ||
-                !aligned(p->v16, 16)))
+                !aligned(p->v16, 16) || (p->qk16_dtype != QK4V8_F16 && p->qk16_dtype != QK4V8_BF16)))
     return QK4V8_ERR_INVALID_ARG;
   const int64_t tiles = static_cast<int64_t>((p->n_q + 127) / 128) * p->batch * p->q_heads;
   if (tiles > 0x7fffffffLL) return QK4V8_ERR_UNSUPPORTED;

@@ -176,7 +176,9 @@ qk4v8_status quantize_mxfp8_v(const void* v, qk4v8_dtype dtype, int32_t batch_he
  * (one dtype), 16-byte aligned; head_dim 64 or 128.
  * q_codes/q_scales/q_tensor_scale, k_...: as quantize_nvfp4's outputs (codes 8-byte aligned).
  * v_codes/v_scales: as quantize_mxfp8_v's outputs (codes 16-byte aligned).
- * q16/k16/v16: optional fp16 copies (all three or none), as those calls' x16 / v16.
+ * q16/k16: optional fp16 copies of Q and K (both or neither), as quantize_nvfp4's x16.
+ * v16: optional fp16 copy of V, as quantize_mxfp8_v's v16, independent of q16/k16 (the
+ * FP16-tile attention needs only this one: it reads the caller's Q and K as they are).
  * workspace >= quantize_qkv_workspace_size() bytes, 4-byte aligned (the amax partials).
  * Errors: QK4V8_ERR_INVALID_ARG for null pointers, bad sizes or alignment, a short workspace;
  * QK4V8_ERR_UNSUPPORTED for another head_dim.
@@ -239,8 +241,9 @@ qk4v8_status tile_score_select(const uint8_t* q_codes, const uint8_t* q_scales,
  * 128-key tiles, P quantized to E4M3 as P*448 against the running max after each tile,
  * O += P V on block-scaled FP8 tensor cores, O / l with l the sum of the quantized weights.
  * With fp16_bitmap set, a marked tile (ThriftAttention, method step 3) instead computes
- * S = fp16(q) fp16(k), P = fp16(448 exp(s - m)), O += P fp16(v) on FP16 tensor cores, merged
- * into the same (m, l, O).
+ * S = q k from the caller's 16-bit Q and K (fp16 or bf16, multiplied exactly by the 16-bit
+ * tensor cores), P = fp16(448 exp(s - m)), O += P fp16(v) on FP16 tensor cores, merged into
+ * the same (m, l, O).
  * Causal masking keeps key j <= query i and needs n_q == n_k.
  */
 typedef struct {
@@ -256,8 +259,9 @@ typedef struct {
   int32_t causal;
   float softmax_scale;         /* e.g. 1/sqrt(head_dim) */
   const uint8_t* fp16_bitmap;  /* optional [B*Hq, ceil(Nq/128), ceil(Nk/128)]; or NULL */
-  const void* q16;             /* fp16 [B, Hq, Nq, D] when fp16_bitmap is set */
-  const void* k16;             /* fp16 [B, Hkv, Nk, D] */
+  const void* q16;             /* when fp16_bitmap is set: the 16-bit Q [B, Hq, Nq, D] (the
+                                  tensor q_codes was quantized from; type qk16_dtype) */
+  const void* k16;             /* the 16-bit K [B, Hkv, Nk, D] (type qk16_dtype) */
   const void* v16;             /* fp16 [B, Hkv, D, Nk_pad] (quantize_mxfp8_v's v16) */
   qk4v8_dtype out_dtype;
   void* out;                   /* [B, Hq, Nq, D] out (out_dtype), 16-byte aligned */
@@ -270,6 +274,8 @@ typedef struct {
                                   MMAs into one accumulator; NULL for one Q tensor; not with
                                   fp16_bitmap */
   const uint8_t* q2_scales;
+  qk4v8_dtype qk16_dtype;      /* QK4V8_F16 or QK4V8_BF16: the type of q16 and k16 (read
+                                  only when fp16_bitmap is set) */
 } qk4v8_fwd_params;
 
 qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* params, cudaStream_t stream);

@@ -31,9 +31,12 @@ Readings (the pages are silent on each): l sums the quantized p, so constant V g
 to that constant and the weights sum to one exactly; P is encoded against the running max
 after the tile is included; no clipping of QK^T; causal means j <= i with Nq == Nk.
 
-FP16 tile (a tile marked in the selection): s_j from the FP16-rounded inputs, and
+FP16 tile (a tile marked in the selection): s_j from the 16-bit inputs as given (fp16 or bf16
+values; a 16-bit tensor core multiplies either exactly, so the page's "FP16" is read as the
+16-bit precision of the inputs, not a re-rounding of bf16 Q and K to fp16), and
 p_j = fp16(448 p~_j) / 448 (the FP16 branch works in the same P*448 units as the E4M3
-branch, so both accumulate into one O); V from its FP16-rounded copy.
+branch, so both accumulate into one O); V from its FP16-rounded copy (P and V meet in one
+FP16 product).
 
 Underflow-aware probability scaling (sns.style BitDecoding-FP4 summary, the second algorithm
 item: long-context probabilities are tiny, the E4M3 encoding of P can round whole blocks to
@@ -92,7 +95,8 @@ def attention_rows(q: np.ndarray, row_pos: np.ndarray, k: np.ndarray, v: np.ndar
     keys [128 t, 128 t + 128)).
 
     ``fp16_select(q_tile_of_rows [R], t) -> bool [R]`` marks rows whose (query tile, key
-    tile) pair takes the FP16 branch; q16/k16/v16 are then the FP16-rounded operands.
+    tile) pair takes the FP16 branch; q16/k16/v16 are then that branch's operands (Q and K as
+    given, V rounded to FP16).
     Returns the un-normalised state (m, l, O) in float64.
     """
     q = np.asarray(q, dtype=np.float64)

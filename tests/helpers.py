@@ -108,7 +108,8 @@ def oracle_prefill_rows(q, k, v, hq, rows, causal, scale, hkv_of=None, fp16_sele
     vh = OQ.mxfp8_dequantize_v(vc, vs, v.shape[2])
     kw = {}
     if fp16_select is not None:
-        kw = dict(fp16_select=fp16_select, q16=OF.fp16_round(f32(q[0, hq, rows])),
-                  k16=OF.fp16_round(f32(k[0, hk])), v16=OF.fp16_round(f32(v[0, hk])))
+        # FP16 tiles: Q and K as given (16-bit values, multiplied exactly), V rounded to fp16
+        kw = dict(fp16_select=fp16_select, q16=f32(q[0, hq, rows]).astype(np.float64),
+                  k16=f32(k[0, hk]).astype(np.float64), v16=OF.fp16_round(f32(v[0, hk])))
     m, l, o = OA.attention_rows(qh, np.asarray(rows), kh, vh, causal, scale, **kw)
     return OA.finish(m, l, o)

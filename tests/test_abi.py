@@ -107,7 +107,8 @@ def test_quantize_qkv_validation(lib):
     assert f(p(q_rows=0), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(p(head_dim=96), FAKE, wsb, None) == _lib.QK4V8_ERR_UNSUPPORTED
     assert f(p(q=FAKE + 8), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG   # misaligned
-    assert f(p(q16=FAKE), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG     # copies: all or none
+    assert f(p(q16=FAKE), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG     # Q, K copies: both or neither
+    assert f(p(v16=FAKE + 8), FAKE, wsb, None) == _lib.QK4V8_ERR_INVALID_ARG # V copy misaligned
 
 
 def test_quantize_mxfp8_validation(lib):
@@ -153,7 +154,8 @@ def test_fwd_validation(lib):
     assert f(_fwd(head_dim=96)) == _lib.QK4V8_ERR_UNSUPPORTED
     assert f(_fwd(out=FAKE + 4)) == _lib.QK4V8_ERR_INVALID_ARG
     assert f(_fwd(softmax_scale=0.0)) == _lib.QK4V8_ERR_INVALID_ARG
-    assert f(_fwd(fp16_bitmap=FAKE)) == _lib.QK4V8_ERR_INVALID_ARG  # bitmap without fp16 copies
+    assert f(_fwd(fp16_bitmap=FAKE)) == _lib.QK4V8_ERR_INVALID_ARG  # bitmap without 16-bit operands
+    assert f(_fwd(fp16_bitmap=FAKE, q16=FAKE, k16=FAKE, v16=FAKE, qk16_dtype=2)) == _lib.QK4V8_ERR_INVALID_ARG
     assert lib.attn_qk4v8_fwd(None, None) == _lib.QK4V8_ERR_INVALID_ARG
 
 

@@ -11,10 +11,14 @@ DEVICE_ERR = "contiguous tensors on one CUDA device"
 
 
 def _prefill(B, Hq, Hkv, Nq, Nk, D, fp16=False):
-    q = api._nvfp4_empty((B, Hq, Nq, D), "cpu", fp16)
-    k = api._nvfp4_empty((B, Hkv, Nk, D), "cpu", fp16)
+    q = api._nvfp4_empty((B, Hq, Nq, D), "cpu")
+    k = api._nvfp4_empty((B, Hkv, Nk, D), "cpu")
     v = api._mxfp8_empty((B, Hkv, Nk, D), "cpu", fp16)
     return q, k, v
+
+
+def _inputs16(B, Hq, Hkv, Nq, Nk, D, dtype=torch.bfloat16):
+    return torch.empty(B, Hq, Nq, D, dtype=dtype), torch.empty(B, Hkv, Nk, D, dtype=dtype)
 
 
 def _bitmap(B, Hq, N):
@@ -37,8 +41,10 @@ def test_fwd_accepts_producer_shapes(B, Hq, Hkv, Nq, Nk, D):
 @pytest.mark.parametrize("N", [128, 700, 16384])
 def test_fwd_fp16_tiles_accept_producer_shapes(N):
     q, k, v = _prefill(1, 4, 2, N, N, 128, fp16=True)
-    with pytest.raises(ValueError, match=DEVICE_ERR):
-        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, N))
+    for dt in (torch.bfloat16, torch.float16):
+        q16, k16 = _inputs16(1, 4, 2, N, N, 128, dt)
+        with pytest.raises(ValueError, match=DEVICE_ERR):
+            api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, N), q16=q16, k16=k16)
     with pytest.raises(ValueError, match=DEVICE_ERR):
         api.tile_score_select(q, k, True, 500)
 
@@ -65,14 +71,23 @@ def test_fwd_refuses_mismatched_buffers():
 
 
 def test_fwd_fp16_tiles_need_their_copies_and_a_full_bitmap():
-    q, k, v = _prefill(1, 4, 2, 700, 700, 128)                      # no FP16 copies
-    with pytest.raises(ValueError, match="want_fp16"):
-        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700))
+    q16, k16 = _inputs16(1, 4, 2, 700, 700, 128)
+    q, k, v = _prefill(1, 4, 2, 700, 700, 128)                      # no fp16 copy of V
+    with pytest.raises(ValueError, match="want_fp16_v"):
+        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700), q16=q16, k16=k16)
     q, k, v = _prefill(1, 4, 2, 700, 700, 128, fp16=True)
+    with pytest.raises(ValueError, match="q16 and k16"):
+        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700))
+    with pytest.raises(TypeError, match="k16"):                       # Q and K of two types
+        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700), q16=q16, k16=k16.half())
+    with pytest.raises(TypeError, match="q16"):
+        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700), q16=q16.float(), k16=k16)
+    with pytest.raises(ValueError, match="k16"):                      # K of another length
+        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700), q16=q16, k16=k16[:, :, :600])
     with pytest.raises(ValueError, match="fp16_bitmap"):
-        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 2, 700))
+        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 2, 700), q16=q16, k16=k16)
     with pytest.raises(ValueError, match="second Q"):
-        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700), q2=q)
+        api.attn_qk4v8_fwd(q, k, v, True, fp16_bitmap=_bitmap(1, 4, 700), q2=q, q16=q16, k16=k16)
 
 
 def test_strided_views_are_refused_before_any_call():
