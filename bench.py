@@ -25,6 +25,7 @@ import math
 import os
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -82,16 +83,49 @@ def decode_bytes(lay):
 
 
 class Clocks:
-    """nvidia-smi sampler running during the timed region."""
+    """SM clock and throttle-reason sampler running during the timed region: NVML polled every
+    2 ms from a thread (the device matched by PCI bus id), else an nvidia-smi loop."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, device_index):
         self.idx = device_index
         self.proc = None
+        self.nvml = None
+        self.samples = []          # (sm MHz, max MHz, reason names)
+        self.out = ""
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.idx)
+        bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def _poll(self, nv, h):
+        bits = [nv.nvmlClocksEventReasonHwSlowdown, nv.nvmlClocksEventReasonHwThermalSlowdown,
+                nv.nvmlClocksEventReasonSwThermalSlowdown, nv.nvmlClocksEventReasonSwPowerCap]
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), [n for n, bit in zip(self.NAMES, bits) if r & bit]))
+            except Exception:
+                break
+            self.stop.wait(0.002)
 
     def __enter__(self):
+        try:
+            nv, h = self._nvml_handle()
+            self.stop = threading.Event()
+            self.nvml = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.nvml.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
@@ -101,7 +135,9 @@ class Clocks:
         return self
 
     def __exit__(self, *a):
-        self.out = ""
+        if self.nvml is not None:
+            self.stop.set()
+            self.nvml.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -112,7 +148,10 @@ class Clocks:
 
     def summary(self):
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s_mhz, m_mhz, names in self.samples:
+            sm.append(s_mhz)
+            mx = m_mhz
+            reasons.update(names)
         for ln in (self.out or "").splitlines():
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
@@ -122,13 +161,13 @@ class Clocks:
                 mx = float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(self.NAMES, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvml" if self.samples else "nvidia-smi"}
 
 
 def dist_setup(args):

@@ -10,6 +10,7 @@
 #include "quantize.cuh"
 #include "tilescore.cuh"
 #include "attn_fwd.cuh"
+#include "attn_pp.cuh"
 #include "decode.cuh"
 #include "append.cuh"
 
@@ -510,6 +511,48 @@ static qk4v8_status launch_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   return launch_status();
 }
 
+// The FP4-only path: two query tiles per CTA, one softmax warpgroup each (attn_pp.cuh).
+template <int D>
+static qk4v8_status launch_pp(const qk4v8_fwd_params* p, cudaStream_t stream) {
+  using L = PPLayout<D>;
+  const int32_t B = p->batch, Hq = p->q_heads, Hkv = p->kv_heads;
+  const int32_t Nq = p->n_q, Nk = p->n_k;
+  const int32_t npad = (Nk + 127) / 128 * 128;
+  const CUtensorMapSwizzle qk_sw = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUtensorMap tq, tk, tv;
+  const uint64_t dq[3] = {D / 2, static_cast<uint64_t>(Nq), static_cast<uint64_t>(B) * Hq};
+  const uint64_t sq[2] = {D / 2, static_cast<uint64_t>(Nq) * (D / 2)};
+  const uint32_t bq[3] = {D / 2, 128, 1};
+  if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p->q_codes, dq, sq, bq, qk_sw)) return QK4V8_ERR_CUDA;
+  const uint64_t dk[3] = {D / 2, static_cast<uint64_t>(Nk), static_cast<uint64_t>(B) * Hkv};
+  const uint64_t sk[2] = {D / 2, static_cast<uint64_t>(Nk) * (D / 2)};
+  if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, p->k_codes, dk, sk, bq, qk_sw)) return QK4V8_ERR_CUDA;
+  const uint64_t dv[2] = {static_cast<uint64_t>(npad), static_cast<uint64_t>(B) * Hkv * D};
+  const uint64_t sv[1] = {static_cast<uint64_t>(npad)};
+  const uint32_t bv[2] = {128, D};
+  if (!make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->v_codes, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
+  static PerDeviceOnce opt_in;
+  if (!opt_in.run(current_device(), [] { return set_smem(attn_pp_kernel<D>, L::SMEM_ALLOC); }))
+    return QK4V8_ERR_CUDA;
+  FwdArgs a;
+  a.q_scales = p->q_scales; a.k_scales = p->k_scales; a.v_scales = p->v_scales;
+  a.q2_scales = nullptr;
+  a.q_ts = p->q_tensor_scale; a.k_ts = p->k_tensor_scale;
+  a.bitmap = nullptr; a.out = p->out; a.lse = p->lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.Npad = npad;
+  a.Tq = (Nq + 127) / 128; a.Tk = (Nk + 127) / 128;
+  a.causal = p->causal ? 1 : 0;
+  a.softmax_scale = p->softmax_scale;
+  a.out_kind = static_cast<int32_t>(p->out_dtype);
+  a.qk16_bf16 = 0;
+  const int64_t items = static_cast<int64_t>(a.Tq) * B * Hq;     // an upper bound of the pairs
+  if (items > INT32_MAX / 2) return QK4V8_ERR_UNSUPPORTED;
+  const int64_t n_pairs = pp_items(B, Hq, Hkv, a.Tq);
+  const int64_t grid = n_pairs < sm_count() ? n_pairs : sm_count();
+  attn_pp_kernel<D><<<static_cast<unsigned>(grid), L::THREADS, L::SMEM_ALLOC, stream>>>(tq, tk, tv, a);
+  return launch_status();
+}
+
 extern "C" {
 qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
   if (p == nullptr) return QK4V8_ERR_INVALID_ARG;
@@ -550,8 +593,8 @@ qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* p, cudaStream_t stream) {
     if (p->p_underflow_aware) return dq ? launch_fwd<64, false, true, true>(p, stream) : launch_fwd<64, false, true>(p, stream);
     return launch_fwd<64, false, false, true>(p, stream);
   }
-  if (p->head_dim == 128) return mixed ? launch_fwd<128, true>(p, stream) : launch_fwd<128, false>(p, stream);
-  return mixed ? launch_fwd<64, true>(p, stream) : launch_fwd<64, false>(p, stream);
+  if (p->head_dim == 128) return mixed ? launch_fwd<128, true>(p, stream) : launch_pp<128>(p, stream);
+  return mixed ? launch_fwd<64, true>(p, stream) : launch_pp<64>(p, stream);
 }
 
 // ------------------------------------------------------------------------------------------
