@@ -68,6 +68,9 @@ def test_workload_full_parity(name):
     (1, 2, 2, 200, 700, 128, False),     # Nq != Nk
     (1, 1, 1, 1, 1, 128, True),          # one token
     (1, 3, 3, 129, 129, 64, True),
+    (1, 3, 1, 300, 300, 128, True),      # odd GQA ratio: consecutive query tiles paired, the last alone
+    (2, 2, 2, 520, 520, 64, True),       # five query tiles a head: pairs and a lone last tile
+    (1, 2, 2, 390, 390, 128, False),     # the same without the causal mask
 ])
 def test_ragged_shapes(B, Hq, Hkv, Nq, Nk, D, causal):
     g = torch.Generator().manual_seed(Nq * 7 + Nk)
