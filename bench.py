@@ -43,9 +43,9 @@ METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of H
 # kernel on the workload (dram__bytes_read.sum + dram__bytes_write.sum). Only workloads with a
 # capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
-    "prefill_h16_n4096": 18_159_616 + 6_656,
-    "prefill_gqa_n32768": 134_921_984 + 214_016_512,
-    "mixed_prefill_n16384": 186_574_080 + 80_747_008,
+    "prefill_h16_n4096": 18_173_184 + 0,
+    "prefill_gqa_n32768": 150_773_504 + 217_906_688,
+    "mixed_prefill_n16384": 185_389_824 + 80_766_464,
     "paged_decode_s64": 2_170_382_000 + 13_552_384,
 }
 KERNEL_TIMING = "CUDA graph of the kernel(s) alone, replayed after a 256 MB L2 flush, CUDA events"
@@ -574,7 +574,9 @@ def measure(name, args, world):
         peak = pk["bf16_tflops"] * FP4_OVER_BF16
         roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "traffic": NCU_TRAFFIC_BYTES.get(name),
-                "kernel": "attn_fwd_kernel", "kernel_ms": kern_ms, "timing": KERNEL_TIMING,
+                # FP16-tile workloads run the FP16-tile instance; FP4-only ones the paired kernel
+                "kernel": "attn_fwd_kernel" if st["cfg"].get("frac_bp", 0) > 0 else "attn_pp_kernel",
+                "kernel_ms": kern_ms, "timing": KERNEL_TIMING,
                 "peak_source": f"{src} bf16 x {FP4_OVER_BF16:g} (FP4 dense)",
                 "mixed_fp4_fp8_bound_tflops": peak / 1.5}
     else:
