@@ -99,6 +99,10 @@ struct PPLayout {
   static constexpr uint32_t QK_SW = (D == 128) ? kSw64 : kSw32;
   static constexpr uint32_t QK_SBO = 8 * D / 2;
   static constexpr int THREADS = 384;
+  // Registers: 168 a thread at launch (384 threads); warpgroup 0 (producer, issuers) gives
+  // some to the two softmax warpgroups: 4*32*96 + 8*32*200 <= 384*168.
+  static constexpr int REGS_LAUNCH = 168, REGS_WG0 = 96, REGS_SOFTMAX = 200;
+  static_assert(4 * 32 * REGS_WG0 + 8 * 32 * REGS_SOFTMAX <= THREADS * REGS_LAUNCH, "register split");
 };
 
 template <int D>
@@ -179,6 +183,8 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     return bounded_wait(bar, parity, abort_flag, site(bar, tile));
   };
 
+  if (warp < 4) {
+  setmaxnreg_to<L::REGS_WG0, L::REGS_LAUNCH>();
   if (warp == 0) {
     // ================================ producer ================================
     if (lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); }
@@ -371,7 +377,9 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_wait(mma_final + 1, 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_to<L::REGS_SOFTMAX, L::REGS_LAUNCH>();
     // ================================ softmax ================================
     const int wq = warp & 3;                 // TMEM lane quadrant
     const int unit = (warp - 4) >> 2;        // the query tile this warpgroup owns
@@ -432,8 +440,12 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           x[c] = ex2_approx(t.x);
           x[c + 1] = ex2_approx(t.y);
         }
-        // The P buffer and O were last used by PV of this unit's previous tile.
-        if (n >= 1 && !waitw(pv_done + unit, (n - 1) & 1, n)) { ok = false; break; }
+        // The P buffer and O were last used by PV of this unit's previous tile (all lanes poll:
+        // the scores are live here).
+        if (n >= 1 && !bounded_wait_warp_all(pv_done + unit, (n - 1) & 1, abort_flag, site(pv_done + unit, n))) {
+          ok = false;
+          break;
+        }
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {               // 16 keys per 16-byte chunk
           uint32_t w4[4];

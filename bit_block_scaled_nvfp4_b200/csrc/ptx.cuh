@@ -110,6 +110,27 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
   if (mbar_try_wait(bar, parity)) return true;
   return bounded_wait_slow(bar, parity, flag, site);
 }
+// The same with every lane polling until the phase completes (no divergent slow path), for
+// waits while a thread holds many live values: a lane-0-only slow path there leaves the
+// register allocator without room when the warp's register count is set by setmaxnreg.
+__device__ __forceinline__ bool bounded_wait_warp_all(uint64_t* bar, uint32_t parity,
+                                                      volatile int* flag, uint64_t site) {
+  if (__any_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (__any_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if (__any_sync(0xffffffffu, *flag != 0)) return false;
+    if (__any_sync(0xffffffffu, clock64() - t0 > kWaitLimitCycles)) {
+      if ((threadIdx.x & 31) == 0) {
+        flag_error(kStatusTimeout);
+        record_timeout(site);
+        *flag = 1;
+      }
+      __syncwarp();
+      return false;
+    }
+  }
+}
 // The same for a whole (converged) warp: every lane polls once (one instruction, so every
 // lane sees the same phase); a pending phase is then waited for by lane 0 alone and the
 // outcome broadcast, so that every lane agrees.
@@ -133,6 +154,26 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+// A warpgroup's register count moved from the launch's per-thread count kLaunch to N (once, by
+// all four warps of the warpgroup, at the start of its role): .inc above it, .dec below it,
+// nothing when equal (an .inc or .dec the other way round is not a valid instruction). The
+// warpgroups' counts must not add up to more than the launch allocated, or an .inc waits for
+// registers that never free.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N, int kLaunch>
+__device__ __forceinline__ void setmaxnreg_to() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256 && kLaunch % 8 == 0, "setmaxnreg count");
+  if constexpr (N > kLaunch) setmaxnreg_inc<N>();
+  else if constexpr (N < kLaunch) setmaxnreg_dec<N>();
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -531,8 +531,16 @@ static qk4v8_status launch_pp(const qk4v8_fwd_params* p, cudaStream_t stream) {
   const uint64_t sv[1] = {static_cast<uint64_t>(npad)};
   const uint32_t bv[2] = {128, D};
   if (!make_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->v_codes, dv, sv, bv, CU_TENSOR_MAP_SWIZZLE_128B)) return QK4V8_ERR_CUDA;
+  // One-time set-up per device: the shared-memory opt-in, and a check that the kernel launches
+  // with the register count its setmaxnreg split is computed from (a split above the launch's
+  // registers would leave the softmax warps waiting for registers that never free).
   static PerDeviceOnce opt_in;
-  if (!opt_in.run(current_device(), [] { return set_smem(attn_pp_kernel<D>, L::SMEM_ALLOC); }))
+  if (!opt_in.run(current_device(), [] {
+        cudaFuncAttributes fa;
+        return set_smem(attn_pp_kernel<D>, L::SMEM_ALLOC) &&
+               cudaFuncGetAttributes(&fa, attn_pp_kernel<D>) == cudaSuccess &&
+               fa.numRegs == L::REGS_LAUNCH;
+      }))
     return QK4V8_ERR_CUDA;
   FwdArgs a;
   a.q_scales = p->q_scales; a.k_scales = p->k_scales; a.v_scales = p->v_scales;
