@@ -43,8 +43,8 @@ METRIC = "QK4V8 attention TFLOPS & % of FP4 tensor peak; decode KV GB/s & % of H
 # kernel on the workload (dram__bytes_read.sum + dram__bytes_write.sum). Only workloads with a
 # capture of the current kernel have an entry; the others report null.
 NCU_TRAFFIC_BYTES = {
-    "prefill_h16_n4096": 18_173_184 + 0,
-    "prefill_gqa_n32768": 150_773_504 + 217_906_688,
+    "prefill_h16_n4096": 18_167_040 + 1_280,
+    "prefill_gqa_n32768": 154_096_128 + 217_831_168,
     "mixed_prefill_n16384": 185_389_824 + 80_766_464,
     "paged_decode_s64": 2_170_382_000 + 13_552_384,
 }
