@@ -450,11 +450,11 @@ def _inputs(name):
     return _INPUTS[name]
 
 
-def oracle_sample(name, rows=256, heads=1):
+def oracle_sample(name, rows=256, heads=1, seqs=1):
     """Time the oracle, as it stands, on a bounded sample of the workload: ``heads`` query
     heads x ``rows`` query rows spread over the sequence (prefill; the whole-tensor scales
-    are computed once), or ``rows // 64`` sequences' worth of decode steps. Returns
-    (seconds, algorithmic units (FLOPs or bytes) done, description)."""
+    are computed once), or one decode step of the ``seqs`` shortest sequences (decode).
+    Returns (seconds, algorithmic units (FLOPs or bytes) done, description)."""
     from oracle import attention as OA
     from oracle import quant as OQ
     from oracle import paged as OP
@@ -462,23 +462,29 @@ def oracle_sample(name, rows=256, heads=1):
         lay = _inputs(name)
         cfg = lay.cfg
         q = workloads.make_decode_query(lay).float().numpy()
+        lens = lay.lens.numpy()
+        picked = [int(i) for i in np.argsort(lens, kind="stable")[:max(1, seqs)]]
+        seqs_kv = [workloads.make_decode_sequence(lay, s) for s in picked]
+        per_tok = cfg["d"] // 2 + cfg["d"] // 16 + cfg["d"] + cfg["d"] // 32
+        g = cfg["Hq"] // cfg["Hkv"]
         t0 = time.perf_counter()
         qc, qs, qt = OQ.nvfp4_quantize(q)
         qh = OQ.nvfp4_dequantize(qc, qs, qt)
-        s = int(np.argmin(lay.lens.numpy()))
-        k, v = workloads.make_decode_sequence(lay, s)
-        n = int(lay.lens[s])
-        kc, ks, vc, vs = OP.quantize_sequence(k.float().numpy(), v.float().numpy(),
-                                              workloads.DECODE_K_TENSOR_SCALE)
-        kh = OQ.nvfp4_dequantize(kc, ks, np.float32(workloads.DECODE_K_TENSOR_SCALE))
-        vh = OQ.mxfp8_dequantize_v(vc, vs, n)
-        g = cfg["Hq"] // cfg["Hkv"]
-        for h in range(cfg["Hkv"]):
-            OA.decode_rows(qh[s, h * g:(h + 1) * g], kh[h], vh[h], n, 1 / math.sqrt(cfg["d"]), 4096)
+        units = 0
+        for s, (k, v) in zip(picked, seqs_kv):
+            n = int(lens[s])
+            kc, ks, vc, vs = OP.quantize_sequence(k.float().numpy(), v.float().numpy(),
+                                                  workloads.DECODE_K_TENSOR_SCALE)
+            kh = OQ.nvfp4_dequantize(kc, ks, np.float32(workloads.DECODE_K_TENSOR_SCALE))
+            vh = OQ.mxfp8_dequantize_v(vc, vs, n)
+            for h in range(cfg["Hkv"]):
+                OA.decode_rows(qh[s, h * g:(h + 1) * g], kh[h], vh[h], n,
+                               1 / math.sqrt(cfg["d"]), 4096)
+            units += ((n + 63) // 64) * 64 * cfg["Hkv"] * per_tok
         dt = time.perf_counter() - t0
-        per_tok = cfg["d"] // 2 + cfg["d"] // 16 + cfg["d"] + cfg["d"] // 32
-        units = ((n + 63) // 64) * 64 * cfg["Hkv"] * per_tok
-        return dt, float(units), f"1 sequence ({n} tokens) x {cfg['Hkv']} KV heads of one decode step"
+        toks = "+".join(str(int(lens[s])) for s in picked)
+        return dt, float(units), (f"{len(picked)} sequence(s) ({toks} tokens) x {cfg['Hkv']} "
+                                  f"KV heads of one decode step")
     w = _inputs(name)
     cfg = w.cfg
     N, d = cfg["N"], cfg["d"]
@@ -620,7 +626,8 @@ def measure(name, args, world):
                         "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                         "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
     if world == 1 and not args.no_cpu_baseline:          # the oracle is timed at N = 1 only
-        dt, u, desc = oracle_sample(name, rows=64, heads=1)
+        # about ten seconds of host work on 16 cores: 3 query heads x 4096 rows, or 3 sequences
+        dt, u, desc = oracle_sample(name, rows=4096, heads=3, seqs=3)
         cv = u / dt / (1e12 if st["kind"] == "prefill" else 1e9)
         out["cpu_baseline"] = {"value": cv, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
                                "sample": desc, "seconds": dt}
