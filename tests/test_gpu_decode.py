@@ -91,6 +91,25 @@ def test_decode_parity(lens, hq, hkv, split):
     assert api.check_status() == 0
 
 
+def test_one_split_per_sequence_is_the_one_pass_method():
+    """With split_tokens at least the longest context (16384, the largest split the kernel
+    takes), every sequence is a single split and the kernel computes the sequential method of
+    the BitDecoding-FP4 summary (one running max over the whole cache): parity at the bar
+    against the oracle's decode without splits, at 1, 333, 5000 and 16384 tokens."""
+    lens, hq, hkv, d = [16384, 5000, 333, 1], 32, 8, 128
+    cache, table, seqs = _build(lens, hkv, d, seed=41)
+    g = torch.Generator().manual_seed(43)
+    q = torch.randn(len(lens), hq, d, generator=g).to(torch.bfloat16)
+    q4 = api.quantize_nvfp4(q.to(DEV))
+    ctx = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    out, lse = api.attn_qk4v8_decode_paged(q4, cache, table.to(DEV), ctx, max(lens), 16384,
+                                           want_lse=True, out_dtype=torch.float32)
+    want, wlse = _oracle_decode(q, seqs, lens, hq, hkv, 0, 1 / math.sqrt(d))
+    assert_attention_close(f32(out), want, "decode, one split per sequence vs one pass")
+    assert np.max(np.abs(lse.cpu().numpy() - wlse)) < 1e-3
+    assert api.check_status() == 0
+
+
 def test_page_permutation_is_bit_invariant():
     lens = [900, 300]
     c1, t1, seqs = _build(lens, 2, 128, seed=5, shuffle=False)
