@@ -14,7 +14,8 @@ Timing: inputs resident in HBM; W warm-up steps; then K steps, each bracketed by
 on the launching stream, with a 256 MB L2 flush between steps (outside the events); barrier +
 synchronize on both sides; max over ranks. `e2e` repeats the step through the same public
 API with the inputs copied from pinned host memory and the output read back inside the timed
-region. Multi-GPU (torchrun): independent replicas, one per GPU (no collective in the path).
+region, one after another; `e2e_overlapped` runs the same with each step's copies on copy
+streams of their own, overlapped with the neighbouring steps' compute. Multi-GPU (torchrun): independent replicas, one per GPU (no collective in the path).
 `--impl reference` times the CPU oracle on a bounded sample of the same workload instead.
 """
 from __future__ import annotations
@@ -254,8 +255,9 @@ def make_prefill_step(name):
     qbytes = (nq + nk) * (2 + 0.5 + 1 / 16) + nv * (2 + 1 + 1 / 32) + (2 * nv if mixed else 0)
     # algorithmic scoring bytes: the Q and K codes and E4M3 scales read once
     sbytes = (nq + nk) * (0.5 + 1 / 16)
-    return dict(cfg=cfg, step=step, inputs=(q, k, v), host=host, launches=launches,
-                flops=prefill_flops(cfg), kind="prefill", quant=quant, quant_bytes=qbytes,
+    return dict(cfg=cfg, step=step, step_on=lambda ins: step(*ins), inputs=(q, k, v), host=host,
+                launches=launches, flops=prefill_flops(cfg), kind="prefill", quant=quant,
+                quant_bytes=qbytes, device_bytes=sum(t.numel() * t.element_size() for t in (q, k, v)),
                 score=(score_only, sbytes) if mixed else None,
                 attn_only=attn_only)
 
@@ -284,6 +286,15 @@ def make_decode_step(name):
     def step(q=q):
         return plan.run(quant(q))
 
+    plans = {table.data_ptr(): plan}
+
+    def step_on(ins):
+        # one step on another set of device inputs (query, page table, lengths): a plan per set
+        q_, t_, c_ = ins
+        if t_.data_ptr() not in plans:
+            plans[t_.data_ptr()] = api.DecodePlan(cache, t_, c_, max(lens), split, cfg["S"], cfg["Hq"])
+        return plans[t_.data_ptr()].run(quant(q_))
+
     prep = {}
 
     def attn_only():
@@ -294,7 +305,8 @@ def make_decode_step(name):
 
     kv, total = decode_bytes(lay)
     host = [workloads.make_decode_query(lay).pin_memory(), lay.page_table.pin_memory(), lay.lens.pin_memory()]
-    return dict(cfg=cfg, step=step, inputs=(q, table, ctx), host=host, launches=4, kv_bytes=kv,
+    return dict(cfg=cfg, step=step, step_on=step_on, inputs=(q, table, ctx), host=host, launches=4,
+                kv_bytes=kv, device_bytes=kv,
                 bytes=total, kind="decode", split=split, lay=lay, quant=quant, attn_only=attn_only,
                 quant_bytes=q.numel() * (2 + 0.5 + 1 / 16))
 
@@ -402,6 +414,74 @@ def time_steps(st, K, W, world):
     kern_ms = sum(a.elapsed_time(b) for a, b in zip(k0, k1)) / K
     st["quant_ms"] = sum(a.elapsed_time(b) for a, b in zip(q0, q1)) / K
     return step_ms, kern_ms
+
+
+L2_BYTES = 126 << 20
+
+
+def time_e2e_overlapped(st, K, world):
+    """The same steps through the public API as a streaming caller runs them: each step's inputs
+    copied from pinned host memory on a copy stream into one of two device input sets used in
+    turn, the step on the compute stream once its copy has landed, and its output read back into
+    pinned memory on a third stream, so that one step's copies overlap its neighbours' compute.
+    A set is refilled only after the step that read it, and a step's output buffer is reused
+    only after its read-back. Device time from the first copy in to the last copy out over K
+    steps (after one untimed pass that allocates); ms per step. Inputs smaller than twice the
+    L2 get a 256 MB flush on the compute stream before each step, inside the timed region."""
+    host = st["host"]
+    sets = [list(st["inputs"]), [t.clone() for t in st["inputs"]]]
+    run = st["step_on"]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if st["device_bytes"] < 2 * L2_BYTES else None
+    cs = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    out_host = [None, None]
+
+    def one_pass(n, timed):
+        freed = [None, None]          # the compute stream has finished the step that read set b
+        read_back = [None, None]      # the read-back of the last output made from set b is done
+        t0 = t1 = None
+        if timed:
+            t0 = torch.cuda.Event(enable_timing=True)
+            t0.record(s_in)
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                if freed[b] is not None:
+                    s_in.wait_event(freed[b])
+                for d_, h_ in zip(sets[b], host):
+                    d_.copy_(h_, non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(s_in)
+            cs.wait_event(landed)
+            if read_back[b] is not None:
+                cs.wait_event(read_back[b])
+            if flush is not None:
+                flush.zero_()
+            out = run(sets[b])
+            out = out[0] if isinstance(out, tuple) else out
+            done = torch.cuda.Event()
+            done.record(cs)
+            freed[b] = done
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done)
+                if out_host[b] is None:
+                    out_host[b] = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+                out_host[b].copy_(out, non_blocking=True)
+                rb = torch.cuda.Event()
+                rb.record(s_out)
+                read_back[b] = rb
+            out.record_stream(s_out)
+        if timed:
+            t1 = torch.cuda.Event(enable_timing=True)
+            t1.record(s_out)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n if timed else None
+
+    barrier(world)
+    one_pass(2, False)
+    ms = one_pass(K, True)
+    barrier(world)
+    return ms
 
 
 def time_e2e(st, K, world):
@@ -557,6 +637,7 @@ def measure(name, args, world):
         with Clocks(torch.cuda.current_device()) as clk:
             step_ms, kern_ms = time_steps(st, args.steps, args.warmup, world)
         e2e_ms, h2d, d2h = time_e2e(st, max(3, args.steps // 3), world)
+        e2e_ov_ms = time_e2e_overlapped(st, max(4, args.steps // 3), world)
         status = api.check_status()
         # every rank takes the same decision, so that all of them run the same collectives
         agreed = max_over_ranks(float(status), world)
@@ -569,12 +650,14 @@ def measure(name, args, world):
     step_ms = max_over_ranks(step_ms, world)
     kern_ms = max_over_ranks(kern_ms, world)
     e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_ov_ms = max_over_ranks(e2e_ov_ms, world)
     quant_ms = max_over_ranks(st["quant_ms"], world)
     pk, src = peaks()
     if st["kind"] == "prefill":
         units = st["flops"]
         value = units * world / (step_ms * 1e-3) / 1e12
         e2e_v = units * world / (e2e_ms * 1e-3) / 1e12
+        e2e_ov = units * world / (e2e_ov_ms * 1e-3) / 1e12
         unit = "TFLOP/s"
         ach = units / (kern_ms * 1e-3) / 1e12
         peak = pk["bf16_tflops"] * FP4_OVER_BF16
@@ -589,6 +672,7 @@ def measure(name, args, world):
         units = st["bytes"]
         value = units * world / (step_ms * 1e-3) / 1e9
         e2e_v = units * world / (e2e_ms * 1e-3) / 1e9
+        e2e_ov = units * world / (e2e_ov_ms * 1e-3) / 1e9
         unit = "GB/s"
         ach = st["kv_bytes"] / (kern_ms * 1e-3) / 1e9
         peak = pk["hbm_gbs"]
@@ -599,6 +683,10 @@ def measure(name, args, world):
     out = {"value": value, "unit": unit, "ms_per_step": step_ms, "config": config_of(name),
            "roofline": roof,
            "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           # the same with each step's copies overlapped with its neighbours' compute
+           "e2e_overlapped": {"value": e2e_ov, "unit": unit, "ms_per_step": e2e_ov_ms,
+                              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                              "streams": "copy in, compute, copy out; two input sets in turn"},
            "gpu_launches": st["launches"] * args.steps,
            # the quantize kernels of the step, timed as a graph of their own after an L2 flush
            # (algorithmic bytes: the amax pass's second read of each input is not counted)
@@ -626,8 +714,8 @@ def measure(name, args, world):
                         "achieved_gbs": nbytes / (ms * 1e-3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                         "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
     if world == 1 and not args.no_cpu_baseline:          # the oracle is timed at N = 1 only
-        # about ten seconds of host work on 16 cores: 3 query heads x 4096 rows, or 3 sequences
-        dt, u, desc = oracle_sample(name, rows=4096, heads=3, seqs=3)
+        # about ten seconds of host work on 16 cores: 5 query heads x 4096 rows, or 8 sequences
+        dt, u, desc = oracle_sample(name, rows=4096, heads=5, seqs=8)
         cv = u / dt / (1e12 if st["kind"] == "prefill" else 1e9)
         out["cpu_baseline"] = {"value": cv, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
                                "sample": desc, "seconds": dt}
