@@ -108,9 +108,8 @@ struct FwdLayout {
   // softmax groups fall into step and contend for the exponential unit at the same time. In
   // the FP16-tile kernel a selected tile takes two consecutive stages, its FP16 K in the first
   // and its FP16 V in the second, so a stage is large enough for either.
-  static constexpr bool kSplit = false;
   static constexpr int NK = 4;
-  static constexpr int NVS = 4;
+  static constexpr int NVS = NK;                        // V shares each K stage
   // P buffers, one per tile parity: the exponentials of tile g wait for PV(g - 2).
   static constexpr int NP = 2;
   static constexpr int KSTEPS = D / 64;                 // FP4 MMAs per QK (K = 64 each)
@@ -124,7 +123,6 @@ struct FwdLayout {
   static constexpr int OFF_PSF = OFF_QSF + 2048;                          // all 1.0 (E8M0 127)
   // Stage s: one block [K | V (+ ones rows) | K scales | V scales] (measured faster than
   // separate K and V arrays).
-  static constexpr bool kInterleaved = true;
   // P scale factors of the underflow-aware variant, two chunks by tile parity (row r's four
   // 32-key block scales in the word at (r % 32) * 16 + (r / 32) * 4)
   static constexpr int OFF_PSFU = OFF_PSF + 1024;
@@ -132,21 +130,11 @@ struct FwdLayout {
   static constexpr int F16_TILE = 128 * D * 2;     // FP16 Q, K or V (no ones rows) of a tile
   static constexpr int STG_FP4 = K_BYTES + V_BYTES + 2048;
   static constexpr int STG_BYTES = (kMixed && F16_TILE > STG_FP4) ? F16_TILE : STG_FP4;
-  static constexpr int OFF_VSTG = OFF_STG + NK * (K_BYTES + 1024);
-  __device__ static constexpr int k_off(int s) {
-    return kInterleaved ? OFF_STG + s * STG_BYTES : OFF_STG + s * (K_BYTES + 1024);
-  }
-  __device__ static constexpr int k_sf_off(int s) {
-    return kInterleaved ? k_off(s) + K_BYTES + V_BYTES : k_off(s) + K_BYTES;
-  }
-  __device__ static constexpr int v_off(int s) {
-    return kInterleaved ? k_off(s) + K_BYTES : OFF_VSTG + s * (V_BYTES + 1024);
-  }
-  __device__ static constexpr int v_sf_off(int s) {
-    return kInterleaved ? k_off(s) + K_BYTES + V_BYTES + 1024 : v_off(s) + V_BYTES;
-  }
-  static constexpr int OFF_P = kInterleaved ? OFF_STG + NK * STG_BYTES
-                                            : OFF_VSTG + NVS * (V_BYTES + 1024);  // NP x 16 KB
+  __device__ static constexpr int k_off(int s) { return OFF_STG + s * STG_BYTES; }
+  __device__ static constexpr int k_sf_off(int s) { return k_off(s) + K_BYTES + V_BYTES; }
+  __device__ static constexpr int v_off(int s) { return k_off(s) + K_BYTES; }
+  __device__ static constexpr int v_sf_off(int s) { return k_off(s) + K_BYTES + V_BYTES + 1024; }
+  static constexpr int OFF_P = OFF_STG + NK * STG_BYTES;                   // NP x 16 KB
   static constexpr int OFF_RED = OFF_P + NP * 16384;   // running max hand-off [2][128], final [128]
   static constexpr int OFF_Q16 = OFF_RED + 2048;
   // The FP16 PV's ones rows (the row sum l in column D of O): 16 rows of 1.0 for each 64-key
@@ -158,11 +146,12 @@ struct FwdLayout {
   static constexpr int OFF_Q2 = OFF_ONES16 + (kMixed ? 2 * 2048 : 0);
   static constexpr int OFF_Q2SF = OFF_Q2 + (kDQ ? 2 * Q_BYTES : 0);
   static constexpr int OFF_BAR = OFF_Q2SF + (kDQ ? 2048 : 0);
+  // barriers: 4 for Q, a full/empty pair per stage, 2 NK spare words (kept so the layout
+  // is unchanged), 2 NP for P and 17 singles and pairs (kernel head)
   static constexpr int N_BARS = 2 * NK + 2 * NVS + 2 * NP + 17;
   static constexpr int SMEM_BYTES = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;                     // alignment slack
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory");
-  static_assert(NK == NVS, "a single ring has one stage count");
   static_assert(STG_BYTES % 1024 == 0 && OFF_STG % 1024 == 0 && OFF_Q16 % 1024 == 0 &&
                 OFF_ONES16 % 1024 == 0, "1024-byte aligned operand atoms");
   // TMEM columns. S_b at T_S + 128 b; Q scale factors in two slots by item parity, K and V
@@ -202,8 +191,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   uint64_t* q_empty = bars + 2;            // [2], by item parity
   uint64_t* k_full = bars + 4;             // [NK]
   uint64_t* k_empty = k_full + L::NK;
-  uint64_t* v_full = L::kSplit ? k_empty + L::NK : k_full;       // [NVS]
-  uint64_t* v_empty = L::kSplit ? v_full + L::NVS : k_empty;
+  uint64_t* v_full = k_full;               // V lands on its stage's full barrier with K
+  uint64_t* v_empty = k_empty;             // ... and frees it with K (two commits)
   uint64_t* s_full = bars + 4 + 2 * L::NK + 2 * L::NVS;          // [2], by tile parity
   uint64_t* s_free = s_full + 2;           // [2], by tile parity
   uint64_t* m_ready = s_full + 4;          // [2], by tile parity: running max handed on
@@ -225,12 +214,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int i = 0; i < 2; ++i) { mbar_init(q_full + i, 33); mbar_init(q_empty + i, 1); }
     // full: the TMA's expect-tx arrival plus one cp.async arrival per producer lane (a single
     // ring: K and V on one barrier; its empty barrier takes both issuers' commits)
-    if constexpr (L::kSplit) {
-      for (int s = 0; s < L::NK; ++s) { mbar_init(k_full + s, 33); mbar_init(k_empty + s, 1); }
-      for (int s = 0; s < L::NVS; ++s) { mbar_init(v_full + s, 33); mbar_init(v_empty + s, 1); }
-    } else {
-      for (int s = 0; s < L::NK; ++s) { mbar_init(k_full + s, 33); mbar_init(k_empty + s, 2); }
-    }
+    for (int s = 0; s < L::NK; ++s) { mbar_init(k_full + s, 33); mbar_init(k_empty + s, 2); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_free + i, 4);
       mbar_init(s_full + i, 1);
