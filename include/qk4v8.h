@@ -168,9 +168,9 @@ qk4v8_status quantize_mxfp8_v(const void* v, qk4v8_dtype dtype, int32_t batch_he
  * quantize_qkv — Q and K to NVFP4 (each with its own dynamic tensor scale, exactly as
  * quantize_nvfp4 with tensor_scale_in <= 0) and V to MXFP8 (exactly as quantize_mxfp8_v), for
  * one attention call, in two launches: the amax pass of Q and K (per-CTA maxima, no grid-wide
- * wait), then one launch that encodes all three. The encode launch takes Q and K from their
- * last 16-element blocks to their first, so the parts the amax pass read last, still cached in
- * L2, are read again first. Same formats and arithmetic as the per-tensor calls (the tqpw.cn
+ * wait) together with V's MXFP8 encode (V needs no tensor scale), then one launch that encodes
+ * Q and K. The encode launch takes Q and K from their last 16-element blocks to their first,
+ * so the parts the amax pass read last, still cached in L2, are read again first. Same formats and arithmetic as the per-tensor calls (the tqpw.cn
  * article §2.2 for NVFP4, §2.1 for MXFP8); outputs are bit-identical to theirs.
  * q [q_rows, head_dim], k [k_rows, head_dim], v [v_bh, v_tokens, head_dim]: dense fp16/bf16
  * (one dtype), 16-byte aligned; head_dim 64 or 128.
@@ -286,7 +286,8 @@ qk4v8_status attn_qk4v8_fwd(const qk4v8_fwd_params* params, cudaStream_t stream)
  * tensor-core MMA; P quantization fused). Split-K: the keys of a sequence are cut into
  * splits of split_tokens keys (a multiple of 128); each split runs the QK4V8 online softmax
  * from its own running max, and the splits merge exactly (M = max m_s,
- * O = sum e^(m_s - M) O_s / sum e^(m_s - M) l_s).
+ * O = sum e^(m_s - M) O_s / sum e^(m_s - M) l_s). With split_tokens at least the longest
+ * context every sequence is one split: the sequential method with one running max.
  * Page layout (64 tokens per page, per page and KV head):
  *   K codes [64, D/2], K scales [64, D/16] (NVFP4, one FP32 scale for the whole cache),
  *   V codes [D, 64] (token-contiguous), V scales [D, 2] (E8M0 per 32 tokens).
